@@ -1,0 +1,452 @@
+/*
+ * dspark_oracle.c -- TEST INFRASTRUCTURE, NOT PART OF THE PRODUCT.
+ *
+ * A plain, slow, double-precision CPU statement of DSpark's per-step
+ * speculative-decoding hot path: the Markov-head draft, the
+ * confidence-scheduled prefix cut and the lossless rejection-sampling
+ * verify.  Only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The CUDA library
+ * shares no code, header, table or helper with it, and neither side
+ * includes or calls the other.
+ *
+ * Sources (page title, section):
+ *   [yage]       yage.ai, "DSpark speculative decoding hardware scheduling":
+ *                the first-order Markov head paragraph (the formula
+ *                p(x_k|x_{k-1}) = softmax(base_logit_k + transition_bias)),
+ *                the rejection-sampling paragraph (exact per-token p_d),
+ *                the SPS(B) scheduler paragraph (rank by calibrated
+ *                survival, stop before throughput drops).
+ *   [freeaitool] freeaitool.com, "DeepSeek DSpark complete guide":
+ *                section 3.1 (Markov head, rank-256 low-rank transition),
+ *                section 4.1 (confidence head c_k, sequential temperature
+ *                scaling), section 4.2 (greedy ordering + early stop).
+ *   [legalagi]   legalagi.cn, "读懂 DSpark：一个律师外行眼里的 DeepSeek 推理新论文":
+ *                section 三 (draft -> verify -> keep the longest accepted
+ *                prefix; lossless), section 五 (early stop keeps it lossless).
+ * The accept/residual/bonus rule itself is the textbook speculative
+ * sampling rule (Leviathan, Kalman & Matias 2023; Chen et al. 2023): the
+ * pages only say that verification compares draft and target
+ * probabilities and needs the exact p_d.
+ *
+ * Parity status (what pins each function; the tests live in
+ * tests/test_oracle_pins.py):
+ *   oracle_draft_row / oracle_draft : pinned (W=0 reduces to independent
+ *       categorical sampling checked against numpy searchsorted; a
+ *       constructed deterministic transition chain; exact enumeration of
+ *       the Markov chain on V=4, K=3 against a 10^6-sample histogram; a
+ *       hand-worked V=4 example under tests/golden/).
+ *   oracle_prefix : pinned (flat / steep cost limits, T_k=1 reduces to the
+ *       logistic function, prefix property, linear cost without knee equals
+ *       the argmax over prefix lengths of the sorted survival list).
+ *   oracle_verify : pinned (p_d = p_t accepts everything, E[accept] =
+ *       1 - TV, chi-square losslessness on V=8 at positions 1 and 2, exact
+ *       E[n_acc] by enumeration).
+ *
+ * Numerical conventions (stated once, used everywhere):
+ *   - inputs are read exactly (fp32 and bf16 values are exact in double);
+ *   - 1/T is supplied by the caller as an fp32 value and used as is;
+ *   - inverse CDF: the smallest index i with C_i > u*Z, where C_i is the
+ *     running sum of the weights; if rounding leaves no such i, the last
+ *     index with non-zero weight;
+ *   - margin of a draw = min(u*Z - C_{i-1}, C_i - u*Z) / Z.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ */
+/* scalar helpers                                                      */
+/* ------------------------------------------------------------------ */
+
+static double bf16_value(uint16_t h)
+{
+    uint32_t bits = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+/* element (row, col) of a [rows, r] matrix stored as fp32 or bf16 */
+static double mat_at(const void *m, int is_bf16, int r, long row, int col)
+{
+    if (is_bf16)
+        return bf16_value(((const uint16_t *)m)[row * (long)r + col]);
+    return (double)((const float *)m)[row * (long)r + col];
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* ------------------------------------------------------------------ */
+/* draft                                                               */
+/* ------------------------------------------------------------------ */
+
+/*
+ * One draft distribution row, as logits:
+ *   l_v = (base_v + sum_i U[x_prev, i] * W[v, i]) * inv_temp
+ * [yage, Markov-head paragraph]: the transition bias is a lookup of the
+ * previous token in a V x V low-rank matrix, here U[x_prev] . W^T with
+ * rank r ([freeaitool 3.1]).  x_prev < 0 means "no previous token": the
+ * bias is left out.
+ */
+void oracle_draft_row(const float *base_row, const void *U, const void *W,
+                      int uw_bf16, int V, int r, int x_prev, double inv_temp,
+                      double *logits)
+{
+    double *u = NULL;
+    if (x_prev >= 0) {
+        u = (double *)malloc(sizeof(double) * (size_t)r);
+        for (int i = 0; i < r; ++i)
+            u[i] = mat_at(U, uw_bf16, r, x_prev, i);
+    }
+    for (int v = 0; v < V; ++v) {
+        double bias = 0.0;
+        if (u) {
+            for (int i = 0; i < r; ++i)
+                bias += u[i] * mat_at(W, uw_bf16, r, v, i);
+        }
+        logits[v] = ((double)base_row[v] + bias) * inv_temp;
+    }
+    free(u);
+}
+
+/* softmax weights w_v = exp(l_v - max l); returns Z = sum w, sets *m */
+static double softmax_weights(const double *l, int V, double *w, double *m)
+{
+    double mx = -INFINITY;
+    for (int v = 0; v < V; ++v)
+        if (l[v] > mx)
+            mx = l[v];
+    double z = 0.0;
+    for (int v = 0; v < V; ++v) {
+        w[v] = exp(l[v] - mx);
+        z += w[v];
+    }
+    *m = mx;
+    return z;
+}
+
+/* inverse CDF over weights w (total Z): smallest i with C_i > u*Z */
+static int inverse_cdf(const double *w, int V, double total, double u,
+                       double *margin)
+{
+    double target = u * total;
+    double c = 0.0;
+    for (int v = 0; v < V; ++v) {
+        double prev = c;
+        c += w[v];
+        if (c > target) {
+            double a = target - prev, b = c - target;
+            *margin = (a < b ? a : b) / total;
+            return v;
+        }
+    }
+    /* rounding left no crossing: last index with non-zero weight */
+    for (int v = V - 1; v >= 0; --v)
+        if (w[v] > 0.0) {
+            *margin = 0.0;
+            return v;
+        }
+    *margin = 0.0;
+    return 0;
+}
+
+/*
+ * The semi-autoregressive Markov-head draft for a batch of B requests,
+ * K sequential positions each ([freeaitool 3.1]: parallel backbone gives
+ * base logits for every position, the sequential head corrects them from
+ * the token actually sampled at the previous position; [yage, Markov-head
+ * paragraph] for the formula).
+ *
+ *   base       [B, K, V] fp32        base_logit_k per request and position
+ *   U, W       [V, r] fp32 or bf16   low-rank transition factors
+ *   prev_token [B]                   token before position 1 (<0: no bias)
+ *   inv_temp   [B] or NULL           fp32 1/T_b (NULL: 1)
+ *   u_draft    [B, K]                uniforms in [0, 1)
+ * outputs
+ *   tokens [B, K], p_tok [B, K] = p_d(x_k), lse [B, K] = log sum exp(l),
+ *   margin [B, K] = CDF margin of each draw.
+ */
+int oracle_draft(const float *base, const void *U, const void *W, int uw_bf16,
+                 int V, int r, int B, int K, const int32_t *prev_token,
+                 const float *inv_temp, const float *u_draft, int32_t *tokens,
+                 double *p_tok, double *lse, double *margin)
+{
+    if (V <= 0 || r <= 0 || B < 0 || K < 0)
+        return 1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+        double *l = (double *)malloc(sizeof(double) * (size_t)V);
+        double *w = (double *)malloc(sizeof(double) * (size_t)V);
+        double it = inv_temp ? (double)inv_temp[b] : 1.0;
+        int x = prev_token[b];
+        for (int k = 0; k < K; ++k) {
+            const float *brow = base + ((size_t)b * K + k) * (size_t)V;
+            oracle_draft_row(brow, U, W, uw_bf16, V, r, x, it, l);
+            double m;
+            double z = softmax_weights(l, V, w, &m);
+            double mg;
+            int xk = inverse_cdf(w, V, z, (double)u_draft[(size_t)b * K + k], &mg);
+            size_t o = (size_t)b * K + k;
+            tokens[o] = xk;
+            p_tok[o] = w[xk] / z;
+            lse[o] = m + log(z);
+            margin[o] = mg;
+            x = xk;
+        }
+        free(l);
+        free(w);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* confidence-scheduled prefix cut                                     */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Cost (ms) of a verify batch of n tokens: piecewise-linear interpolation
+ * of the profiled table (tokens ascending), extended linearly from the
+ * first and last segments.  [yage, SPS(B) paragraph]: the throughput
+ * profile is measured at start-up and consulted by the scheduler.
+ */
+double oracle_cost_ms(const float *xs, const float *ys, int n, double tokens)
+{
+    int i = 0;
+    while (i < n - 2 && tokens > (double)xs[i + 1])
+        ++i;
+    double x0 = xs[i], x1 = xs[i + 1], y0 = ys[i], y1 = ys[i + 1];
+    return y0 + (y1 - y0) * (tokens - x0) / (x1 - x0);
+}
+
+typedef struct {
+    double s;
+    int k;
+    int b;
+} cand_t;
+
+/* survival descending, then position ascending, then request ascending */
+static int cand_cmp(const void *pa, const void *pb)
+{
+    const cand_t *a = (const cand_t *)pa, *b = (const cand_t *)pb;
+    if (a->s > b->s) return -1;
+    if (a->s < b->s) return 1;
+    if (a->k != b->k) return a->k < b->k ? -1 : 1;
+    if (a->b != b->b) return a->b < b->b ? -1 : 1;
+    return 0;
+}
+
+/*
+ * [freeaitool 4.1]: c_k in (0,1) is the probability that position k is
+ * accepted given every earlier position was; sequential temperature
+ * scaling calibrates it position by position, applied here as
+ * c_k = sigmoid(z_k / T_k).  [yage, SPS(B) paragraph]: the survival of a
+ * draft token together with everything before it is the running product
+ * S_k = prod_{j<=k} c_j; all requests' candidates are ranked by it, the
+ * most probable added first, stopping before the batch-size cost makes
+ * the throughput fall ([freeaitool 4.2] greedy ordering + early stop;
+ * [legalagi 五] the early stop keeps the method lossless).
+ *
+ * Objective: expected emitted tokens per ms, E / t(N), with N the verify
+ * tokens (every request verifies at least one position, so N starts at
+ * B) and E the expected emitted tokens (every request emits at least one
+ * token, so E starts at B).  A candidate is committed while it strictly
+ * raises the objective; the first one that does not ends the scan.
+ *
+ * outputs: c, S [B, K]; L [B] = committed positions per request;
+ * objective = E / t(N) of the committed set; margin = relative objective
+ * gap at the stopping decision (+inf when every candidate was taken).
+ */
+int oracle_prefix(const float *z, const float *temps, const float *cost_tokens,
+                  const float *cost_ms, int n_pts, int B, int K, int enable,
+                  double *c, double *S, int32_t *L, double *objective,
+                  double *margin)
+{
+    if (B < 0 || K < 0 || n_pts < 2)
+        return 1;
+    for (int b = 0; b < B; ++b) {
+        double run = 1.0;
+        for (int k = 0; k < K; ++k) {
+            size_t o = (size_t)b * K + k;
+            double ck = 1.0 / (1.0 + exp(-(double)z[o] / (double)temps[k]));
+            run *= ck;
+            c[o] = ck;
+            S[o] = run;
+        }
+    }
+    if (!enable) {
+        double E = B;
+        for (size_t o = 0; o < (size_t)B * K; ++o)
+            E += S[o];
+        for (int b = 0; b < B; ++b)
+            L[b] = K;
+        *objective = E / oracle_cost_ms(cost_tokens, cost_ms, n_pts,
+                                        (double)B + (double)B * K);
+        *margin = INFINITY;
+        return 0;
+    }
+    size_t n = (size_t)B * K;
+    cand_t *cand = (cand_t *)malloc(sizeof(cand_t) * (n ? n : 1));
+    for (int b = 0; b < B; ++b)
+        for (int k = 0; k < K; ++k) {
+            size_t o = (size_t)b * K + k;
+            cand[o].s = S[o];
+            cand[o].k = k;
+            cand[o].b = b;
+        }
+    qsort(cand, n, sizeof(cand_t), cand_cmp);
+    for (int b = 0; b < B; ++b)
+        L[b] = 0;
+    double E = B, N = B;
+    double obj = E / oracle_cost_ms(cost_tokens, cost_ms, n_pts, N);
+    *margin = INFINITY;
+    for (size_t i = 0; i < n; ++i) {
+        double E2 = E + cand[i].s, N2 = N + 1.0;
+        double obj2 = E2 / oracle_cost_ms(cost_tokens, cost_ms, n_pts, N2);
+        if (!(obj2 > obj)) {
+            *margin = fabs(obj2 - obj) / obj;
+            break;
+        }
+        L[cand[i].b] += 1;
+        E = E2;
+        N = N2;
+        obj = obj2;
+    }
+    *objective = obj;
+    free(cand);
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* verify                                                              */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Rejection-sampling verify of one step ([legalagi 三]: the target checks
+ * the whole draft in one pass and the longest accepted prefix is kept;
+ * [yage, rejection-sampling paragraph]: the check compares draft and
+ * target probabilities, which is why p_d must be exact).  Textbook rule:
+ * position k is accepted iff u_acc < p_t(x_k) / p_d(x_k); at the first
+ * rejected position j the replacement token is drawn from
+ * normalize(max(0, p_t - p_d)); if all L_b positions are accepted a bonus
+ * token is drawn from the target row after them.  The same uniform
+ * u_res[b] serves the residual draw or the bonus draw (only one happens).
+ * If the residual mass is zero the draw falls back to p_t.
+ *
+ *   target     rows [n_rows, V] fp32; request b, position p (0-based)
+ *              reads row row_start[b] + p, p = 0..L_b (row L_b: bonus)
+ *   verify_len [B] L_b in [0, K]
+ *   base, U, W, prev_token, inv_temp  as for oracle_draft (used to
+ *              rebuild the full draft row at the rejected position)
+ *   tokens [B, K], p_d [B, K]  the draft's tokens and their probabilities
+ *   u_accept [B, K], u_res [B]
+ * outputs
+ *   n_acc [B]; out_tokens [B, K+1] (accepted tokens, then the
+ *   correction/bonus token, then -1); accept_margin [B] = min |u - ratio|
+ *   over the tested positions (+inf if none); res_margin [B] = CDF margin
+ *   of the correction/bonus draw.
+ */
+int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
+                  const int32_t *verify_len, const float *base, const void *U,
+                  const void *W, int uw_bf16, int V, int r, int B, int K,
+                  const int32_t *prev_token, const float *inv_temp,
+                  const int32_t *tokens, const double *p_d,
+                  const float *u_accept, const float *u_res, int32_t *n_acc,
+                  int32_t *out_tokens, double *accept_margin,
+                  double *res_margin)
+{
+    for (int b = 0; b < B; ++b) {
+        int L = verify_len[b];
+        if (L < 0 || L > K || row_start[b] < 0 || row_start[b] + L >= n_rows)
+            return 2;
+    }
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int b = 0; b < B; ++b) {
+        double *lt = (double *)malloc(sizeof(double) * (size_t)V);
+        double *pt = (double *)malloc(sizeof(double) * (size_t)V);
+        double *ld = (double *)malloc(sizeof(double) * (size_t)V);
+        double *pd = (double *)malloc(sizeof(double) * (size_t)V);
+        int L = verify_len[b];
+        double it = inv_temp ? (double)inv_temp[b] : 1.0;
+        int n = 0, rejected = 0;
+        double amg = INFINITY;
+        for (int p = 0; p < L; ++p) {
+            const float *trow = target + (size_t)(row_start[b] + p) * (size_t)V;
+            for (int v = 0; v < V; ++v)
+                lt[v] = (double)trow[v] * it;
+            double m;
+            double zt = softmax_weights(lt, V, pt, &m);
+            int x = tokens[(size_t)b * K + p];
+            if (x < 0 || x >= V) {
+                bad = 1;
+                break;
+            }
+            double ratio = (pt[x] / zt) / p_d[(size_t)b * K + p];
+            double u = (double)u_accept[(size_t)b * K + p];
+            double d = fabs(u - ratio);
+            if (d < amg)
+                amg = d;
+            if (u < ratio) {
+                ++n;
+            } else {
+                rejected = 1;
+                break;
+            }
+        }
+        int j = n; /* position of the correction (or bonus) token */
+        const float *trow = target + (size_t)(row_start[b] + j) * (size_t)V;
+        for (int v = 0; v < V; ++v)
+            lt[v] = (double)trow[v] * it;
+        double m;
+        double zt = softmax_weights(lt, V, pt, &m);
+        for (int v = 0; v < V; ++v)
+            pt[v] /= zt;
+        int tok;
+        double mg;
+        double u = (double)u_res[b];
+        if (rejected) {
+            int xp = (j == 0) ? prev_token[b] : tokens[(size_t)b * K + j - 1];
+            const float *brow = base + ((size_t)b * K + j) * (size_t)V;
+            oracle_draft_row(brow, U, W, uw_bf16, V, r, xp, it, ld);
+            double md;
+            double zd = softmax_weights(ld, V, pd, &md);
+            double q = 0.0;
+            for (int v = 0; v < V; ++v) {
+                double d = pt[v] - pd[v] / zd;
+                pd[v] = d > 0.0 ? d : 0.0; /* reuse pd as the residual */
+                q += pd[v];
+            }
+            if (q > 0.0)
+                tok = inverse_cdf(pd, V, q, u, &mg);
+            else
+                tok = inverse_cdf(pt, V, 1.0, u, &mg);
+        } else {
+            tok = inverse_cdf(pt, V, 1.0, u, &mg);
+        }
+        int32_t *out = out_tokens + (size_t)b * (K + 1);
+        for (int p = 0; p < K + 1; ++p)
+            out[p] = -1;
+        for (int p = 0; p < n; ++p)
+            out[p] = tokens[(size_t)b * K + p];
+        out[n] = tok;
+        n_acc[b] = n;
+        accept_margin[b] = amg;
+        res_margin[b] = mg;
+        free(lt);
+        free(pt);
+        free(ld);
+        free(pd);
+    }
+    return bad ? 3 : 0;
+}
