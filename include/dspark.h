@@ -1,0 +1,226 @@
+/*
+ * dspark.h -- C ABI of the DSpark per-step speculative-decoding hot path
+ * (B200 / sm_100a).
+ *
+ * Three calls make one decode step, in this order on one stream:
+ *   1. dspark_draft_markov       the semi-autoregressive Markov-head draft
+ *   2. dspark_confidence_prefix  the confidence-scheduled prefix cut
+ *   3. dspark_verify             the lossless rejection-sampling verify
+ *
+ * Sources (page title, section):
+ *   yage.ai "DSpark speculative decoding hardware scheduling": the
+ *     first-order Markov head paragraph (p(x_k|x_{k-1}) =
+ *     softmax(base_logit_k + transition_bias(x_{k-1}, x_k)), the bias read
+ *     from a V x V low-rank matrix with the previous token); the rejection
+ *     sampling paragraph (the draft must give the exact single-step
+ *     p_d(x_k)); the SPS(B) scheduler paragraph (rank every draft token of
+ *     the batch by calibrated survival, add the most probable first, stop
+ *     before the throughput curve turns down); the variable-length verify
+ *     paragraph (verify rows flattened into one tensor, no padding).
+ *   freeaitool.com "DeepSeek DSpark complete guide": 3.1 (Markov head,
+ *     rank 256), 4.1 (confidence c_k, sequential temperature scaling),
+ *     4.2 (greedy ordering with early stop against a profiled curve).
+ *   legalagi.cn "读懂 DSpark": 三 (keep the longest accepted prefix;
+ *     lossless), 五 (early stop keeps the scheduler lossless).
+ * The accept / residual / bonus rule is textbook speculative sampling
+ * (Leviathan et al. 2023; Chen et al. 2023).
+ *
+ * Conventions shared by every call
+ *   - Every pointer argument is DEVICE memory owned by the caller, unless
+ *     stated otherwise.  The library allocates nothing and keeps no state
+ *     between calls.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Every call only enqueues work on it: no host
+ *     synchronisation, fixed launch shapes for fixed sizes, so a whole
+ *     step can be captured in a CUDA graph.
+ *   - Argument errors (NULL required pointers, bad sizes, misaligned
+ *     pointers, too small workspace) are reported synchronously by the
+ *     return value, before anything is enqueued.
+ *   - Data errors found on the device (a token id outside [0,V), a verify
+ *     length outside [0,K], a target row outside the buffer, a
+ *     non-positive or non-finite 1/T, a non-finite partition sum, a cost
+ *     table that is not ascending) set bits in a status word kept at the
+ *     start of the call's workspace; each call clears that word first.
+ *     Read it with dspark_get_device_status (synchronises the stream).
+ *     The kernels clamp offending values so every access stays in bounds.
+ *   - Layouts are row-major and contiguous.  V, r, B, K are counts.
+ *     Uniforms are fp32 in [0, 1).  Sampling is by inverse CDF: the
+ *     smallest index whose running probability exceeds u.
+ *   - All base / target logits are fp32; U and W are bf16 (tensor-core
+ *     path for B > 16) or fp32 (CUDA-core path); arithmetic is fp32 with
+ *     fp32 accumulation, partition sums and CDF scans in fp64.
+ *   - Alignment: base_logits, target_logits, U, W and the workspace must
+ *     be 16-byte aligned (256 for the workspace); V % 4 == 0; r % 8 == 0.
+ */
+#ifndef DSPARK_H_
+#define DSPARK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSPARK_OK = 0,
+    DSPARK_ERR_INVALID_ARG = 1,  /* bad argument, reported before any launch */
+    DSPARK_ERR_CUDA = 2,         /* a CUDA runtime call failed */
+    DSPARK_ERR_TIMEOUT = 3,      /* a bounded device-side wait gave up */
+    DSPARK_ERR_UNSUPPORTED = 4,  /* sizes outside what this build supports */
+    DSPARK_ERR_DEVICE_DATA = 5,  /* device found bad data (see status flags) */
+    DSPARK_ERR_WORKSPACE = 6     /* workspace missing, misaligned or too small */
+} dspark_status;
+
+typedef enum { DSPARK_F32 = 0, DSPARK_BF16 = 1 } dspark_dtype;
+
+/* Device status flag bits (dspark_get_device_flags). */
+#define DSPARK_FLAG_BAD_TOKEN   0x01u /* token id outside [0, V) */
+#define DSPARK_FLAG_BAD_LENGTH  0x02u /* verify_len outside [0,K] or row outside target */
+#define DSPARK_FLAG_NONFINITE   0x04u /* non-finite or zero partition sum */
+#define DSPARK_FLAG_BAD_TEMP    0x08u /* inv_temp <= 0 or non-finite */
+#define DSPARK_FLAG_TIMEOUT     0x10u /* a bounded device wait gave up */
+#define DSPARK_FLAG_BAD_TABLE   0x20u /* cost table not ascending or cost <= 0 */
+
+/* ---------------------------------------------------------------------- */
+/* 1. Markov-head draft                                                    */
+/* ---------------------------------------------------------------------- */
+
+/* Workspace bytes dspark_draft_markov needs for these sizes. */
+size_t dspark_draft_workspace_size(int V, int r, int B, int K);
+
+/*
+ * For every request b and position k = 1..K, sequentially in k:
+ *   x_0       = prev_token[b]
+ *   l_v       = (base_logits[b,k,v] + U[x_{k-1}] . W[v]) * inv_temp[b]
+ *   p(.)      = softmax(l)
+ *   x_k       = inverse-CDF draw from p with u_draft[b,k]
+ * (yage.ai, Markov-head paragraph; freeaitool 3.1).  The bias term is
+ * left out when x_{k-1} < 0 (only possible at k = 1).
+ *
+ * Inputs
+ *   base_logits [B,K,V] fp32   base logits from the parallel backbone
+ *   U, W        [V,r]          low-rank transition factors, uw_dtype
+ *   prev_token  [B] int32      last committed token (<0: no bias at k=1)
+ *   inv_temp    [B] fp32 or NULL (NULL: 1)
+ *   u_draft     [B,K] fp32 uniforms
+ * Outputs
+ *   tokens   [B,K] int32   x_k
+ *   p_tok    [B,K] fp32    p_d(x_k), the exact draft probability of x_k
+ *   lse      [B,K] fp32    log sum_v exp(l_v)
+ *   ref_max  [B,K] fp32    M: the reference maximum of the un-tempered
+ *                          logits (base + bias) used by the sampler
+ *   ref_sum  [B,K] fp32    Z = sum_v exp((base_v + bias_v - M) * inv_temp);
+ *                          p_d(v) = exp((base_v + bias_v - M)*inv_temp) / Z.
+ *                          dspark_verify needs ref_max / ref_sum to rebuild
+ *                          the draft row at a rejected position exactly.
+ *   draft_logits [B,K,V] fp32 or NULL: the tempered logits l, if wanted.
+ */
+dspark_status dspark_draft_markov(
+    const float *base_logits, const void *U, const void *W, dspark_dtype uw_dtype,
+    int V, int r, int B, int K,
+    const int32_t *prev_token, const float *inv_temp, const float *u_draft,
+    int32_t *tokens, float *p_tok, float *lse, float *ref_max, float *ref_sum,
+    float *draft_logits, void *workspace, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* 2. Confidence-scheduled prefix cut                                      */
+/* ---------------------------------------------------------------------- */
+
+size_t dspark_prefix_workspace_size(int B, int K, int n_pts);
+
+/*
+ * Sequential temperature scaling, survival and the hardware-aware greedy
+ * prefix cut (freeaitool 4.1-4.2; yage.ai SPS(B) paragraph; legalagi 五):
+ *   c[b,k]        = sigmoid(z[b,k] / temps[k])
+ *   survival[b,k] = prod_{j<=k} c[b,j]
+ *   candidates (b,k) in order of survival descending, ties by k then b
+ *   ascending; starting from N = B verify tokens and E = B expected
+ *   emitted tokens, a candidate is committed while E'/t(N') > E/t(N) with
+ *   E' = E + survival, N' = N + 1; the first candidate that does not raise
+ *   the objective ends the scan.  t(N) = piecewise-linear interpolation of
+ *   (cost_tokens, cost_ms), extended linearly past both ends.
+ *   verify_len[b] = committed positions of request b (a prefix 1..L_b).
+ *   objective[0]  = E / t(N) of the committed set.
+ * enable == 0: verify_len[b] = K for every b (c and survival still filled).
+ * Inputs: z [B,K], temps [K], cost_tokens [n_pts] (ascending), cost_ms
+ * [n_pts]; n_pts >= 2; B*K <= 8192.  Computed in fp64 on the device.
+ */
+dspark_status dspark_confidence_prefix(
+    const float *z, const float *temps, const float *cost_tokens,
+    const float *cost_ms, int n_pts, int B, int K, int enable,
+    float *c, float *survival, int32_t *verify_len, float *objective,
+    void *workspace, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* 3. Rejection-sampling verify                                            */
+/* ---------------------------------------------------------------------- */
+
+size_t dspark_verify_workspace_size(int V, int r, int B, int K);
+
+/*
+ * Lossless verify of one step (legalagi 三; yage.ai rejection-sampling
+ * paragraph; textbook speculative sampling):
+ *   p_t(row)   = softmax(target_logits[row] * inv_temp[b])
+ *   for k = 1..L_b (L_b = verify_len[b]), row = row_start[b] + k - 1:
+ *       accept iff u_accept[b,k] < p_t(x_k) / p_tok[b,k]; stop at the first
+ *       rejection.  n_accepted[b] = accepted prefix length.
+ *   rejected at position j: the correction token is drawn with
+ *       u_resample[b] from normalize(max(0, p_t - p_d)) where p_d is the
+ *       draft distribution at position j, rebuilt from base_logits, U, W,
+ *       the previous token, ref_max[b,j] and ref_sum[b,j] (falls back to
+ *       p_t if the residual mass is zero);
+ *   all accepted: a bonus token is drawn with u_resample[b] from p_t of
+ *       row row_start[b] + L_b.
+ *   out_tokens[b, 0..n] = accepted draft tokens then the correction/bonus
+ *   token; the rest of the row (up to K) is -1.
+ *
+ * Inputs
+ *   target_logits [n_target_rows, V] fp32: flattened ragged verify rows;
+ *       request b uses rows row_start[b] .. row_start[b] + L_b.
+ *   row_start [B] int64; verify_len [B] int32 (L_b in [0,K], read on device)
+ *   base_logits, U, W, uw_dtype, prev_token, inv_temp: as for the draft
+ *   tokens, p_tok, ref_max, ref_sum [B,K]: the draft's outputs
+ *   u_accept [B,K], u_resample [B] fp32 uniforms
+ * Outputs
+ *   n_accepted [B] int32; out_tokens [B,K+1] int32;
+ *   last_token [B] int32 or NULL: the last emitted token (the next step's
+ *       prev_token).
+ */
+dspark_status dspark_verify(
+    const float *target_logits, int64_t n_target_rows, const int64_t *row_start,
+    const int32_t *verify_len, const float *base_logits, const void *U,
+    const void *W, dspark_dtype uw_dtype, int V, int r, int B, int K,
+    const int32_t *prev_token, const float *inv_temp, const int32_t *tokens,
+    const float *p_tok, const float *ref_max, const float *ref_sum,
+    const float *u_accept, const float *u_resample, int32_t *n_accepted,
+    int32_t *out_tokens, int32_t *last_token, void *workspace, size_t ws_bytes,
+    void *stream);
+
+/* ---------------------------------------------------------------------- */
+/* status                                                                  */
+/* ---------------------------------------------------------------------- */
+
+/* Synchronises `stream`, reads the status word of `workspace` and maps it
+ * to DSPARK_OK / DSPARK_ERR_TIMEOUT / DSPARK_ERR_DEVICE_DATA. */
+dspark_status dspark_get_device_status(const void *workspace, void *stream);
+
+/* Synchronises `stream`; returns the raw DSPARK_FLAG_* bits (or -1 on a
+ * CUDA error). */
+int dspark_get_device_flags(const void *workspace, void *stream);
+
+/* Static string for a status code. */
+const char *dspark_status_string(dspark_status s);
+
+/* Name of the draft projection path these sizes take:
+ * "cuda-core" (fp32 U/W or B <= 16) or "tcgen05" (bf16, B > 16). */
+const char *dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype);
+
+/* Library ABI version (major*100 + minor). */
+int dspark_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSPARK_H_ */

@@ -1,0 +1,360 @@
+// api.cu -- the C ABI (include/dspark.h): argument validation, workspace
+// layout and kernel launches.  No entry point allocates memory or
+// synchronises the stream (except the status readers).
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "prefix.cuh"
+#include "proj_simt.cuh"
+#include "proj_tc.cuh"
+#include "sample.cuh"
+#include "verify.cuh"
+
+using namespace dspark;
+
+namespace {
+
+constexpr int kMaxK = 64;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Workspace of the draft: header, then chunk partials [B][n_chunks].
+struct DraftWs {
+  size_t part_off, total;
+};
+DraftWs draft_ws(int V, int B) {
+  DraftWs w;
+  w.part_off = kHeaderBytes;
+  w.total = w.part_off + align256((size_t)B * n_chunks_of(V) * sizeof(float2));
+  return w;
+}
+
+// Workspace of the verify: header, target partials [B*(K+1)][n_segs],
+// ResInfo [B], residual partials [B][n_chunks].
+struct VerifyWs {
+  size_t tpart_off, info_off, rpart_off, total;
+};
+VerifyWs verify_ws(int V, int B, int K) {
+  VerifyWs w;
+  w.tpart_off = kHeaderBytes;
+  w.info_off = w.tpart_off + align256((size_t)B * (K + 1) * n_segs_of(V) * sizeof(float2));
+  w.rpart_off = w.info_off + align256((size_t)B * sizeof(ResInfo));
+  w.total = w.rpart_off + align256((size_t)B * n_chunks_of(V) * sizeof(float2));
+  return w;
+}
+
+dspark_status check_launch() {
+  return cudaGetLastError() == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
+dspark_status clear_status(void* ws, cudaStream_t s) {
+  return cudaMemsetAsync(ws, 0, sizeof(unsigned), s) == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
+// Shape checks shared by draft and verify.
+dspark_status check_shapes(int V, int r, int B, int K, dspark_dtype dt) {
+  if (V <= 0 || r <= 0 || B < 0 || K < 0) return DSPARK_ERR_INVALID_ARG;
+  if (dt != DSPARK_F32 && dt != DSPARK_BF16) return DSPARK_ERR_INVALID_ARG;
+  if (V % 4 != 0 || r % 8 != 0) return DSPARK_ERR_UNSUPPORTED;
+  if (r > kMaxRank || K > kMaxK) return DSPARK_ERR_UNSUPPORTED;
+  if ((long long)V * (K + 1) > (1ll << 40)) return DSPARK_ERR_UNSUPPORTED;
+  return DSPARK_OK;
+}
+
+int simt_group(int B) {
+  int nb = 1;
+  while (nb < B && nb < 16) nb <<= 1;
+  return nb;
+}
+
+template <typename TW, int NB>
+void launch_draft_proj_simt(const float* base, const void* U, const void* W, int V, int r, int B,
+                            int K, int k, const int32_t* prev, const int32_t* tokens,
+                            const float* it, float* dl, float2* part, unsigned* flags,
+                            cudaStream_t s) {
+  const int nc = n_chunks_of(V);
+  const size_t smem = (size_t)NB * r * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(draft_proj_simt_kernel<TW, NB>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, NB * kMaxRank * 4);
+    attr = true;
+  }
+  dim3 grid((nc + 7) / 8, (B + NB - 1) / NB);
+  draft_proj_simt_kernel<TW, NB><<<grid, 256, smem, s>>>(
+      base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, B, K, k, prev, tokens, it,
+      dl, part, nc, flags);
+}
+
+template <typename TW, int NB>
+void launch_res_proj_simt(const float* target, const float* base, const void* U, const void* W,
+                          int V, int r, int B, int K, const ResInfo* info, const float* it,
+                          float2* rpart, unsigned* flags, cudaStream_t s) {
+  const int nc = n_chunks_of(V);
+  const size_t smem = (size_t)NB * r * sizeof(float);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(residual_proj_simt_kernel<TW, NB>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize, NB * kMaxRank * 4);
+    attr = true;
+  }
+  dim3 grid((nc + 7) / 8, (B + NB - 1) / NB);
+  residual_proj_simt_kernel<TW, NB><<<grid, 256, smem, s>>>(
+      target, base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, B, K, info, it,
+      rpart, nc, flags);
+}
+
+template <typename TW>
+void draft_proj_simt(int nb, const float* base, const void* U, const void* W, int V, int r, int B,
+                     int K, int k, const int32_t* prev, const int32_t* tokens, const float* it,
+                     float* dl, float2* part, unsigned* flags, cudaStream_t s) {
+  switch (nb) {
+    case 1: launch_draft_proj_simt<TW, 1>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
+    case 2: launch_draft_proj_simt<TW, 2>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
+    case 4: launch_draft_proj_simt<TW, 4>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
+    case 8: launch_draft_proj_simt<TW, 8>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
+    default: launch_draft_proj_simt<TW, 16>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
+  }
+}
+
+template <typename TW>
+void res_proj_simt(int nb, const float* target, const float* base, const void* U, const void* W,
+                   int V, int r, int B, int K, const ResInfo* info, const float* it, float2* rpart,
+                   unsigned* flags, cudaStream_t s) {
+  switch (nb) {
+    case 1: launch_res_proj_simt<TW, 1>(target, base, U, W, V, r, B, K, info, it, rpart, flags, s); break;
+    case 2: launch_res_proj_simt<TW, 2>(target, base, U, W, V, r, B, K, info, it, rpart, flags, s); break;
+    case 4: launch_res_proj_simt<TW, 4>(target, base, U, W, V, r, B, K, info, it, rpart, flags, s); break;
+    case 8: launch_res_proj_simt<TW, 8>(target, base, U, W, V, r, B, K, info, it, rpart, flags, s); break;
+    default: launch_res_proj_simt<TW, 16>(target, base, U, W, V, r, B, K, info, it, rpart, flags, s); break;
+  }
+}
+
+// Which projection path a draft / residual of these sizes takes.
+bool use_tc(int V, int r, int B, dspark_dtype dt) {
+  return dt == DSPARK_BF16 && B > 16 && tc_supported(V, r, B);
+}
+
+template <typename TW>
+dspark_status draft_impl(const float* base, const void* U, const void* W, dspark_dtype dt, int V,
+                         int r, int B, int K, const int32_t* prev, const float* it,
+                         const float* ud, int32_t* tokens, float* p_tok, float* lse, float* rmax,
+                         float* rsum, float* dl, unsigned char* ws, cudaStream_t s) {
+  const DraftWs w = draft_ws(V, B);
+  unsigned* flags = reinterpret_cast<unsigned*>(ws);
+  float2* part = reinterpret_cast<float2*>(ws + w.part_off);
+  const int nc = n_chunks_of(V);
+  const bool tc = use_tc(V, r, B, dt);
+  TcPlan plan;
+  if (tc) {
+    dspark_status st = tc_plan_draft(plan, base, U, W, V, r, B, K);
+    if (st != DSPARK_OK) return st;
+  }
+  const int nb = simt_group(B);
+  for (int k = 0; k < K; ++k) {
+    if (tc) {
+      tc_launch_draft(plan, k, prev, tokens, it, dl, part, flags, s);
+    } else {
+      draft_proj_simt<TW>(nb, base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s);
+    }
+    draft_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
+        base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, k, prev, tokens, it,
+        ud, part, nc, p_tok, lse, rmax, rsum, flags);
+  }
+  return check_launch();
+}
+
+template <typename TW>
+dspark_status verify_impl(const float* target, long long n_rows, const int64_t* row_start,
+                          const int32_t* vlen, const float* base, const void* U, const void* W,
+                          dspark_dtype dt, int V, int r, int B, int K, const int32_t* prev,
+                          const float* it, const int32_t* tokens, const float* p_tok,
+                          const float* rmax, const float* rsum, const float* ua, const float* ur,
+                          int32_t* n_acc, int32_t* out, int32_t* last, unsigned char* ws,
+                          cudaStream_t s) {
+  const VerifyWs w = verify_ws(V, B, K);
+  unsigned* flags = reinterpret_cast<unsigned*>(ws);
+  float2* tpart = reinterpret_cast<float2*>(ws + w.tpart_off);
+  ResInfo* info = reinterpret_cast<ResInfo*>(ws + w.info_off);
+  float2* rpart = reinterpret_cast<float2*>(ws + w.rpart_off);
+  const int ns = n_segs_of(V), nc = n_chunks_of(V);
+  dim3 sgrid(ns, B * (K + 1));
+  target_stats_kernel<<<sgrid, kStatsThreads, 0, s>>>(target, n_rows, row_start, vlen, it, V, K,
+                                                       tpart, ns, flags);
+  accept_kernel<<<(B + 3) / 4, 128, 0, s>>>(target, n_rows, row_start, vlen, it, V, B, K, prev,
+                                            tokens, p_tok, rmax, rsum, ua, tpart, ns, n_acc, out,
+                                            info, flags);
+  if (use_tc(V, r, B, dt)) {
+    TcPlan plan;
+    dspark_status st = tc_plan_residual(plan, target, base, U, W, V, r, B, K);
+    if (st != DSPARK_OK) return st;
+    tc_launch_residual(plan, info, it, rpart, flags, s);
+  } else {
+    res_proj_simt<TW>(simt_group(B), target, base, U, W, V, r, B, K, info, it, rpart, flags, s);
+  }
+  residual_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
+      target, base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, it, ur, info,
+      rpart, nc, out, last, flags);
+  return check_launch();
+}
+
+}  // namespace
+
+extern "C" {
+
+int dspark_version(void) { return 100; }
+
+const char* dspark_status_string(dspark_status s) {
+  switch (s) {
+    case DSPARK_OK: return "ok";
+    case DSPARK_ERR_INVALID_ARG: return "invalid argument";
+    case DSPARK_ERR_CUDA: return "CUDA runtime error";
+    case DSPARK_ERR_TIMEOUT: return "device wait timed out";
+    case DSPARK_ERR_UNSUPPORTED: return "sizes not supported by this build";
+    case DSPARK_ERR_DEVICE_DATA: return "device found invalid data";
+    case DSPARK_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+const char* dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype) {
+  (void)K;
+  return use_tc(V, r, B, uw_dtype) ? "tcgen05" : "cuda-core";
+}
+
+size_t dspark_draft_workspace_size(int V, int r, int B, int K) {
+  (void)r;
+  (void)K;
+  if (V <= 0 || B < 0) return 0;
+  return draft_ws(V, B).total;
+}
+
+size_t dspark_verify_workspace_size(int V, int r, int B, int K) {
+  (void)r;
+  if (V <= 0 || B < 0 || K < 0) return 0;
+  return verify_ws(V, B, K).total;
+}
+
+size_t dspark_prefix_workspace_size(int B, int K, int n_pts) {
+  (void)B;
+  (void)K;
+  (void)n_pts;
+  return kHeaderBytes;
+}
+
+dspark_status dspark_draft_markov(const float* base_logits, const void* U, const void* W,
+                                  dspark_dtype uw_dtype, int V, int r, int B, int K,
+                                  const int32_t* prev_token, const float* inv_temp,
+                                  const float* u_draft, int32_t* tokens, float* p_tok, float* lse,
+                                  float* ref_max, float* ref_sum, float* draft_logits,
+                                  void* workspace, size_t ws_bytes, void* stream) {
+  dspark_status st = check_shapes(V, r, B, K, uw_dtype);
+  if (st != DSPARK_OK) return st;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < dspark_draft_workspace_size(V, r, B, K))
+    return DSPARK_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 0 || K == 0) return clear_status(workspace, s);
+  if (!base_logits || !U || !W || !prev_token || !u_draft || !tokens || !p_tok || !lse ||
+      !ref_max || !ref_sum)
+    return DSPARK_ERR_INVALID_ARG;
+  if (!aligned(base_logits, 16) || !aligned(U, 16) || !aligned(W, 16) ||
+      (draft_logits && !aligned(draft_logits, 16)))
+    return DSPARK_ERR_INVALID_ARG;
+  if ((st = clear_status(workspace, s)) != DSPARK_OK) return st;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (uw_dtype == DSPARK_BF16)
+    return draft_impl<__nv_bfloat16>(base_logits, U, W, uw_dtype, V, r, B, K, prev_token,
+                                     inv_temp, u_draft, tokens, p_tok, lse, ref_max, ref_sum,
+                                     draft_logits, ws, s);
+  return draft_impl<float>(base_logits, U, W, uw_dtype, V, r, B, K, prev_token, inv_temp, u_draft,
+                           tokens, p_tok, lse, ref_max, ref_sum, draft_logits, ws, s);
+}
+
+dspark_status dspark_verify(const float* target_logits, int64_t n_target_rows,
+                            const int64_t* row_start, const int32_t* verify_len,
+                            const float* base_logits, const void* U, const void* W,
+                            dspark_dtype uw_dtype, int V, int r, int B, int K,
+                            const int32_t* prev_token, const float* inv_temp,
+                            const int32_t* tokens, const float* p_tok, const float* ref_max,
+                            const float* ref_sum, const float* u_accept, const float* u_resample,
+                            int32_t* n_accepted, int32_t* out_tokens, int32_t* last_token,
+                            void* workspace, size_t ws_bytes, void* stream) {
+  dspark_status st = check_shapes(V, r, B, K, uw_dtype);
+  if (st != DSPARK_OK) return st;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < dspark_verify_workspace_size(V, r, B, K))
+    return DSPARK_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 0) return clear_status(workspace, s);
+  if (!target_logits || n_target_rows <= 0 || !row_start || !verify_len || !base_logits || !U ||
+      !W || !prev_token || !u_resample || !n_accepted || !out_tokens)
+    return DSPARK_ERR_INVALID_ARG;
+  if (K > 0 && (!tokens || !p_tok || !ref_max || !ref_sum || !u_accept))
+    return DSPARK_ERR_INVALID_ARG;
+  if (!aligned(target_logits, 16) || !aligned(base_logits, 16) || !aligned(U, 16) ||
+      !aligned(W, 16))
+    return DSPARK_ERR_INVALID_ARG;
+  if ((long long)B * (K + 1) > (1ll << 31) - 1) return DSPARK_ERR_UNSUPPORTED;
+  if ((st = clear_status(workspace, s)) != DSPARK_OK) return st;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (uw_dtype == DSPARK_BF16)
+    return verify_impl<__nv_bfloat16>(target_logits, n_target_rows, row_start, verify_len,
+                                      base_logits, U, W, uw_dtype, V, r, B, K, prev_token,
+                                      inv_temp, tokens, p_tok, ref_max, ref_sum, u_accept,
+                                      u_resample, n_accepted, out_tokens, last_token, ws, s);
+  return verify_impl<float>(target_logits, n_target_rows, row_start, verify_len, base_logits, U, W,
+                            uw_dtype, V, r, B, K, prev_token, inv_temp, tokens, p_tok, ref_max,
+                            ref_sum, u_accept, u_resample, n_accepted, out_tokens, last_token, ws,
+                            s);
+}
+
+dspark_status dspark_confidence_prefix(const float* z, const float* temps,
+                                       const float* cost_tokens, const float* cost_ms, int n_pts,
+                                       int B, int K, int enable, float* c, float* survival,
+                                       int32_t* verify_len, float* objective, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+  if (B < 0 || K < 0 || n_pts < 2 || n_pts > 64) return DSPARK_ERR_INVALID_ARG;
+  if ((long long)B * K > kMaxCand) return DSPARK_ERR_UNSUPPORTED;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < dspark_prefix_workspace_size(B, K, n_pts))
+    return DSPARK_ERR_WORKSPACE;
+  if (!cost_tokens || !cost_ms || !verify_len || !objective) return DSPARK_ERR_INVALID_ARG;
+  if (B * K > 0 && (!z || !temps || !c || !survival)) return DSPARK_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dspark_status st = clear_status(workspace, s);
+  if (st != DSPARK_OK) return st;
+  int npad = 1;
+  while (npad < B * K) npad <<= 1;
+  const size_t smem = (size_t)npad * (sizeof(double) + sizeof(int)) + (size_t)B * sizeof(int);
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kMaxCand * 12 + 8192 * 4);
+    attr = true;
+  }
+  if (smem > (size_t)kMaxCand * 12 + 8192 * 4) return DSPARK_ERR_UNSUPPORTED;
+  prefix_kernel<<<1, kPrefixThreads, smem, s>>>(z, temps, cost_tokens, cost_ms, n_pts, B, K, enable,
+                                               c, survival, verify_len, objective,
+                                               static_cast<unsigned*>(workspace));
+  return check_launch();
+}
+
+int dspark_get_device_flags(const void* workspace, void* stream) {
+  if (!workspace) return -1;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned h = 0;
+  if (cudaMemcpyAsync(&h, workspace, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return -1;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return -1;
+  return (int)h;
+}
+
+dspark_status dspark_get_device_status(const void* workspace, void* stream) {
+  const int f = dspark_get_device_flags(workspace, stream);
+  if (f < 0) return DSPARK_ERR_CUDA;
+  if (f & DSPARK_FLAG_TIMEOUT) return DSPARK_ERR_TIMEOUT;
+  if (f) return DSPARK_ERR_DEVICE_DATA;
+  return DSPARK_OK;
+}
+
+}  // extern "C"

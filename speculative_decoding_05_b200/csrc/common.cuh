@@ -1,0 +1,207 @@
+// common.cuh -- device helpers shared by the DSpark kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "../../include/dspark.h"
+
+namespace dspark {
+
+// ---------------------------------------------------------------------------
+// sizes and workspace layout
+// ---------------------------------------------------------------------------
+
+// Rows of the vocabulary summarised by one softmax partial (one warp's rows).
+constexpr int kChunk = 32;
+// Elements of a target row reduced by one CTA in the target-statistics pass.
+constexpr int kSeg = 8192;
+// The workspace starts with a 256-byte header whose first word is the
+// device status (DSPARK_FLAG_* bits).
+constexpr size_t kHeaderBytes = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__host__ __device__ inline int n_chunks_of(int V) { return (V + kChunk - 1) / kChunk; }
+__host__ __device__ inline int n_segs_of(int V) { return (V + kSeg - 1) / kSeg; }
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// ---------------------------------------------------------------------------
+// status word
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void raise_flag(unsigned* flags, unsigned f) { atomicOr(flags, f); }
+
+// A token id read from memory, clamped into [0, V) (or -1 for "none" when
+// allowed); an id outside the range raises DSPARK_FLAG_BAD_TOKEN.
+__device__ __forceinline__ int checked_token(int x, int V, bool allow_none, unsigned* flags) {
+  if (x < 0) {
+    if (allow_none) return -1;
+    raise_flag(flags, DSPARK_FLAG_BAD_TOKEN);
+    return 0;
+  }
+  if (x >= V) {
+    raise_flag(flags, DSPARK_FLAG_BAD_TOKEN);
+    return allow_none ? -1 : V - 1;
+  }
+  return x;
+}
+
+// 1/T for request b; a non-positive or non-finite value raises
+// DSPARK_FLAG_BAD_TEMP and is replaced by 1.
+__device__ __forceinline__ float checked_inv_temp(const float* inv_temp, int b, unsigned* flags) {
+  if (inv_temp == nullptr) return 1.0f;
+  float it = inv_temp[b];
+  if (!(it > 0.0f) || !isfinite(it)) {
+    raise_flag(flags, DSPARK_FLAG_BAD_TEMP);
+    return 1.0f;
+  }
+  return it;
+}
+
+// ---------------------------------------------------------------------------
+// arithmetic
+// ---------------------------------------------------------------------------
+
+// 2^x on the SFU (relative error of a couple of ulp; subnormal results
+// flush to zero, far below anything a sampling decision can see).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+// Inclusive prefix sum over the lanes of a warp (lane order), in fp64.
+__device__ __forceinline__ double warp_incl_scan_d(double v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    double n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// ---------------------------------------------------------------------------
+// loads
+// ---------------------------------------------------------------------------
+
+// 8 consecutive elements of a W / U row as fp32.  Row starts are 16-byte
+// aligned (r % 8 == 0, base pointer 16-byte aligned).
+__device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&o)[8]) {
+  uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
+  o[0] = __uint_as_float(q.x << 16); o[1] = __uint_as_float(q.x & 0xffff0000u);
+  o[2] = __uint_as_float(q.y << 16); o[3] = __uint_as_float(q.y & 0xffff0000u);
+  o[4] = __uint_as_float(q.z << 16); o[5] = __uint_as_float(q.z & 0xffff0000u);
+  o[6] = __uint_as_float(q.w << 16); o[7] = __uint_as_float(q.w & 0xffff0000u);
+}
+__device__ __forceinline__ void load8(const float* p, float (&o)[8]) {
+  float4 a = __ldg(reinterpret_cast<const float4*>(p));
+  float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(float x) { return x; }
+
+// L2 policy for data read exactly once (logit streams): evict first, so
+// that it does not displace data that is re-read (W, partials).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+// 128-bit streaming load with an L2 cache policy, not allocated in L1.
+__device__ __forceinline__ float4 ld_stream4(const float* p, uint64_t pol) {
+  float4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.f32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+// The transition bias U[x] . W[v] for one vocabulary row, accumulated in
+// fp32 in ascending index order (fmaf).  The projection kernels and the
+// samplers call this same function, so a re-computed chunk reproduces the
+// projection's bias bit for bit on the CUDA-core path.
+template <typename TW>
+__device__ __forceinline__ float dot_row(const TW* __restrict__ wrow, const float* __restrict__ u, int r) {
+  float acc = 0.0f;
+  for (int i = 0; i < r; i += 8) {
+    float w8[8];
+    load8(wrow + i, w8);
+    float4 ua = *reinterpret_cast<const float4*>(u + i);
+    float4 ub = *reinterpret_cast<const float4*>(u + i + 4);
+    acc = fmaf(w8[0], ua.x, acc); acc = fmaf(w8[1], ua.y, acc);
+    acc = fmaf(w8[2], ua.z, acc); acc = fmaf(w8[3], ua.w, acc);
+    acc = fmaf(w8[4], ub.x, acc); acc = fmaf(w8[5], ub.y, acc);
+    acc = fmaf(w8[6], ub.z, acc); acc = fmaf(w8[7], ub.w, acc);
+  }
+  return acc;
+}
+
+// ---------------------------------------------------------------------------
+// block-wide reductions / scans over 256 threads (8 warps)
+// ---------------------------------------------------------------------------
+
+template <int NT>
+__device__ __forceinline__ float block_max(float v, float* sh) {
+  v = warp_max(v);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  float r = (lane < NT / 32) ? sh[lane] : -CUDART_INF_F;
+  return warp_max(r);
+}
+
+template <int NT>
+__device__ __forceinline__ double block_sum_d(double v, double* sh) {
+  v = warp_sum_d(v);
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __syncthreads();
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  double r = (lane < NT / 32) ? sh[lane] : 0.0;
+  return warp_sum_d(r);
+}
+
+// Exclusive prefix sum over the threads of a block (thread order), fp64.
+// The result is non-decreasing in thread order when every v >= 0 (each
+// value is a rounded running sum, never "inclusive minus v").
+// Returns the exclusive prefix; *total receives the block total.
+template <int NT>
+__device__ __forceinline__ double block_excl_scan_d(double v, double* sh, double* total) {
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const double incl = warp_incl_scan_d(v);
+  double ex = __shfl_up_sync(0xffffffffu, incl, 1);
+  if (lane == 0) ex = 0.0;
+  __syncthreads();
+  if (lane == 31) sh[w] = incl;
+  __syncthreads();
+  double wpre = 0.0;
+  for (int i = 0; i < w; ++i) wpre += sh[i];
+  double tot = 0.0;
+  for (int i = 0; i < NT / 32; ++i) tot += sh[i];
+  *total = tot;
+  return (lane == 0) ? wpre : wpre + ex;
+}
+
+}  // namespace dspark

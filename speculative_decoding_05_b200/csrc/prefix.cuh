@@ -1,0 +1,153 @@
+// prefix.cuh -- sequential temperature scaling, survival and the greedy
+// hardware-aware prefix cut, in one CTA.
+//
+// The whole batch has at most kMaxCand = 8192 candidates (B*K); they are
+// sorted in shared memory (bitonic, key = survival descending, ties by
+// candidate index k*B + b ascending, i.e. position then request), the
+// expected-emitted-token prefix sums are a block scan in fp64, and the
+// early stop is the first index where E/t(N) does not increase.
+#pragma once
+
+#include "common.cuh"
+
+namespace dspark {
+
+constexpr int kPrefixThreads = 1024;
+constexpr int kMaxCand = 8192;
+
+// Piecewise-linear cost (ms) of a verify batch of n tokens, extended
+// linearly past both ends of the table.
+__device__ __forceinline__ double cost_at(const float* __restrict__ xs, const float* __restrict__ ys,
+                                          int n, double tokens) {
+  int i = 0;
+  while (i < n - 2 && tokens > (double)xs[i + 1]) ++i;
+  const double x0 = xs[i], x1 = xs[i + 1], y0 = ys[i], y1 = ys[i + 1];
+  return y0 + (y1 - y0) * (tokens - x0) / (x1 - x0);
+}
+
+// key order: larger survival first; equal survival: smaller index first
+__device__ __forceinline__ bool cand_before(double sa, int ia, double sb, int ib) {
+  return sa > sb || (sa == sb && ia < ib);
+}
+
+__global__ void __launch_bounds__(kPrefixThreads)
+prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
+              const float* __restrict__ cost_tokens, const float* __restrict__ cost_ms, int n_pts,
+              int B, int K, int enable, float* __restrict__ c_out, float* __restrict__ s_out,
+              int32_t* __restrict__ verify_len, float* __restrict__ objective, unsigned* flags) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int n = B * K;
+  int npad = 1;
+  while (npad < n) npad <<= 1;
+  double* key = reinterpret_cast<double*>(smem_raw);           // [npad]
+  int* idx = reinterpret_cast<int*>(key + npad);               // [npad]
+  int* lcount = idx + npad;                                     // [B]
+  __shared__ float s_xs[64], s_ys[64];
+  __shared__ double shd[32];
+  __shared__ int s_stop;
+  const int tid = threadIdx.x;
+
+  // cost table into shared memory; it must be ascending in tokens
+  for (int i = tid; i < n_pts; i += kPrefixThreads) {
+    s_xs[i] = cost_tokens[i];
+    s_ys[i] = cost_ms[i];
+  }
+  __syncthreads();
+  if (tid == 0) {
+    bool ok = true;
+    for (int i = 0; i + 1 < n_pts; ++i) ok = ok && (s_xs[i + 1] > s_xs[i]);
+    if (!ok) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
+    s_stop = n;
+  }
+
+  // c = sigmoid(z / T_k) and survival = running product over k, in fp64
+  for (int b = tid; b < B; b += kPrefixThreads) {
+    double run = 1.0;
+    for (int k = 0; k < K; ++k) {
+      const size_t o = (size_t)b * K + k;
+      const double ck = 1.0 / (1.0 + exp(-(double)z[o] / (double)temps[k]));
+      run *= ck;
+      c_out[o] = (float)ck;
+      s_out[o] = (float)run;
+      key[k * B + b] = run;
+      idx[k * B + b] = k * B + b;
+    }
+    lcount[b] = 0;
+  }
+  for (int i = n + tid; i < npad; i += kPrefixThreads) {
+    key[i] = -1.0;  // padding sorts last
+    idx[i] = 0x7fffffff;
+  }
+  __syncthreads();
+
+  if (!enable) {
+    double e = 0.0;
+    for (int i = tid; i < n; i += kPrefixThreads) e += key[i];
+    const double E = (double)B + block_sum_d<kPrefixThreads>(e, shd);
+    for (int b = tid; b < B; b += kPrefixThreads) verify_len[b] = K;
+    if (tid == 0) {
+      const double t = cost_at(s_xs, s_ys, n_pts, (double)B + (double)n);
+      if (!(t > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
+      objective[0] = (float)(E / t);
+    }
+    return;
+  }
+
+  // bitonic sort of (key, idx) in the order of cand_before
+  for (int size = 2; size <= npad; size <<= 1) {
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      for (int i = tid; i < npad; i += kPrefixThreads) {
+        const int j = i ^ stride;
+        if (j > i) {
+          const bool up = (i & size) == 0;  // this half sorts in cand_before order
+          const double ki = key[i], kj = key[j];
+          const int ii = idx[i], ij = idx[j];
+          const bool jfirst = cand_before(kj, ij, ki, ii);
+          if (jfirst == up) {
+            key[i] = kj; key[j] = ki;
+            idx[i] = ij; idx[j] = ii;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+
+  // E_i = B + sum of the first i survivals; each thread owns a contiguous run
+  const int per = npad / kPrefixThreads > 0 ? npad / kPrefixThreads : 1;
+  const int i0 = tid * per;
+  double run = 0.0;
+  for (int i = i0; i < i0 + per && i < n; ++i) run += key[i];
+  double total;
+  const double excl = block_excl_scan_d<kPrefixThreads>(run, shd, &total);
+  // candidate i (0-based) raises the objective iff E_{i+1}/t(B+i+1) > E_i/t(B+i)
+  double E = (double)B + excl;
+  for (int i = i0; i < i0 + per && i < n; ++i) {
+    const double t0 = cost_at(s_xs, s_ys, n_pts, (double)B + (double)i);
+    const double t1 = cost_at(s_xs, s_ys, n_pts, (double)B + (double)i + 1.0);
+    const double E1 = E + key[i];
+    if (!(t0 > 0.0) || !(t1 > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
+    if (!(E1 / t1 > E / t0)) {
+      atomicMin(&s_stop, i);
+      break;
+    }
+    E = E1;
+  }
+  __syncthreads();
+  const int n_commit = s_stop;
+  for (int i = tid; i < n_commit; i += kPrefixThreads) atomicAdd(&lcount[idx[i] % B], 1);
+  __syncthreads();
+  for (int b = tid; b < B; b += kPrefixThreads) verify_len[b] = lcount[b];
+  // objective of the committed set: E at n_commit from the owning thread's run
+  const bool owner = (n_commit == n) ? (tid == 0) : (n_commit >= i0 && n_commit < i0 + per);
+  if (owner) {
+    double Ec = (double)B + total;
+    if (n_commit < n) {
+      Ec = (double)B + excl;
+      for (int i = i0; i < n_commit; ++i) Ec += key[i];
+    }
+    objective[0] = (float)(Ec / cost_at(s_xs, s_ys, n_pts, (double)B + (double)n_commit));
+  }
+}
+
+}  // namespace dspark

@@ -1,0 +1,191 @@
+"""Thin Python binding of the C ABI in include/dspark.h (ctypes).
+
+Argument marshalling only: tensors are turned into device pointers and
+sizes, every step of the hot path runs in libdspark.so.  The functions carry
+the C names.  Loading fails loudly if the CUDA library is missing; there is
+no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdspark.so")
+
+DSPARK_F32 = 0
+DSPARK_BF16 = 1
+
+STATUS = {0: "DSPARK_OK", 1: "DSPARK_ERR_INVALID_ARG", 2: "DSPARK_ERR_CUDA",
+          3: "DSPARK_ERR_TIMEOUT", 4: "DSPARK_ERR_UNSUPPORTED",
+          5: "DSPARK_ERR_DEVICE_DATA", 6: "DSPARK_ERR_WORKSPACE"}
+
+FLAG_BAD_TOKEN = 0x01
+FLAG_BAD_LENGTH = 0x02
+FLAG_NONFINITE = 0x04
+FLAG_BAD_TEMP = 0x08
+FLAG_TIMEOUT = 0x10
+FLAG_BAD_TABLE = 0x20
+
+# every symbol include/dspark.h declares
+SYMBOLS = [
+    "dspark_draft_workspace_size", "dspark_draft_markov",
+    "dspark_prefix_workspace_size", "dspark_confidence_prefix",
+    "dspark_verify_workspace_size", "dspark_verify",
+    "dspark_get_device_status", "dspark_get_device_flags",
+    "dspark_status_string", "dspark_draft_path", "dspark_version",
+]
+
+
+class DSparkError(RuntimeError):
+    def __init__(self, where: str, code: int):
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({status_string(code)})")
+        self.code = code
+
+
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load libdspark.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"CUDA library not built: {p} (run speculative_decoding_05_b200.build)")
+    lib = ctypes.CDLL(p)
+    P, I, L, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    lib.dspark_draft_workspace_size.argtypes = [I, I, I, I]
+    lib.dspark_draft_workspace_size.restype = S
+    lib.dspark_verify_workspace_size.argtypes = [I, I, I, I]
+    lib.dspark_verify_workspace_size.restype = S
+    lib.dspark_prefix_workspace_size.argtypes = [I, I, I]
+    lib.dspark_prefix_workspace_size.restype = S
+    lib.dspark_draft_markov.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, S, P]
+    lib.dspark_draft_markov.restype = I
+    lib.dspark_verify.argtypes = [P, L, P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P,
+                                  P, P, S, P]
+    lib.dspark_verify.restype = I
+    lib.dspark_confidence_prefix.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P, S, P]
+    lib.dspark_confidence_prefix.restype = I
+    lib.dspark_get_device_status.argtypes = [P, P]
+    lib.dspark_get_device_status.restype = I
+    lib.dspark_get_device_flags.argtypes = [P, P]
+    lib.dspark_get_device_flags.restype = I
+    lib.dspark_status_string.argtypes = [I]
+    lib.dspark_status_string.restype = ctypes.c_char_p
+    lib.dspark_draft_path.argtypes = [I, I, I, I, I]
+    lib.dspark_draft_path.restype = ctypes.c_char_p
+    lib.dspark_version.argtypes = []
+    lib.dspark_version.restype = I
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(where, rc):
+    if rc != 0:
+        raise DSparkError(where, rc)
+
+
+def _dtype_code(U):
+    return DSPARK_BF16 if U.dtype == torch.bfloat16 else DSPARK_F32
+
+
+def status_string(code: int) -> str:
+    try:
+        return load().dspark_status_string(int(code)).decode()
+    except Exception:  # the library may be missing when formatting an error
+        return STATUS.get(code, "unknown")
+
+
+dspark_status_string = status_string
+
+
+def dspark_version() -> int:
+    return int(load().dspark_version())
+
+
+def dspark_draft_path(V, r, B, K, uw_dtype) -> str:
+    code = uw_dtype if isinstance(uw_dtype, int) else (
+        DSPARK_BF16 if uw_dtype == torch.bfloat16 else DSPARK_F32)
+    return load().dspark_draft_path(V, r, B, K, code).decode()
+
+
+def dspark_draft_workspace_size(V, r, B, K) -> int:
+    return int(load().dspark_draft_workspace_size(V, r, B, K))
+
+
+def dspark_verify_workspace_size(V, r, B, K) -> int:
+    return int(load().dspark_verify_workspace_size(V, r, B, K))
+
+
+def dspark_prefix_workspace_size(B, K, n_pts) -> int:
+    return int(load().dspark_prefix_workspace_size(B, K, n_pts))
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned device byte buffer (torch's allocator aligns to 512)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def dspark_draft_markov(base_logits, U, W, prev_token, inv_temp, u_draft, tokens, p_tok, lse,
+                        ref_max, ref_sum, workspace, draft_logits=None, stream=None):
+    B, K, V = base_logits.shape
+    r = W.shape[1]
+    rc = load().dspark_draft_markov(
+        _ptr(base_logits), _ptr(U), _ptr(W), _dtype_code(U), V, r, B, K, _ptr(prev_token),
+        _ptr(inv_temp), _ptr(u_draft), _ptr(tokens), _ptr(p_tok), _ptr(lse), _ptr(ref_max),
+        _ptr(ref_sum), _ptr(draft_logits), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("dspark_draft_markov", rc)
+
+
+def dspark_confidence_prefix(z, temps, cost_tokens, cost_ms, enable, c, survival, verify_len,
+                             objective, workspace, stream=None):
+    B, K = z.shape
+    rc = load().dspark_confidence_prefix(
+        _ptr(z), _ptr(temps), _ptr(cost_tokens), _ptr(cost_ms), cost_tokens.numel(), B, K,
+        int(bool(enable)), _ptr(c), _ptr(survival), _ptr(verify_len), _ptr(objective),
+        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("dspark_confidence_prefix", rc)
+
+
+def dspark_verify(target_logits, row_start, verify_len, base_logits, U, W, prev_token, inv_temp,
+                  tokens, p_tok, ref_max, ref_sum, u_accept, u_resample, n_accepted, out_tokens,
+                  workspace, last_token=None, stream=None):
+    n_rows, V = target_logits.shape
+    B, K = tokens.shape
+    r = W.shape[1]
+    rc = load().dspark_verify(
+        _ptr(target_logits), n_rows, _ptr(row_start), _ptr(verify_len), _ptr(base_logits),
+        _ptr(U), _ptr(W), _dtype_code(U), V, r, B, K, _ptr(prev_token), _ptr(inv_temp),
+        _ptr(tokens), _ptr(p_tok), _ptr(ref_max), _ptr(ref_sum), _ptr(u_accept),
+        _ptr(u_resample), _ptr(n_accepted), _ptr(out_tokens), _ptr(last_token),
+        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("dspark_verify", rc)
+
+
+def dspark_get_device_flags(workspace, stream=None) -> int:
+    f = int(load().dspark_get_device_flags(_ptr(workspace), _stream(stream)))
+    if f < 0:
+        raise DSparkError("dspark_get_device_flags", 2)
+    return f
+
+
+def dspark_get_device_status(workspace, stream=None) -> int:
+    return int(load().dspark_get_device_status(_ptr(workspace), _stream(stream)))

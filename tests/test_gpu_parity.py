@@ -1,0 +1,169 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Small shapes (several chunks, a ragged tail, every request) and the five
+workloads at full size in the launch configuration the benchmark times
+(sampled requests for the large batches).
+"""
+import numpy as np
+import pytest
+import torch
+
+from speculative_decoding_05_b200 import dspark as D
+from speculative_decoding_05_b200 import workloads as WL
+from speculative_decoding_05_b200.step import DSparkStep
+
+from tests.parity import compare_step, host
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(w, enable=None, seed=None, requests=None, oracle=None, inp=None):
+    inp = inp or WL.make_inputs(w, device="cuda", seed=seed)
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+    en = w.scheduler if enable is None else enable
+    step.run(inp, enable_prefix=en)
+    torch.cuda.synchronize()
+    flags = step.flags()
+    assert all(f == 0 for f in flags.values()), flags
+    rep = compare_step(oracle, inp, step, en, requests=requests)
+    return rep, step, inp
+
+
+def _assert_ok(rep):
+    print(rep)
+    assert not rep.failures, rep.failures[:10]
+    # near-margin cases are allowed but must stay rare
+    assert sum(rep.near.values()) <= max(2, sum(rep.checked.values()) // 200), rep
+
+
+def test_tiny_full(oracle_mod):
+    rep, _, _ = _run(WL.get("tiny"), oracle=oracle_mod)
+    _assert_ok(rep)
+    assert rep.checked["draft"] == 2 * 4
+
+
+@pytest.mark.parametrize("bf16", [True, False])
+@pytest.mark.parametrize("V,r,B,K", [(1000, 64, 3, 5), (4096, 32, 7, 3), (2056, 256, 16, 4)])
+def test_small_shapes(oracle_mod, bf16, V, r, B, K):
+    w = WL.get("serving", V=V, r=r, B=B, K=K, uw_bf16=bf16, seed=11 + V + B)
+    inp = WL.make_inputs(w, device="cuda")
+    inp["prev_token"][0] = -1  # no bias at position 1 for request 0
+    rep, _, _ = _run(w, oracle=oracle_mod, inp=inp)
+    _assert_ok(rep)
+    assert rep.checked["draft"] >= B
+
+
+def test_temperatures_and_flat_peaked(oracle_mod):
+    w = WL.get("stress", V=3072, r=64, B=24, K=6, seed=5)
+    rep, _, _ = _run(w, oracle=oracle_mod)
+    _assert_ok(rep)
+    w = WL.get("batched", V=3072, r=64, B=12, K=5, seed=6)
+    rep, _, _ = _run(w, oracle=oracle_mod)
+    _assert_ok(rep)
+
+
+def test_draft_logits_output(oracle_mod):
+    w = WL.get("single", V=2048, r=64, B=2, K=3, seed=9)
+    inp = WL.make_inputs(w, device="cuda")
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+    dl = torch.empty_like(inp["base"])
+    step.draft(inp, draft_logits=dl)
+    torch.cuda.synchronize()
+    U, W = WL.host_uw(inp["U"]), WL.host_uw(inp["W"])
+    tok = host(step.tokens)
+    for b in range(w.B):
+        x = int(host(inp["prev_token"])[b])
+        for k in range(w.K):
+            ref = oracle_mod.draft_row(host(inp["base"][b, k]), U, W, x, float(host(inp["inv_temp"])[b]))
+            np.testing.assert_allclose(host(dl[b, k]), ref, atol=1e-5, rtol=1e-6)
+            x = int(tok[b, k])
+
+
+@pytest.mark.parametrize("name", ["single", "batched", "serving", "stress"])
+def test_full_size(oracle_mod, name):
+    w = WL.get(name)
+    requests = None if w.B <= 4 else np.random.default_rng(0).choice(w.B, size=6, replace=False)
+    rep, _, _ = _run(w, oracle=oracle_mod, requests=requests)
+    _assert_ok(rep)
+    del rep
+    torch.cuda.empty_cache()
+
+
+def test_stress_sequential_steps(oracle_mod):
+    """Three sequential steps; each side feeds its own last emitted token
+    into the next step (the oracle never reads the GPU's tokens)."""
+    w = WL.get("stress", V=8192, r=256, B=32, K=16, seed=21)
+    inp = WL.make_inputs(w, device="cuda")
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+    req = np.arange(w.B)
+    prev_gpu = inp["prev_token"].clone()
+    prev_or = host(inp["prev_token"]).copy()
+    for s in range(3):
+        if s > 0:
+            inp.update(WL.step_uniforms(w, s, device="cuda"))
+        step.run(inp, enable_prefix=True, prev_token=prev_gpu)
+        torch.cuda.synchronize()
+        oinp = dict(inp)
+        oinp["prev_token"] = torch.as_tensor(prev_or, device="cuda")
+        rep = compare_step(oracle_mod, oinp, step, True, requests=req)
+        _assert_ok(rep)
+        # next step: GPU uses its own last token, the oracle its own
+        prev_gpu = step.last_token.clone()
+        pr = oracle_mod.prefix(host(inp["z"]), host(inp["temps"]), host(inp["cost_tokens"]),
+                               host(inp["cost_ms"]))
+        d = oracle_mod.draft(host(inp["base"]), WL.host_uw(inp["U"]), WL.host_uw(inp["W"]), prev_or,
+                             host(inp["u_draft"]), inv_temp=host(inp["inv_temp"]))
+        v = oracle_mod.verify(host(inp["target"]), host(inp["row_start"]), pr["L"], host(inp["base"]),
+                              WL.host_uw(inp["U"]), WL.host_uw(inp["W"]), prev_or, d["tokens"],
+                              d["p_tok"], host(inp["u_accept"]), host(inp["u_res"]),
+                              inv_temp=host(inp["inv_temp"]))
+        prev_or = v["out_tokens"][np.arange(w.B), v["n_acc"]].astype(np.int32)
+
+
+def test_edge_cases(oracle_mod):
+    # B = 1, K = 1, every verify length 0 and K
+    for L in (0, 1):
+        w = WL.get("single", V=512, r=16, B=1, K=1, seed=30 + L)
+        inp = WL.make_inputs(w, device="cuda")
+        step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+        step.draft(inp)
+        step.verify_len.fill_(L)
+        step.verify(inp)
+        torch.cuda.synchronize()
+        assert int(step.n_accepted[0]) <= L
+        assert 0 <= int(step.out_tokens[0, int(step.n_accepted[0])]) < w.V
+
+
+def test_empty_batch_is_noop():
+    w = WL.get("single", V=512, r=16, B=1, K=2)
+    inp = WL.make_inputs(w, device="cuda")
+    ws = D.workspace(D.dspark_draft_workspace_size(512, 16, 0, 2), "cuda")
+    e = torch.empty(0, 2, device="cuda")
+    D.dspark_draft_markov(inp["base"][:0], inp["U"], inp["W"], inp["prev_token"][:0], None,
+                          e, e.int(), e, e, e, e, ws)
+    assert D.dspark_get_device_flags(ws) == 0
+
+
+def test_device_flags_on_bad_data():
+    w = WL.get("single", V=1024, r=16, B=4, K=3, seed=40)
+    inp = WL.make_inputs(w, device="cuda")
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+    step.draft(inp)
+    step.prefix(inp, enable=False)
+    step.tokens[1, 0] = w.V + 7      # out-of-range token id
+    step.verify_len[2] = w.K + 5     # out-of-range verify length
+    step.verify(inp)
+    f = D.dspark_get_device_flags(step.ws_verify)
+    assert f & D.FLAG_BAD_TOKEN and f & D.FLAG_BAD_LENGTH
+    assert D.dspark_get_device_status(step.ws_verify) == 5
+    bad = inp["inv_temp"].clone()
+    bad[0] = 0.0
+    inp2 = dict(inp, inv_temp=bad)
+    step.draft(inp2)
+    assert D.dspark_get_device_flags(step.ws_draft) & D.FLAG_BAD_TEMP
+    xs = inp["cost_tokens"].flip(0).contiguous()
+    step.prefix(dict(inp, cost_tokens=xs), enable=True)
+    assert D.dspark_get_device_flags(step.ws_prefix) & D.FLAG_BAD_TABLE
+    # a clean call clears the status word again
+    step.draft(inp)
+    assert D.dspark_get_device_flags(step.ws_draft) == 0

@@ -1,0 +1,93 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads,
+exports every symbol include/dspark.h declares, and rejects bad arguments
+before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from speculative_decoding_05_b200 import build
+from speculative_decoding_05_b200 import dspark as D
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return D.load()
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"\b(dspark_\w+)\s*\(", txt))
+    return names
+
+
+def test_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert declared, "no declarations found"
+    out = subprocess.run(["nm", "-D", "--defined-only", D.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\b(dspark_\w+)\b", out))
+    assert declared <= exported, declared - exported
+    assert set(D.SYMBOLS) <= declared
+    for name in declared:
+        assert hasattr(lib, name)
+
+
+def test_status_strings_and_paths(lib):
+    for code in range(7):
+        assert D.status_string(code)
+    assert D.dspark_version() >= 100
+    assert D.dspark_draft_path(151936, 256, 1, 16, D.DSPARK_BF16) == "cuda-core"
+    assert D.dspark_draft_path(1024, 16, 64, 4, D.DSPARK_F32) == "cuda-core"
+
+
+def test_workspace_sizes(lib):
+    V, r, B, K = 151936, 256, 512, 16
+    nch = (V + 31) // 32
+    assert lib.dspark_draft_workspace_size(V, r, B, K) >= 256 + B * nch * 8
+    assert lib.dspark_verify_workspace_size(V, r, B, K) >= 256 + B * nch * 8
+    assert lib.dspark_prefix_workspace_size(B, K, 16) >= 4
+    assert lib.dspark_draft_workspace_size(0, r, B, K) == 0
+
+
+def _draft(lib, V=1024, r=16, B=2, K=3, base=1 << 20, U=1 << 21, W=1 << 22, ws=1 << 24,
+           ws_bytes=None, dtype=D.DSPARK_BF16):
+    if ws_bytes is None:
+        ws_bytes = lib.dspark_draft_workspace_size(V, r, B, K)
+    P = ctypes.c_void_p
+    p = P(1 << 23)
+    return lib.dspark_draft_markov(P(base), P(U), P(W), dtype, V, r, B, K, p, None, p, p, p, p, p,
+                                   p, None, P(ws), ws_bytes, None)
+
+
+def test_argument_validation_before_launch(lib):
+    # every case below must be rejected on the host, before any CUDA call
+    assert _draft(lib, V=1022) == 4            # V % 4 != 0 -> unsupported
+    assert _draft(lib, r=12) == 4              # r % 8 != 0
+    assert _draft(lib, r=2048) == 4            # r too large
+    assert _draft(lib, K=65) == 4              # K too large
+    assert _draft(lib, V=-4) == 1
+    assert _draft(lib, dtype=7) == 1
+    assert _draft(lib, ws_bytes=16) == 6       # workspace too small
+    assert _draft(lib, ws=(1 << 24) + 8) == 6  # workspace misaligned
+    assert _draft(lib, base=(1 << 20) + 4) == 1  # base not 16-byte aligned
+    assert _draft(lib, U=0) == 1               # NULL required pointer
+    P = ctypes.c_void_p
+    p = P(1 << 23)
+    ws = P(1 << 24)
+    # prefix: too many candidates, bad table size
+    assert lib.dspark_confidence_prefix(p, p, p, p, 16, 1024, 9, 1, p, p, p, p, ws, 256, None) == 4
+    assert lib.dspark_confidence_prefix(p, p, p, p, 1, 4, 4, 1, p, p, p, p, ws, 256, None) == 1
+    # verify: missing target
+    vb = lib.dspark_verify_workspace_size(1024, 16, 2, 3)
+    assert lib.dspark_verify(None, 10, p, p, p, p, p, 1, 1024, 16, 2, 3, p, None, p, p, p, p, p,
+                             p, p, p, None, ws, vb, None) == 1
