@@ -115,13 +115,20 @@ size_t dspark_draft_workspace_size(int V, int r, int B, int K);
  *                          dspark_verify needs ref_max / ref_sum to rebuild
  *                          the draft row at a rejected position exactly.
  *   draft_logits [B,K,V] fp32 or NULL: the tempered logits l, if wanted.
+ *   draft_bias   [B,K,V] fp32 or NULL: the transition bias U[x_{k-1}] . W[v]
+ *                of every drafted position.  Passing it on to
+ *                dspark_verify lets the verify rebuild the draft row at a
+ *                rejected position without another pass over W (worth it
+ *                for small B; for large B the re-projection is cheaper
+ *                than writing B*K*V floats).
  */
 dspark_status dspark_draft_markov(
     const float *base_logits, const void *U, const void *W, dspark_dtype uw_dtype,
     int V, int r, int B, int K,
     const int32_t *prev_token, const float *inv_temp, const float *u_draft,
     int32_t *tokens, float *p_tok, float *lse, float *ref_max, float *ref_sum,
-    float *draft_logits, void *workspace, size_t ws_bytes, void *stream);
+    float *draft_logits, float *draft_bias, void *workspace, size_t ws_bytes,
+    void *stream);
 
 /* ---------------------------------------------------------------------- */
 /* 2. Confidence-scheduled prefix cut                                      */
@@ -181,6 +188,8 @@ size_t dspark_verify_workspace_size(int V, int r, int B, int K);
  *   row_start [B] int64; verify_len [B] int32 (L_b in [0,K], read on device)
  *   base_logits, U, W, uw_dtype, prev_token, inv_temp: as for the draft
  *   tokens, p_tok, ref_max, ref_sum [B,K]: the draft's outputs
+ *   draft_bias [B,K,V] or NULL: the draft's bias rows (see the draft); NULL
+ *       makes the verify re-project U[x_{j-1}] . W for the rejected row
  *   u_accept [B,K], u_resample [B] fp32 uniforms
  * Outputs
  *   n_accepted [B] int32; out_tokens [B,K+1] int32;
@@ -193,7 +202,8 @@ dspark_status dspark_verify(
     const void *W, dspark_dtype uw_dtype, int V, int r, int B, int K,
     const int32_t *prev_token, const float *inv_temp, const int32_t *tokens,
     const float *p_tok, const float *ref_max, const float *ref_sum,
-    const float *u_accept, const float *u_resample, int32_t *n_accepted,
+    const float *draft_bias, const float *u_accept, const float *u_resample,
+    int32_t *n_accepted,
     int32_t *out_tokens, int32_t *last_token, void *workspace, size_t ws_bytes,
     void *stream);
 
@@ -213,7 +223,9 @@ int dspark_get_device_flags(const void *workspace, void *stream);
 const char *dspark_status_string(dspark_status s);
 
 /* Name of the draft projection path these sizes take:
- * "cuda-core" (fp32 U/W or B <= 16) or "tcgen05" (bf16, B > 16). */
+ * "tcgen05-persistent" (bf16, B <= 16: all K positions in one launch),
+ * "tcgen05" (bf16, B > 16: one launch per position) or "cuda-core"
+ * (fp32 U/W, or shapes outside the tensor-core paths). */
 const char *dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype);
 
 /* Library ABI version (major*100 + minor). */

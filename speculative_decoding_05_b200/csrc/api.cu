@@ -10,6 +10,7 @@
 #include "prefix.cuh"
 #include "proj_simt.cuh"
 #include "proj_tc.cuh"
+#include "draft_persist.cuh"
 #include "sample.cuh"
 #include "verify.cuh"
 
@@ -21,14 +22,19 @@ constexpr int kMaxK = 64;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Workspace of the draft: header, then chunk partials [B][n_chunks].
+// Workspace of the draft: header (status word at 0, grid-barrier counter
+// at 64), chunk partials [B][n_chunks], then (persistent path) per-CTA
+// partials [B][<=1024] and bias rows [B][V].
+constexpr size_t kCounterOff = 64;
 struct DraftWs {
-  size_t part_off, total;
+  size_t part_off, cta_off, bias_off, total;
 };
 DraftWs draft_ws(int V, int B) {
   DraftWs w;
   w.part_off = kHeaderBytes;
-  w.total = w.part_off + align256((size_t)B * n_chunks_of(V) * sizeof(float2));
+  w.cta_off = w.part_off + align256((size_t)B * n_chunks_of(V) * sizeof(float2));
+  w.bias_off = w.cta_off + align256((size_t)(B <= kPMaxB ? B : 0) * 1024 * sizeof(float2));
+  w.total = w.bias_off + align256((size_t)(B <= kPMaxB ? B : 0) * V * sizeof(float));
   return w;
 }
 
@@ -50,8 +56,9 @@ dspark_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
+// Clears the status word and the grid-barrier counter of a workspace.
 dspark_status clear_status(void* ws, cudaStream_t s) {
-  return cudaMemsetAsync(ws, 0, sizeof(unsigned), s) == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+  return cudaMemsetAsync(ws, 0, 128, s) == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
 // Shape checks shared by draft and verify.
@@ -73,8 +80,8 @@ int simt_group(int B) {
 template <typename TW, int NB>
 void launch_draft_proj_simt(const float* base, const void* U, const void* W, int V, int r, int B,
                             int K, int k, const int32_t* prev, const int32_t* tokens,
-                            const float* it, float* dl, float2* part, unsigned* flags,
-                            cudaStream_t s) {
+                            const float* it, float* dl, float* dbias, float2* part,
+                            unsigned* flags, cudaStream_t s) {
   const int nc = n_chunks_of(V);
   const size_t smem = (size_t)NB * r * sizeof(float);
   static bool attr = false;
@@ -86,7 +93,7 @@ void launch_draft_proj_simt(const float* base, const void* U, const void* W, int
   dim3 grid((nc + 7) / 8, (B + NB - 1) / NB);
   draft_proj_simt_kernel<TW, NB><<<grid, 256, smem, s>>>(
       base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, B, K, k, prev, tokens, it,
-      dl, part, nc, flags);
+      dl, dbias, part, nc, flags);
 }
 
 template <typename TW, int NB>
@@ -110,13 +117,13 @@ void launch_res_proj_simt(const float* target, const float* base, const void* U,
 template <typename TW>
 void draft_proj_simt(int nb, const float* base, const void* U, const void* W, int V, int r, int B,
                      int K, int k, const int32_t* prev, const int32_t* tokens, const float* it,
-                     float* dl, float2* part, unsigned* flags, cudaStream_t s) {
+                     float* dl, float* dbias, float2* part, unsigned* flags, cudaStream_t s) {
   switch (nb) {
-    case 1: launch_draft_proj_simt<TW, 1>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
-    case 2: launch_draft_proj_simt<TW, 2>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
-    case 4: launch_draft_proj_simt<TW, 4>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
-    case 8: launch_draft_proj_simt<TW, 8>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
-    default: launch_draft_proj_simt<TW, 16>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s); break;
+    case 1: launch_draft_proj_simt<TW, 1>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, dbias, part, flags, s); break;
+    case 2: launch_draft_proj_simt<TW, 2>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, dbias, part, flags, s); break;
+    case 4: launch_draft_proj_simt<TW, 4>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, dbias, part, flags, s); break;
+    case 8: launch_draft_proj_simt<TW, 8>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, dbias, part, flags, s); break;
+    default: launch_draft_proj_simt<TW, 16>(base, U, W, V, r, B, K, k, prev, tokens, it, dl, dbias, part, flags, s); break;
   }
 }
 
@@ -137,16 +144,50 @@ void res_proj_simt(int nb, const float* target, const float* base, const void* U
 bool use_tc(int V, int r, int B, dspark_dtype dt) {
   return dt == DSPARK_BF16 && B > 16 && tc_supported(V, r, B);
 }
+bool use_persist(int V, int r, int B, dspark_dtype dt) {
+  return dt == DSPARK_BF16 && persist_supported(V, r, B);
+}
 
 template <typename TW>
 dspark_status draft_impl(const float* base, const void* U, const void* W, dspark_dtype dt, int V,
                          int r, int B, int K, const int32_t* prev, const float* it,
                          const float* ud, int32_t* tokens, float* p_tok, float* lse, float* rmax,
-                         float* rsum, float* dl, unsigned char* ws, cudaStream_t s) {
+                         float* rsum, float* dl, float* dbias, unsigned char* ws, cudaStream_t s) {
   const DraftWs w = draft_ws(V, B);
   unsigned* flags = reinterpret_cast<unsigned*>(ws);
   float2* part = reinterpret_cast<float2*>(ws + w.part_off);
   const int nc = n_chunks_of(V);
+  if (use_persist(V, r, B, dt)) {
+    CUtensorMap tm_w;
+    if (!encode_w_map(&tm_w, W, V, r)) return DSPARK_ERR_CUDA;
+    PersistArgs a;
+    a.base = base;
+    a.U = static_cast<const __nv_bfloat16*>(U);
+    a.prev_token = prev;
+    a.inv_temp = it;
+    a.u_draft = ud;
+    a.tokens = tokens;
+    a.p_tok = p_tok;
+    a.lse = lse;
+    a.ref_max = rmax;
+    a.ref_sum = rsum;
+    a.draft_logits = dl;
+    a.part = part;
+    a.cta_part = reinterpret_cast<float2*>(ws + w.cta_off);
+    a.bias_buf = reinterpret_cast<float*>(ws + w.bias_off);
+    a.draft_bias = dbias;
+    a.flags = flags;
+    a.grid_counter = reinterpret_cast<unsigned*>(ws + kCounterOff);
+    a.V = V;
+    a.r = r;
+    a.B = B;
+    a.K = K;
+    a.n_chunks = nc;
+    a.n_tiles = (V + kTileN - 1) / kTileN;
+    dspark_status st = persist_launch(tm_w, a, s);
+    if (st != DSPARK_OK) return st;
+    return check_launch();
+  }
   const bool tc = use_tc(V, r, B, dt);
   TcPlan plan;
   if (tc) {
@@ -156,13 +197,13 @@ dspark_status draft_impl(const float* base, const void* U, const void* W, dspark
   const int nb = simt_group(B);
   for (int k = 0; k < K; ++k) {
     if (tc) {
-      tc_launch_draft(plan, k, prev, tokens, it, dl, part, flags, s);
+      tc_launch_draft(plan, k, prev, tokens, it, dl, dbias, part, flags, s);
     } else {
-      draft_proj_simt<TW>(nb, base, U, W, V, r, B, K, k, prev, tokens, it, dl, part, flags, s);
+      draft_proj_simt<TW>(nb, base, U, W, V, r, B, K, k, prev, tokens, it, dl, dbias, part, flags, s);
     }
     draft_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
         base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, k, prev, tokens, it,
-        ud, part, nc, p_tok, lse, rmax, rsum, flags);
+        ud, part, nc, dbias, p_tok, lse, rmax, rsum, flags);
   }
   return check_launch();
 }
@@ -172,9 +213,9 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
                           const int32_t* vlen, const float* base, const void* U, const void* W,
                           dspark_dtype dt, int V, int r, int B, int K, const int32_t* prev,
                           const float* it, const int32_t* tokens, const float* p_tok,
-                          const float* rmax, const float* rsum, const float* ua, const float* ur,
-                          int32_t* n_acc, int32_t* out, int32_t* last, unsigned char* ws,
-                          cudaStream_t s) {
+                          const float* rmax, const float* rsum, const float* dbias,
+                          const float* ua, const float* ur, int32_t* n_acc, int32_t* out,
+                          int32_t* last, unsigned char* ws, cudaStream_t s) {
   const VerifyWs w = verify_ws(V, B, K);
   unsigned* flags = reinterpret_cast<unsigned*>(ws);
   float2* tpart = reinterpret_cast<float2*>(ws + w.tpart_off);
@@ -187,7 +228,11 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
   accept_kernel<<<(B + 3) / 4, 128, 0, s>>>(target, n_rows, row_start, vlen, it, V, B, K, prev,
                                             tokens, p_tok, rmax, rsum, ua, tpart, ns, n_acc, out,
                                             info, flags);
-  if (use_tc(V, r, B, dt)) {
+  if (dbias != nullptr) {
+    dim3 rgrid((nc + 7) / 8, B);
+    residual_bias_kernel<<<rgrid, 256, 0, s>>>(target, base, dbias, V, K, info, it, rpart, nc,
+                                                flags);
+  } else if (use_tc(V, r, B, dt)) {
     TcPlan plan;
     dspark_status st = tc_plan_residual(plan, target, base, U, W, V, r, B, K);
     if (st != DSPARK_OK) return st;
@@ -197,7 +242,7 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
   }
   residual_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
       target, base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, it, ur, info,
-      rpart, nc, out, last, flags);
+      rpart, nc, dbias, out, last, flags);
   return check_launch();
 }
 
@@ -222,6 +267,7 @@ const char* dspark_status_string(dspark_status s) {
 
 const char* dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype) {
   (void)K;
+  if (use_persist(V, r, B, uw_dtype)) return "tcgen05-persistent";
   return use_tc(V, r, B, uw_dtype) ? "tcgen05" : "cuda-core";
 }
 
@@ -250,7 +296,8 @@ dspark_status dspark_draft_markov(const float* base_logits, const void* U, const
                                   const int32_t* prev_token, const float* inv_temp,
                                   const float* u_draft, int32_t* tokens, float* p_tok, float* lse,
                                   float* ref_max, float* ref_sum, float* draft_logits,
-                                  void* workspace, size_t ws_bytes, void* stream) {
+                                  float* draft_bias, void* workspace, size_t ws_bytes,
+                                  void* stream) {
   dspark_status st = check_shapes(V, r, B, K, uw_dtype);
   if (st != DSPARK_OK) return st;
   if (!workspace || !aligned(workspace, 256) || ws_bytes < dspark_draft_workspace_size(V, r, B, K))
@@ -261,16 +308,16 @@ dspark_status dspark_draft_markov(const float* base_logits, const void* U, const
       !ref_max || !ref_sum)
     return DSPARK_ERR_INVALID_ARG;
   if (!aligned(base_logits, 16) || !aligned(U, 16) || !aligned(W, 16) ||
-      (draft_logits && !aligned(draft_logits, 16)))
+      (draft_logits && !aligned(draft_logits, 16)) || (draft_bias && !aligned(draft_bias, 16)))
     return DSPARK_ERR_INVALID_ARG;
   if ((st = clear_status(workspace, s)) != DSPARK_OK) return st;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   if (uw_dtype == DSPARK_BF16)
     return draft_impl<__nv_bfloat16>(base_logits, U, W, uw_dtype, V, r, B, K, prev_token,
                                      inv_temp, u_draft, tokens, p_tok, lse, ref_max, ref_sum,
-                                     draft_logits, ws, s);
+                                     draft_logits, draft_bias, ws, s);
   return draft_impl<float>(base_logits, U, W, uw_dtype, V, r, B, K, prev_token, inv_temp, u_draft,
-                           tokens, p_tok, lse, ref_max, ref_sum, draft_logits, ws, s);
+                           tokens, p_tok, lse, ref_max, ref_sum, draft_logits, draft_bias, ws, s);
 }
 
 dspark_status dspark_verify(const float* target_logits, int64_t n_target_rows,
@@ -279,8 +326,9 @@ dspark_status dspark_verify(const float* target_logits, int64_t n_target_rows,
                             dspark_dtype uw_dtype, int V, int r, int B, int K,
                             const int32_t* prev_token, const float* inv_temp,
                             const int32_t* tokens, const float* p_tok, const float* ref_max,
-                            const float* ref_sum, const float* u_accept, const float* u_resample,
-                            int32_t* n_accepted, int32_t* out_tokens, int32_t* last_token,
+                            const float* ref_sum, const float* draft_bias, const float* u_accept,
+                            const float* u_resample, int32_t* n_accepted, int32_t* out_tokens,
+                            int32_t* last_token,
                             void* workspace, size_t ws_bytes, void* stream) {
   dspark_status st = check_shapes(V, r, B, K, uw_dtype);
   if (st != DSPARK_OK) return st;
@@ -302,12 +350,13 @@ dspark_status dspark_verify(const float* target_logits, int64_t n_target_rows,
   if (uw_dtype == DSPARK_BF16)
     return verify_impl<__nv_bfloat16>(target_logits, n_target_rows, row_start, verify_len,
                                       base_logits, U, W, uw_dtype, V, r, B, K, prev_token,
-                                      inv_temp, tokens, p_tok, ref_max, ref_sum, u_accept,
-                                      u_resample, n_accepted, out_tokens, last_token, ws, s);
+                                      inv_temp, tokens, p_tok, ref_max, ref_sum, draft_bias,
+                                      u_accept, u_resample, n_accepted, out_tokens, last_token, ws,
+                                      s);
   return verify_impl<float>(target_logits, n_target_rows, row_start, verify_len, base_logits, U, W,
                             uw_dtype, V, r, B, K, prev_token, inv_temp, tokens, p_tok, ref_max,
-                            ref_sum, u_accept, u_resample, n_accepted, out_tokens, last_token, ws,
-                            s);
+                            ref_sum, draft_bias, u_accept, u_resample, n_accepted, out_tokens,
+                            last_token, ws, s);
 }
 
 dspark_status dspark_confidence_prefix(const float* z, const float* temps,

@@ -144,15 +144,22 @@ __device__ __forceinline__ float4 ld_stream4(const float* p, uint64_t pol) {
 template <typename TW>
 __device__ __forceinline__ float dot_row(const TW* __restrict__ wrow, const float* __restrict__ u, int r) {
   float acc = 0.0f;
-  for (int i = 0; i < r; i += 8) {
-    float w8[8];
-    load8(wrow + i, w8);
-    float4 ua = *reinterpret_cast<const float4*>(u + i);
-    float4 ub = *reinterpret_cast<const float4*>(u + i + 4);
-    acc = fmaf(w8[0], ua.x, acc); acc = fmaf(w8[1], ua.y, acc);
-    acc = fmaf(w8[2], ua.z, acc); acc = fmaf(w8[3], ua.w, acc);
-    acc = fmaf(w8[4], ub.x, acc); acc = fmaf(w8[5], ub.y, acc);
-    acc = fmaf(w8[6], ub.z, acc); acc = fmaf(w8[7], ub.w, acc);
+  for (int i0 = 0; i0 < r; i0 += 64) {
+    // issue up to eight independent 16-byte loads before using any of them
+    float w[8][8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      if (i0 + 8 * q < r) load8(wrow + i0 + 8 * q, w[q]);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      if (i0 + 8 * q >= r) break;
+      const float4 ua = *reinterpret_cast<const float4*>(u + i0 + 8 * q);
+      const float4 ub = *reinterpret_cast<const float4*>(u + i0 + 8 * q + 4);
+      acc = fmaf(w[q][0], ua.x, acc); acc = fmaf(w[q][1], ua.y, acc);
+      acc = fmaf(w[q][2], ua.z, acc); acc = fmaf(w[q][3], ua.w, acc);
+      acc = fmaf(w[q][4], ub.x, acc); acc = fmaf(w[q][5], ub.y, acc);
+      acc = fmaf(w[q][6], ub.z, acc); acc = fmaf(w[q][7], ub.w, acc);
+    }
   }
   return acc;
 }

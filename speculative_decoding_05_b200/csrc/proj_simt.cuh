@@ -85,7 +85,8 @@ draft_proj_simt_kernel(const float* __restrict__ base, const TW* __restrict__ U,
                        const TW* __restrict__ W, int V, int r, int B, int K, int k,
                        const int32_t* __restrict__ prev_token, const int32_t* __restrict__ tokens,
                        const float* __restrict__ inv_temp, float* __restrict__ draft_logits,
-                       float2* __restrict__ part, int n_chunks, unsigned* flags) {
+                       float* __restrict__ draft_bias, float2* __restrict__ part, int n_chunks,
+                       unsigned* flags) {
   extern __shared__ __align__(16) float u_s[];  // [NB][r]
   __shared__ int x[NB];
   __shared__ float it2[NB], it[NB];
@@ -131,6 +132,7 @@ draft_proj_simt_kernel(const float* __restrict__ base, const TW* __restrict__ U,
       const float s = warp_sum(e);
       if (lane == 0) part[(size_t)gb * n_chunks + c] = make_float2(A, s);
       if (draft_logits != nullptr && valid) draft_logits[row + v] = a * it[b];
+      if (draft_bias != nullptr && valid) draft_bias[row + v] = acc[b];
     }
   }
 }
@@ -190,6 +192,34 @@ residual_proj_simt_kernel(const float* __restrict__ target, const float* __restr
       const float Q = warp_sum(q), P = warp_sum(pt);
       if (lane == 0) rpart[(size_t)gb * n_chunks + c] = make_float2(Q, P);
     }
+  }
+}
+
+// Residual partials when the draft's bias rows are available: the draft row
+// at position j is rebuilt from base + bias without touching W.  Grid
+// (chunk groups, B); one warp per 32-row chunk, lane = vocabulary row.
+__global__ void __launch_bounds__(256)
+residual_bias_kernel(const float* __restrict__ target, const float* __restrict__ base,
+                     const float* __restrict__ draft_bias, int V, int K,
+                     const ResInfo* __restrict__ info, const float* __restrict__ inv_temp,
+                     float2* __restrict__ rpart, int n_chunks, unsigned* flags) {
+  const int b = blockIdx.y;
+  const ResInfo ri = info[b];
+  const float it2 = checked_inv_temp(inv_temp, b, flags) * kLog2e;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const float* trow = target + (size_t)ri.row * V;
+  const size_t drow = ((size_t)b * K + (ri.bonus ? 0 : ri.j)) * (size_t)V;
+  for (int c = blockIdx.x * 8 + warp; c < n_chunks; c += gridDim.x * 8) {
+    const int v = c * kChunk + lane;
+    float q = 0.0f, pt = 0.0f;
+    if (v < V) {
+      const float t = trow[v];
+      const float bv = ri.bonus ? 0.0f : base[drow + v];
+      const float bias = ri.bonus ? 0.0f : draft_bias[drow + v];
+      q = residual_q(t, bv, bias, ri, it2, &pt);
+    }
+    const float Q = warp_sum(q), P = warp_sum(pt);
+    if (lane == 0) rpart[(size_t)b * n_chunks + c] = make_float2(Q, P);
   }
 }
 

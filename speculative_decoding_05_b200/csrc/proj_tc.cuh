@@ -1,32 +1,447 @@
-// proj_tc.cuh -- tensor-core (tcgen05) projection path for large batches.
+// proj_tc.cuh -- tensor-core (tcgen05) projection for large batches.
+//
+// bias[b, v] = U[x_b] . W[v] is a [B, r] x [r, V] GEMM once B is large.
+// Each CTA owns a block of kBlockM = 128 requests (MMA M; rows past B are
+// zero) and a contiguous range of vocabulary tiles of kTileN = 128 rows
+// (MMA N); K = r (64..256).  The gathered U rows (operand A) are written to
+// shared memory once per launch in the 128-byte-swizzled K-major layout;
+// W tiles (operand B) stream through a TMA ring and the accumulator lives
+// in TMEM (two 128-column buffers, so the epilogue of tile t overlaps the
+// MMAs of tile t+1).  The epilogue thread of request b reads its TMEM row
+// (tcgen05.ld) and reduces every 32-row chunk of its row to a softmax
+// partial locally -- no cross-thread reduction, because the request is the
+// TMEM lane.
+//
+//   warp 0       W producer (TMA, evict-last: W is re-read every position)
+//   warp 1       TMEM allocator + MMA issuer (one thread)
+//   warp 2       base-logit producer (TMA 3-D boxes, evict-first)   [draft]
+//   warps 3..6   epilogue (128 threads = 128 requests)
+//
+// Draft mode streams base[b, k, v0:v0+32] boxes through a second TMA ring.
+// Residual mode reads the per-request rows base[b, j_b, :] and
+// target[row_b, :] directly (each thread owns one request's contiguous
+// row segment), since j_b differs between requests.
 #pragma once
 
+#include <cudaTypedefs.h>
+
 #include "proj_simt.cuh"
+#include "tc_common.cuh"
 
 namespace dspark {
 
+constexpr int kTcThreads = 224;
+constexpr int kBlockM = 128;
+constexpr int kTileN = 128;
+constexpr int kWStages = 4;
+constexpr int kBStages = 5;
+constexpr int kStageBytes = 16384;  // 128 rows x 128 bytes
+constexpr int kTmemCols = 256;
+
 struct TcPlan {
+  CUtensorMap tm_w;
+  CUtensorMap tm_base;
+  const float* base;
+  const float* target;
+  const __nv_bfloat16* U;
   int V, r, B, K;
+  int n_tiles, n_bb, ctas_per_bb;
 };
 
-inline bool tc_supported(int V, int r, int B) {
-  (void)V;
-  (void)r;
-  (void)B;
-  return false;
+inline size_t tc_smem_bytes(int r, bool residual) {
+  return 1024 + (size_t)(r / 64) * kStageBytes + (size_t)kWStages * kStageBytes +
+         (residual ? 0 : (size_t)kBStages * kStageBytes) + 256;
 }
 
-inline dspark_status tc_plan_draft(TcPlan&, const float*, const void*, const void*, int, int, int,
-                                   int) {
-  return DSPARK_ERR_UNSUPPORTED;
+inline bool tc_supported(int V, int r, int B) {
+  return B > 16 && r % 64 == 0 && r >= 64 && r <= 256 && V % 4 == 0 && V >= kTileN;
 }
-inline dspark_status tc_plan_residual(TcPlan&, const float*, const float*, const void*, const void*,
-                                      int, int, int, int) {
-  return DSPARK_ERR_UNSUPPORTED;
+
+template <bool kRes>
+__global__ void __launch_bounds__(kTcThreads, 1)
+proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_base,
+               const __nv_bfloat16* __restrict__ U, int V, int r, int B, int K, int k,
+               const int32_t* __restrict__ prev_token, const int32_t* __restrict__ tokens,
+               const float* __restrict__ inv_temp, const float* __restrict__ target,
+               const float* __restrict__ base, const ResInfo* __restrict__ info,
+               float* __restrict__ draft_logits, float* __restrict__ draft_bias,
+               float2* __restrict__ part, int n_chunks, int n_tiles, int ctas_per_bb,
+               unsigned* flags) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nkb = r >> 6;
+  uint8_t* sA = sm;
+  uint8_t* sW = sA + nkb * kStageBytes;
+  uint8_t* sBase = sW + kWStages * kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + (kRes ? 0 : kBStages * kStageBytes));
+  uint64_t* fullW = bars;
+  uint64_t* emptyW = fullW + kWStages;
+  uint64_t* fullB = emptyW + kWStages;
+  uint64_t* emptyB = fullB + kBStages;
+  uint64_t* accFull = emptyB + kBStages;
+  uint64_t* accEmpty = accFull + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accEmpty + 2);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bb = blockIdx.x / ctas_per_bb, pi = blockIdx.x % ctas_per_bb;
+  const int t0 = (int)((long long)pi * n_tiles / ctas_per_bb);
+  const int t1 = (int)((long long)(pi + 1) * n_tiles / ctas_per_bb);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kWStages; ++i) {
+      mbar_init(&fullW[i], 1);
+      mbar_init(&emptyW[i], 1);
+    }
+    for (int i = 0; i < kBStages; ++i) {
+      mbar_init(&fullB[i], 1);
+      mbar_init(&emptyB[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&accFull[i], 1);
+      mbar_init(&accEmpty[i], 4);
+    }
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+
+  // operand A: the previous-token rows of U for this block of requests
+  const int cpr = r >> 3;  // 16-byte chunks per row
+  for (int q = threadIdx.x; q < kBlockM * cpr; q += kTcThreads) {
+    const int m = q / cpr, c = q % cpr;
+    const int b = bb * kBlockM + m;
+    int x = -1;
+    if (b < B) {
+      if (kRes) {
+        const ResInfo& ri = info[b];
+        x = ri.bonus ? -1 : ri.x_prev;
+      } else {
+        x = (k == 0) ? prev_token[b] : tokens[(size_t)b * K + (k - 1)];
+        if (x >= V || (k > 0 && x < 0)) {
+          if (c == 0) raise_flag(flags, DSPARK_FLAG_BAD_TOKEN);
+          x = (k > 0) ? (x < 0 ? 0 : V - 1) : -1;
+        }
+      }
+    }
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (x >= 0) val = __ldg(reinterpret_cast<const uint4*>(U + (size_t)x * r) + c);
+    const int kb = c >> 3, j = c & 7;
+    *reinterpret_cast<uint4*>(sA + kb * kStageBytes + m * 128 + ((j ^ (m & 7)) << 4)) = val;
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- W producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int it = 0;
+      for (int t = t0; t < t1 && !*s_abort; ++t) {
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kWStages;
+          const uint32_t ph = (uint32_t)(it / kWStages) & 1u;
+          if (!mbar_wait(&emptyW[s], ph ^ 1u)) {
+            *s_abort = 1;
+            raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+            break;
+          }
+          mbar_arrive_expect_tx(&fullW[s], kStageBytes);
+          tma_load_2d_hint(sW + s * kStageBytes, &tm_w, &fullW[s], kb * 64, t * kTileN, pol);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(kBlockM, kTileN);
+      const uint32_t a0 = smem_u32(sA), w0 = smem_u32(sW);
+      int it = 0;
+      for (int t = t0; t < t1 && !*s_abort; ++t) {
+        const int a = (t - t0) & 1;
+        const uint32_t aph = (uint32_t)((t - t0) >> 1) & 1u;
+        if (!mbar_wait(&accEmpty[a], aph ^ 1u)) {
+          *s_abort = 1;
+          raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = it % kWStages;
+          const uint32_t ph = (uint32_t)(it / kWStages) & 1u;
+          if (!mbar_wait(&fullW[s], ph)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t ad = sdesc_sw128(a0 + kb * kStageBytes + kk * 32);
+            const uint64_t bd = sdesc_sw128(w0 + s * kStageBytes + kk * 32);
+            mma_bf16_ss(tmem + a * kTileN, ad, bd, idesc, (kb | kk) != 0);
+          }
+          mma_commit(&emptyW[s]);
+        }
+        if (!ok) {
+          *s_abort = 1;
+          raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+          break;
+        }
+        mma_commit(&accFull[a]);
+      }
+    }
+  } else if (warp == 2) {
+    // ---------------- base-logit producer (draft only)
+    if (!kRes && lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      int it = 0;
+      for (int t = t0; t < t1 && !*s_abort; ++t) {
+        for (int cb = 0; cb < kTileN / 32; ++cb, ++it) {
+          const int s = it % kBStages;
+          const uint32_t ph = (uint32_t)(it / kBStages) & 1u;
+          if (!mbar_wait(&emptyB[s], ph ^ 1u)) {
+            *s_abort = 1;
+            raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+            break;
+          }
+          mbar_arrive_expect_tx(&fullB[s], kStageBytes);
+          tma_load_3d_hint(sBase + s * kStageBytes, &tm_base, &fullB[s], t * kTileN + cb * 32, k,
+                           bb * kBlockM, pol);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue: thread = request (TMEM lane)
+    const int quarter = warp & 3;
+    const int m = quarter * 32 + lane;
+    const int b = bb * kBlockM + m;
+    const bool bval = b < B;
+    const float it = bval ? checked_inv_temp(inv_temp, b, flags) : 1.0f;
+    const float it2 = it * kLog2e;
+    ResInfo ri{};
+    if (kRes && bval) ri = info[b];
+    const uint64_t pol = policy_evict_first();
+    int itB = 0;
+    for (int t = t0; t < t1; ++t) {
+      const int a = (t - t0) & 1;
+      const uint32_t aph = (uint32_t)((t - t0) >> 1) & 1u;
+      if (*s_abort || !mbar_wait(&accFull[a], aph)) {
+        *s_abort = 1;
+        raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      float2 pp[kTileN / 32];
+#pragma unroll 1
+      for (int cb = 0; cb < kTileN / 32; ++cb) {
+        float d[32], bv[32];
+        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
+        const int v0 = t * kTileN + cb * 32;
+        if (!kRes) {
+          const int s = itB % kBStages;
+          const uint32_t ph = (uint32_t)(itB / kBStages) & 1u;
+          ++itB;
+          if (!mbar_wait(&fullB[s], ph)) {
+            *s_abort = 1;
+            raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+          }
+          const uint8_t* row = sBase + s * kStageBytes + m * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const float4 q4 = *reinterpret_cast<const float4*>(row + ((j ^ (m & 7)) << 4));
+            bv[4 * j] = q4.x; bv[4 * j + 1] = q4.y; bv[4 * j + 2] = q4.z; bv[4 * j + 3] = q4.w;
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&emptyB[s]);
+          float A = -CUDART_INF_F;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (v0 + j < V) A = fmaxf(A, bv[j] + d[j]);
+          float sum = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (v0 + j < V) sum += ex2(((bv[j] - A) + d[j]) * it2);
+          pp[cb] = make_float2(A, sum);
+          if (draft_bias != nullptr && bval) {
+            float* dst = draft_bias + ((size_t)b * K + k) * (size_t)V + v0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              if (v0 + j < V)
+                *reinterpret_cast<float4*>(dst + j) = make_float4(d[j], d[j + 1], d[j + 2], d[j + 3]);
+          }
+          if (draft_logits != nullptr && bval) {
+            float* dst = draft_logits + ((size_t)b * K + k) * (size_t)V + v0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              if (v0 + j < V)
+                *reinterpret_cast<float4*>(dst + j) =
+                    make_float4((bv[j] + d[j]) * it, (bv[j + 1] + d[j + 1]) * it,
+                                (bv[j + 2] + d[j + 2]) * it, (bv[j + 3] + d[j + 3]) * it);
+          }
+        } else {
+          float tq[32];
+          if (bval) {
+            const float* trow = target + (size_t)ri.row * V + v0;
+            const float* brow = base + ((size_t)b * K + (ri.bonus ? 0 : ri.j)) * (size_t)V + v0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+              float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = t4;
+              if (v0 + j < V) {
+                t4 = ld_stream4(trow + j, pol);
+                if (!ri.bonus) b4 = ld_stream4(brow + j, pol);
+              }
+              tq[j] = t4.x; tq[j + 1] = t4.y; tq[j + 2] = t4.z; tq[j + 3] = t4.w;
+              bv[j] = b4.x; bv[j + 1] = b4.y; bv[j + 2] = b4.z; bv[j + 3] = b4.w;
+            }
+          }
+          float qs = 0.0f, ps = 0.0f;
+          if (bval) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              if (v0 + j < V) {
+                float pt;
+                qs += residual_q(tq[j], bv[j], d[j], ri, it2, &pt);
+                ps += pt;
+              }
+            }
+          }
+          pp[cb] = make_float2(qs, ps);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&accEmpty[a]);
+      if (bval) {
+        float2* dst = part + (size_t)b * n_chunks + t * (kTileN / 32);
+#pragma unroll
+        for (int cb = 0; cb < kTileN / 32; ++cb)
+          if (t * (kTileN / 32) + cb < n_chunks) dst[cb] = pp[cb];
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
-inline void tc_launch_draft(const TcPlan&, int, const int32_t*, const int32_t*, const float*, float*,
-                            float2*, unsigned*, cudaStream_t) {}
-inline void tc_launch_residual(const TcPlan&, const ResInfo*, const float*, float2*, unsigned*,
-                               cudaStream_t) {}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+inline int num_sms() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+// W [V, r] bf16 as 64 x 128 boxes (128-byte rows), 128-byte swizzle.
+inline bool encode_w_map(CUtensorMap* m, const void* W, int V, int r) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)r, (cuuint64_t)V};
+  cuuint64_t strides[1] = {(cuuint64_t)r * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kTileN};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(W), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// base [B, K, V] fp32 as 32 (v) x 1 (k) x 128 (b) boxes, 128-byte swizzle.
+inline bool encode_base_map(CUtensorMap* m, const float* base, int V, int K, int B) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)V, (cuuint64_t)K, (cuuint64_t)B};
+  cuuint64_t strides[2] = {(cuuint64_t)V * 4, (cuuint64_t)K * V * 4};
+  cuuint32_t box[3] = {32, 1, (cuuint32_t)kBlockM};
+  cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline void tc_grid(TcPlan& p) {
+  p.n_tiles = (p.V + kTileN - 1) / kTileN;
+  p.n_bb = (p.B + kBlockM - 1) / kBlockM;
+  int per = num_sms() / p.n_bb;
+  if (per < 1) per = 1;
+  if (per > p.n_tiles) per = p.n_tiles;
+  p.ctas_per_bb = per;
+}
+
+inline dspark_status tc_plan_draft(TcPlan& p, const float* base, const void* U, const void* W,
+                                   int V, int r, int B, int K) {
+  p.V = V; p.r = r; p.B = B; p.K = K;
+  p.base = base;
+  p.target = nullptr;
+  p.U = static_cast<const __nv_bfloat16*>(U);
+  if (!encode_w_map(&p.tm_w, W, V, r) || !encode_base_map(&p.tm_base, base, V, K, B))
+    return DSPARK_ERR_CUDA;
+  tc_grid(p);
+  return DSPARK_OK;
+}
+
+inline dspark_status tc_plan_residual(TcPlan& p, const float* target, const float* base,
+                                      const void* U, const void* W, int V, int r, int B, int K) {
+  p.V = V; p.r = r; p.B = B; p.K = K;
+  p.base = base;
+  p.target = target;
+  p.U = static_cast<const __nv_bfloat16*>(U);
+  if (!encode_w_map(&p.tm_w, W, V, r)) return DSPARK_ERR_CUDA;
+  p.tm_base = p.tm_w;  // unused in residual mode
+  tc_grid(p);
+  return DSPARK_OK;
+}
+
+template <bool kRes>
+inline void tc_set_attr() {
+  static bool done = false;
+  if (!done) {
+    cudaFuncSetAttribute(proj_tc_kernel<kRes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)tc_smem_bytes(256, kRes));
+    done = true;
+  }
+}
+
+inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const int32_t* tokens,
+                            const float* it, float* dl, float* dbias, float2* part,
+                            unsigned* flags, cudaStream_t s) {
+  tc_set_attr<false>();
+  proj_tc_kernel<false><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, false), s>>>(
+      p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, k, prev, tokens, it, nullptr, p.base, nullptr,
+      dl, dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, flags);
+}
+
+inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,
+                               float2* rpart, unsigned* flags, cudaStream_t s) {
+  tc_set_attr<true>();
+  proj_tc_kernel<true><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, true), s>>>(
+      p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, 0, nullptr, nullptr, it, p.target, p.base, info,
+      nullptr, nullptr, rpart, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, flags);
+}
 
 }  // namespace dspark

@@ -118,7 +118,8 @@ draft_sample_kernel(const float* __restrict__ base, const TW* __restrict__ U,
                     const TW* __restrict__ W, int V, int r, int K, int k,
                     const int32_t* __restrict__ prev_token, int32_t* __restrict__ tokens,
                     const float* __restrict__ inv_temp, const float* __restrict__ u_draft,
-                    const float2* __restrict__ part, int n_chunks, float* __restrict__ p_tok,
+                    const float2* __restrict__ part, int n_chunks,
+                    const float* __restrict__ draft_bias, float* __restrict__ p_tok,
                     float* __restrict__ lse, float* __restrict__ ref_max,
                     float* __restrict__ ref_sum, unsigned* flags) {
   __shared__ __align__(16) float u_s[kMaxRank];
@@ -140,7 +141,7 @@ draft_sample_kernel(const float* __restrict__ base, const TW* __restrict__ U,
 
   int xp = (k == 0) ? prev_token[b] : tokens[(size_t)b * K + (k - 1)];
   xp = checked_token(xp, V, k == 0, flags);
-  if (xp >= 0)
+  if (xp >= 0 && draft_bias == nullptr)
     for (int i = threadIdx.x; i < r; i += kSampleThreads) u_s[i] = to_f32(U[(size_t)xp * r + i]);
   __syncthreads();
 
@@ -150,8 +151,11 @@ draft_sample_kernel(const float* __restrict__ base, const TW* __restrict__ U,
     const bool valid = v < V;
     float e = 0.0f;
     if (valid) {
-      const float bias = (xp >= 0) ? dot_row(W + (size_t)v * r, u_s, r) : 0.0f;
-      const float bv = base[((size_t)b * K + k) * (size_t)V + v];
+      const size_t row = ((size_t)b * K + k) * (size_t)V;
+      const float bias = draft_bias != nullptr ? draft_bias[row + v]
+                         : (xp >= 0)           ? dot_row(W + (size_t)v * r, u_s, r)
+                                               : 0.0f;
+      const float bv = base[row + v];
       e = ex2(((bv - M) + bias) * it2);
     }
     const int pick = pick_lane(valid ? (double)e : 0.0, pk.before, pk.target);
@@ -185,7 +189,8 @@ residual_sample_kernel(const float* __restrict__ target, const float* __restrict
                        const TW* __restrict__ U, const TW* __restrict__ W, int V, int r, int K,
                        const float* __restrict__ inv_temp, const float* __restrict__ u_res,
                        const ResInfo* __restrict__ info, const float2* __restrict__ rpart,
-                       int n_chunks, int32_t* __restrict__ out_tokens,
+                       int n_chunks, const float* __restrict__ draft_bias,
+                       int32_t* __restrict__ out_tokens,
                        int32_t* __restrict__ last_token, unsigned* flags) {
   __shared__ __align__(16) float u_s[kMaxRank];
   __shared__ double shd[32];
@@ -206,7 +211,7 @@ residual_sample_kernel(const float* __restrict__ target, const float* __restrict
   });
 
   const int xp = ri.bonus ? -1 : ri.x_prev;
-  if (xp >= 0)
+  if (xp >= 0 && draft_bias == nullptr)
     for (int i = threadIdx.x; i < r; i += kSampleThreads) u_s[i] = to_f32(U[(size_t)xp * r + i]);
   __syncthreads();
 
@@ -216,9 +221,14 @@ residual_sample_kernel(const float* __restrict__ target, const float* __restrict
     const bool valid = v < V;
     double e = 0.0;
     if (valid) {
-      const float bias = (xp >= 0) ? dot_row(W + (size_t)v * r, u_s, r) : 0.0f;
+      const size_t drow = ((size_t)b * K + (ri.bonus ? 0 : ri.j)) * (size_t)V;
+      float bias = 0.0f;
+      if (!ri.bonus) {
+        if (draft_bias != nullptr) bias = draft_bias[drow + v];
+        else if (xp >= 0) bias = dot_row(W + (size_t)v * r, u_s, r);
+      }
       const float t = target[(size_t)ri.row * V + v];
-      const float bv = ri.bonus ? 0.0f : base[((size_t)b * K + ri.j) * (size_t)V + v];
+      const float bv = ri.bonus ? 0.0f : base[drow + v];
       float pt;
       const float qv = residual_q(t, bv, bias, ri, it2, &pt);
       e = (double)(use_q ? qv : pt);

@@ -64,10 +64,11 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.dspark_verify_workspace_size.restype = S
     lib.dspark_prefix_workspace_size.argtypes = [I, I, I]
     lib.dspark_prefix_workspace_size.restype = S
-    lib.dspark_draft_markov.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, S, P]
+    lib.dspark_draft_markov.argtypes = [P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P,
+                                        S, P]
     lib.dspark_draft_markov.restype = I
     lib.dspark_verify.argtypes = [P, L, P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P,
-                                  P, P, S, P]
+                                  P, P, P, S, P]
     lib.dspark_verify.restype = I
     lib.dspark_confidence_prefix.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P, S, P]
     lib.dspark_confidence_prefix.restype = I
@@ -145,13 +146,15 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 
 
 def dspark_draft_markov(base_logits, U, W, prev_token, inv_temp, u_draft, tokens, p_tok, lse,
-                        ref_max, ref_sum, workspace, draft_logits=None, stream=None):
+                        ref_max, ref_sum, workspace, draft_logits=None, draft_bias=None,
+                        stream=None):
     B, K, V = base_logits.shape
     r = W.shape[1]
     rc = load().dspark_draft_markov(
         _ptr(base_logits), _ptr(U), _ptr(W), _dtype_code(U), V, r, B, K, _ptr(prev_token),
         _ptr(inv_temp), _ptr(u_draft), _ptr(tokens), _ptr(p_tok), _ptr(lse), _ptr(ref_max),
-        _ptr(ref_sum), _ptr(draft_logits), _ptr(workspace), workspace.numel(), _stream(stream))
+        _ptr(ref_sum), _ptr(draft_logits), _ptr(draft_bias), _ptr(workspace), workspace.numel(),
+        _stream(stream))
     _check("dspark_draft_markov", rc)
 
 
@@ -167,14 +170,14 @@ def dspark_confidence_prefix(z, temps, cost_tokens, cost_ms, enable, c, survival
 
 def dspark_verify(target_logits, row_start, verify_len, base_logits, U, W, prev_token, inv_temp,
                   tokens, p_tok, ref_max, ref_sum, u_accept, u_resample, n_accepted, out_tokens,
-                  workspace, last_token=None, stream=None):
+                  workspace, last_token=None, draft_bias=None, stream=None):
     n_rows, V = target_logits.shape
     B, K = tokens.shape
     r = W.shape[1]
     rc = load().dspark_verify(
         _ptr(target_logits), n_rows, _ptr(row_start), _ptr(verify_len), _ptr(base_logits),
         _ptr(U), _ptr(W), _dtype_code(U), V, r, B, K, _ptr(prev_token), _ptr(inv_temp),
-        _ptr(tokens), _ptr(p_tok), _ptr(ref_max), _ptr(ref_sum), _ptr(u_accept),
+        _ptr(tokens), _ptr(p_tok), _ptr(ref_max), _ptr(ref_sum), _ptr(draft_bias), _ptr(u_accept),
         _ptr(u_resample), _ptr(n_accepted), _ptr(out_tokens), _ptr(last_token),
         _ptr(workspace), workspace.numel(), _stream(stream))
     _check("dspark_verify", rc)

@@ -17,9 +17,10 @@ from tests.parity import compare_step, host
 pytestmark = pytest.mark.gpu
 
 
-def _run(w, enable=None, seed=None, requests=None, oracle=None, inp=None):
+def _run(w, enable=None, seed=None, requests=None, oracle=None, inp=None, keep_bias=None):
     inp = inp or WL.make_inputs(w, device="cuda", seed=seed)
-    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype,
+                      keep_bias=keep_bias)
     en = w.scheduler if enable is None else enable
     step.run(inp, enable_prefix=en)
     torch.cuda.synchronize()
@@ -51,6 +52,64 @@ def test_small_shapes(oracle_mod, bf16, V, r, B, K):
     rep, _, _ = _run(w, oracle=oracle_mod, inp=inp)
     _assert_ok(rep)
     assert rep.checked["draft"] >= B
+
+
+@pytest.mark.parametrize("V,r,B,K", [(4096, 64, 40, 3), (1000, 128, 130, 2), (3000, 256, 17, 4),
+                                     (2048, 192, 257, 2)])
+def test_tensor_core_path(oracle_mod, V, r, B, K):
+    """B > 16 with bf16 U/W takes the tcgen05 projection (ragged last
+    vocabulary tile, partial request blocks, several request blocks)."""
+    w = WL.get("stress", V=V, r=r, B=B, K=K, seed=3 * V + B)
+    assert D.dspark_draft_path(V, r, B, K, D.DSPARK_BF16) == "tcgen05"
+    inp = WL.make_inputs(w, device="cuda")
+    inp["prev_token"][1] = -1
+    req = np.unique(np.r_[0, 1, B - 1, np.random.default_rng(V).choice(B, size=min(B, 12), replace=False)])
+    rep, _, _ = _run(w, oracle=oracle_mod, inp=inp, requests=req)
+    _assert_ok(rep)
+
+
+@pytest.mark.parametrize("V,r,B,K,keep", [(4096, 64, 3, 5, True), (1000, 128, 1, 4, False),
+                                          (20000, 256, 16, 6, True), (151936, 256, 2, 3, False),
+                                          (8192, 192, 9, 16, False)])
+def test_persistent_draft(oracle_mod, V, r, B, K, keep):
+    """B <= 16 with bf16 U/W: all K positions in one persistent launch
+    (resident + streamed W tiles, grid barrier, redundant sampler); the
+    verify either reuses the draft's bias rows or re-projects."""
+    w = WL.get("stress", V=V, r=r, B=B, K=K, seed=7 * V + B)
+    assert D.dspark_draft_path(V, r, B, K, D.DSPARK_BF16) == "tcgen05-persistent"
+    inp = WL.make_inputs(w, device="cuda")
+    inp["prev_token"][0] = -1
+    rep, step, _ = _run(w, oracle=oracle_mod, inp=inp, keep_bias=keep)
+    _assert_ok(rep)
+    assert rep.checked["draft"] >= B
+
+
+def test_graph_capture_matches_eager():
+    """A whole step captured in a CUDA graph replays to the same outputs as
+    the eager calls (fixed launch shapes, no host synchronisation)."""
+    for name, over in [("single", dict(V=16384, K=6, seed=12)), ("batched", dict(V=8192, B=40, K=3, seed=13))]:
+        w = WL.get(name, **over)
+        inp = WL.make_inputs(w, device="cuda")
+        step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+        step.run(inp, enable_prefix=True)
+        torch.cuda.synchronize()
+        ref = [t.clone() for t in (step.tokens, step.p_tok, step.lse, step.verify_len,
+                                    step.n_accepted, step.out_tokens, step.last_token)]
+        for t in (step.tokens, step.p_tok, step.out_tokens):
+            t.zero_()
+        s = torch.cuda.Stream()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            step.run(inp, enable_prefix=True)
+        for _ in range(2):
+            g.replay()
+        torch.cuda.synchronize()
+        got = (step.tokens, step.p_tok, step.lse, step.verify_len, step.n_accepted,
+               step.out_tokens, step.last_token)
+        for a, b in zip(ref, got):
+            assert torch.equal(a, b)
+        assert all(f == 0 for f in step.flags().values())
+        del g
 
 
 def test_temperatures_and_flat_peaked(oracle_mod):

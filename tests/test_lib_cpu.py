@@ -46,8 +46,13 @@ def test_status_strings_and_paths(lib):
     for code in range(7):
         assert D.status_string(code)
     assert D.dspark_version() >= 100
-    assert D.dspark_draft_path(151936, 256, 1, 16, D.DSPARK_BF16) == "cuda-core"
+    assert D.dspark_draft_path(151936, 256, 1, 16, D.DSPARK_BF16) == "tcgen05-persistent"
+    assert D.dspark_draft_path(151936, 256, 16, 16, D.DSPARK_BF16) == "tcgen05-persistent"
+    assert D.dspark_draft_path(1024, 16, 2, 4, D.DSPARK_F32) == "cuda-core"
     assert D.dspark_draft_path(1024, 16, 64, 4, D.DSPARK_F32) == "cuda-core"
+    assert D.dspark_draft_path(151936, 256, 64, 8, D.DSPARK_BF16) == "tcgen05"
+    assert D.dspark_draft_path(151936, 256, 17, 8, D.DSPARK_BF16) == "tcgen05"
+    assert D.dspark_draft_path(1000, 32, 4, 8, D.DSPARK_BF16) == "cuda-core"
 
 
 def test_workspace_sizes(lib):
@@ -66,7 +71,7 @@ def _draft(lib, V=1024, r=16, B=2, K=3, base=1 << 20, U=1 << 21, W=1 << 22, ws=1
     P = ctypes.c_void_p
     p = P(1 << 23)
     return lib.dspark_draft_markov(P(base), P(U), P(W), dtype, V, r, B, K, p, None, p, p, p, p, p,
-                                   p, None, P(ws), ws_bytes, None)
+                                   p, None, None, P(ws), ws_bytes, None)
 
 
 def test_argument_validation_before_launch(lib):
@@ -89,5 +94,5 @@ def test_argument_validation_before_launch(lib):
     assert lib.dspark_confidence_prefix(p, p, p, p, 1, 4, 4, 1, p, p, p, p, ws, 256, None) == 1
     # verify: missing target
     vb = lib.dspark_verify_workspace_size(1024, 16, 2, 3)
-    assert lib.dspark_verify(None, 10, p, p, p, p, p, 1, 1024, 16, 2, 3, p, None, p, p, p, p, p,
-                             p, p, p, None, ws, vb, None) == 1
+    assert lib.dspark_verify(None, 10, p, p, p, p, p, 1, 1024, 16, 2, 3, p, None, p, p, p, p, None,
+                             p, p, p, p, None, ws, vb, None) == 1
