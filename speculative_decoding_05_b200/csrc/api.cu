@@ -22,10 +22,10 @@ constexpr int kMaxK = 64;
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Workspace of the draft: header (status word at 0, grid-barrier counter
-// at 64), chunk partials [B][n_chunks], then (persistent path) per-CTA
-// partials [B][<=1024] and bias rows [B][V].
-constexpr size_t kCounterOff = 64;
+// Workspace of the draft: header (status word at 0, eight grid-barrier
+// counters 128 bytes apart from byte 128), chunk partials [B][n_chunks],
+// then (persistent path) per-CTA partials [B][<=1024] and bias rows [B][V].
+constexpr size_t kCounterOff = 128;
 struct DraftWs {
   size_t part_off, cta_off, bias_off, total;
 };
@@ -56,9 +56,9 @@ dspark_status check_launch() {
   return cudaGetLastError() == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
-// Clears the status word and the grid-barrier counter of a workspace.
+// Clears the status word and the grid-barrier counters of a workspace.
 dspark_status clear_status(void* ws, cudaStream_t s) {
-  return cudaMemsetAsync(ws, 0, 128, s) == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+  return cudaMemsetAsync(ws, 0, kHeaderBytes, s) == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
 // Shape checks shared by draft and verify.
@@ -163,6 +163,7 @@ dspark_status draft_impl(const float* base, const void* U, const void* W, dspark
     PersistArgs a;
     a.base = base;
     a.U = static_cast<const __nv_bfloat16*>(U);
+    a.W = static_cast<const __nv_bfloat16*>(W);
     a.prev_token = prev;
     a.inv_temp = it;
     a.u_draft = ud;
@@ -267,7 +268,8 @@ const char* dspark_status_string(dspark_status s) {
 
 const char* dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype) {
   (void)K;
-  if (use_persist(V, r, B, uw_dtype)) return "tcgen05-persistent";
+  if (use_persist(V, r, B, uw_dtype))
+    return B <= kSimtMaxB ? "persistent-cuda-core" : "tcgen05-persistent";
   return use_tc(V, r, B, uw_dtype) ? "tcgen05" : "cuda-core";
 }
 

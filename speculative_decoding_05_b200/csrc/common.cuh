@@ -18,9 +18,10 @@ namespace dspark {
 constexpr int kChunk = 32;
 // Elements of a target row reduced by one CTA in the target-statistics pass.
 constexpr int kSeg = 8192;
-// The workspace starts with a 256-byte header whose first word is the
-// device status (DSPARK_FLAG_* bits).
-constexpr size_t kHeaderBytes = 256;
+// The workspace starts with a 2 KB header whose first word is the device
+// status (DSPARK_FLAG_* bits); the persistent draft keeps its grid-barrier
+// counters there.
+constexpr size_t kHeaderBytes = 2048;
 constexpr float kLog2e = 1.4426950408889634f;
 
 __host__ __device__ inline int n_chunks_of(int V) { return (V + kChunk - 1) / kChunk; }

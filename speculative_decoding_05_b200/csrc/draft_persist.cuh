@@ -2,26 +2,35 @@
 // (B <= 16): all K sequential positions in one launch.
 //
 // One CTA per SM owns a contiguous range of 128-row vocabulary tiles for
-// the whole call.  The first tiles of the range stay resident in shared
-// memory for all K positions; the rest stream from L2 through a TMA ring
-// whose producer runs ahead across positions (the tiles do not depend on
-// the sampled tokens).  Per position:
-//   1. gather U[x_{k-1}] for the B requests into the MMA B operand
-//      (N = 16 rows, zero-padded);
-//   2. tcgen05 MMAs D[v, b] = W_tile[v, :] . u_b (M = 128 vocabulary rows,
-//      N = 16, K = r), one TMEM slot per tile;
-//   3. epilogue (thread = vocabulary row): a = base + bias, per 32-row chunk
+// the whole call.  Its W tiles stream from L2 through one deep TMA ring
+// whose producer runs ahead across positions: the tiles do not depend on
+// the sampled tokens, so while the grid waits at a barrier and samples,
+// the ring already fills with the next position's tiles (as good as
+// keeping that much of W resident).  The base-logit rows of the CTA's
+// range are bulk-copied into shared memory one position ahead by another
+// producer warp.  Per position:
+//   1. tcgen05 MMAs D[v, b] = W_tile[v, :] . U[x_b] (M = 128 vocabulary
+//      rows, N = 16 requests zero-padded, K = r) into an 8-slot TMEM
+//      accumulator ring.  The first three tiles of every CTA's range stay
+//      resident in TMEM for the whole call and feed the MMA as its A operand
+//      straight from tensor memory (28 MB of W on chip across the GPU), so
+//      the part that streams each position (about 49 MB at V = 151936,
+//      r = 256) stays L2-resident; the rest comes from the TMA ring;
+//   2. epilogue (thread = vocabulary row): a = base + bias, per 32-row chunk
 //      the softmax partial (max, sum exp) per request via warp shuffles,
 //      the bias values to a scratch row (so the sampler needs no W), and a
 //      per-CTA partial;
-//   4. grid barrier (bounded spin on a counter in the workspace);
-//   5. every CTA samples every request redundantly in three levels (CTA
-//      partials -> chunk partials of the chosen CTA -> the 32 stored values
-//      of the chosen chunk), so the next position starts without a second
-//      barrier; CTA 0 writes the outputs.
+//   3. grid barrier: a release reduction on one counter, relaxed polling
+//      with a time limit, one acquire fence;
+//   4. every CTA samples every request redundantly in three dependent
+//      loads (CTA partials -> chunk partials of the chosen CTA -> the 32
+//      stored values of the chosen chunk), so the next position needs no
+//      second barrier; the sampling warp writes U[x_k] straight into the
+//      MMA operand; CTA 0 writes the outputs.
 //
-// Warp roles: warp 0 TMA producer, warp 1 TMEM allocator + MMA issuer,
-// warps 4..7 epilogue + sampler (TMEM lane quarters 0..3); warps 2..3 idle.
+// Warp roles: warp 0 W producer (TMA), warp 1 TMEM allocator + MMA issuer,
+// warp 2 base producer (bulk copies), warps 4..7 epilogue + sampler (TMEM
+// lane quarters 0..3); warp 3 idle.
 #pragma once
 
 #include "proj_tc.cuh"
@@ -30,18 +39,25 @@
 namespace dspark {
 
 constexpr int kPThreads = 256;
-constexpr int kPN = 16;            // MMA N: requests, zero-padded
+constexpr int kPN = 16;          // MMA N: requests, zero-padded
 constexpr int kPMaxB = 16;
-constexpr int kPStages = 5;        // streaming ring: 16 KB K-blocks
-constexpr int kPMaxTiles = 16;     // tiles per CTA (one 16-column TMEM slot each)
-constexpr int kPResidentBytes = 131072;
-constexpr int kPTmemCols = 256;
-constexpr int kPEpiWarp0 = 4;      // first epilogue warp
+constexpr int kPMaxTiles = 16;   // tiles per CTA
+constexpr int kPTmemCols = 512;
+constexpr int kPDSlots = 8;      // accumulator ring: 8 x 16 TMEM columns
+constexpr int kPACol = 128;      // first TMEM column of the resident W tiles
+constexpr int kPMaxTmemTiles = 3;  // W tiles resident in TMEM (128 columns each)
+constexpr int kPGroup = 1;       // tiles whose MMAs are issued together
+constexpr int kPEpiWarp0 = 4;    // first epilogue warp
 constexpr int kPEpiThreads = 128;
+constexpr int kPMaxG = 256;      // grid limit of the sampler's register arrays
+constexpr int kPMinStages = 4;
+constexpr int kPMaxStages = 24;
+constexpr int kPSmemLimit = 232448;  // 227 KB of dynamic shared memory
 
 struct PersistArgs {
   const float* base;
   const __nv_bfloat16* U;
+  const __nv_bfloat16* W;
   const int32_t* prev_token;
   const float* inv_temp;
   const float* u_draft;
@@ -51,24 +67,50 @@ struct PersistArgs {
   float* ref_max;
   float* ref_sum;
   float* draft_logits;
-  float2* part;      // [B][n_chunks]
-  float2* cta_part;  // [B][G]
-  float* bias_buf;   // [B][V] scratch, used when draft_bias is NULL
-  float* draft_bias; // [B][K][V] or NULL
+  float2* part;       // [B][n_chunks]
+  float2* cta_part;   // [B][G]
+  float* bias_buf;    // [B][V] scratch, used when draft_bias is NULL
+  float* draft_bias;  // [B][K][V] or NULL
   unsigned* flags;
   unsigned* grid_counter;
   int V, r, B, K, n_chunks, n_tiles;
+  int max_nt;         // tiles of the largest CTA range
+  int n_stages;       // W ring stages (16 KB each)
 };
 
 __host__ __device__ inline int p_tile_begin(int cta, int G, int n_tiles) {
   return (int)((long long)cta * n_tiles / G);
 }
 
-inline size_t persist_smem_bytes(int r) {
-  const int nkb = r / 64;
-  const int tile = nkb * kStageBytes;
-  const int nres = kPResidentBytes / tile;
-  return 1024 + (size_t)nres * tile + (size_t)kPStages * kStageBytes + (size_t)nkb * 2048 + 1024;
+struct PersistLayout {
+  int G, max_nt, n_stages;
+  size_t u_bytes, base_bytes, smem;
+};
+
+inline int persist_grid(int V) {
+  const int n_tiles = (V + kTileN - 1) / kTileN;
+  int G = num_sms();
+  if (G > n_tiles) G = n_tiles;
+  if (G > kPMaxG) G = kPMaxG;
+  return G;
+}
+
+// Up to this many requests the persistent draft runs its projection on the
+// CUDA cores; above it, on tcgen05 with N = 16.
+constexpr int kSimtMaxB = 4;
+
+inline PersistLayout persist_layout(int V, int r, int B) {
+  PersistLayout L;
+  const int n_tiles = (V + kTileN - 1) / kTileN;
+  L.G = persist_grid(V);
+  L.max_nt = (n_tiles + L.G - 1) / L.G;
+  L.u_bytes = B <= kSimtMaxB ? (size_t)B * r * 4 : (size_t)(r / 64) * 2048;
+  L.base_bytes = (((size_t)B * L.max_nt * kTileN * 4) + 1023) & ~size_t(1023);
+  const size_t fixed = 1024 /*align*/ + L.u_bytes + L.base_bytes + 2048 /*barriers, scratch*/;
+  L.n_stages = fixed >= (size_t)kPSmemLimit ? 0 : (int)((kPSmemLimit - fixed) / kStageBytes);
+  if (L.n_stages > kPMaxStages) L.n_stages = kPMaxStages;
+  L.smem = fixed + (size_t)L.n_stages * kStageBytes;
+  return L;
 }
 
 // epilogue-group barrier (warps 4..7 only)
@@ -90,81 +132,292 @@ __device__ __forceinline__ void merge_partial(float& M, float& S, float A, float
   M = Mn;
 }
 
+__device__ __forceinline__ double partial_weight(float2 q, float M, float it2) {
+  return (q.x == -CUDART_INF_F) ? 0.0 : (double)(q.y * ex2((q.x - M) * it2));
+}
+
+// Write U[x] (or zeros) into row n of the 128-byte swizzled K-major B
+// operand, one 16-byte chunk per lane step.
+__device__ __forceinline__ void store_u_row(uint8_t* sU, const __nv_bfloat16* U, int x, int n, int r,
+                                            int lane) {
+  const int cpr = r >> 3;
+  for (int c = lane; c < cpr; c += 32) {
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (x >= 0) val = __ldg(reinterpret_cast<const uint4*>(U + (size_t)x * r) + c);
+    const int kb = c >> 3, j = c & 7;
+    *reinterpret_cast<uint4*>(sU + kb * 2048 + n * 128 + ((j ^ (n & 7)) << 4)) = val;
+  }
+}
+
+// Grid barrier of position k, called by one thread per CTA: a release
+// reduction on the counter, relaxed polling with a time limit, then one
+// acquire fence.  Returns false on timeout (DSPARK_FLAG_TIMEOUT raised).
+__device__ __forceinline__ bool persist_grid_barrier(unsigned* counter, int k, int G,
+                                                     unsigned* flags) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
+  const unsigned target = (unsigned)(k + 1) * (unsigned)G;
+  const uint64_t tstart = global_timer_ns();
+  bool ok = true;
+  for (;;) {
+    unsigned seen;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(counter) : "memory");
+    if (seen >= target) break;
+    if (global_timer_ns() - tstart > kWaitLimitNs) {
+      raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+      ok = false;
+      break;
+    }
+  }
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+  return ok;
+}
+
+// Redundant three-level sampler of request b at position k, one full warp:
+// CTA partials -> chunk partials of the chosen CTA -> the 32 stored bias
+// values of the chosen chunk.  Every CTA computes the same token; CTA 0
+// writes the outputs.  Returns the token (in every lane).
+__device__ __noinline__ int persist_sample(const PersistArgs& p, int b, int k, int G, int cta,
+                                           float it2b, float itvb) {
+  const int lane = threadIdx.x & 31;
+  const int K = p.K, V = p.V;
+        const double u = (double)p.u_draft[(size_t)b * K + k];
+        const float2* cp = p.cta_part + (size_t)b * G;
+        // level 1: CTA partials (contiguous ranges of at most 8 CTAs per lane)
+        const int per = (G + 31) / 32;
+        const int c0 = min(lane * per, G), c1 = min(c0 + per, G);
+        float2 q[kPMaxG / 32];
+#pragma unroll
+        for (int i = 0; i < kPMaxG / 32; ++i)
+          q[i] = (c0 + i < c1) ? __ldcg(&cp[c0 + i]) : make_float2(-CUDART_INF_F, 0.0f);
+        float m = -CUDART_INF_F;
+#pragma unroll
+        for (int i = 0; i < kPMaxG / 32; ++i) m = fmaxf(m, q[i].x);
+        const float M = warp_max(m);
+        double wsum = 0.0;
+#pragma unroll
+        for (int i = 0; i < kPMaxG / 32; ++i) wsum += partial_weight(q[i], M, it2b);
+        const double incl = warp_incl_scan_d(wsum);
+        const double Z = __shfl_sync(0xffffffffu, incl, 31);
+        const double T = u * Z;
+        double start = __shfl_up_sync(0xffffffffu, incl, 1);
+        if (lane == 0) start = 0.0;
+        const unsigned own = __ballot_sync(0xffffffffu, start <= T && T < incl && wsum > 0.0);
+        int cstar = -1;
+        double before = 0.0;
+        {
+          double cum = start, lastb = start, pb = start;
+          int pick = -1, lastp = -1;
+#pragma unroll
+          for (int i = 0; i < kPMaxG / 32; ++i) {
+            const double w = partial_weight(q[i], M, it2b);
+            if (pick < 0 && w > 0.0) {
+              lastp = c0 + i;
+              lastb = cum;
+              if (cum + w > T) {
+                pick = c0 + i;
+                pb = cum;
+              }
+            }
+            cum += w;
+          }
+          if (pick < 0) {
+            pick = lastp;
+            pb = lastb;
+          }
+          if (own) {
+            const int ol = __ffs(own) - 1;
+            cstar = __shfl_sync(0xffffffffu, pick, ol);
+            before = __shfl_sync(0xffffffffu, pb, ol);
+          } else {  // no crossing (u*Z rounded to Z): last CTA with mass
+            const unsigned pos = __ballot_sync(0xffffffffu, lastp >= 0);
+            const int pl = pos ? 31 - __clz(pos) : 0;
+            cstar = __shfl_sync(0xffffffffu, lastp, pl);
+            before = -CUDART_INF;
+            if (cstar < 0) cstar = 0;
+          }
+        }
+        // level 2: chunk partials of CTA cstar (<= 64 chunks, two per lane)
+        const int ch0 = p_tile_begin(cstar, G, p.n_tiles) * (kTileN / kChunk);
+        const int ch1 = min(p_tile_begin(cstar + 1, G, p.n_tiles) * (kTileN / kChunk), p.n_chunks);
+        const float2* pp = p.part + (size_t)b * p.n_chunks;
+        const int ca = ch0 + 2 * lane, cb2 = ca + 1;
+        const float2 qa = (ca < ch1) ? __ldcg(&pp[ca]) : make_float2(-CUDART_INF_F, 0.0f);
+        const float2 qb = (cb2 < ch1) ? __ldcg(&pp[cb2]) : make_float2(-CUDART_INF_F, 0.0f);
+        const double wA = partial_weight(qa, M, it2b), wB = partial_weight(qb, M, it2b);
+        const double pin = warp_incl_scan_d(wA + wB);
+        double lstart = __shfl_up_sync(0xffffffffu, pin, 1);
+        if (lane == 0) lstart = 0.0;
+        lstart += before;
+        int chunk = -1;
+        double before2 = 0.0;
+        {
+          const bool hitA = wA > 0.0 && lstart + wA > T;
+          const bool hitB = wB > 0.0 && lstart + wA + wB > T;
+          const unsigned h = __ballot_sync(0xffffffffu, hitA || hitB);
+          if (h) {
+            const int hl = __ffs(h) - 1;
+            const int myc = hitA ? ca : cb2;
+            const double myb = hitA ? lstart : lstart + wA;
+            chunk = __shfl_sync(0xffffffffu, myc, hl);
+            before2 = __shfl_sync(0xffffffffu, myb, hl);
+          } else {  // rounding: last chunk of the CTA with positive weight
+            const unsigned hp = __ballot_sync(0xffffffffu, wA > 0.0 || wB > 0.0);
+            const int hl = hp ? 31 - __clz(hp) : 0;
+            const int myc = (wB > 0.0) ? cb2 : ca;
+            chunk = __shfl_sync(0xffffffffu, myc, hl);
+            if (!hp) chunk = ch0;
+            before2 = -CUDART_INF;
+          }
+        }
+        // level 3: the 32 stored values of the chunk
+        const int v = chunk * kChunk + lane;
+        const bool valid = v < V;
+        double e = 0.0;
+        float ef = 0.0f;
+        if (valid) {
+          const float bias = p.draft_bias != nullptr
+                                 ? __ldcg(&p.draft_bias[((size_t)b * K + k) * (size_t)V + v])
+                                 : __ldcg(&p.bias_buf[(size_t)b * V + v]);
+          const float bv = p.base[((size_t)b * K + k) * (size_t)V + v];
+          ef = ex2(((bv - M) + bias) * it2b);
+          e = (double)ef;
+        }
+        const int pick = pick_lane(e, before2, T);
+        const int x = __shfl_sync(0xffffffffu, valid ? v : 0, pick);
+        if (lane == pick && cta == 0) {
+          const size_t o = (size_t)b * K + k;
+          if (!(Z > 0.0) || !isfinite(Z)) {
+            raise_flag(p.flags, DSPARK_FLAG_NONFINITE);
+            p.tokens[o] = 0;
+            p.p_tok[o] = 0.0f;
+            p.lse[o] = CUDART_NAN_F;
+            p.ref_max[o] = M;
+            p.ref_sum[o] = 1.0f;
+          } else {
+            p.tokens[o] = x;
+            p.p_tok[o] = (float)((double)ef / Z);
+            p.lse[o] = (float)((double)M * (double)itvb + log(Z));
+            p.ref_max[o] = M;
+            p.ref_sum[o] = (float)Z;
+          }
+        }
+  return x;
+}
+
 __global__ void __launch_bounds__(kPThreads, 1)
 draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nkb = p.r >> 6;
-  const int tile_bytes = nkb * kStageBytes;
-  const int max_res = kPResidentBytes / tile_bytes;
   const int G = gridDim.x, cta = blockIdx.x;
   const int t0 = p_tile_begin(cta, G, p.n_tiles), t1 = p_tile_begin(cta + 1, G, p.n_tiles);
   const int nt = t1 - t0;
-  const int nres = min(nt, max_res);
+  const int B = p.B, K = p.K, V = p.V;
+  const int S = p.n_stages;
+  const int base_stride = p.max_nt * kTileN;  // floats per request in sBase
+  const int nres = min(nt, kPMaxTmemTiles);   // tiles resident in TMEM
 
-  uint8_t* sRes = sm;
-  uint8_t* sRing = sRes + max_res * tile_bytes;
-  uint8_t* sU = sRing + kPStages * kStageBytes;
-  uint64_t* ringFull = reinterpret_cast<uint64_t*>(sU + nkb * 2048);
-  uint64_t* ringEmpty = ringFull + kPStages;
-  uint64_t* dFull = ringEmpty + kPStages;   // [kPMaxTiles]
-  uint64_t* uReady = dFull + kPMaxTiles;
-  uint64_t* resReady = uReady + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(resReady + 1);
+  uint8_t* sRing = sm;
+  uint8_t* sU = sRing + S * kStageBytes;
+  float* sBase = reinterpret_cast<float*>(sU + nkb * 2048);
+  uint8_t* misc = reinterpret_cast<uint8_t*>(sBase) +
+                  ((((size_t)B * base_stride * 4) + 1023) & ~size_t(1023));
+  uint64_t* ringFull = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* ringEmpty = ringFull + kPMaxStages;
+  uint64_t* dFull = ringEmpty + kPMaxStages;  // [kPDSlots]
+  uint64_t* dEmpty = dFull + kPDSlots;        // [kPDSlots]
+  uint64_t* uReady = dEmpty + kPDSlots;
+  uint64_t* baseFull = uReady + 1;
+  uint64_t* baseEmpty = baseFull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(baseEmpty + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_tok = const_cast<int*>(reinterpret_cast<volatile int*>(s_abort + 1));  // [kPMaxB]
-  float* s_wm = reinterpret_cast<float*>(s_tok + kPMaxB);                        // [4][kPMaxB]
-  float* s_ws = s_wm + 4 * kPMaxB;                                                // [4][kPMaxB]
+  float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [4][kPMaxB]
+  float* s_ws = s_wm + 4 * kPMaxB;                        // [4][kPMaxB]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int B = p.B, K = p.K, V = p.V;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kPStages; ++i) {
+    for (int i = 0; i < S; ++i) {
       mbar_init(&ringFull[i], 1);
       mbar_init(&ringEmpty[i], 1);
     }
-    for (int i = 0; i < kPMaxTiles; ++i) mbar_init(&dFull[i], 1);
+    for (int i = 0; i < kPDSlots; ++i) {
+      mbar_init(&dFull[i], 1);
+      mbar_init(&dEmpty[i], 4);
+    }
     mbar_init(uReady, 1);
-    mbar_init(resReady, 1);
+    mbar_init(baseFull, 1);
+    mbar_init(baseEmpty, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kPTmemCols);
-  // zero the padded request rows of the B operand once (rows >= B stay zero)
+  // operand B of position 1: U[prev_token] rows, zero rows past B
   for (int i = threadIdx.x; i < nkb * 2048 / 16; i += kPThreads)
     reinterpret_cast<uint4*>(sU)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  if (warp >= kPEpiWarp0) {
+    const int ew = warp - kPEpiWarp0;
+    for (int b = ew; b < B; b += 4) {
+      const int x = checked_token(p.prev_token[b], V, true, p.flags);
+      store_u_row(sU, p.U, x, b, p.r, lane);
+    }
+  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp >= kPEpiWarp0) {
+    // resident W tiles -> TMEM: lane = tile row, 32-bit column c holds the
+    // bf16 pair (2c, 2c+1) of the row (the A-operand layout of a
+    // tensor-memory MMA)
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    for (int i = 0; i < nres; ++i) {
+      const int v = (t0 + i) * kTileN + row;
+      const uint4* src = reinterpret_cast<const uint4*>(p.W + (size_t)(v < V ? v : 0) * p.r);
+      for (int g = 0; g < (p.r >> 6); ++g) {
+        uint32_t regs[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 val = (v < V) ? __ldg(src + g * 8 + q) : make_uint4(0, 0, 0, 0);
+          regs[4 * q] = val.x;
+          regs[4 * q + 1] = val.y;
+          regs[4 * q + 2] = val.z;
+          regs[4 * q + 3] = val.w;
+        }
+        tmem_st32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(kPACol + i * 128 + g * 32),
+                  regs);
+      }
+    }
+    tmem_st_wait();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
 
   if (warp == 0) {
-    // ------------------------------------------------ TMA producer
+    // ------------------------------------------------ W producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
-      if (nres > 0) {
-        mbar_arrive_expect_tx(resReady, (uint32_t)(nres * tile_bytes));
-        for (int i = 0; i < nres; ++i)
-          for (int kb = 0; kb < nkb; ++kb)
-            tma_load_2d_hint(sRes + i * tile_bytes + kb * kStageBytes, &tm_w, resReady, kb * 64,
-                             (t0 + i) * kTileN, pol);
-      }
       int it = 0;
       for (int k = 0; k < K && !*s_abort; ++k) {
-        for (int i = nres; i < nt && !*s_abort; ++i) {
-          for (int kb = 0; kb < nkb; ++kb, ++it) {
-            const int s = it % kPStages;
-            const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
-            if (!mbar_wait(&ringEmpty[s], ph ^ 1u)) {
-              *s_abort = 1;
-              raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
-              break;
+        for (int g0 = nres; g0 < nt && !*s_abort; g0 += kPGroup) {
+          const int gn = min(kPGroup, nt - g0);
+          for (int kb = 0; kb < nkb && !*s_abort; ++kb) {
+            for (int j = 0; j < gn; ++j, ++it) {
+              const int s = it % S;
+              const uint32_t ph = (uint32_t)(it / S) & 1u;
+              if (!mbar_wait(&ringEmpty[s], ph ^ 1u)) {
+                *s_abort = 1;
+                raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+                break;
+              }
+              mbar_arrive_expect_tx(&ringFull[s], kStageBytes);
+              tma_load_2d_hint(sRing + s * kStageBytes, &tm_w, &ringFull[s], kb * 64,
+                               (t0 + g0 + j) * kTileN, pol);
             }
-            mbar_arrive_expect_tx(&ringFull[s], kStageBytes);
-            tma_load_2d_hint(sRing + s * kStageBytes, &tm_w, &ringFull[s], kb * 64,
-                             (t0 + i) * kTileN, pol);
           }
         }
       }
@@ -173,45 +426,88 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(kTileN, kPN);
-      const uint32_t res0 = smem_u32(sRes), ring0 = smem_u32(sRing), u0 = smem_u32(sU);
+      const uint32_t ring0 = smem_u32(sRing), u0 = smem_u32(sU);
       int it = 0;
-      bool ok = nres == 0 || mbar_wait(resReady, 0);
+      bool ok = true;
       for (int k = 0; k < K && ok; ++k) {
-        if (!mbar_wait(uReady, (uint32_t)k & 1u) || *s_abort) {
+        if (!mbar_wait_spin(uReady, (uint32_t)k & 1u) || *s_abort) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int i = 0; i < nt && ok; ++i) {
-          const uint32_t d = tmem + (uint32_t)(i * kPN);
-          for (int kb = 0; kb < nkb; ++kb) {
-            uint32_t a_base;
-            int s = -1;
-            if (i < nres) {
-              a_base = res0 + i * tile_bytes + kb * kStageBytes;
-            } else {
-              s = it % kPStages;
-              const uint32_t ph = (uint32_t)(it / kPStages) & 1u;
-              ++it;
-              if (!mbar_wait(&ringFull[s], ph)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              a_base = ring0 + s * kStageBytes;
-            }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16_ss(d, sdesc_sw128(a_base + kk * 32), sdesc_sw128(u0 + kb * 2048 + kk * 32),
-                          idesc, (kb | kk) != 0);
-            if (s >= 0) mma_commit(&ringEmpty[s]);
+        // groups: the TMEM-resident tiles, then streamed tiles kPGroup at a time
+        for (int g0 = 0; g0 < nt && ok;) {
+          const bool resident = g0 < nres;
+          const int gn = min(kPGroup, (resident ? nres : nt) - g0);
+          uint32_t dcol[kPGroup];
+          for (int j = 0; j < gn && ok; ++j) {
+            const int i = g0 + j, slot = i % kPDSlots;
+            const int per_step = (nt - slot + kPDSlots - 1) / kPDSlots;  // uses per position
+            const uint32_t use = (uint32_t)(k * per_step + i / kPDSlots);
+            ok = mbar_wait_spin(&dEmpty[slot], (use & 1u) ^ 1u);
+            dcol[j] = tmem + (uint32_t)(slot * kPN);
           }
-          mma_commit(&dFull[i]);
+          if (!ok) break;
+          tc_fence_after();
+          if (resident) {
+            for (int kb = 0; kb < nkb; ++kb) {
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd = sdesc_sw128(u0 + kb * 2048 + kk * 32);
+                for (int j = 0; j < gn; ++j)
+                  mma_bf16_ts(dcol[j], tmem + (uint32_t)(kPACol + (g0 + j) * 128 + (kb * 4 + kk) * 8),
+                              bd, idesc, (kb | kk) != 0);
+              }
+            }
+          } else {
+            for (int kb = 0; kb < nkb && ok; ++kb) {
+              int st[kPGroup];
+              for (int j = 0; j < gn; ++j, ++it) {
+                st[j] = it % S;
+                if (!mbar_wait_spin(&ringFull[st[j]], (uint32_t)(it / S) & 1u)) {
+                  ok = false;
+                  break;
+                }
+              }
+              if (!ok) break;
+              tc_fence_after();
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd = sdesc_sw128(u0 + kb * 2048 + kk * 32);
+                for (int j = 0; j < gn; ++j)
+                  mma_bf16_ss(dcol[j], sdesc_sw128(ring0 + st[j] * kStageBytes + kk * 32), bd, idesc,
+                              (kb | kk) != 0);
+              }
+              for (int j = 0; j < gn; ++j) mma_commit(&ringEmpty[st[j]]);
+            }
+          }
+          if (!ok) break;
+          for (int j = 0; j < gn; ++j) mma_commit(&dFull[(g0 + j) % kPDSlots]);
+          g0 += gn;
         }
       }
       if (!ok) {
         *s_abort = 1;
         raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ base producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      const int v0 = t0 * kTileN;
+      const int nval = min(nt * kTileN, V - v0);
+      const uint32_t bytes = (uint32_t)nval * 4u;
+      for (int k = 0; k < K && !*s_abort; ++k) {
+        if (!mbar_wait(baseEmpty, ((uint32_t)k & 1u) ^ 1u)) {
+          *s_abort = 1;
+          raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(baseFull, bytes * (uint32_t)B);
+        for (int b = 0; b < B; ++b)
+          bulk_load(sBase + (size_t)b * base_stride, p.base + ((size_t)b * K + k) * (size_t)V + v0,
+                    bytes, baseFull, pol);
       }
     }
   } else if (warp >= kPEpiWarp0) {
@@ -225,45 +521,40 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
       itv[b] = (b < B) ? checked_inv_temp(p.inv_temp, b, p.flags) : 1.0f;
       it2[b] = itv[b] * kLog2e;
     }
-    const int cpr = p.r >> 3;  // 16-byte chunks per U row
+    if (et == 0) mbar_arrive(uReady);  // operand B of position 1 is in place
     for (int k = 0; k < K; ++k) {
-      // 1. previous-token rows of U -> operand B (rows < B)
-      for (int q = et; q < B * cpr; q += kPEpiThreads) {
-        const int n = q / cpr, c = q % cpr;
-        int x = (k == 0) ? p.prev_token[n] : s_tok[n];
-        if (k == 0) x = checked_token(x, V, true, p.flags);
-        uint4 val = make_uint4(0, 0, 0, 0);
-        if (x >= 0) val = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)x * p.r) + c);
-        const int kb = c >> 3, j = c & 7;
-        *reinterpret_cast<uint4*>(sU + kb * 2048 + n * 128 + ((j ^ (n & 7)) << 4)) = val;
-      }
-      fence_proxy_async_smem();
-      epi_sync();
-      if (et == 0) mbar_arrive(uReady);
-
-      // 2.-3. epilogue per tile
+      // ---- epilogue over the CTA's tiles
       float wm[kPMaxB], ws[kPMaxB];
 #pragma unroll
       for (int b = 0; b < kPMaxB; ++b) {
         wm[b] = -CUDART_INF_F;
         ws[b] = 0.0f;
       }
+      bool ok = mbar_wait_spin(baseFull, (uint32_t)k & 1u);
       for (int i = 0; i < nt; ++i) {
-        if (!mbar_wait(&dFull[i], (uint32_t)k & 1u)) {
+        const int slot = i % kPDSlots;
+        const int per_step = (nt - slot + kPDSlots - 1) / kPDSlots;
+        const uint32_t use = (uint32_t)(k * per_step + i / kPDSlots);
+        ok = ok && mbar_wait_spin(&dFull[slot], use & 1u);
+        if (!ok) {
           *s_abort = 1;
           raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
         }
         tc_fence_after();
         float d[16];
-        tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * kPN), d);
-        const int v = (t0 + i) * kTileN + quarter * 32 + lane;
+        tmem_ld16(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(slot * kPN), d);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dEmpty[slot]);
+        const int vl = i * kTileN + quarter * 32 + lane;  // row within the CTA range
+        const int v = t0 * kTileN + vl;
         const bool valid = v < V;
         const int chunk = v >> 5;
 #pragma unroll
         for (int b = 0; b < kPMaxB; ++b) {
           if (b >= B) break;
           const size_t row = ((size_t)b * K + k) * (size_t)V;
-          const float bv = valid ? p.base[row + v] : 0.0f;
+          const float bv = valid ? sBase[(size_t)b * base_stride + vl] : 0.0f;
           const float a = valid ? bv + d[b] : -CUDART_INF_F;
           const float A = warp_max(a);
           const float e = valid ? ex2(((bv - A) + d[b]) * it2[b]) : 0.0f;
@@ -280,7 +571,6 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
         }
       }
       tc_fence_before();
-      // per-CTA partial of each request
       if (lane == 0) {
 #pragma unroll
         for (int b = 0; b < kPMaxB; ++b) {
@@ -289,175 +579,305 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
         }
       }
       epi_sync();
+      if (et == 0) mbar_arrive(baseEmpty);  // sBase may take the next position
       if (et < B) {
         const int b = et;
-        float M = -CUDART_INF_F, S = 0.0f;
+        float M = -CUDART_INF_F, Sm = 0.0f;
         for (int w2 = 0; w2 < 4; ++w2)
-          merge_partial(M, S, s_wm[w2 * kPMaxB + b], s_ws[w2 * kPMaxB + b], it2[b]);
-        p.cta_part[(size_t)b * G + cta] = make_float2(M, S);
+          merge_partial(M, Sm, s_wm[w2 * kPMaxB + b], s_ws[w2 * kPMaxB + b], it2[b]);
+        p.cta_part[(size_t)b * G + cta] = make_float2(M, Sm);
       }
-      // 4. grid barrier
+      // ---- grid barrier
       epi_sync();
-      if (et == 0) {
-        __threadfence();
-        atomicAdd(p.grid_counter, 1u);
-        const unsigned target = (unsigned)(k + 1) * (unsigned)G;
-        const uint64_t tstart = global_timer_ns();
-        while (ld_acquire_u32(p.grid_counter) < target) {
-          if (global_timer_ns() - tstart > kWaitLimitNs) {
-            *s_abort = 1;
-            raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
-            break;
-          }
-        }
-        __threadfence();
-      }
+      if (et == 0 && !persist_grid_barrier(p.grid_counter, k, G, p.flags)) *s_abort = 1;
       epi_sync();
       if (*s_abort) {
         if (et == 0 && k + 1 < K) mbar_arrive(uReady);  // release the MMA thread
         break;
       }
 
-      // 5. redundant three-level sampler: warp ew handles requests ew, ew+4, ...
+      // ---- redundant sampler: warp ew handles requests ew, ew+4, ...
       for (int b = ew; b < B; b += 4) {
-        const double u = (double)p.u_draft[(size_t)b * K + k];
-        const float2* cp = p.cta_part + (size_t)b * G;
-        // level 1: CTA partials, contiguous CTA ranges per lane
-        const int per = (G + 31) / 32;
-        const int c0 = min(lane * per, G), c1 = min(c0 + per, G);
-        float m = -CUDART_INF_F;
-        for (int c = c0; c < c1; ++c) m = fmaxf(m, __ldcg(&cp[c]).x);
-        const float M = warp_max(m);
-        double wsum = 0.0;
-        for (int c = c0; c < c1; ++c) {
-          const float2 q = __ldcg(&cp[c]);
-          wsum += (q.x == -CUDART_INF_F) ? 0.0 : (double)(q.y * ex2((q.x - M) * it2[b]));
-        }
-        const double incl = warp_incl_scan_d(wsum);
-        const double Z = __shfl_sync(0xffffffffu, incl, 31);
-        const double T = u * Z;
-        const double excl = incl - wsum;
-        // lane owning the target (intervals [excl, incl) of consecutive lanes)
-        const double prev_incl = __shfl_up_sync(0xffffffffu, incl, 1);
-        const double start = lane == 0 ? 0.0 : prev_incl;
-        unsigned own = __ballot_sync(0xffffffffu, start <= T && T < incl && wsum > 0.0);
-        int cstar = -1;
-        double before = 0.0;
-        if (own) {
-          const int ol = __ffs(own) - 1;
-          if (lane == ol) {
-            double cum = start;
-            int lastp = -1;
-            double lastb = start;
-            for (int c = c0; c < c1; ++c) {
-              const float2 q = __ldcg(&cp[c]);
-              const double w = (q.x == -CUDART_INF_F) ? 0.0 : (double)(q.y * ex2((q.x - M) * it2[b]));
-              if (w > 0.0) {
-                lastp = c;
-                lastb = cum;
-              }
-              if (cum + w > T && w > 0.0) {
-                cstar = c;
-                before = cum;
-                break;
-              }
-              cum += w;
+        const int x = persist_sample(p, b, k, G, cta, it2[b], itv[b]);
+        // operand B of the next position: U[x] into row b
+        if (k + 1 < K) store_u_row(sU, p.U, x, b, p.r, lane);
+      }
+      fence_proxy_async_smem();
+      epi_sync();
+      if (et == 0 && k + 1 < K) mbar_arrive(uReady);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kPTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core variant for the smallest batches
+// ---------------------------------------------------------------------------
+//
+// At N = 16 a tcgen05 MMA instruction costs about as much as at several
+// times the width, so for one to a few requests the projection is a GEMV
+// on the CUDA cores (the thread owns one vocabulary row and accumulates the
+// row's dot product with U[x_{k-1}] in fp32, ascending index order).  The
+// memory plan stays the same: four W tiles per SM resident in TMEM for the
+// whole call (read back with tcgen05.ld, 38 MB of W on chip across the
+// GPU), the rest streamed from L2 through the TMA ring into shared memory,
+// base rows bulk-copied one position ahead.  Eight compute warps: tile i
+// belongs to warp group (i & 1); the warp with TMEM lane quarter q owns
+// rows 32q..32q+31 of the tile, i.e. one 32-row softmax chunk.
+constexpr int kSThreads = 384;
+constexpr int kSCompWarp0 = 4;
+constexpr int kSCompThreads = 256;
+constexpr int kSMaxTmemTiles = 4;
+
+__device__ __forceinline__ void comp_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kSCompThreads) : "memory");
+}
+
+// acc[b] += sum_e w_e * u_b[e0 + e] over the 8 bf16 values packed in q
+template <int NB>
+__device__ __forceinline__ void fma8(uint4 q, const float* __restrict__ u_s, int r, int e0, int B,
+                                     float (&acc)[NB]) {
+  float w[8];
+  w[0] = __uint_as_float(q.x << 16); w[1] = __uint_as_float(q.x & 0xffff0000u);
+  w[2] = __uint_as_float(q.y << 16); w[3] = __uint_as_float(q.y & 0xffff0000u);
+  w[4] = __uint_as_float(q.z << 16); w[5] = __uint_as_float(q.z & 0xffff0000u);
+  w[6] = __uint_as_float(q.w << 16); w[7] = __uint_as_float(q.w & 0xffff0000u);
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    if (b >= B) break;
+    const float4 ua = *reinterpret_cast<const float4*>(u_s + b * r + e0);
+    const float4 ub = *reinterpret_cast<const float4*>(u_s + b * r + e0 + 4);
+    float a = acc[b];
+    a = fmaf(w[0], ua.x, a); a = fmaf(w[1], ua.y, a);
+    a = fmaf(w[2], ua.z, a); a = fmaf(w[3], ua.w, a);
+    a = fmaf(w[4], ub.x, a); a = fmaf(w[5], ub.y, a);
+    a = fmaf(w[6], ub.z, a); a = fmaf(w[7], ub.w, a);
+    acc[b] = a;
+  }
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kSThreads, 1)
+draft_persist_simt_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int nkb = p.r >> 6;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int t0 = p_tile_begin(cta, G, p.n_tiles), t1 = p_tile_begin(cta + 1, G, p.n_tiles);
+  const int nt = t1 - t0;
+  const int B = p.B, K = p.K, V = p.V, r = p.r;
+  const int S = p.n_stages;
+  const int base_stride = p.max_nt * kTileN;
+  const int nres = min(nt, kSMaxTmemTiles);
+  const int nstream = nt - nres;
+
+  uint8_t* sRing = sm;
+  float* u_s = reinterpret_cast<float*>(sRing + S * kStageBytes);  // [B][r] fp32
+  float* sBase = u_s + (size_t)B * r;
+  uint8_t* misc = reinterpret_cast<uint8_t*>(sBase) +
+                  ((((size_t)B * base_stride * 4) + 1023) & ~size_t(1023));
+  uint64_t* ringFull = reinterpret_cast<uint64_t*>(misc);
+  uint64_t* ringEmpty = ringFull + kPMaxStages;
+  uint64_t* baseFull = ringEmpty + kPMaxStages;
+  uint64_t* baseEmpty = baseFull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(baseEmpty + 1);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [8][kPMaxB]
+  float* s_ws = s_wm + 8 * kPMaxB;                        // [8][kPMaxB]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(&ringFull[i], 1);
+      mbar_init(&ringEmpty[i], 4);
+    }
+    mbar_init(baseFull, 1);
+    mbar_init(baseEmpty, 1);
+    *s_abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, kPTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ W producer (streamed tiles)
+    if (lane == 0 && nstream > 0) {
+      const uint64_t pol = policy_evict_last();
+      int it = 0;
+      for (int k = 0; k < K && !*s_abort; ++k) {
+        for (int i = nres; i < nt && !*s_abort; ++i) {
+          for (int kb = 0; kb < nkb; ++kb, ++it) {
+            const int s = it % S;
+            if (!mbar_wait(&ringEmpty[s], ((uint32_t)(it / S) & 1u) ^ 1u)) {
+              *s_abort = 1;
+              raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+              break;
             }
-            if (cstar < 0) {
-              cstar = lastp;
-              before = lastb;
-            }
-          }
-          cstar = __shfl_sync(0xffffffffu, cstar, ol);
-          before = __shfl_sync(0xffffffffu, before, ol);
-        }
-        bool fallback = false;
-        if (cstar < 0) {  // no crossing (u*Z rounded to Z): last CTA with mass
-          const unsigned pos = __ballot_sync(0xffffffffu, wsum > 0.0);
-          const int pl = pos ? 31 - __clz(pos) : 0;
-          int lastc = -1;
-          if (lane == pl)
-            for (int c = c0; c < c1; ++c)
-              if (__ldcg(&cp[c]).x != -CUDART_INF_F && __ldcg(&cp[c]).y > 0.0f) lastc = c;
-          cstar = __shfl_sync(0xffffffffu, lastc, pl);
-          if (cstar < 0) cstar = 0;
-          fallback = true;
-        }
-        (void)excl;
-        // level 2: chunk partials of CTA cstar (<= 64 chunks, two per lane)
-        const int ch0 = p_tile_begin(cstar, G, p.n_tiles) * (kTileN / kChunk);
-        const int ch1 = min(p_tile_begin(cstar + 1, G, p.n_tiles) * (kTileN / kChunk), p.n_chunks);
-        const float2* pp = p.part + (size_t)b * p.n_chunks;
-        double wA = 0.0, wB = 0.0;
-        const int ca = ch0 + 2 * lane, cb2 = ca + 1;
-        if (ca < ch1) {
-          const float2 q = __ldcg(&pp[ca]);
-          wA = (q.x == -CUDART_INF_F) ? 0.0 : (double)(q.y * ex2((q.x - M) * it2[b]));
-        }
-        if (cb2 < ch1) {
-          const float2 q = __ldcg(&pp[cb2]);
-          wB = (q.x == -CUDART_INF_F) ? 0.0 : (double)(q.y * ex2((q.x - M) * it2[b]));
-        }
-        const double pin = warp_incl_scan_d(wA + wB);
-        const double lstart = before + (pin - (wA + wB));
-        int chunk = -1;
-        double before2 = 0.0;
-        if (!fallback) {
-          const bool hitA = wA > 0.0 && lstart + wA > T;
-          const bool hitB = wB > 0.0 && lstart + wA + wB > T;
-          const unsigned h = __ballot_sync(0xffffffffu, hitA || hitB);
-          if (h) {
-            const int hl = __ffs(h) - 1;
-            const int myc = hitA ? ca : cb2;
-            const double myb = hitA ? lstart : lstart + wA;
-            chunk = __shfl_sync(0xffffffffu, myc, hl);
-            before2 = __shfl_sync(0xffffffffu, myb, hl);
-          }
-        }
-        if (chunk < 0) {  // last chunk of the CTA with positive weight
-          const unsigned h = __ballot_sync(0xffffffffu, wA > 0.0 || wB > 0.0);
-          const int hl = h ? 31 - __clz(h) : 0;
-          const int myc = (wB > 0.0) ? cb2 : ca;
-          chunk = __shfl_sync(0xffffffffu, myc, hl);
-          before2 = -CUDART_INF;
-          if (!h) chunk = ch0;
-        }
-        // level 3: the 32 stored values of the chunk
-        const int v = chunk * kChunk + lane;
-        const bool valid = v < V;
-        double e = 0.0;
-        float ef = 0.0f;
-        if (valid) {
-          const float bias = p.draft_bias != nullptr
-                                 ? __ldcg(&p.draft_bias[((size_t)b * K + k) * (size_t)V + v])
-                                 : __ldcg(&p.bias_buf[(size_t)b * V + v]);
-          const float bv = p.base[((size_t)b * K + k) * (size_t)V + v];
-          ef = ex2(((bv - M) + bias) * it2[b]);
-          e = (double)ef;
-        }
-        const int pick = pick_lane(e, before2, T);
-        if (lane == pick) {
-          s_tok[b] = valid ? v : 0;
-          if (cta == 0) {
-            const size_t o = (size_t)b * K + k;
-            if (!(Z > 0.0) || !isfinite(Z)) {
-              raise_flag(p.flags, DSPARK_FLAG_NONFINITE);
-              p.tokens[o] = 0;
-              p.p_tok[o] = 0.0f;
-              p.lse[o] = CUDART_NAN_F;
-              p.ref_max[o] = M;
-              p.ref_sum[o] = 1.0f;
-            } else {
-              p.tokens[o] = valid ? v : 0;
-              p.p_tok[o] = (float)((double)ef / Z);
-              p.lse[o] = (float)((double)M * (double)itv[b] + log(Z));
-              p.ref_max[o] = M;
-              p.ref_sum[o] = (float)Z;
-            }
+            mbar_arrive_expect_tx(&ringFull[s], kStageBytes);
+            tma_load_2d_hint(sRing + s * kStageBytes, &tm_w, &ringFull[s], kb * 64,
+                             (t0 + i) * kTileN, pol);
           }
         }
       }
-      epi_sync();  // s_tok visible to the next position's gather
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------ base producer
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_first();
+      const int v0 = t0 * kTileN;
+      const uint32_t bytes = (uint32_t)min(nt * kTileN, V - v0) * 4u;
+      for (int k = 0; k < K && !*s_abort; ++k) {
+        if (!mbar_wait(baseEmpty, ((uint32_t)k & 1u) ^ 1u)) {
+          *s_abort = 1;
+          raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+          break;
+        }
+        mbar_arrive_expect_tx(baseFull, bytes * (uint32_t)B);
+        for (int b = 0; b < B; ++b)
+          bulk_load(sBase + (size_t)b * base_stride, p.base + ((size_t)b * K + k) * (size_t)V + v0,
+                    bytes, baseFull, pol);
+      }
+    }
+  } else if (warp >= kSCompWarp0) {
+    // ------------------------------------------------ compute + epilogue + sampler
+    const int ct = threadIdx.x - kSCompWarp0 * 32;  // 0..255
+    const int cw = warp - kSCompWarp0;              // 0..7
+    const int half = cw >> 2;                       // tile parity owned by this warp
+    const int quarter = warp & 3;                   // TMEM lane quarter
+    const int m = quarter * 32 + lane;              // row within a tile
+    float it2[NB], itv[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      itv[b] = (b < B) ? checked_inv_temp(p.inv_temp, b, p.flags) : 1.0f;
+      it2[b] = itv[b] * kLog2e;
+    }
+    // resident W tiles -> TMEM (rows of this warp's quarter, tiles of its half)
+    for (int i = half; i < nres; i += 2) {
+      const int v = (t0 + i) * kTileN + m;
+      const uint4* src = reinterpret_cast<const uint4*>(p.W + (size_t)(v < V ? v : 0) * r);
+      for (int g = 0; g < nkb; ++g) {
+        uint32_t regs[32];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const uint4 val = (v < V) ? __ldg(src + g * 8 + q) : make_uint4(0, 0, 0, 0);
+          regs[4 * q] = val.x;
+          regs[4 * q + 1] = val.y;
+          regs[4 * q + 2] = val.z;
+          regs[4 * q + 3] = val.w;
+        }
+        tmem_st32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + g * 32), regs);
+      }
+    }
+    tmem_st_wait();
+    // operand of position 1: U[prev_token] as fp32
+    for (int b = cw; b < B; b += 8) {
+      const int x = checked_token(p.prev_token[b], V, true, p.flags);
+      for (int e = lane; e < r; e += 32) u_s[b * r + e] = (x >= 0) ? to_f32(p.U[(size_t)x * r + e]) : 0.0f;
+    }
+    tc_fence_before();
+    comp_sync();
+    tc_fence_after();
+
+    for (int k = 0; k < K; ++k) {
+      float wm[NB], ws[NB];
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        wm[b] = -CUDART_INF_F;
+        ws[b] = 0.0f;
+      }
+      bool ok = mbar_wait_spin(baseFull, (uint32_t)k & 1u);
+      for (int i = half; i < nt; i += 2) {
+        float acc[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) acc[b] = 0.0f;
+        if (i < nres) {
+          for (int g = 0; g < nkb; ++g) {
+            float wf[32];
+            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + g * 32), wf);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint4 pk = make_uint4(__float_as_uint(wf[4 * q]), __float_as_uint(wf[4 * q + 1]),
+                                          __float_as_uint(wf[4 * q + 2]), __float_as_uint(wf[4 * q + 3]));
+              fma8<NB>(pk, u_s, r, g * 64 + q * 8, B, acc);
+            }
+          }
+        } else {
+          const int itb = (k * nstream + (i - nres)) * nkb;
+          for (int kb = 0; kb < nkb; ++kb) {
+            const int it = itb + kb, s = it % S;
+            ok = ok && mbar_wait_spin(&ringFull[s], (uint32_t)(it / S) & 1u);
+            const uint8_t* rowp = sRing + s * kStageBytes + m * 128;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint4 pk = *reinterpret_cast<const uint4*>(rowp + ((j ^ (m & 7)) << 4));
+              fma8<NB>(pk, u_s, r, kb * 64 + j * 8, B, acc);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ringEmpty[s]);
+          }
+        }
+        if (!ok) {
+          *s_abort = 1;
+          raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+        }
+        const int vl = i * kTileN + m;
+        const int v = t0 * kTileN + vl;
+        const bool valid = v < V;
+        const int chunk = v >> 5;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b >= B) break;
+          const size_t row = ((size_t)b * K + k) * (size_t)V;
+          const float bv = valid ? sBase[(size_t)b * base_stride + vl] : 0.0f;
+          const float a = valid ? bv + acc[b] : -CUDART_INF_F;
+          const float A = warp_max(a);
+          const float e = valid ? ex2(((bv - A) + acc[b]) * it2[b]) : 0.0f;
+          const float sm2 = warp_sum(e);
+          if (valid) {
+            if (p.draft_bias != nullptr) p.draft_bias[row + v] = acc[b];
+            else p.bias_buf[(size_t)b * V + v] = acc[b];
+            if (p.draft_logits != nullptr) p.draft_logits[row + v] = a * itv[b];
+          }
+          if (lane == 0 && chunk < p.n_chunks) {
+            p.part[(size_t)b * p.n_chunks + chunk] = make_float2(A, sm2);
+            merge_partial(wm[b], ws[b], A, sm2, it2[b]);
+          }
+        }
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          s_wm[cw * kPMaxB + b] = wm[b];
+          s_ws[cw * kPMaxB + b] = ws[b];
+        }
+      }
+      comp_sync();
+      if (ct == 0) mbar_arrive(baseEmpty);  // sBase may take the next position
+      if (ct < B) {
+        const int b = ct;
+        float M = -CUDART_INF_F, Sm = 0.0f;
+        for (int w2 = 0; w2 < 8; ++w2)
+          merge_partial(M, Sm, s_wm[w2 * kPMaxB + b], s_ws[w2 * kPMaxB + b], it2[b]);
+        p.cta_part[(size_t)b * G + cta] = make_float2(M, Sm);
+      }
+      comp_sync();
+      if (ct == 0 && !persist_grid_barrier(p.grid_counter, k, G, p.flags)) *s_abort = 1;
+      comp_sync();
+      if (*s_abort) break;
+      for (int b = cw; b < B; b += 8) {
+        const int x = persist_sample(p, b, k, G, cta, it2[b], itv[b]);
+        if (k + 1 < K)
+          for (int e = lane; e < r; e += 32) u_s[b * r + e] = to_f32(p.U[(size_t)x * r + e]);
+      }
+      comp_sync();
     }
   }
 
@@ -471,46 +891,51 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
 // host side
 // ---------------------------------------------------------------------------
 
-inline int persist_grid(int V) {
-  const int n_tiles = (V + kTileN - 1) / kTileN;
-  int G = num_sms();
-  if (G > n_tiles) G = n_tiles;
-  return G;
-}
-
 inline bool persist_supported(int V, int r, int B) {
   if (B < 1 || B > kPMaxB || r % 64 != 0 || r < 64 || r > 256 || V % 4 != 0 || V < kTileN)
     return false;
-  const int n_tiles = (V + kTileN - 1) / kTileN;
-  const int G = persist_grid(V);
-  return (n_tiles + G - 1) / G <= kPMaxTiles;
+  const PersistLayout L = persist_layout(V, r, B);
+  return L.max_nt <= kPMaxTiles && L.n_stages >= kPMinStages;
 }
 
-// Workspace bytes the persistent draft needs beyond the chunk partials:
-// per-CTA partials and the bias rows.
-inline size_t persist_extra_bytes(int V, int B) {
-  return align256((size_t)B * 1024 * sizeof(float2)) + align256((size_t)B * V * sizeof(float));
-}
-
-inline dspark_status persist_launch(const CUtensorMap& tm_w, const PersistArgs& a, cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(draft_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)persist_smem_bytes(256));
-    attr = true;
-  }
+template <typename Kern>
+inline dspark_status persist_launch_kernel(Kern kern, int threads, const CUtensorMap& tm_w,
+                                           const PersistArgs& a, const PersistLayout& L,
+                                           cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(persist_grid(a.V));
-  cfg.blockDim = dim3(kPThreads);
-  cfg.dynamicSmemBytes = persist_smem_bytes(a.r);
+  cfg.gridDim = dim3(L.G);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = L.smem;
   cfg.stream = s;
   cudaLaunchAttribute attrs[1];
   attrs[0].id = cudaLaunchAttributeCooperative;
   attrs[0].val.cooperative = 1;
   cfg.attrs = attrs;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, draft_persist_kernel, tm_w, a) == cudaSuccess ? DSPARK_OK
-                                                                                 : DSPARK_ERR_CUDA;
+  return cudaLaunchKernelEx(&cfg, kern, tm_w, a) == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
+inline dspark_status persist_launch(const CUtensorMap& tm_w, PersistArgs a, cudaStream_t s) {
+  static bool attr = false;
+  if (!attr) {
+    cudaFuncSetAttribute(draft_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kPSmemLimit);
+    cudaFuncSetAttribute(draft_persist_simt_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kPSmemLimit);
+    cudaFuncSetAttribute(draft_persist_simt_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kPSmemLimit);
+    cudaFuncSetAttribute(draft_persist_simt_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kPSmemLimit);
+    attr = true;
+  }
+  const PersistLayout L = persist_layout(a.V, a.r, a.B);
+  a.max_nt = L.max_nt;
+  a.n_stages = L.n_stages;
+  if (a.B == 1) return persist_launch_kernel(draft_persist_simt_kernel<1>, kSThreads, tm_w, a, L, s);
+  if (a.B == 2) return persist_launch_kernel(draft_persist_simt_kernel<2>, kSThreads, tm_w, a, L, s);
+  if (a.B <= kSimtMaxB)
+    return persist_launch_kernel(draft_persist_simt_kernel<4>, kSThreads, tm_w, a, L, s);
+  return persist_launch_kernel(draft_persist_kernel, kPThreads, tm_w, a, L, s);
 }
 
 }  // namespace dspark

@@ -46,7 +46,9 @@ def test_status_strings_and_paths(lib):
     for code in range(7):
         assert D.status_string(code)
     assert D.dspark_version() >= 100
-    assert D.dspark_draft_path(151936, 256, 1, 16, D.DSPARK_BF16) == "tcgen05-persistent"
+    assert D.dspark_draft_path(151936, 256, 1, 16, D.DSPARK_BF16) == "persistent-cuda-core"
+    assert D.dspark_draft_path(151936, 256, 4, 16, D.DSPARK_BF16) == "persistent-cuda-core"
+    assert D.dspark_draft_path(151936, 256, 5, 16, D.DSPARK_BF16) == "tcgen05-persistent"
     assert D.dspark_draft_path(151936, 256, 16, 16, D.DSPARK_BF16) == "tcgen05-persistent"
     assert D.dspark_draft_path(1024, 16, 2, 4, D.DSPARK_F32) == "cuda-core"
     assert D.dspark_draft_path(1024, 16, 64, 4, D.DSPARK_F32) == "cuda-core"
