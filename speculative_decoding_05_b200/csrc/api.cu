@@ -27,14 +27,16 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 // then (persistent path) per-CTA partials [B][<=1024] and bias rows [B][V].
 constexpr size_t kCounterOff = 128;
 struct DraftWs {
-  size_t part_off, cta_off, bias_off, total;
+  size_t part_off, cta_off, bias_off, rec_off, total;
 };
 DraftWs draft_ws(int V, int B) {
   DraftWs w;
+  const int Bp = B <= kPMaxB ? B : 0;  // persistent paths only
   w.part_off = kHeaderBytes;
   w.cta_off = w.part_off + align256((size_t)B * n_chunks_of(V) * sizeof(float2));
-  w.bias_off = w.cta_off + align256((size_t)(B <= kPMaxB ? B : 0) * 1024 * sizeof(float2));
-  w.total = w.bias_off + align256((size_t)(B <= kPMaxB ? B : 0) * V * sizeof(float));
+  w.bias_off = w.cta_off + align256((size_t)Bp * 1024 * sizeof(float2));
+  w.rec_off = w.bias_off + align256((size_t)Bp * V * sizeof(float));
+  w.total = w.rec_off + align256(Bp ? gemv_rec_bytes(Bp) : 0);
   return w;
 }
 
@@ -185,7 +187,13 @@ dspark_status draft_impl(const float* base, const void* U, const void* W, dspark
     a.K = K;
     a.n_chunks = nc;
     a.n_tiles = (V + kTileN - 1) / kTileN;
-    dspark_status st = persist_launch(tm_w, a, s);
+    GemvRecs recs;
+    recs.cta = reinterpret_cast<unsigned long long*>(ws + w.rec_off);
+    recs.tok = recs.cta + (size_t)2 * B * kPMaxG * 2;
+    if (gemv_path(r, B) &&
+        cudaMemsetAsync(ws + w.rec_off, 0, gemv_rec_bytes(B), s) != cudaSuccess)
+      return DSPARK_ERR_CUDA;
+    dspark_status st = persist_launch(tm_w, a, recs, s);
     if (st != DSPARK_OK) return st;
     return check_launch();
   }
@@ -269,7 +277,7 @@ const char* dspark_status_string(dspark_status s) {
 const char* dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype) {
   (void)K;
   if (use_persist(V, r, B, uw_dtype))
-    return B <= kSimtMaxB ? "persistent-cuda-core" : "tcgen05-persistent";
+    return gemv_path(r, B) ? "persistent-cuda-core" : "tcgen05-persistent";
   return use_tc(V, r, B, uw_dtype) ? "tcgen05" : "cuda-core";
 }
 

@@ -95,17 +95,24 @@ inline int persist_grid(int V) {
   return G;
 }
 
-// Up to this many requests the persistent draft runs its projection on the
-// CUDA cores; above it, on tcgen05 with N = 16.
-constexpr int kSimtMaxB = 4;
+// Up to this many requests (at r = 256) the persistent draft runs its
+// projection as a CUDA-core GEMV; above it, on tcgen05 with N = 16.
+constexpr int kSimtMaxB = 2;
+inline bool gemv_path(int r, int B) { return B <= kSimtMaxB && r == 256; }
 
 inline PersistLayout persist_layout(int V, int r, int B) {
   PersistLayout L;
   const int n_tiles = (V + kTileN - 1) / kTileN;
   L.G = persist_grid(V);
   L.max_nt = (n_tiles + L.G - 1) / L.G;
-  L.u_bytes = B <= kSimtMaxB ? (size_t)B * r * 4 : (size_t)(r / 64) * 2048;
-  L.base_bytes = (((size_t)B * L.max_nt * kTileN * 4) + 1023) & ~size_t(1023);
+  if (gemv_path(r, B)) {
+    // sBias [B][rows] + sBase [2][B][rows] + sPart [B][max_nt*4]
+    L.u_bytes = 0;
+    L.base_bytes = (size_t)3 * B * L.max_nt * kTileN * 4 + (size_t)B * L.max_nt * 4 * 8 + 16;
+  } else {
+    L.u_bytes = (size_t)(r / 64) * 2048;
+    L.base_bytes = (((size_t)B * L.max_nt * kTileN * 4) + 1023) & ~size_t(1023);
+  }
   const size_t fixed = 1024 /*align*/ + L.u_bytes + L.base_bytes + 2048 /*barriers, scratch*/;
   L.n_stages = fixed >= (size_t)kPSmemLimit ? 0 : (int)((kPSmemLimit - fixed) / kStageBytes);
   if (L.n_stages > kPMaxStages) L.n_stages = kPMaxStages;
@@ -615,79 +622,122 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
 }
 
 // ---------------------------------------------------------------------------
-// CUDA-core variant for the smallest batches
+// GEMV variant for one or two requests (r = 256)
 // ---------------------------------------------------------------------------
 //
-// At N = 16 a tcgen05 MMA instruction costs about as much as at several
-// times the width, so for one to a few requests the projection is a GEMV
-// on the CUDA cores (the thread owns one vocabulary row and accumulates the
-// row's dot product with U[x_{k-1}] in fp32, ascending index order).  The
-// memory plan stays the same: four W tiles per SM resident in TMEM for the
-// whole call (read back with tcgen05.ld, 38 MB of W on chip across the
-// GPU), the rest streamed from L2 through the TMA ring into shared memory,
-// base rows bulk-copied one position ahead.  Eight compute warps: tile i
-// belongs to warp group (i & 1); the warp with TMEM lane quarter q owns
-// rows 32q..32q+31 of the tile, i.e. one 32-row softmax chunk.
-constexpr int kSThreads = 384;
-constexpr int kSCompWarp0 = 4;
-constexpr int kSCompThreads = 256;
-constexpr int kSMaxTmemTiles = 4;
+// An N = 16 tcgen05 MMA costs about as much as a much wider one, so for one
+// or two requests the projection is a GEMV on the CUDA cores.  It is laid
+// out "transposed": lane l of a warp owns the K slice [8l, 8l+8) of every
+// row, so the previous-token vector U[x] stays in eight registers per
+// request, each lane accumulates the dot products of 32 rows at once, and
+// a 31-shuffle butterfly hands lane l the finished bias of row l.  Memory
+// plan: four W tiles per SM resident in TMEM for the whole call, stored in
+// the same transposed order (lane = K slice, four 32-bit columns = 8 bf16
+// per row) and read back with tcgen05.ld; the rest streams through the TMA
+// ring; base rows are bulk-copied one position ahead (double-buffered).
+//
+// No grid barrier: after its tiles each CTA publishes its softmax partial
+// as self-validating 8-byte {value, sequence} records; every CTA polls all
+// records of the position (one round trip once the last one lands), finds
+// the CTA whose range holds the sample, and only that CTA resolves the
+// chunk and the token from its own shared memory (chunk partials, bias and
+// base values of its rows).  It writes the outputs and publishes U[x] as
+// sequence-tagged records, which every CTA polls straight into its
+// registers for the next position.  Records are double-buffered by
+// position parity; a CTA can only overwrite a parity after every CTA has
+// consumed it (it needs everyone's next records first).
+constexpr int kGThreads = 384;
+constexpr int kGCompWarp0 = 4;
+constexpr int kGCompThreads = 256;
+constexpr int kGMaxB = 2;
+constexpr int kGRank = 256;
+constexpr int kGMaxTmemTiles = 4;
+constexpr int kTokRec = kGRank + 1;  // U row values + the token id
 
-__device__ __forceinline__ void comp_sync() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kSCompThreads) : "memory");
+__device__ __forceinline__ void gemv_sync() {
+  asm volatile("bar.sync 1, %0;" ::"r"(kGCompThreads) : "memory");
+}
+__device__ __forceinline__ void st_rec(unsigned long long* p, uint32_t lo, uint32_t seq) {
+  const unsigned long long v = ((unsigned long long)seq << 32) | lo;
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_rec(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
 }
 
-// acc[b] += sum_e w_e * u_b[e0 + e] over the 8 bf16 values packed in q
+// lane l receives sum over lanes of v[l] (butterfly transpose-reduce)
+__device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool upper = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < o; ++i) {
+      const float send = upper ? v[i] : v[i + o];
+      const float keep = upper ? v[i + o] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+// pr[b][row] += sum_{e<8} w_e * u[b][e] over the 8 bf16 packed in q
 template <int NB>
-__device__ __forceinline__ void fma8(uint4 q, const float* __restrict__ u_s, int r, int e0, int B,
-                                     float (&acc)[NB]) {
-  float w[8];
-  w[0] = __uint_as_float(q.x << 16); w[1] = __uint_as_float(q.x & 0xffff0000u);
-  w[2] = __uint_as_float(q.y << 16); w[3] = __uint_as_float(q.y & 0xffff0000u);
-  w[4] = __uint_as_float(q.z << 16); w[5] = __uint_as_float(q.z & 0xffff0000u);
-  w[6] = __uint_as_float(q.w << 16); w[7] = __uint_as_float(q.w & 0xffff0000u);
+__device__ __forceinline__ void gemv8(uint4 q, const float (&u)[NB][8], int B, float (&pr)[NB][32],
+                                      int row) {
+  const float w0 = __uint_as_float(q.x << 16), w1 = __uint_as_float(q.x & 0xffff0000u);
+  const float w2 = __uint_as_float(q.y << 16), w3 = __uint_as_float(q.y & 0xffff0000u);
+  const float w4 = __uint_as_float(q.z << 16), w5 = __uint_as_float(q.z & 0xffff0000u);
+  const float w6 = __uint_as_float(q.w << 16), w7 = __uint_as_float(q.w & 0xffff0000u);
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     if (b >= B) break;
-    const float4 ua = *reinterpret_cast<const float4*>(u_s + b * r + e0);
-    const float4 ub = *reinterpret_cast<const float4*>(u_s + b * r + e0 + 4);
-    float a = acc[b];
-    a = fmaf(w[0], ua.x, a); a = fmaf(w[1], ua.y, a);
-    a = fmaf(w[2], ua.z, a); a = fmaf(w[3], ua.w, a);
-    a = fmaf(w[4], ub.x, a); a = fmaf(w[5], ub.y, a);
-    a = fmaf(w[6], ub.z, a); a = fmaf(w[7], ub.w, a);
-    acc[b] = a;
+    float a = pr[b][row];
+    a = fmaf(w0, u[b][0], a); a = fmaf(w1, u[b][1], a);
+    a = fmaf(w2, u[b][2], a); a = fmaf(w3, u[b][3], a);
+    a = fmaf(w4, u[b][4], a); a = fmaf(w5, u[b][5], a);
+    a = fmaf(w6, u[b][6], a); a = fmaf(w7, u[b][7], a);
+    pr[b][row] = a;
   }
 }
 
+struct GemvRecs {
+  unsigned long long* cta;  // [2][B][G][2]: {M, seq}, {S, seq}
+  unsigned long long* tok;  // [2][B][kTokRec]: U row values, then the token id
+};
+
 template <int NB>
-__global__ void __launch_bounds__(kSThreads, 1)
-draft_persist_simt_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p) {
+__global__ void __launch_bounds__(kGThreads, 1)
+draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p, const GemvRecs rec) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int nkb = p.r >> 6;
+  constexpr int nkb = kGRank / 64;
   const int G = gridDim.x, cta = blockIdx.x;
   const int t0 = p_tile_begin(cta, G, p.n_tiles), t1 = p_tile_begin(cta + 1, G, p.n_tiles);
   const int nt = t1 - t0;
-  const int B = p.B, K = p.K, V = p.V, r = p.r;
+  const int B = p.B, K = p.K, V = p.V;
   const int S = p.n_stages;
-  const int base_stride = p.max_nt * kTileN;
-  const int nres = min(nt, kSMaxTmemTiles);
+  const int rows_cap = p.max_nt * kTileN;  // row slots per request in sBias / sBase
+  const int nres = min(nt, kGMaxTmemTiles);
   const int nstream = nt - nres;
+  const int nrows = min(nt * kTileN, V - t0 * kTileN);   // valid rows of this CTA
+  const int nloc = (nrows + kChunk - 1) / kChunk;        // chunks of this CTA
 
   uint8_t* sRing = sm;
-  float* u_s = reinterpret_cast<float*>(sRing + S * kStageBytes);  // [B][r] fp32
-  float* sBase = u_s + (size_t)B * r;
-  uint8_t* misc = reinterpret_cast<uint8_t*>(sBase) +
-                  ((((size_t)B * base_stride * 4) + 1023) & ~size_t(1023));
+  float* sBias = reinterpret_cast<float*>(sRing + S * kStageBytes);  // [B][rows_cap]
+  float* sBase = sBias + (size_t)B * rows_cap;                       // [2][B][rows_cap]
+  float2* sPart = reinterpret_cast<float2*>(sBase + (size_t)2 * B * rows_cap);  // [B][max_nt*4]
+  uint8_t* misc = reinterpret_cast<uint8_t*>(sPart + (size_t)B * p.max_nt * 4);
+  misc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(misc) + 15) & ~uintptr_t(15));
   uint64_t* ringFull = reinterpret_cast<uint64_t*>(misc);
   uint64_t* ringEmpty = ringFull + kPMaxStages;
-  uint64_t* baseFull = ringEmpty + kPMaxStages;
-  uint64_t* baseEmpty = baseFull + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(baseEmpty + 1);
+  uint64_t* baseFull = ringEmpty + kPMaxStages;  // [2]
+  uint64_t* baseEmpty = baseFull + 2;            // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(baseEmpty + 2);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [8][kPMaxB]
-  float* s_ws = s_wm + 8 * kPMaxB;                        // [8][kPMaxB]
+  float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [8][kGMaxB]
+  float* s_ws = s_wm + 8 * kGMaxB;                        // [8][kGMaxB]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -696,8 +746,10 @@ draft_persist_simt_kernel(const __grid_constant__ CUtensorMap tm_w, const Persis
       mbar_init(&ringFull[i], 1);
       mbar_init(&ringEmpty[i], 4);
     }
-    mbar_init(baseFull, 1);
-    mbar_init(baseEmpty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&baseFull[i], 1);
+      mbar_init(&baseEmpty[i], 1);
+    }
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -729,125 +781,140 @@ draft_persist_simt_kernel(const __grid_constant__ CUtensorMap tm_w, const Persis
       }
     }
   } else if (warp == 2) {
-    // ------------------------------------------------ base producer
+    // ------------------------------------------------ base producer (double-buffered)
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       const int v0 = t0 * kTileN;
-      const uint32_t bytes = (uint32_t)min(nt * kTileN, V - v0) * 4u;
+      const uint32_t bytes = (uint32_t)nrows * 4u;
       for (int k = 0; k < K && !*s_abort; ++k) {
-        if (!mbar_wait(baseEmpty, ((uint32_t)k & 1u) ^ 1u)) {
+        const int buf = k & 1;
+        if (!mbar_wait(&baseEmpty[buf], ((uint32_t)(k >> 1) & 1u) ^ 1u)) {
           *s_abort = 1;
           raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
           break;
         }
-        mbar_arrive_expect_tx(baseFull, bytes * (uint32_t)B);
+        mbar_arrive_expect_tx(&baseFull[buf], bytes * (uint32_t)B);
         for (int b = 0; b < B; ++b)
-          bulk_load(sBase + (size_t)b * base_stride, p.base + ((size_t)b * K + k) * (size_t)V + v0,
-                    bytes, baseFull, pol);
+          bulk_load(sBase + ((size_t)buf * B + b) * rows_cap,
+                    p.base + ((size_t)b * K + k) * (size_t)V + v0, bytes, &baseFull[buf], pol);
       }
     }
-  } else if (warp >= kSCompWarp0) {
-    // ------------------------------------------------ compute + epilogue + sampler
-    const int ct = threadIdx.x - kSCompWarp0 * 32;  // 0..255
-    const int cw = warp - kSCompWarp0;              // 0..7
-    const int half = cw >> 2;                       // tile parity owned by this warp
-    const int quarter = warp & 3;                   // TMEM lane quarter
-    const int m = quarter * 32 + lane;              // row within a tile
+  } else if (warp >= kGCompWarp0) {
+    // ------------------------------------------------ GEMV, epilogue, sampling
+    const int cw = warp - kGCompWarp0;  // 0..7
+    const int half = cw >> 2;           // tile parity owned by this warp
+    const int quarter = warp & 3;       // TMEM lane quarter = rows 32q..32q+31 of a tile
+    const int kb_l = lane >> 3, j8 = lane & 7;  // this lane's K slice: k-block, 16-byte chunk
     float it2[NB], itv[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
       itv[b] = (b < B) ? checked_inv_temp(p.inv_temp, b, p.flags) : 1.0f;
       it2[b] = itv[b] * kLog2e;
     }
-    // resident W tiles -> TMEM (rows of this warp's quarter, tiles of its half)
+    // resident tiles -> TMEM in transposed order
     for (int i = half; i < nres; i += 2) {
-      const int v = (t0 + i) * kTileN + m;
-      const uint4* src = reinterpret_cast<const uint4*>(p.W + (size_t)(v < V ? v : 0) * r);
-      for (int g = 0; g < nkb; ++g) {
+      for (int cb = 0; cb < 4; ++cb) {
         uint32_t regs[32];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const uint4 val = (v < V) ? __ldg(src + g * 8 + q) : make_uint4(0, 0, 0, 0);
-          regs[4 * q] = val.x;
-          regs[4 * q + 1] = val.y;
-          regs[4 * q + 2] = val.z;
-          regs[4 * q + 3] = val.w;
+        for (int j = 0; j < 8; ++j) {
+          const int row = (t0 + i) * kTileN + quarter * 32 + cb * 8 + j;
+          const uint4 val = (row < V) ? __ldg(reinterpret_cast<const uint4*>(p.W + (size_t)row * kGRank) + lane)
+                                      : make_uint4(0, 0, 0, 0);
+          regs[4 * j] = val.x;
+          regs[4 * j + 1] = val.y;
+          regs[4 * j + 2] = val.z;
+          regs[4 * j + 3] = val.w;
         }
-        tmem_st32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + g * 32), regs);
+        tmem_st32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + cb * 32), regs);
       }
     }
     tmem_st_wait();
-    // operand of position 1: U[prev_token] as fp32
-    for (int b = cw; b < B; b += 8) {
-      const int x = checked_token(p.prev_token[b], V, true, p.flags);
-      for (int e = lane; e < r; e += 32) u_s[b * r + e] = (x >= 0) ? to_f32(p.U[(size_t)x * r + e]) : 0.0f;
+    // U[prev_token] slice of this lane
+    float u[NB][8];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int x = (b < B) ? checked_token(p.prev_token[b], V, true, p.flags) : -1;
+      uint4 val = make_uint4(0, 0, 0, 0);
+      if (x >= 0) val = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)x * kGRank) + lane);
+      u[b][0] = __uint_as_float(val.x << 16); u[b][1] = __uint_as_float(val.x & 0xffff0000u);
+      u[b][2] = __uint_as_float(val.y << 16); u[b][3] = __uint_as_float(val.y & 0xffff0000u);
+      u[b][4] = __uint_as_float(val.z << 16); u[b][5] = __uint_as_float(val.z & 0xffff0000u);
+      u[b][6] = __uint_as_float(val.w << 16); u[b][7] = __uint_as_float(val.w & 0xffff0000u);
     }
     tc_fence_before();
-    comp_sync();
+    gemv_sync();
     tc_fence_after();
 
-    for (int k = 0; k < K; ++k) {
+    for (int k = 0; k < K && !*s_abort; ++k) {
+      const int buf = k & 1, par = k & 1;
+      const uint32_t seq = (uint32_t)k + 1u;
+      const float* bse = sBase + (size_t)buf * B * rows_cap;
       float wm[NB], ws[NB];
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         wm[b] = -CUDART_INF_F;
         ws[b] = 0.0f;
       }
-      bool ok = mbar_wait_spin(baseFull, (uint32_t)k & 1u);
+      bool ok = mbar_wait_spin(&baseFull[buf], (uint32_t)(k >> 1) & 1u);
       for (int i = half; i < nt; i += 2) {
-        float acc[NB];
+        float pr[NB][32];
 #pragma unroll
-        for (int b = 0; b < NB; ++b) acc[b] = 0.0f;
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pr[b][j] = 0.0f;
         if (i < nres) {
-          for (int g = 0; g < nkb; ++g) {
-            float wf[32];
-            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + g * 32), wf);
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-              const uint4 pk = make_uint4(__float_as_uint(wf[4 * q]), __float_as_uint(wf[4 * q + 1]),
-                                          __float_as_uint(wf[4 * q + 2]), __float_as_uint(wf[4 * q + 3]));
-              fma8<NB>(pk, u_s, r, g * 64 + q * 8, B, acc);
+          for (int cb = 0; cb < 4; ++cb) {
+            float wf[32];
+            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + cb * 32), wf);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const uint4 q = make_uint4(__float_as_uint(wf[4 * j]), __float_as_uint(wf[4 * j + 1]),
+                                         __float_as_uint(wf[4 * j + 2]), __float_as_uint(wf[4 * j + 3]));
+              gemv8<NB>(q, u, B, pr, cb * 8 + j);
             }
           }
         } else {
           const int itb = (k * nstream + (i - nres)) * nkb;
           for (int kb = 0; kb < nkb; ++kb) {
-            const int it = itb + kb, s = it % S;
-            ok = ok && mbar_wait_spin(&ringFull[s], (uint32_t)(it / S) & 1u);
-            const uint8_t* rowp = sRing + s * kStageBytes + m * 128;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint4 pk = *reinterpret_cast<const uint4*>(rowp + ((j ^ (m & 7)) << 4));
-              fma8<NB>(pk, u_s, r, kb * 64 + j * 8, B, acc);
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ringEmpty[s]);
+            const int it = itb + kb;
+            ok = ok && mbar_wait_spin(&ringFull[it % S], (uint32_t)(it / S) & 1u);
           }
+          const uint8_t* stg = sRing + ((itb + kb_l) % S) * kStageBytes;
+#pragma unroll
+          for (int rr = 0; rr < 32; ++rr) {
+            const int m = quarter * 32 + rr;
+            const uint4 q = *reinterpret_cast<const uint4*>(stg + m * 128 + ((j8 ^ (m & 7)) << 4));
+            gemv8<NB>(q, u, B, pr, rr);
+          }
+          __syncwarp();
+          if (lane == 0)
+            for (int kb = 0; kb < nkb; ++kb) mbar_arrive(&ringEmpty[(itb + kb) % S]);
         }
         if (!ok) {
           *s_abort = 1;
           raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
         }
-        const int vl = i * kTileN + m;
+        const int vl = i * kTileN + quarter * 32 + lane;  // row within the CTA range
         const int v = t0 * kTileN + vl;
         const bool valid = v < V;
-        const int chunk = v >> 5;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           if (b >= B) break;
-          const size_t row = ((size_t)b * K + k) * (size_t)V;
-          const float bv = valid ? sBase[(size_t)b * base_stride + vl] : 0.0f;
-          const float a = valid ? bv + acc[b] : -CUDART_INF_F;
+          const float bias = transpose_reduce32(pr[b], lane);
+          const float bv = valid ? bse[(size_t)b * rows_cap + vl] : 0.0f;
+          const float a = valid ? bv + bias : -CUDART_INF_F;
           const float A = warp_max(a);
-          const float e = valid ? ex2(((bv - A) + acc[b]) * it2[b]) : 0.0f;
+          const float e = valid ? ex2(((bv - A) + bias) * it2[b]) : 0.0f;
           const float sm2 = warp_sum(e);
+          sBias[(size_t)b * rows_cap + vl] = bias;
           if (valid) {
-            if (p.draft_bias != nullptr) p.draft_bias[row + v] = acc[b];
-            else p.bias_buf[(size_t)b * V + v] = acc[b];
+            const size_t row = ((size_t)b * K + k) * (size_t)V;
+            if (p.draft_bias != nullptr) p.draft_bias[row + v] = bias;
             if (p.draft_logits != nullptr) p.draft_logits[row + v] = a * itv[b];
           }
-          if (lane == 0 && chunk < p.n_chunks) {
-            p.part[(size_t)b * p.n_chunks + chunk] = make_float2(A, sm2);
+          if (lane == 0) {
+            sPart[(size_t)b * p.max_nt * 4 + i * 4 + quarter] = make_float2(A, sm2);
             merge_partial(wm[b], ws[b], A, sm2, it2[b]);
           }
         }
@@ -855,29 +922,182 @@ draft_persist_simt_kernel(const __grid_constant__ CUtensorMap tm_w, const Persis
       if (lane == 0) {
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          s_wm[cw * kPMaxB + b] = wm[b];
-          s_ws[cw * kPMaxB + b] = ws[b];
+          s_wm[cw * kGMaxB + b] = wm[b];
+          s_ws[cw * kGMaxB + b] = ws[b];
         }
       }
-      comp_sync();
-      if (ct == 0) mbar_arrive(baseEmpty);  // sBase may take the next position
-      if (ct < B) {
-        const int b = ct;
+      gemv_sync();
+      // publish this CTA's partial of every request
+      if (cw == 0 && lane < B) {
+        const int b = lane;
         float M = -CUDART_INF_F, Sm = 0.0f;
         for (int w2 = 0; w2 < 8; ++w2)
-          merge_partial(M, Sm, s_wm[w2 * kPMaxB + b], s_ws[w2 * kPMaxB + b], it2[b]);
-        p.cta_part[(size_t)b * G + cta] = make_float2(M, Sm);
+          merge_partial(M, Sm, s_wm[w2 * kGMaxB + b], s_ws[w2 * kGMaxB + b], it2[b]);
+        unsigned long long* r0 = rec.cta + (((size_t)par * B + b) * G + cta) * 2;
+        st_rec(r0, __float_as_uint(M), seq);
+        st_rec(r0 + 1, __float_as_uint(Sm), seq);
       }
-      comp_sync();
-      if (ct == 0 && !persist_grid_barrier(p.grid_counter, k, G, p.flags)) *s_abort = 1;
-      comp_sync();
-      if (*s_abort) break;
-      for (int b = cw; b < B; b += 8) {
-        const int x = persist_sample(p, b, k, G, cta, it2[b], itv[b]);
-        if (k + 1 < K)
-          for (int e = lane; e < r; e += 32) u_s[b * r + e] = to_f32(p.U[(size_t)x * r + e]);
+      // warp b: level 1 over all CTAs; the owning CTA resolves chunk and token
+      if (cw < B) {
+        const int b = cw;
+        const unsigned long long* cr = rec.cta + (((size_t)par * B + b) * G) * 2;
+        const int per = (G + 31) / 32;
+        const int c0 = min(lane * per, G), c1 = min(c0 + per, G);
+        float2 q[kPMaxG / 32];
+        const uint64_t tstart = global_timer_ns();
+        for (;;) {
+          bool mine = true;
+#pragma unroll
+          for (int i = 0; i < kPMaxG / 32; ++i) {
+            q[i] = make_float2(-CUDART_INF_F, 0.0f);
+            if (c0 + i < c1) {
+              const unsigned long long m0 = ld_rec(cr + 2 * (c0 + i));
+              const unsigned long long m1 = ld_rec(cr + 2 * (c0 + i) + 1);
+              if ((uint32_t)(m0 >> 32) != seq || (uint32_t)(m1 >> 32) != seq) mine = false;
+              q[i] = make_float2(__uint_as_float((uint32_t)m0), __uint_as_float((uint32_t)m1));
+            }
+          }
+          if (__all_sync(0xffffffffu, mine)) break;
+          if (global_timer_ns() - tstart > kWaitLimitNs) {
+            *s_abort = 1;
+            raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+            break;
+          }
+        }
+        float mx = -CUDART_INF_F;
+#pragma unroll
+        for (int i = 0; i < kPMaxG / 32; ++i) mx = fmaxf(mx, q[i].x);
+        const float M = warp_max(mx);
+        double wsum = 0.0;
+#pragma unroll
+        for (int i = 0; i < kPMaxG / 32; ++i) wsum += partial_weight(q[i], M, it2[b]);
+        const double incl = warp_incl_scan_d(wsum);
+        const double Z = __shfl_sync(0xffffffffu, incl, 31);
+        const double T = (double)p.u_draft[(size_t)b * K + k] * Z;
+        double start = __shfl_up_sync(0xffffffffu, incl, 1);
+        if (lane == 0) start = 0.0;
+        const unsigned own = __ballot_sync(0xffffffffu, start <= T && T < incl && wsum > 0.0);
+        int cstar, pick = -1, lastp = -1;
+        double before = start, lastb = start;
+        {
+          double cum = start;
+#pragma unroll
+          for (int i = 0; i < kPMaxG / 32; ++i) {
+            const double w = partial_weight(q[i], M, it2[b]);
+            if (pick < 0 && w > 0.0) {
+              lastp = c0 + i;
+              lastb = cum;
+              if (cum + w > T) {
+                pick = c0 + i;
+                before = cum;
+              }
+            }
+            cum += w;
+          }
+        }
+        if (pick < 0) {
+          pick = lastp;
+          before = lastb;
+        }
+        if (own) {
+          const int ol = __ffs(own) - 1;
+          cstar = __shfl_sync(0xffffffffu, pick, ol);
+          before = __shfl_sync(0xffffffffu, before, ol);
+        } else {  // no crossing (u*Z rounded to Z): last CTA with mass
+          const unsigned pos = __ballot_sync(0xffffffffu, lastp >= 0);
+          const int pl = pos ? 31 - __clz(pos) : 0;
+          cstar = __shfl_sync(0xffffffffu, lastp, pl);
+          if (cstar < 0) cstar = 0;
+          before = -CUDART_INF;
+        }
+        if (cstar == cta) {
+          // level 2: this CTA's chunk partials (shared memory), two per lane
+          const float2* lp = sPart + (size_t)b * p.max_nt * 4;
+          const int ca = 2 * lane, cb2 = ca + 1;
+          const double wA = (ca < nloc) ? partial_weight(lp[ca], M, it2[b]) : 0.0;
+          const double wB = (cb2 < nloc) ? partial_weight(lp[cb2], M, it2[b]) : 0.0;
+          const double pin = warp_incl_scan_d(wA + wB);
+          double lstart = __shfl_up_sync(0xffffffffu, pin, 1);
+          if (lane == 0) lstart = 0.0;
+          lstart += before;
+          const bool hitA = wA > 0.0 && lstart + wA > T;
+          const bool hitB = wB > 0.0 && lstart + wA + wB > T;
+          const unsigned h = __ballot_sync(0xffffffffu, hitA || hitB);
+          int chunk;
+          double before2;
+          if (h) {
+            const int hl = __ffs(h) - 1;
+            chunk = __shfl_sync(0xffffffffu, hitA ? ca : cb2, hl);
+            before2 = __shfl_sync(0xffffffffu, hitA ? lstart : lstart + wA, hl);
+          } else {
+            const unsigned hp = __ballot_sync(0xffffffffu, wA > 0.0 || wB > 0.0);
+            const int hl = hp ? 31 - __clz(hp) : 0;
+            chunk = __shfl_sync(0xffffffffu, (wB > 0.0) ? cb2 : ca, hl);
+            if (!hp) chunk = 0;
+            before2 = -CUDART_INF;
+          }
+          // level 3: the chunk's rows from shared memory
+          const int vl = chunk * kChunk + lane;
+          const int v = t0 * kTileN + vl;
+          const bool valid = v < V;
+          float ef = 0.0f;
+          if (valid)
+            ef = ex2(((bse[(size_t)b * rows_cap + vl] - M) + sBias[(size_t)b * rows_cap + vl]) * it2[b]);
+          const int pl = pick_lane((double)ef, before2, T);
+          const int x = __shfl_sync(0xffffffffu, valid ? v : 0, pl);
+          if (lane == pl) {
+            const size_t o = (size_t)b * K + k;
+            if (!(Z > 0.0) || !isfinite(Z)) {
+              raise_flag(p.flags, DSPARK_FLAG_NONFINITE);
+              p.tokens[o] = 0;
+              p.p_tok[o] = 0.0f;
+              p.lse[o] = CUDART_NAN_F;
+              p.ref_max[o] = M;
+              p.ref_sum[o] = 1.0f;
+            } else {
+              p.tokens[o] = x;
+              p.p_tok[o] = (float)((double)ef / Z);
+              p.lse[o] = (float)((double)M * (double)itv[b] + log(Z));
+              p.ref_max[o] = M;
+              p.ref_sum[o] = (float)Z;
+            }
+          }
+          // publish U[x] (one 16-byte slice per lane) and the token id
+          unsigned long long* tr = rec.tok + ((size_t)par * B + b) * kTokRec;
+          const uint4 val = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)x * kGRank) + lane);
+          const uint32_t w8[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            st_rec(tr + 8 * lane + 2 * e, w8[e] << 16, seq);
+            st_rec(tr + 8 * lane + 2 * e + 1, w8[e] & 0xffff0000u, seq);
+          }
+          if (lane == 0) st_rec(tr + kGRank, (uint32_t)x, seq);
+        }
       }
-      comp_sync();
+      // every compute warp: next position's U[x] slice from the records
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        if (b >= B) break;
+        const unsigned long long* tr = rec.tok + ((size_t)par * B + b) * kTokRec + 8 * lane;
+        const uint64_t tstart = global_timer_ns();
+        for (;;) {
+          bool mine = true;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const unsigned long long m = ld_rec(tr + e);
+            if ((uint32_t)(m >> 32) != seq) mine = false;
+            u[b][e] = __uint_as_float((uint32_t)m);
+          }
+          if (__all_sync(0xffffffffu, mine)) break;
+          if (global_timer_ns() - tstart > kWaitLimitNs || *s_abort) {
+            *s_abort = 1;
+            raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+            break;
+          }
+        }
+      }
+      gemv_sync();
+      if (cw == 0 && lane == 0) mbar_arrive(&baseEmpty[buf]);  // buffer free for position k+2
     }
   }
 
@@ -915,27 +1135,46 @@ inline dspark_status persist_launch_kernel(Kern kern, int threads, const CUtenso
   return cudaLaunchKernelEx(&cfg, kern, tm_w, a) == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
 }
 
-inline dspark_status persist_launch(const CUtensorMap& tm_w, PersistArgs a, cudaStream_t s) {
+inline dspark_status persist_launch(const CUtensorMap& tm_w, PersistArgs a, GemvRecs recs,
+                                    cudaStream_t s) {
   static bool attr = false;
   if (!attr) {
     cudaFuncSetAttribute(draft_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kPSmemLimit);
-    cudaFuncSetAttribute(draft_persist_simt_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(draft_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kPSmemLimit);
-    cudaFuncSetAttribute(draft_persist_simt_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kPSmemLimit);
-    cudaFuncSetAttribute(draft_persist_simt_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(draft_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kPSmemLimit);
     attr = true;
   }
   const PersistLayout L = persist_layout(a.V, a.r, a.B);
   a.max_nt = L.max_nt;
   a.n_stages = L.n_stages;
-  if (a.B == 1) return persist_launch_kernel(draft_persist_simt_kernel<1>, kSThreads, tm_w, a, L, s);
-  if (a.B == 2) return persist_launch_kernel(draft_persist_simt_kernel<2>, kSThreads, tm_w, a, L, s);
-  if (a.B <= kSimtMaxB)
-    return persist_launch_kernel(draft_persist_simt_kernel<4>, kSThreads, tm_w, a, L, s);
-  return persist_launch_kernel(draft_persist_kernel, kPThreads, tm_w, a, L, s);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(L.G);
+  cfg.dynamicSmemBytes = L.smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attrs[1];
+  attrs[0].id = cudaLaunchAttributeCooperative;
+  attrs[0].val.cooperative = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 1;
+  cudaError_t e;
+  if (gemv_path(a.r, a.B)) {
+    cfg.blockDim = dim3(kGThreads);
+    e = (a.B == 1) ? cudaLaunchKernelEx(&cfg, draft_gemv_kernel<1>, tm_w, a, recs)
+                   : cudaLaunchKernelEx(&cfg, draft_gemv_kernel<2>, tm_w, a, recs);
+  } else {
+    cfg.blockDim = dim3(kPThreads);
+    e = cudaLaunchKernelEx(&cfg, draft_persist_kernel, tm_w, a);
+  }
+  return e == cudaSuccess ? DSPARK_OK : DSPARK_ERR_CUDA;
+}
+
+// Bytes of the position records of the GEMV variant (zeroed by the caller
+// before each call): CTA partials [2][B][G][2] and token rows [2][B][r+1].
+inline size_t gemv_rec_bytes(int B) {
+  return (size_t)2 * B * kPMaxG * 2 * 8 + (size_t)2 * B * kTokRec * 8;
 }
 
 }  // namespace dspark

@@ -15,7 +15,8 @@
 //   warp 0       W producer (TMA, evict-last: W is re-read every position)
 //   warp 1       TMEM allocator + MMA issuer (one thread)
 //   warp 2       base-logit producer (TMA 3-D boxes, evict-first)   [draft]
-//   warps 3..6   epilogue (128 threads = 128 requests)
+//   warps 3..10  epilogue: two warpgroups of 128 threads (= 128 requests),
+//                each taking half of every tile's 32-column chunks
 //
 // Draft mode streams base[b, k, v0:v0+32] boxes through a second TMA ring.
 // Residual mode reads the per-request rows base[b, j_b, :] and
@@ -30,7 +31,7 @@
 
 namespace dspark {
 
-constexpr int kTcThreads = 224;
+constexpr int kTcThreads = 352;
 constexpr int kBlockM = 128;
 constexpr int kTileN = 128;
 constexpr int kWStages = 4;
@@ -99,7 +100,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accFull[i], 1);
-      mbar_init(&accEmpty[i], 4);
+      mbar_init(&accEmpty[i], 8);
     }
     *s_abort = 0;
     fence_barrier_init();
@@ -216,6 +217,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
   } else {
     // ---------------- epilogue: thread = request (TMEM lane)
+    const int eg = (warp - 3) >> 2;  // warpgroup: chunks 2*eg, 2*eg+1 of every tile
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
     const int b = bb * kBlockM + m;
@@ -225,7 +227,6 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     ResInfo ri{};
     if (kRes && bval) ri = info[b];
     const uint64_t pol = policy_evict_first();
-    int itB = 0;
     for (int t = t0; t < t1; ++t) {
       const int a = (t - t0) & 1;
       const uint32_t aph = (uint32_t)((t - t0) >> 1) & 1u;
@@ -235,16 +236,17 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         break;
       }
       tc_fence_after();
-      float2 pp[kTileN / 32];
+      float2 pp[2];
 #pragma unroll 1
-      for (int cb = 0; cb < kTileN / 32; ++cb) {
+      for (int ci = 0; ci < 2; ++ci) {
+        const int cb = 2 * eg + ci;
         float d[32], bv[32];
         tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
         const int v0 = t * kTileN + cb * 32;
         if (!kRes) {
+          const int itB = (t - t0) * (kTileN / 32) + cb;
           const int s = itB % kBStages;
           const uint32_t ph = (uint32_t)(itB / kBStages) & 1u;
-          ++itB;
           if (!mbar_wait(&fullB[s], ph)) {
             *s_abort = 1;
             raise_flag(flags, DSPARK_FLAG_TIMEOUT);
@@ -265,7 +267,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 #pragma unroll
           for (int j = 0; j < 32; ++j)
             if (v0 + j < V) sum += ex2(((bv[j] - A) + d[j]) * it2);
-          pp[cb] = make_float2(A, sum);
+          pp[ci] = make_float2(A, sum);
           if (draft_bias != nullptr && bval) {
             float* dst = draft_bias + ((size_t)b * K + k) * (size_t)V + v0;
 #pragma unroll
@@ -309,17 +311,21 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
               }
             }
           }
-          pp[cb] = make_float2(qs, ps);
+          pp[ci] = make_float2(qs, ps);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accEmpty[a]);
       if (bval) {
-        float2* dst = part + (size_t)b * n_chunks + t * (kTileN / 32);
-#pragma unroll
-        for (int cb = 0; cb < kTileN / 32; ++cb)
-          if (t * (kTileN / 32) + cb < n_chunks) dst[cb] = pp[cb];
+        const int c0 = t * (kTileN / 32) + 2 * eg;
+        float2* dst = part + (size_t)b * n_chunks + c0;
+        if (c0 + 1 < n_chunks) {
+          dst[0] = pp[0];
+          dst[1] = pp[1];
+        } else if (c0 < n_chunks) {
+          dst[0] = pp[0];
+        }
       }
     }
   }

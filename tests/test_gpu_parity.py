@@ -71,14 +71,15 @@ def test_tensor_core_path(oracle_mod, V, r, B, K):
 @pytest.mark.parametrize("V,r,B,K,keep", [(4096, 64, 3, 5, True), (1000, 128, 1, 4, False),
                                           (20000, 256, 16, 6, True), (151936, 256, 2, 3, False),
                                           (8192, 192, 9, 16, False), (40000, 256, 4, 7, True),
-                                          (30000, 128, 5, 5, True), (151936, 256, 1, 5, True)])
+                                          (30000, 128, 5, 5, True), (151936, 256, 1, 5, True),
+                                          (9000, 256, 2, 9, False), (300, 256, 1, 3, True)])
 def test_persistent_draft(oracle_mod, V, r, B, K, keep):
     """B <= 16 with bf16 U/W: all K positions in one persistent launch
     (resident + streamed W tiles, grid barrier, redundant sampler); the
     verify either reuses the draft's bias rows or re-projects."""
     w = WL.get("stress", V=V, r=r, B=B, K=K, seed=7 * V + B)
     assert D.dspark_draft_path(V, r, B, K, D.DSPARK_BF16) == (
-        "persistent-cuda-core" if B <= 4 else "tcgen05-persistent")
+        "persistent-cuda-core" if B <= 2 and r == 256 else "tcgen05-persistent")
     inp = WL.make_inputs(w, device="cuda")
     inp["prev_token"][0] = -1
     rep, step, _ = _run(w, oracle=oracle_mod, inp=inp, keep_bias=keep)

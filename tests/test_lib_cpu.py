@@ -47,7 +47,9 @@ def test_status_strings_and_paths(lib):
         assert D.status_string(code)
     assert D.dspark_version() >= 100
     assert D.dspark_draft_path(151936, 256, 1, 16, D.DSPARK_BF16) == "persistent-cuda-core"
-    assert D.dspark_draft_path(151936, 256, 4, 16, D.DSPARK_BF16) == "persistent-cuda-core"
+    assert D.dspark_draft_path(151936, 256, 2, 16, D.DSPARK_BF16) == "persistent-cuda-core"
+    assert D.dspark_draft_path(151936, 128, 1, 16, D.DSPARK_BF16) == "tcgen05-persistent"
+    assert D.dspark_draft_path(151936, 256, 4, 16, D.DSPARK_BF16) == "tcgen05-persistent"
     assert D.dspark_draft_path(151936, 256, 5, 16, D.DSPARK_BF16) == "tcgen05-persistent"
     assert D.dspark_draft_path(151936, 256, 16, 16, D.DSPARK_BF16) == "tcgen05-persistent"
     assert D.dspark_draft_path(1024, 16, 2, 4, D.DSPARK_F32) == "cuda-core"
