@@ -636,23 +636,23 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
 // per row) and read back with tcgen05.ld; the rest streams through the TMA
 // ring; base rows are bulk-copied one position ahead (double-buffered).
 //
-// No grid barrier: after its tiles each CTA publishes its softmax partial
-// as self-validating 8-byte {value, sequence} records; every CTA polls all
-// records of the position (one round trip once the last one lands), finds
-// the CTA whose range holds the sample, and only that CTA resolves the
-// chunk and the token from its own shared memory (chunk partials, bias and
-// base values of its rows).  It writes the outputs and publishes U[x] as
-// sequence-tagged records, which every CTA polls straight into its
-// registers for the next position.  Records are double-buffered by
-// position parity; a CTA can only overwrite a parity after every CTA has
-// consumed it (it needs everyone's next records first).
+// One round of global exchange per position: after its tiles each CTA
+// stores its softmax partial and adds to an arrival counter with release
+// semantics; one thread per CTA polls the counter (relaxed loads with a
+// short back-off, so 148 CTAs do not flood one L2 line); then one warp
+// reads all CTA partials, finds the CTA whose range holds the sample, and
+// only that CTA resolves the chunk and the token from its own shared
+// memory (chunk partials, bias and base values of its rows).  It writes the
+// outputs and publishes {position, token} as one 8-byte word; one thread
+// per CTA polls that word and every warp then loads its slice of U[x] for
+// the next position.  The partials are double-buffered by position parity:
+// a CTA can only reach position k+2 after every CTA has finished k.
 constexpr int kGThreads = 384;
 constexpr int kGCompWarp0 = 4;
 constexpr int kGCompThreads = 256;
 constexpr int kGMaxB = 2;
 constexpr int kGRank = 256;
 constexpr int kGMaxTmemTiles = 4;
-constexpr int kTokRec = kGRank + 1;  // U row values + the token id
 
 __device__ __forceinline__ void gemv_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(kGCompThreads) : "memory");
@@ -704,8 +704,27 @@ __device__ __forceinline__ void gemv8(uint4 q, const float (&u)[NB][8], int B, f
 
 struct GemvRecs {
   unsigned long long* cta;  // [2][B][G][2]: {M, seq}, {S, seq}
-  unsigned long long* tok;  // [2][B][kTokRec]: U row values, then the token id
+  unsigned long long* tok;  // [B]: {position + 1, token}
+  unsigned* counter;        // arrival counter (zeroed per call)
 };
+
+__device__ __forceinline__ void backoff_spin_u64(const unsigned long long* p, uint32_t seq,
+                                                 unsigned long long* out, bool* timed_out) {
+  const uint64_t tstart = global_timer_ns();
+  for (;;) {
+    const unsigned long long v = ld_rec(p);
+    if ((uint32_t)(v >> 32) == seq) {
+      *out = v;
+      return;
+    }
+    if (global_timer_ns() - tstart > kWaitLimitNs) {
+      *timed_out = true;
+      *out = 0;
+      return;
+    }
+    __nanosleep(32);
+  }
+}
 
 template <int NB>
 __global__ void __launch_bounds__(kGThreads, 1)
@@ -738,6 +757,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [8][kGMaxB]
   float* s_ws = s_wm + 8 * kGMaxB;                        // [8][kGMaxB]
+  volatile int* s_i = reinterpret_cast<volatile int*>(s_ws + 8 * kGMaxB);  // [4]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -937,6 +957,28 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         st_rec(r0, __float_as_uint(M), seq);
         st_rec(r0 + 1, __float_as_uint(Sm), seq);
       }
+      if (cw == 0) {
+        __syncwarp();
+        if (lane == 0) {
+          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(rec.counter) : "memory");
+          const unsigned target = (unsigned)(k + 1) * (unsigned)G;
+          const uint64_t tstart = global_timer_ns();
+          for (;;) {
+            unsigned seen;
+            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(rec.counter) : "memory");
+            if (seen >= target) break;
+            if (global_timer_ns() - tstart > kWaitLimitNs) {
+              *s_abort = 1;
+              raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+              break;
+            }
+            __nanosleep(20);
+          }
+          asm volatile("fence.acq_rel.gpu;" ::: "memory");
+          s_i[0] = 1;
+        }
+      }
+      gemv_sync();
       // warp b: level 1 over all CTAs; the owning CTA resolves chunk and token
       if (cw < B) {
         const int b = cw;
@@ -944,25 +986,20 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         const int per = (G + 31) / 32;
         const int c0 = min(lane * per, G), c1 = min(c0 + per, G);
         float2 q[kPMaxG / 32];
-        const uint64_t tstart = global_timer_ns();
-        for (;;) {
-          bool mine = true;
+        bool stale = false;
 #pragma unroll
-          for (int i = 0; i < kPMaxG / 32; ++i) {
-            q[i] = make_float2(-CUDART_INF_F, 0.0f);
-            if (c0 + i < c1) {
-              const unsigned long long m0 = ld_rec(cr + 2 * (c0 + i));
-              const unsigned long long m1 = ld_rec(cr + 2 * (c0 + i) + 1);
-              if ((uint32_t)(m0 >> 32) != seq || (uint32_t)(m1 >> 32) != seq) mine = false;
-              q[i] = make_float2(__uint_as_float((uint32_t)m0), __uint_as_float((uint32_t)m1));
-            }
+        for (int i = 0; i < kPMaxG / 32; ++i) {
+          q[i] = make_float2(-CUDART_INF_F, 0.0f);
+          if (c0 + i < c1) {
+            const unsigned long long m0 = ld_rec(cr + 2 * (c0 + i));
+            const unsigned long long m1 = ld_rec(cr + 2 * (c0 + i) + 1);
+            if ((uint32_t)(m0 >> 32) != seq || (uint32_t)(m1 >> 32) != seq) stale = true;
+            q[i] = make_float2(__uint_as_float((uint32_t)m0), __uint_as_float((uint32_t)m1));
           }
-          if (__all_sync(0xffffffffu, mine)) break;
-          if (global_timer_ns() - tstart > kWaitLimitNs) {
-            *s_abort = 1;
-            raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
-            break;
-          }
+        }
+        if (__any_sync(0xffffffffu, stale) && lane == 0) {
+          *s_abort = 1;  // the counter said every partial was in place
+          raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
         }
         float mx = -CUDART_INF_F;
 #pragma unroll
@@ -1062,38 +1099,31 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
               p.ref_sum[o] = (float)Z;
             }
           }
-          // publish U[x] (one 16-byte slice per lane) and the token id
-          unsigned long long* tr = rec.tok + ((size_t)par * B + b) * kTokRec;
-          const uint4 val = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)x * kGRank) + lane);
-          const uint32_t w8[4] = {val.x, val.y, val.z, val.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            st_rec(tr + 8 * lane + 2 * e, w8[e] << 16, seq);
-            st_rec(tr + 8 * lane + 2 * e + 1, w8[e] & 0xffff0000u, seq);
-          }
-          if (lane == 0) st_rec(tr + kGRank, (uint32_t)x, seq);
+          // publish {position, token}
+          if (lane == 0) st_rec(rec.tok + b, (uint32_t)x, seq);
         }
       }
-      // every compute warp: next position's U[x] slice from the records
+      // one thread per CTA waits for the tokens; every warp loads its U[x] slice
+      if (cw == 0 && lane < B) {
+        unsigned long long v;
+        bool to = false;
+        backoff_spin_u64(rec.tok + lane, seq, &v, &to);
+        if (to) {
+          *s_abort = 1;
+          raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+        }
+        s_i[1 + lane] = min(max((int)(uint32_t)v, 0), V - 1);
+      }
+      gemv_sync();
+      if (k + 1 < K) {
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        if (b >= B) break;
-        const unsigned long long* tr = rec.tok + ((size_t)par * B + b) * kTokRec + 8 * lane;
-        const uint64_t tstart = global_timer_ns();
-        for (;;) {
-          bool mine = true;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const unsigned long long m = ld_rec(tr + e);
-            if ((uint32_t)(m >> 32) != seq) mine = false;
-            u[b][e] = __uint_as_float((uint32_t)m);
-          }
-          if (__all_sync(0xffffffffu, mine)) break;
-          if (global_timer_ns() - tstart > kWaitLimitNs || *s_abort) {
-            *s_abort = 1;
-            raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
-            break;
-          }
+        for (int b = 0; b < NB; ++b) {
+          if (b >= B) break;
+          const uint4 val = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)s_i[1 + b] * kGRank) + lane);
+          u[b][0] = __uint_as_float(val.x << 16); u[b][1] = __uint_as_float(val.x & 0xffff0000u);
+          u[b][2] = __uint_as_float(val.y << 16); u[b][3] = __uint_as_float(val.y & 0xffff0000u);
+          u[b][4] = __uint_as_float(val.z << 16); u[b][5] = __uint_as_float(val.z & 0xffff0000u);
+          u[b][6] = __uint_as_float(val.w << 16); u[b][7] = __uint_as_float(val.w & 0xffff0000u);
         }
       }
       gemv_sync();
@@ -1172,9 +1202,9 @@ inline dspark_status persist_launch(const CUtensorMap& tm_w, PersistArgs a, Gemv
 }
 
 // Bytes of the position records of the GEMV variant (zeroed by the caller
-// before each call): CTA partials [2][B][G][2] and token rows [2][B][r+1].
+// before each call): CTA partials [2][B][G][2], token words [B], counter.
 inline size_t gemv_rec_bytes(int B) {
-  return (size_t)2 * B * kPMaxG * 2 * 8 + (size_t)2 * B * kTokRec * 8;
+  return (size_t)2 * B * kPMaxG * 2 * 8 + (size_t)B * 8 + 256;
 }
 
 }  // namespace dspark
