@@ -207,6 +207,46 @@ dspark_status dspark_verify(
     int32_t *out_tokens, int32_t *last_token, void *workspace, size_t ws_bytes,
     void *stream);
 
+/*
+ * dspark_verify without a workspace argument (the pages have no counterpart;
+ * this is a convenience of this library).
+ *
+ * Who needs it: callers that cannot call cudaMalloc -- code that runs while
+ * another component captures a CUDA graph in global capture mode (device
+ * allocation is illegal there), plugins whose host application owns every
+ * device allocation, runtimes with a fixed device-memory budget.  They still
+ * own and pass all inputs and outputs; only the scratch is provided here.
+ *
+ * Scratch: a fixed 2 MiB array inside the library image, held by every GPU
+ * that loads the library until the process exits.  Problems whose
+ * dspark_verify_workspace_size exceeds 2 MiB are rejected with
+ * DSPARK_ERR_UNSUPPORTED before anything is enqueued (at V = 151936 that
+ * is about B <= 50 requests; B <= 16, K <= 16 always fits).
+ *
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and caches it; make that
+ * first call before any stream capture.  The function allocates nothing
+ * (no cudaMalloc, no cudaFree, no allocating library call).
+ *
+ * Sharing: every call on a device uses the same array and leaves its
+ * contents behind; each call clears the part that must start at zero (the
+ * status word).  Calls whose kernels overlap on the GPU (different streams
+ * without ordering) race on the array and give wrong results; order them.
+ * Device-side data checks still clamp bad values, but their status word
+ * lives in the shared array and is not reported through this entry point.
+ *
+ * Arguments and results: exactly those of dspark_verify, minus workspace and
+ * ws_bytes.
+ */
+dspark_status dspark_verify_noalloc(
+    const float *target_logits, int64_t n_target_rows, const int64_t *row_start,
+    const int32_t *verify_len, const float *base_logits, const void *U,
+    const void *W, dspark_dtype uw_dtype, int V, int r, int B, int K,
+    const int32_t *prev_token, const float *inv_temp, const int32_t *tokens,
+    const float *p_tok, const float *ref_max, const float *ref_sum,
+    const float *draft_bias, const float *u_accept, const float *u_resample,
+    int32_t *n_accepted, int32_t *out_tokens, int32_t *last_token, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* status                                                                  */
 /* ---------------------------------------------------------------------- */

@@ -5,6 +5,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "prefix.cuh"
@@ -256,6 +257,38 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
   return check_launch();
 }
 
+// ---------------------------------------------------------------------------
+// Verify without a caller-provided workspace
+// ---------------------------------------------------------------------------
+// Scratch of dspark_verify_noalloc: a fixed array in the library image, so a
+// caller that cannot allocate device memory can still run the verify.  Every
+// GPU that loads the library holds these bytes until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(2) << 20;  // 2 MiB
+static __device__ __align__(256) unsigned char g_verify_scratch[kNoAllocScratchBytes];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch on the current device.  Host code may not
+// use the symbol itself (it names a host-side stand-in); the address comes
+// from cudaGetSymbolAddress, looked up once per device with that device
+// current and cached.
+dspark_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return DSPARK_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return DSPARK_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_verify_scratch) != cudaSuccess || p == nullptr)
+      return DSPARK_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return DSPARK_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -415,6 +448,29 @@ dspark_status dspark_get_device_status(const void* workspace, void* stream) {
   if (f & DSPARK_FLAG_TIMEOUT) return DSPARK_ERR_TIMEOUT;
   if (f) return DSPARK_ERR_DEVICE_DATA;
   return DSPARK_OK;
+}
+
+dspark_status dspark_verify_noalloc(const float* target_logits, int64_t n_target_rows,
+                                    const int64_t* row_start, const int32_t* verify_len,
+                                    const float* base_logits, const void* U, const void* W,
+                                    dspark_dtype uw_dtype, int V, int r, int B, int K,
+                                    const int32_t* prev_token, const float* inv_temp,
+                                    const int32_t* tokens, const float* p_tok,
+                                    const float* ref_max, const float* ref_sum,
+                                    const float* draft_bias, const float* u_accept,
+                                    const float* u_resample, int32_t* n_accepted,
+                                    int32_t* out_tokens, int32_t* last_token, void* stream) {
+  // sizes first: nothing below runs for a problem that does not fit
+  const dspark_status st0 = check_shapes(V, r, B, K, uw_dtype);
+  if (st0 != DSPARK_OK) return st0;
+  if (dspark_verify_workspace_size(V, r, B, K) > kNoAllocScratchBytes) return DSPARK_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  const dspark_status st = noalloc_scratch(&scratch);
+  if (st != DSPARK_OK) return st;
+  return dspark_verify(target_logits, n_target_rows, row_start, verify_len, base_logits, U, W,
+                       uw_dtype, V, r, B, K, prev_token, inv_temp, tokens, p_tok, ref_max, ref_sum,
+                       draft_bias, u_accept, u_resample, n_accepted, out_tokens, last_token, scratch,
+                       kNoAllocScratchBytes, stream);
 }
 
 }  // extern "C"

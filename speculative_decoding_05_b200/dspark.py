@@ -36,6 +36,7 @@ SYMBOLS = [
     "dspark_verify_workspace_size", "dspark_verify",
     "dspark_get_device_status", "dspark_get_device_flags",
     "dspark_status_string", "dspark_draft_path", "dspark_version",
+    "dspark_verify_noalloc",
 ]
 
 
@@ -70,6 +71,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.dspark_verify.argtypes = [P, L, P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P,
                                   P, P, P, S, P]
     lib.dspark_verify.restype = I
+    lib.dspark_verify_noalloc.argtypes = [P, L, P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P,
+                                          P, P, P, P, P, P]
+    lib.dspark_verify_noalloc.restype = I
     lib.dspark_confidence_prefix.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P, S, P]
     lib.dspark_confidence_prefix.restype = I
     lib.dspark_get_device_status.argtypes = [P, P]
@@ -181,6 +185,21 @@ def dspark_verify(target_logits, row_start, verify_len, base_logits, U, W, prev_
         _ptr(u_resample), _ptr(n_accepted), _ptr(out_tokens), _ptr(last_token),
         _ptr(workspace), workspace.numel(), _stream(stream))
     _check("dspark_verify", rc)
+
+
+def dspark_verify_noalloc(target_logits, row_start, verify_len, base_logits, U, W, prev_token,
+                          inv_temp, tokens, p_tok, ref_max, ref_sum, u_accept, u_resample,
+                          n_accepted, out_tokens, last_token=None, draft_bias=None, stream=None):
+    """dspark_verify with the library's built-in scratch (no workspace)."""
+    n_rows, V = target_logits.shape
+    B, K = tokens.shape
+    r = W.shape[1]
+    rc = load().dspark_verify_noalloc(
+        _ptr(target_logits), n_rows, _ptr(row_start), _ptr(verify_len), _ptr(base_logits),
+        _ptr(U), _ptr(W), _dtype_code(U), V, r, B, K, _ptr(prev_token), _ptr(inv_temp),
+        _ptr(tokens), _ptr(p_tok), _ptr(ref_max), _ptr(ref_sum), _ptr(draft_bias), _ptr(u_accept),
+        _ptr(u_resample), _ptr(n_accepted), _ptr(out_tokens), _ptr(last_token), _stream(stream))
+    _check("dspark_verify_noalloc", rc)
 
 
 def dspark_get_device_flags(workspace, stream=None) -> int:
