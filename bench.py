@@ -19,9 +19,8 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
-import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -68,58 +67,126 @@ def algorithmic(w, L):
                 verify_flops=verify_flops)
 
 
+# ------------------------------------------------------------ multi-rank --
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a per-rank value over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
+
+
+# ---------------------------------------------------------------- traffic --
+
+def source_digest() -> str:
+    """Hash of the CUDA sources: a stored DRAM-traffic figure is only valid
+    for the kernels it was measured on."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "speculative_decoding_05_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def kernel_name(path: str, call: str, w) -> str:
+    if call != "dspark_draft_markov":
+        return "dspark_verify kernels"
+    if path == "persistent-cuda-core":
+        return f"draft_gemv_kernel<{w.B}>"
+    if path == "tcgen05-persistent":
+        return "draft_persist_kernel"
+    if path == "tcgen05":
+        return "proj_tc_kernel<false> + draft_sample_kernel"
+    return "draft_proj_simt_kernel + draft_sample_kernel"
+
+
+def measured_traffic(kernel: str, workload: str):
+    """dram bytes (read + write) per launch from the committed ncu summary,
+    or None when absent or measured on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p)).get(f"{kernel}|{workload}")
+    except ValueError:
+        return None
+    if not d or d.get("source_digest") != source_digest():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
 # --------------------------------------------------------------- clocks --
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and throttle reasons sampled every few milliseconds by a
+    host thread through NVML while the timed region runs (read only: no
+    setting of the GPU is touched)."""
+    # clocks-event reason bits of NVML
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, dev_id):
-        self.dev_id = dev_id
-        self.proc = None
-        self.path = None
+    def __init__(self, dev_id, period_s=0.005):
+        self.dev_id = str(dev_id)
+        self.period = period_s
+        self.samples = []
+        self.mask = 0
+        self.max_mhz = None
+        self.thread = None
+        self.nvml = None
+
+    def _handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        self.nvml = pynvml
+        if self.dev_id.startswith(("GPU-", "MIG-")):
+            return pynvml.nvmlDeviceGetHandleByUUID(self.dev_id)
+        return pynvml.nvmlDeviceGetHandleByIndex(int(self.dev_id))
 
     def start(self):
-        fd, self.path = tempfile.mkstemp(suffix=".csv")
-        os.close(fd)
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.dev_id)], stdout=self.f, stderr=subprocess.DEVNULL)
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            h = self._handle()
+            self.max_mhz = float(self.nvml.nvmlDeviceGetMaxClockInfo(h, self.nvml.NVML_CLOCK_SM))
+        except Exception:
+            self.nvml = None
+            return
+        self.stop_evt = threading.Event()
+
+        def loop():
+            nv = self.nvml
+            while not self.stop_evt.is_set():
+                try:
+                    self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                    self.mask |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))
+                except Exception:
+                    pass
+                self.stop_evt.wait(self.period)
+
+        self.thread = threading.Thread(target=loop, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
+        if self.thread is None:
             return None
-        self.proc.terminate()
+        self.stop_evt.set()
+        self.thread.join(timeout=5)
         try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.f.close()
-        rows = [l.split(",") for l in open(self.path).read().strip().splitlines() if l.strip()]
-        os.unlink(self.path)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for row in rows:
-            row = [x.strip() for x in row]
-            if len(row) < 9:
-                continue
-            try:
-                sm.append(float(row[1]))
-                mx = float(row[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, row[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        if not sm:
-            return dict(sm_mhz=None, sm_max_mhz=mx, reasons=sorted(reasons), samples=0)
-        return dict(sm_mhz=statistics.median(sm), sm_max_mhz=mx, reasons=sorted(reasons),
-                    samples=len(sm))
+            self.nvml.nvmlShutdown()
+        except Exception:
+            pass
+        reasons = sorted(n for n, bit in self.REASONS.items() if self.mask & bit)
+        sm = statistics.median(self.samples) if self.samples else None
+        return dict(sm_mhz=sm, sm_max_mhz=self.max_mhz, reasons=reasons,
+                    samples=len(self.samples), source="nvml, 5 ms period")
 
 
 # ------------------------------------------------------------ reference --
@@ -256,6 +323,7 @@ def main():
     flags = step.flags(stream)
     if any(flags.values()):
         raise RuntimeError(f"device status flags after warm-up: {flags}")
+    # one graph per call (breakdown pass) and one graph for the whole step (timed)
     graphs = []
     for fn in (lambda: step.draft(inp), lambda: step.prefix(inp, w.scheduler),
                lambda: step.verify(inp)):
@@ -263,11 +331,18 @@ def main():
         with torch.cuda.graph(g, stream=stream):
             fn()
         graphs.append(g)
+    # timed: the draft call and the rest of the step (prefix + verify) as two
+    # graphs, so the draft's own time comes from the same timed region
+    g_draft = graphs[0]
+    g_rest = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_rest, stream=stream):
+        step.prefix(inp, w.scheduler)
+        step.verify(inp)
     torch.cuda.synchronize()
 
     def replay():
-        for g in graphs:
-            g.replay()
+        g_draft.replay()
+        g_rest.replay()
 
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
@@ -275,7 +350,7 @@ def main():
             replay()
     torch.cuda.synchronize()
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     dev_id = os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank] \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local_rank)
     clocks = ClockSampler(dev_id)
@@ -287,46 +362,52 @@ def main():
     with torch.cuda.stream(stream):
         for i in range(args.steps):
             flush.zero_()
-            e = ev[i]
-            e[0].record(stream)
-            graphs[0].replay()
-            e[1].record(stream)
-            graphs[1].replay()
-            e[2].record(stream)
-            graphs[2].replay()
-            e[3].record(stream)
+            ev[i][0].record(stream)
+            g_draft.replay()
+            ev[i][1].record(stream)
+            g_rest.replay()
+            ev[i][2].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     wall = time.perf_counter() - wall0
     clk = clocks.stop()
-
-    t_step = [e[0].elapsed_time(e[3]) for e in ev]
-    t_draft = [e[0].elapsed_time(e[1]) for e in ev]
-    t_prefix = [e[1].elapsed_time(e[2]) for e in ev]
-    t_verify = [e[2].elapsed_time(e[3]) for e in ev]
-    ms = sum(t_step) / len(t_step)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    t_step = [e[0].elapsed_time(e[2]) for e in ev]
+    t_draft_timed = [e[0].elapsed_time(e[1]) for e in ev]
+    ms = reduce_max(sum(t_step) / len(t_step), dev)
     units_per_rank = w.B * w.K
-    value = units_per_rank * world / (ms * 1e-3)
+    value = whole_job_rate(units_per_rank, world, ms)
+
+    # per-call breakdown (untimed pass, same flushing)
+    n_bd = max(3, min(args.steps, 50))
+    bd = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_bd)]
+    with torch.cuda.stream(stream):
+        for i in range(n_bd):
+            flush.zero_()
+            for j, g in enumerate(graphs):
+                bd[i][j].record(stream)
+                g.replay()
+            bd[i][3].record(stream)
+    torch.cuda.synchronize()
+    t_draft = [e[0].elapsed_time(e[1]) for e in bd]
+    t_prefix = [e[1].elapsed_time(e[2]) for e in bd]
+    t_verify = [e[2].elapsed_time(e[3]) for e in bd]
 
     L = step.verify_len.cpu().tolist()
     na = step.n_accepted.cpu()
     alg = algorithmic(w, L)
     pk = peaks()
-    md, mv = statistics.mean(t_draft), statistics.mean(t_verify)
+    md, mv = statistics.mean(t_draft_timed), statistics.mean(t_verify)
     # dominant part: the draft call (K projection + sampler launches) or the verify call
     if md >= mv:
         dom, dom_ms, dom_bytes = "dspark_draft_markov", md, alg["draft_bytes"]
     else:
         dom, dom_ms, dom_bytes = "dspark_verify", mv, alg["verify_bytes"]
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    kern = kernel_name(step.path, dom, w)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
-                "frac": achieved / pk["hbm"], "traffic": None,
-                "kernel": dom, "peak_source": pk["src"] + " (burst copy)",
+                "frac": achieved / pk["hbm"], "traffic": measured_traffic(kern, w.name),
+                "kernel": kern, "call": dom, "peak_source": pk["src"] + " (burst copy)",
                 "algorithmic_bytes_per_launch": dom_bytes,
                 "step_frac": alg["step_bytes"] / (ms * 1e-3) / 1e9 / pk["hbm"]}
 
@@ -355,15 +436,14 @@ def main():
                     ho.copy_(o, non_blocking=True)
                 e2e_ev[i][1].record(stream)
         torch.cuda.synchronize()
-        e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in e2e_ev)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": units_per_rank * world / (e2e_ms * 1e-3), "unit": UNIT,
+        e2e_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in e2e_ev), dev)
+        e2e = {"value": whole_job_rate(units_per_rank, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    launches_per_step = 2 * w.K + 1 + 4
+    # kernels of one step: persistent draft = 1 launch, otherwise 2 per
+    # position; prefix 1; verify 4 (statistics, accept, residual, sample)
+    launches_per_step = (1 if step.path.startswith(("persistent", "tcgen05-persistent"))
+                         else 2 * w.K) + 1 + 4
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, args.cpu_seconds)
@@ -384,7 +464,8 @@ def main():
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
-        "breakdown_ms": {"draft": md, "prefix": statistics.mean(t_prefix), "verify": mv},
+        "breakdown_ms": {"draft": md, "prefix": statistics.mean(t_prefix), "verify": mv,
+                         "note": "separate graphs per call, untimed pass"},
         "accepted_mean": float(na.float().mean()), "verify_len_mean": sum(L) / len(L),
         "latency_per_emitted_token_us": ms * 1e3 / (float(na.float().sum()) + w.B),
         "wall_s": wall,
