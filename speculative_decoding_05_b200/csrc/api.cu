@@ -191,7 +191,6 @@ dspark_status draft_impl(const float* base, const void* U, const void* W, dspark
     GemvRecs recs;
     recs.cta = reinterpret_cast<unsigned long long*>(ws + w.rec_off);
     recs.tok = recs.cta + (size_t)2 * B * kPMaxG * 2;
-    recs.counter = reinterpret_cast<unsigned*>(recs.tok + B + 16);
     if (gemv_path(r, B) &&
         cudaMemsetAsync(ws + w.rec_off, 0, gemv_rec_bytes(B), s) != cudaSuccess)
       return DSPARK_ERR_CUDA;

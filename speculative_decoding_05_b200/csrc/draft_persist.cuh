@@ -100,15 +100,47 @@ inline int persist_grid(int V) {
 constexpr int kSimtMaxB = 2;
 inline bool gemv_path(int r, int B) { return B <= kSimtMaxB && r == 256; }
 
+// Work split of the GEMV variant: 32-row chunks, a contiguous run per CTA.
+constexpr int kGRank = 256;
+constexpr int kGTailBytes = kChunk * kGRank * 2;    // 16 KB: the tail chunk's W rows
+constexpr int kGMaxChunks = 64;                     // chunks of one CTA (two per lane in level 2)
+
+// First chunk of CTA c: runs balanced to within one chunk.
+__host__ __device__ inline int gemv_chunk_begin(int cta, int G, int n_chunks) {
+  return (int)((long long)cta * n_chunks / G);
+}
+// 1 when a run of nc chunks hands its last chunk to the tail warp.
+__host__ __device__ inline int gemv_tail(int nc) { return (nc % 4 == 1) ? 1 : 0; }
+
+// Largest chunk run of a CTA, and the most 128-row tiles its GEMV warps take.
+inline void gemv_runs(int n_chunks, int G, int* max_chunks, int* max_tiles) {
+  const int q = n_chunks / G, rem = n_chunks % G;
+  *max_chunks = q + (rem ? 1 : 0);
+  int mt = 0;
+  for (int nc = q; nc <= *max_chunks; ++nc) {
+    const int tiles = (nc - gemv_tail(nc) + 3) / 4;
+    if (tiles > mt) mt = tiles;
+  }
+  *max_tiles = mt;
+}
+
 inline PersistLayout persist_layout(int V, int r, int B) {
   PersistLayout L;
   const int n_tiles = (V + kTileN - 1) / kTileN;
   L.G = persist_grid(V);
   L.max_nt = (n_tiles + L.G - 1) / L.G;
   if (gemv_path(r, B)) {
-    // sBias [B][rows] + sBase [2][B][rows] + sPart [B][max_nt*4]
-    L.u_bytes = 0;
-    L.base_bytes = (size_t)3 * B * L.max_nt * kTileN * 4 + (size_t)B * L.max_nt * 4 * 8 + 16;
+    const int n_chunks = n_chunks_of(V);
+    int G = num_sms();
+    if (G > n_chunks) G = n_chunks;
+    if (G > kPMaxG) G = kPMaxG;
+    int max_chunks;
+    L.G = G;
+    gemv_runs(n_chunks, G, &max_chunks, &L.max_nt);
+    // tail rows, sBias [B][rows_cap] + sBase [2][B][rows_cap] + sPart [B][part_cap]
+    const size_t rows_cap = (size_t)L.max_nt * kTileN + kChunk, part_cap = (size_t)L.max_nt * 4 + 1;
+    L.u_bytes = kGTailBytes;
+    L.base_bytes = (size_t)3 * B * rows_cap * 4 + (size_t)B * part_cap * 8 + 16;
   } else {
     L.u_bytes = (size_t)(r / 64) * 2048;
     L.base_bytes = (((size_t)B * L.max_nt * kTileN * 4) + 1023) & ~size_t(1023);
@@ -630,32 +662,57 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
 // out "transposed": lane l of a warp owns the K slice [8l, 8l+8) of every
 // row, so the previous-token vector U[x] stays in eight registers per
 // request, each lane accumulates the dot products of 32 rows at once, and
-// a 31-shuffle butterfly hands lane l the finished bias of row l.  Memory
-// plan: four W tiles per SM resident in TMEM for the whole call, stored in
-// the same transposed order (lane = K slice, four 32-bit columns = 8 bf16
-// per row) and read back with tcgen05.ld; the rest streams through the TMA
-// ring; base rows are bulk-copied one position ahead (double-buffered).
+// a 31-shuffle butterfly hands lane l the finished bias of row l.
 //
-// One round of global exchange per position: after its tiles each CTA
-// stores its softmax partial and adds to an arrival counter with release
-// semantics; one thread per CTA polls the counter (relaxed loads with a
-// short back-off, so 148 CTAs do not flood one L2 line); then one warp
-// reads all CTA partials, finds the CTA whose range holds the sample, and
-// only that CTA resolves the chunk and the token from its own shared
-// memory (chunk partials, bias and base values of its rows).  It writes the
-// outputs and publishes {position, token} as one 8-byte word; one thread
-// per CTA polls that word and every warp then loads its slice of U[x] for
-// the next position.  The partials are double-buffered by position parity:
-// a CTA can only reach position k+2 after every CTA has finished k.
+// Work split: the vocabulary is cut into 32-row chunks and every CTA owns
+// a contiguous run of them, balanced to within one chunk.  Eight GEMV warps
+// take the CTA's chunks four at a time as 128-row tiles (warp (h, q) takes
+// rows 32q..32q+31 of the tiles of parity h).  When a run has one chunk
+// more than a multiple of four, that last chunk goes to warp 3, which keeps
+// its W rows in shared memory for the whole call, instead of giving one GEMV
+// warp a fifth tile.  Memory plan of the GEMV warps: four W tiles per SM
+// resident in TMEM for the whole call, stored in the same transposed order
+// (lane = K slice, four 32-bit columns = 8 bf16 per row) and read back with
+// tcgen05.ld; the rest streams through the TMA ring; base rows are
+// bulk-copied one position ahead (double-buffered).
+//
+// One round of global exchange per position, without fences or counters:
+// after its tiles each CTA stores its softmax partial as two 8-byte words
+// {value, position + 1}.  The warp of request b polls the G partials of b
+// until every word carries the current position (relaxed loads, re-reading
+// only the stale ones, with a short back-off), finds the CTA whose range
+// holds the sample, and only that CTA resolves the chunk and the token from
+// its own shared memory (chunk partials, bias and base values of its rows).
+// It writes the outputs, starts pulling U[x] into L2, and publishes
+// {position + 1, token} as one 8-byte word; one thread per CTA polls that
+// word and every warp then loads its slice of U[x] for the next position.
+// The partials are double-buffered by position parity: a CTA publishes
+// position k+2 only after every CTA has read position k's partials (a token
+// of k+1 needs every CTA's partial of k+1, which each CTA stores after it has
+// read k's).
 constexpr int kGThreads = 384;
+constexpr int kGTailWarp = 3;
 constexpr int kGCompWarp0 = 4;
-constexpr int kGCompThreads = 256;
+constexpr int kGSyncThreads = 288;  // warps 3..11
 constexpr int kGMaxB = 2;
-constexpr int kGRank = 256;
 constexpr int kGMaxTmemTiles = 4;
+constexpr int kGSlots = 9;                          // per-warp partials: 8 GEMV warps + tail warp
 
 __device__ __forceinline__ void gemv_sync() {
-  asm volatile("bar.sync 1, %0;" ::"r"(kGCompThreads) : "memory");
+  asm volatile("bar.sync 1, %0;" ::"r"(kGSyncThreads) : "memory");
+}
+// the same barrier, returning whether any participating thread passed true
+__device__ __forceinline__ bool gemv_sync_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "r"(kGSyncThreads)
+      : "memory");
+  return r != 0;
 }
 __device__ __forceinline__ void st_rec(unsigned long long* p, uint32_t lo, uint32_t seq) {
   const unsigned long long v = ((unsigned long long)seq << 32) | lo;
@@ -665,6 +722,16 @@ __device__ __forceinline__ unsigned long long ld_rec(const unsigned long long* p
   unsigned long long v;
   asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
   return v;
+}
+// the pair of 8-byte words at p (16-byte aligned); each word is read as one
+// single-copy-atomic access, the pair as two
+__device__ __forceinline__ ulonglong2 ld_rec2(const unsigned long long* p) {
+  ulonglong2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2::evict_last [%0];" ::"l"(p));
 }
 
 // lane l receives sum over lanes of v[l] (butterfly transpose-reduce)
@@ -682,30 +749,61 @@ __device__ __forceinline__ float transpose_reduce32(float (&v)[32], int lane) {
   return v[0];
 }
 
-// pr[b][row] += sum_{e<8} w_e * u[b][e] over the 8 bf16 packed in q
+// c + w * u for the low / high bf16 of two packed pairs, accumulated in
+// fp32: the product of two bf16 values is exact in fp32, so this equals
+// fmaf(float(w), float(u), c) with no conversion instructions.
+__device__ __forceinline__ float fma_bf16_lo(uint32_t w, uint32_t u, float c) {
+  float d;
+  asm("{\n\t.reg .b16 wl, wh, ul, uh;\n\t"
+      "mov.b32 {wl, wh}, %1;\n\tmov.b32 {ul, uh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, wl, ul, %3;\n\t}"
+      : "=f"(d) : "r"(w), "r"(u), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fma_bf16_hi(uint32_t w, uint32_t u, float c) {
+  float d;
+  asm("{\n\t.reg .b16 wl, wh, ul, uh;\n\t"
+      "mov.b32 {wl, wh}, %1;\n\tmov.b32 {ul, uh}, %2;\n\t"
+      "fma.rn.f32.bf16 %0, wh, uh, %3;\n\t}"
+      : "=f"(d) : "r"(w), "r"(u), "f"(c));
+  return d;
+}
+
+// pr[b][row] += sum_{e<8} w_e * u_e over the 8 bf16 packed in q and in u[b]
+// (ascending e, one rounding per step)
 template <int NB>
-__device__ __forceinline__ void gemv8(uint4 q, const float (&u)[NB][8], int B, float (&pr)[NB][32],
+__device__ __forceinline__ void gemv8(uint4 q, const uint32_t (&u)[NB][4], int B, float (&pr)[NB][32],
                                       int row) {
-  const float w0 = __uint_as_float(q.x << 16), w1 = __uint_as_float(q.x & 0xffff0000u);
-  const float w2 = __uint_as_float(q.y << 16), w3 = __uint_as_float(q.y & 0xffff0000u);
-  const float w4 = __uint_as_float(q.z << 16), w5 = __uint_as_float(q.z & 0xffff0000u);
-  const float w6 = __uint_as_float(q.w << 16), w7 = __uint_as_float(q.w & 0xffff0000u);
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
     if (b >= B) break;
     float a = pr[b][row];
-    a = fmaf(w0, u[b][0], a); a = fmaf(w1, u[b][1], a);
-    a = fmaf(w2, u[b][2], a); a = fmaf(w3, u[b][3], a);
-    a = fmaf(w4, u[b][4], a); a = fmaf(w5, u[b][5], a);
-    a = fmaf(w6, u[b][6], a); a = fmaf(w7, u[b][7], a);
+    a = fma_bf16_lo(q.x, u[b][0], a); a = fma_bf16_hi(q.x, u[b][0], a);
+    a = fma_bf16_lo(q.y, u[b][1], a); a = fma_bf16_hi(q.y, u[b][1], a);
+    a = fma_bf16_lo(q.z, u[b][2], a); a = fma_bf16_hi(q.z, u[b][2], a);
+    a = fma_bf16_lo(q.w, u[b][3], a); a = fma_bf16_hi(q.w, u[b][3], a);
     pr[b][row] = a;
+  }
+}
+
+// u[b] = the 8 bf16 of U[x_b][8 lane .. 8 lane + 7], packed (zeros for x < 0)
+template <int NB>
+__device__ __forceinline__ void load_u_slice(const __nv_bfloat16* U, const int (&x)[NB], int B, int lane,
+                                             uint32_t (&u)[NB][4]) {
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (b < B && x[b] >= 0) val = __ldg(reinterpret_cast<const uint4*>(U + (size_t)x[b] * kGRank) + lane);
+    u[b][0] = val.x;
+    u[b][1] = val.y;
+    u[b][2] = val.z;
+    u[b][3] = val.w;
   }
 }
 
 struct GemvRecs {
   unsigned long long* cta;  // [2][B][G][2]: {M, seq}, {S, seq}
   unsigned long long* tok;  // [B]: {position + 1, token}
-  unsigned* counter;        // arrival counter (zeroed per call)
 };
 
 __device__ __forceinline__ void backoff_spin_u64(const unsigned long long* p, uint32_t seq,
@@ -726,6 +824,13 @@ __device__ __forceinline__ void backoff_spin_u64(const unsigned long long* p, ui
   }
 }
 
+// Bounded wait, at the end of the call, for the copies a producer issued:
+// the last issue into each of the n_slots slots of a ring of `issued` issues.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int n_slots, int issued) {
+  for (int j = max(0, issued - n_slots); j < issued; ++j)
+    (void)mbar_wait(&full[j % n_slots], (uint32_t)(j / n_slots) & 1u);
+}
+
 template <int NB>
 __global__ void __launch_bounds__(kGThreads, 1)
 draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p, const GemvRecs rec) {
@@ -733,21 +838,27 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int nkb = kGRank / 64;
   const int G = gridDim.x, cta = blockIdx.x;
-  const int t0 = p_tile_begin(cta, G, p.n_tiles), t1 = p_tile_begin(cta + 1, G, p.n_tiles);
-  const int nt = t1 - t0;
   const int B = p.B, K = p.K, V = p.V;
   const int S = p.n_stages;
-  const int rows_cap = p.max_nt * kTileN;  // row slots per request in sBias / sBase
+  const int c_begin = gemv_chunk_begin(cta, G, p.n_chunks);
+  const int nc = gemv_chunk_begin(cta + 1, G, p.n_chunks) - c_begin;  // chunks of this CTA
+  const int tail = gemv_tail(nc);
+  const int mainc = nc - tail;                   // chunks of the GEMV warps
+  const int nt = (mainc + 3) / 4;                // their 128-row tiles
+  const int v0 = c_begin * kChunk;               // first vocabulary row of this CTA
+  const int nrows = min(nc * kChunk, V - v0);    // valid rows of this CTA
+  const int main_rows = min(mainc * kChunk, nrows);
+  const int rows_cap = p.max_nt * kTileN + kChunk;  // row slots per request in sBias / sBase
+  const int part_cap = p.max_nt * 4 + 1;            // chunk slots per request in sPart
   const int nres = min(nt, kGMaxTmemTiles);
   const int nstream = nt - nres;
-  const int nrows = min(nt * kTileN, V - t0 * kTileN);   // valid rows of this CTA
-  const int nloc = (nrows + kChunk - 1) / kChunk;        // chunks of this CTA
 
   uint8_t* sRing = sm;
-  float* sBias = reinterpret_cast<float*>(sRing + S * kStageBytes);  // [B][rows_cap]
-  float* sBase = sBias + (size_t)B * rows_cap;                       // [2][B][rows_cap]
-  float2* sPart = reinterpret_cast<float2*>(sBase + (size_t)2 * B * rows_cap);  // [B][max_nt*4]
-  uint8_t* misc = reinterpret_cast<uint8_t*>(sPart + (size_t)B * p.max_nt * 4);
+  uint8_t* sTail = sRing + S * kStageBytes;                                  // [32 rows][512 B]
+  float* sBias = reinterpret_cast<float*>(sTail + kGTailBytes);              // [B][rows_cap]
+  float* sBase = sBias + (size_t)B * rows_cap;                               // [2][B][rows_cap]
+  float2* sPart = reinterpret_cast<float2*>(sBase + (size_t)2 * B * rows_cap);  // [B][part_cap]
+  uint8_t* misc = reinterpret_cast<uint8_t*>(sPart + (size_t)B * part_cap);
   misc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(misc) + 15) & ~uintptr_t(15));
   uint64_t* ringFull = reinterpret_cast<uint64_t*>(misc);
   uint64_t* ringEmpty = ringFull + kPMaxStages;
@@ -755,9 +866,9 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   uint64_t* baseEmpty = baseFull + 2;            // [2]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(baseEmpty + 2);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [8][kGMaxB]
-  float* s_ws = s_wm + 8 * kGMaxB;                        // [8][kGMaxB]
-  volatile int* s_i = reinterpret_cast<volatile int*>(s_ws + 8 * kGMaxB);  // [4]
+  float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [kGSlots][kGMaxB]
+  float* s_ws = s_wm + kGSlots * kGMaxB;                  // [kGSlots][kGMaxB]
+  volatile int* s_i = reinterpret_cast<volatile int*>(s_ws + kGSlots * kGMaxB);  // [4]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -786,7 +897,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       int it = 0;
       for (int k = 0; k < K && !*s_abort; ++k) {
         for (int i = nres; i < nt && !*s_abort; ++i) {
-          for (int kb = 0; kb < nkb; ++kb, ++it) {
+          for (int kb = 0; kb < nkb; ++kb) {
             const int s = it % S;
             if (!mbar_wait(&ringEmpty[s], ((uint32_t)(it / S) & 1u) ^ 1u)) {
               *s_abort = 1;
@@ -794,18 +905,19 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
               break;
             }
             mbar_arrive_expect_tx(&ringFull[s], kStageBytes);
-            tma_load_2d_hint(sRing + s * kStageBytes, &tm_w, &ringFull[s], kb * 64,
-                             (t0 + i) * kTileN, pol);
+            tma_load_2d_hint(sRing + s * kStageBytes, &tm_w, &ringFull[s], kb * 64, v0 + i * kTileN, pol);
+            ++it;
           }
         }
       }
+      drain_ring(ringFull, S, it);
     }
   } else if (warp == 2) {
     // ------------------------------------------------ base producer (double-buffered)
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
-      const int v0 = t0 * kTileN;
       const uint32_t bytes = (uint32_t)nrows * 4u;
+      int issued = 0;
       for (int k = 0; k < K && !*s_abort; ++k) {
         const int buf = k & 1;
         if (!mbar_wait(&baseEmpty[buf], ((uint32_t)(k >> 1) & 1u) ^ 1u)) {
@@ -817,13 +929,17 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         for (int b = 0; b < B; ++b)
           bulk_load(sBase + ((size_t)buf * B + b) * rows_cap,
                     p.base + ((size_t)b * K + k) * (size_t)V + v0, bytes, &baseFull[buf], pol);
+        ++issued;
       }
+      drain_ring(baseFull, 2, issued);
     }
-  } else if (warp >= kGCompWarp0) {
+  } else if (warp >= kGTailWarp) {
     // ------------------------------------------------ GEMV, epilogue, sampling
-    const int cw = warp - kGCompWarp0;  // 0..7
-    const int half = cw >> 2;           // tile parity owned by this warp
-    const int quarter = warp & 3;       // TMEM lane quarter = rows 32q..32q+31 of a tile
+    const bool gemv = warp >= kGCompWarp0;
+    const int cw = warp - kGCompWarp0;          // 0..7 for the GEMV warps, -1 for the tail warp
+    const int slot = gemv ? cw : kGSlots - 1;   // this warp's partial slot
+    const int half = cw >> 1 >> 1;              // tile parity owned by a GEMV warp
+    const int quarter = warp & 3;               // TMEM lane quarter = rows 32q..32q+31 of a tile
     const int kb_l = lane >> 3, j8 = lane & 7;  // this lane's K slice: k-block, 16-byte chunk
     float it2[NB], itv[NB];
 #pragma unroll
@@ -831,41 +947,48 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       itv[b] = (b < B) ? checked_inv_temp(p.inv_temp, b, p.flags) : 1.0f;
       it2[b] = itv[b] * kLog2e;
     }
-    // resident tiles -> TMEM in transposed order
-    for (int i = half; i < nres; i += 2) {
-      for (int cb = 0; cb < 4; ++cb) {
-        uint32_t regs[32];
+    if (gemv) {
+      // resident tiles -> TMEM in transposed order
+      for (int i = half; i < nres; i += 2) {
+        for (int cb = 0; cb < 4; ++cb) {
+          uint32_t regs[32];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int row = (t0 + i) * kTileN + quarter * 32 + cb * 8 + j;
-          const uint4 val = (row < V) ? __ldg(reinterpret_cast<const uint4*>(p.W + (size_t)row * kGRank) + lane)
-                                      : make_uint4(0, 0, 0, 0);
-          regs[4 * j] = val.x;
-          regs[4 * j + 1] = val.y;
-          regs[4 * j + 2] = val.z;
-          regs[4 * j + 3] = val.w;
+          for (int j = 0; j < 8; ++j) {
+            const int row = v0 + i * kTileN + quarter * 32 + cb * 8 + j;
+            const uint4 val = (row < V) ? __ldg(reinterpret_cast<const uint4*>(p.W + (size_t)row * kGRank) + lane)
+                                        : make_uint4(0, 0, 0, 0);
+            regs[4 * j] = val.x;
+            regs[4 * j + 1] = val.y;
+            regs[4 * j + 2] = val.z;
+            regs[4 * j + 3] = val.w;
+          }
+          tmem_st32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + cb * 32), regs);
         }
-        tmem_st32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + cb * 32), regs);
+      }
+      tmem_st_wait();
+    } else if (tail) {
+      // the tail chunk's W rows -> shared memory, row-major (512 B per row)
+      for (int rr = 0; rr < kChunk; ++rr) {
+        const int row = v0 + main_rows + rr;
+        const uint4 val = (main_rows + rr < nrows)
+                              ? __ldg(reinterpret_cast<const uint4*>(p.W + (size_t)row * kGRank) + lane)
+                              : make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(sTail + rr * (kGRank * 2) + lane * 16) = val;
       }
     }
-    tmem_st_wait();
     // U[prev_token] slice of this lane
-    float u[NB][8];
+    uint32_t u[NB][4];
+    {
+      int x[NB];
 #pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      const int x = (b < B) ? checked_token(p.prev_token[b], V, true, p.flags) : -1;
-      uint4 val = make_uint4(0, 0, 0, 0);
-      if (x >= 0) val = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)x * kGRank) + lane);
-      u[b][0] = __uint_as_float(val.x << 16); u[b][1] = __uint_as_float(val.x & 0xffff0000u);
-      u[b][2] = __uint_as_float(val.y << 16); u[b][3] = __uint_as_float(val.y & 0xffff0000u);
-      u[b][4] = __uint_as_float(val.z << 16); u[b][5] = __uint_as_float(val.z & 0xffff0000u);
-      u[b][6] = __uint_as_float(val.w << 16); u[b][7] = __uint_as_float(val.w & 0xffff0000u);
+      for (int b = 0; b < NB; ++b) x[b] = (b < B) ? checked_token(p.prev_token[b], V, true, p.flags) : -1;
+      load_u_slice<NB>(p.U, x, B, lane, u);
     }
     tc_fence_before();
     gemv_sync();
     tc_fence_after();
 
-    for (int k = 0; k < K && !*s_abort; ++k) {
+    for (int k = 0; k < K; ++k) {
       const int buf = k & 1, par = k & 1;
       const uint32_t seq = (uint32_t)k + 1u;
       const float* bse = sBase + (size_t)buf * B * rows_cap;
@@ -876,48 +999,10 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         ws[b] = 0.0f;
       }
       bool ok = mbar_wait_spin(&baseFull[buf], (uint32_t)(k >> 1) & 1u);
-      for (int i = half; i < nt; i += 2) {
-        float pr[NB][32];
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) pr[b][j] = 0.0f;
-        if (i < nres) {
-#pragma unroll
-          for (int cb = 0; cb < 4; ++cb) {
-            float wf[32];
-            tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + cb * 32), wf);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint4 q = make_uint4(__float_as_uint(wf[4 * j]), __float_as_uint(wf[4 * j + 1]),
-                                         __float_as_uint(wf[4 * j + 2]), __float_as_uint(wf[4 * j + 3]));
-              gemv8<NB>(q, u, B, pr, cb * 8 + j);
-            }
-          }
-        } else {
-          const int itb = (k * nstream + (i - nres)) * nkb;
-          for (int kb = 0; kb < nkb; ++kb) {
-            const int it = itb + kb;
-            ok = ok && mbar_wait_spin(&ringFull[it % S], (uint32_t)(it / S) & 1u);
-          }
-          const uint8_t* stg = sRing + ((itb + kb_l) % S) * kStageBytes;
-#pragma unroll
-          for (int rr = 0; rr < 32; ++rr) {
-            const int m = quarter * 32 + rr;
-            const uint4 q = *reinterpret_cast<const uint4*>(stg + m * 128 + ((j8 ^ (m & 7)) << 4));
-            gemv8<NB>(q, u, B, pr, rr);
-          }
-          __syncwarp();
-          if (lane == 0)
-            for (int kb = 0; kb < nkb; ++kb) mbar_arrive(&ringEmpty[(itb + kb) % S]);
-        }
-        if (!ok) {
-          *s_abort = 1;
-          raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
-        }
-        const int vl = i * kTileN + quarter * 32 + lane;  // row within the CTA range
-        const int v = t0 * kTileN + vl;
-        const bool valid = v < V;
+
+      // per 32-row unit: bias of lane `lane`'s row, its softmax partial, stores
+      auto finish_unit = [&](float (&pr)[NB][32], int vl, bool valid, int chunk) {
+        const int v = v0 + vl;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
           if (b >= B) break;
@@ -934,16 +1019,74 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             if (p.draft_logits != nullptr) p.draft_logits[row + v] = a * itv[b];
           }
           if (lane == 0) {
-            sPart[(size_t)b * p.max_nt * 4 + i * 4 + quarter] = make_float2(A, sm2);
+            sPart[(size_t)b * part_cap + chunk] = make_float2(A, sm2);
             merge_partial(wm[b], ws[b], A, sm2, it2[b]);
           }
         }
+      };
+
+      if (gemv) {
+        for (int i = half; i < nt; i += 2) {
+          float pr[NB][32];
+#pragma unroll
+          for (int b = 0; b < NB; ++b)
+#pragma unroll
+            for (int j = 0; j < 32; ++j) pr[b][j] = 0.0f;
+          if (i < nres) {
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+              float wf[32];
+              tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + cb * 32), wf);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                const uint4 q = make_uint4(__float_as_uint(wf[4 * j]), __float_as_uint(wf[4 * j + 1]),
+                                           __float_as_uint(wf[4 * j + 2]), __float_as_uint(wf[4 * j + 3]));
+                gemv8<NB>(q, u, B, pr, cb * 8 + j);
+              }
+            }
+          } else {
+            const int itb = (k * nstream + (i - nres)) * nkb;
+            for (int kb = 0; kb < nkb; ++kb) {
+              const int it = itb + kb;
+              ok = ok && mbar_wait_spin(&ringFull[it % S], (uint32_t)(it / S) & 1u);
+            }
+            const uint8_t* stg = sRing + ((itb + kb_l) % S) * kStageBytes;
+#pragma unroll
+            for (int rr = 0; rr < 32; ++rr) {
+              const int m = quarter * 32 + rr;
+              const uint4 q = *reinterpret_cast<const uint4*>(stg + m * 128 + ((j8 ^ (m & 7)) << 4));
+              gemv8<NB>(q, u, B, pr, rr);
+            }
+            __syncwarp();
+            if (lane == 0)
+              for (int kb = 0; kb < nkb; ++kb) mbar_arrive(&ringEmpty[(itb + kb) % S]);
+          }
+          const int vl = i * kTileN + quarter * 32 + lane;  // row within the CTA range
+          finish_unit(pr, vl, vl < main_rows, i * 4 + quarter);
+        }
+      } else if (tail) {
+        float pr[NB][32];
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+#pragma unroll
+          for (int j = 0; j < 32; ++j) pr[b][j] = 0.0f;
+#pragma unroll
+        for (int rr = 0; rr < 32; ++rr) {
+          const uint4 q = *reinterpret_cast<const uint4*>(sTail + rr * (kGRank * 2) + lane * 16);
+          gemv8<NB>(q, u, B, pr, rr);
+        }
+        const int vl = main_rows + lane;
+        finish_unit(pr, vl, vl < nrows, mainc);
+      }
+      if (!ok) {
+        *s_abort = 1;
+        raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
       }
       if (lane == 0) {
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          s_wm[cw * kGMaxB + b] = wm[b];
-          s_ws[cw * kGMaxB + b] = ws[b];
+          s_wm[slot * kGMaxB + b] = wm[b];
+          s_ws[slot * kGMaxB + b] = ws[b];
         }
       }
       gemv_sync();
@@ -951,55 +1094,48 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       if (cw == 0 && lane < B) {
         const int b = lane;
         float M = -CUDART_INF_F, Sm = 0.0f;
-        for (int w2 = 0; w2 < 8; ++w2)
+        for (int w2 = 0; w2 < kGSlots; ++w2)
           merge_partial(M, Sm, s_wm[w2 * kGMaxB + b], s_ws[w2 * kGMaxB + b], it2[b]);
         unsigned long long* r0 = rec.cta + (((size_t)par * B + b) * G + cta) * 2;
         st_rec(r0, __float_as_uint(M), seq);
         st_rec(r0 + 1, __float_as_uint(Sm), seq);
       }
-      if (cw == 0) {
-        __syncwarp();
-        if (lane == 0) {
-          asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(rec.counter) : "memory");
-          const unsigned target = (unsigned)(k + 1) * (unsigned)G;
-          const uint64_t tstart = global_timer_ns();
-          for (;;) {
-            unsigned seen;
-            asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(rec.counter) : "memory");
-            if (seen >= target) break;
-            if (global_timer_ns() - tstart > kWaitLimitNs) {
-              *s_abort = 1;
-              raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
-              break;
-            }
-            __nanosleep(20);
-          }
-          asm volatile("fence.acq_rel.gpu;" ::: "memory");
-          s_i[0] = 1;
-        }
-      }
-      gemv_sync();
-      // warp b: level 1 over all CTAs; the owning CTA resolves chunk and token
-      if (cw < B) {
+      // warp b: gathers the partials of request b from every CTA (level 1);
+      // the CTA that holds the sample resolves chunk and token
+      if (gemv && cw < B) {
         const int b = cw;
         const unsigned long long* cr = rec.cta + (((size_t)par * B + b) * G) * 2;
         const int per = (G + 31) / 32;
         const int c0 = min(lane * per, G), c1 = min(c0 + per, G);
         float2 q[kPMaxG / 32];
-        bool stale = false;
+        unsigned pend = 0;
 #pragma unroll
         for (int i = 0; i < kPMaxG / 32; ++i) {
           q[i] = make_float2(-CUDART_INF_F, 0.0f);
-          if (c0 + i < c1) {
-            const unsigned long long m0 = ld_rec(cr + 2 * (c0 + i));
-            const unsigned long long m1 = ld_rec(cr + 2 * (c0 + i) + 1);
-            if ((uint32_t)(m0 >> 32) != seq || (uint32_t)(m1 >> 32) != seq) stale = true;
-            q[i] = make_float2(__uint_as_float((uint32_t)m0), __uint_as_float((uint32_t)m1));
-          }
+          if (c0 + i < c1) pend |= 1u << i;
         }
-        if (__any_sync(0xffffffffu, stale) && lane == 0) {
-          *s_abort = 1;  // the counter said every partial was in place
-          raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+        const uint64_t tstart = global_timer_ns();
+        for (;;) {
+          ulonglong2 m[kPMaxG / 32];
+#pragma unroll
+          for (int i = 0; i < kPMaxG / 32; ++i)
+            if (pend & (1u << i)) m[i] = ld_rec2(cr + 2 * (c0 + i));
+#pragma unroll
+          for (int i = 0; i < kPMaxG / 32; ++i) {
+            if ((pend & (1u << i)) && (uint32_t)(m[i].x >> 32) == seq && (uint32_t)(m[i].y >> 32) == seq) {
+              q[i] = make_float2(__uint_as_float((uint32_t)m[i].x), __uint_as_float((uint32_t)m[i].y));
+              pend &= ~(1u << i);
+            }
+          }
+          if (!__any_sync(0xffffffffu, pend != 0)) break;
+          if (__any_sync(0xffffffffu, global_timer_ns() - tstart > kWaitLimitNs)) {
+            if (lane == 0) {
+              *s_abort = 1;
+              raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+            }
+            break;
+          }
+          __nanosleep(32);
         }
         float mx = -CUDART_INF_F;
 #pragma unroll
@@ -1049,10 +1185,10 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         }
         if (cstar == cta) {
           // level 2: this CTA's chunk partials (shared memory), two per lane
-          const float2* lp = sPart + (size_t)b * p.max_nt * 4;
+          const float2* lp = sPart + (size_t)b * part_cap;
           const int ca = 2 * lane, cb2 = ca + 1;
-          const double wA = (ca < nloc) ? partial_weight(lp[ca], M, it2[b]) : 0.0;
-          const double wB = (cb2 < nloc) ? partial_weight(lp[cb2], M, it2[b]) : 0.0;
+          const double wA = (ca < nc) ? partial_weight(lp[ca], M, it2[b]) : 0.0;
+          const double wB = (cb2 < nc) ? partial_weight(lp[cb2], M, it2[b]) : 0.0;
           const double pin = warp_incl_scan_d(wA + wB);
           double lstart = __shfl_up_sync(0xffffffffu, pin, 1);
           if (lane == 0) lstart = 0.0;
@@ -1075,13 +1211,16 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           }
           // level 3: the chunk's rows from shared memory
           const int vl = chunk * kChunk + lane;
-          const int v = t0 * kTileN + vl;
-          const bool valid = v < V;
+          const int v = v0 + vl;
+          const bool valid = vl < nrows;
           float ef = 0.0f;
           if (valid)
             ef = ex2(((bse[(size_t)b * rows_cap + vl] - M) + sBias[(size_t)b * rows_cap + vl]) * it2[b]);
           const int pl = pick_lane((double)ef, before2, T);
           const int x = __shfl_sync(0xffffffffu, valid ? v : 0, pl);
+          // start pulling U[x] into L2 for every CTA's next position
+          if (k + 1 < K && lane < (kGRank * 2) / 128)
+            prefetch_l2(reinterpret_cast<const uint8_t*>(p.U + (size_t)x * kGRank) + lane * 128);
           if (lane == pl) {
             const size_t o = (size_t)b * K + k;
             if (!(Z > 0.0) || !isfinite(Z)) {
@@ -1103,7 +1242,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           if (lane == 0) st_rec(rec.tok + b, (uint32_t)x, seq);
         }
       }
-      // one thread per CTA waits for the tokens; every warp loads its U[x] slice
+      // one thread per request waits for the token; every warp then loads its U[x] slice
       if (cw == 0 && lane < B) {
         unsigned long long v;
         bool to = false;
@@ -1114,20 +1253,16 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         }
         s_i[1 + lane] = min(max((int)(uint32_t)v, 0), V - 1);
       }
-      gemv_sync();
-      if (k + 1 < K) {
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          if (b >= B) break;
-          const uint4 val = __ldg(reinterpret_cast<const uint4*>(p.U + (size_t)s_i[1 + b] * kGRank) + lane);
-          u[b][0] = __uint_as_float(val.x << 16); u[b][1] = __uint_as_float(val.x & 0xffff0000u);
-          u[b][2] = __uint_as_float(val.y << 16); u[b][3] = __uint_as_float(val.y & 0xffff0000u);
-          u[b][4] = __uint_as_float(val.z << 16); u[b][5] = __uint_as_float(val.z & 0xffff0000u);
-          u[b][6] = __uint_as_float(val.w << 16); u[b][7] = __uint_as_float(val.w & 0xffff0000u);
-        }
-      }
-      gemv_sync();
+      // every reader of sBase[buf], sBias and sPart for position k is past this barrier
+      const bool abort = gemv_sync_or(*s_abort != 0);
       if (cw == 0 && lane == 0) mbar_arrive(&baseEmpty[buf]);  // buffer free for position k+2
+      if (abort) break;
+      if (k + 1 < K) {
+        int x[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) x[b] = (b < B) ? s_i[1 + b] : -1;
+        load_u_slice<NB>(p.U, x, B, lane, u);
+      }
     }
   }
 
@@ -1145,6 +1280,11 @@ inline bool persist_supported(int V, int r, int B) {
   if (B < 1 || B > kPMaxB || r % 64 != 0 || r < 64 || r > 256 || V % 4 != 0 || V < kTileN)
     return false;
   const PersistLayout L = persist_layout(V, r, B);
+  if (gemv_path(r, B)) {
+    int max_chunks, max_tiles;
+    gemv_runs(n_chunks_of(V), L.G, &max_chunks, &max_tiles);
+    if (max_chunks > kGMaxChunks) return false;
+  }
   return L.max_nt <= kPMaxTiles && L.n_stages >= kPMinStages;
 }
 
@@ -1202,7 +1342,7 @@ inline dspark_status persist_launch(const CUtensorMap& tm_w, PersistArgs a, Gemv
 }
 
 // Bytes of the position records of the GEMV variant (zeroed by the caller
-// before each call): CTA partials [2][B][G][2], token words [B], counter.
+// before each call): CTA partials [2][B][G][2], token words [B].
 inline size_t gemv_rec_bytes(int B) {
   return (size_t)2 * B * kPMaxG * 2 * 8 + (size_t)B * 8 + 256;
 }
