@@ -414,21 +414,25 @@ dspark_status dspark_confidence_prefix(const float* z, const float* temps,
   if (!cost_tokens || !cost_ms || !verify_len || !objective) return DSPARK_ERR_INVALID_ARG;
   if (B * K > 0 && (!z || !temps || !c || !survival)) return DSPARK_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  dspark_status st = clear_status(workspace, s);
-  if (st != DSPARK_OK) return st;
   int npad = 1;
   while (npad < B * K) npad <<= 1;
   const size_t smem = (size_t)npad * (sizeof(double) + sizeof(int)) + (size_t)B * sizeof(int);
   static bool attr = false;
   if (!attr) {
-    cudaFuncSetAttribute(prefix_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaFuncSetAttribute(prefix_kernel<kPrefixThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kMaxCand * 12 + 8192 * 4);
     attr = true;
   }
   if (smem > (size_t)kMaxCand * 12 + 8192 * 4) return DSPARK_ERR_UNSUPPORTED;
-  prefix_kernel<<<1, kPrefixThreads, smem, s>>>(z, temps, cost_tokens, cost_ms, n_pts, B, K, enable,
-                                               c, survival, verify_len, objective,
-                                               static_cast<unsigned*>(workspace));
+  // the kernel clears the status word itself (one CTA: before any flag is raised)
+  if (npad <= kPrefixSmallCand)
+    prefix_kernel<kPrefixThreadsSmall><<<1, kPrefixThreadsSmall, smem, s>>>(
+        z, temps, cost_tokens, cost_ms, n_pts, B, K, enable, c, survival, verify_len, objective,
+        static_cast<unsigned*>(workspace));
+  else
+    prefix_kernel<kPrefixThreads><<<1, kPrefixThreads, smem, s>>>(
+        z, temps, cost_tokens, cost_ms, n_pts, B, K, enable, c, survival, verify_len, objective,
+        static_cast<unsigned*>(workspace));
   return check_launch();
 }
 

@@ -104,6 +104,8 @@ inline bool gemv_path(int r, int B) { return B <= kSimtMaxB && r == 256; }
 constexpr int kGRank = 256;
 constexpr int kGTailBytes = kChunk * kGRank * 2;    // 16 KB: the tail chunk's W rows
 constexpr int kGMaxChunks = 64;                     // chunks of one CTA (two per lane in level 2)
+constexpr int kGPerLane = 5;                        // CTA partials per lane in level 1
+constexpr int kGMaxG = 32 * kGPerLane;              // grid limit of the GEMV variant
 
 // First chunk of CTA c: runs balanced to within one chunk.
 __host__ __device__ inline int gemv_chunk_begin(int cta, int G, int n_chunks) {
@@ -133,7 +135,7 @@ inline PersistLayout persist_layout(int V, int r, int B) {
     const int n_chunks = n_chunks_of(V);
     int G = num_sms();
     if (G > n_chunks) G = n_chunks;
-    if (G > kPMaxG) G = kPMaxG;
+    if (G > kGMaxG) G = kGMaxG;
     int max_chunks;
     L.G = G;
     gemv_runs(n_chunks, G, &max_chunks, &L.max_nt);
@@ -668,7 +670,7 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
 // a contiguous run of them, balanced to within one chunk.  Eight GEMV warps
 // take the CTA's chunks four at a time as 128-row tiles (warp (h, q) takes
 // rows 32q..32q+31 of the tiles of parity h).  When a run has one chunk
-// more than a multiple of four, that last chunk goes to warp 3, which keeps
+// more than a multiple of four, that last chunk goes to warp 2, which keeps
 // its W rows in shared memory for the whole call, instead of giving one GEMV
 // warp a fifth tile.  Memory plan of the GEMV warps: four W tiles per SM
 // resident in TMEM for the whole call, stored in the same transposed order
@@ -680,7 +682,7 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
 // after its tiles each CTA stores its softmax partial as two 8-byte words
 // {value, position + 1}.  The warp of request b polls the G partials of b
 // until every word carries the current position (relaxed loads, re-reading
-// only the stale ones, with a short back-off), finds the CTA whose range
+// only the stale ones), finds the CTA whose range
 // holds the sample, and only that CTA resolves the chunk and the token from
 // its own shared memory (chunk partials, bias and base values of its rows).
 // It writes the outputs, starts pulling U[x] into L2, and publishes
@@ -690,10 +692,14 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
 // position k+2 only after every CTA has read position k's partials (a token
 // of k+1 needs every CTA's partial of k+1, which each CTA stores after it has
 // read k's).
-constexpr int kGThreads = 384;
-constexpr int kGTailWarp = 3;
-constexpr int kGCompWarp0 = 4;
-constexpr int kGSyncThreads = 288;  // warps 3..11
+//
+// Warp roles: warp 0 TMEM allocator + W producer (TMA), warp 1 base
+// producer (bulk copies), warp 2 tail chunk, warps 3..10 GEMV (TMEM lane
+// quarter = warp % 4; warps 3..6 take the even tiles, 7..10 the odd ones).
+constexpr int kGThreads = 352;
+constexpr int kGTailWarp = 2;
+constexpr int kGCompWarp0 = 3;
+constexpr int kGSyncThreads = 288;  // warps 2..10
 constexpr int kGMaxB = 2;
 constexpr int kGMaxTmemTiles = 4;
 constexpr int kGSlots = 9;                          // per-warp partials: 8 GEMV warps + tail warp
@@ -820,7 +826,6 @@ __device__ __forceinline__ void backoff_spin_u64(const unsigned long long* p, ui
       *out = 0;
       return;
     }
-    __nanosleep(32);
   }
 }
 
@@ -884,7 +889,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
     *s_abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(tmem_slot, kPTmemCols);
+  if (warp == 0) tmem_alloc(tmem_slot, kPTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -912,7 +917,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       }
       drain_ring(ringFull, S, it);
     }
-  } else if (warp == 2) {
+  } else if (warp == 1) {
     // ------------------------------------------------ base producer (double-buffered)
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
@@ -1025,58 +1030,65 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         }
       };
 
-      if (gemv) {
-        for (int i = half; i < nt; i += 2) {
-          float pr[NB][32];
-#pragma unroll
-          for (int b = 0; b < NB; ++b)
-#pragma unroll
-            for (int j = 0; j < 32; ++j) pr[b][j] = 0.0f;
-          if (i < nres) {
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-              float wf[32];
-              tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128 + cb * 32), wf);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                const uint4 q = make_uint4(__float_as_uint(wf[4 * j]), __float_as_uint(wf[4 * j + 1]),
-                                           __float_as_uint(wf[4 * j + 2]), __float_as_uint(wf[4 * j + 3]));
-                gemv8<NB>(q, u, B, pr, cb * 8 + j);
-              }
-            }
-          } else {
-            const int itb = (k * nstream + (i - nres)) * nkb;
-            for (int kb = 0; kb < nkb; ++kb) {
-              const int it = itb + kb;
-              ok = ok && mbar_wait_spin(&ringFull[it % S], (uint32_t)(it / S) & 1u);
-            }
-            const uint8_t* stg = sRing + ((itb + kb_l) % S) * kStageBytes;
-#pragma unroll
-            for (int rr = 0; rr < 32; ++rr) {
-              const int m = quarter * 32 + rr;
-              const uint4 q = *reinterpret_cast<const uint4*>(stg + m * 128 + ((j8 ^ (m & 7)) << 4));
-              gemv8<NB>(q, u, B, pr, rr);
-            }
-            __syncwarp();
-            if (lane == 0)
-              for (int kb = 0; kb < nkb; ++kb) mbar_arrive(&ringEmpty[(itb + kb) % S]);
-          }
-          const int vl = i * kTileN + quarter * 32 + lane;  // row within the CTA range
-          finish_unit(pr, vl, vl < main_rows, i * 4 + quarter);
-        }
-      } else if (tail) {
+      // units of 32 rows: the GEMV warps' tiles i = half, half + 2, ...; the
+      // tail warp's single chunk
+      const int n_units = gemv ? (nt - half + 1) / 2 : tail;
+      for (int n = 0; n < n_units; ++n) {
+        const int i = half + 2 * n;
         float pr[NB][32];
 #pragma unroll
         for (int b = 0; b < NB; ++b)
 #pragma unroll
           for (int j = 0; j < 32; ++j) pr[b][j] = 0.0f;
+        if (!gemv) {
 #pragma unroll
-        for (int rr = 0; rr < 32; ++rr) {
-          const uint4 q = *reinterpret_cast<const uint4*>(sTail + rr * (kGRank * 2) + lane * 16);
-          gemv8<NB>(q, u, B, pr, rr);
+          for (int rr = 0; rr < 32; ++rr) {
+            if (rr == 16) asm volatile("" ::: "memory");
+            const uint4 q = *reinterpret_cast<const uint4*>(sTail + rr * (kGRank * 2) + lane * 16);
+            gemv8<NB>(q, u, B, pr, rr);
+          }
+        } else if (i < nres) {
+          // eight 16-column groups (4 rows each), the next group's
+          // tcgen05.ld in flight while the current one is multiplied
+          const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128);
+          uint32_t wa[16], wb[16];
+          tmem_ld16_issue(ta, wa);
+          tmem_ld16_wait(wa);
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            uint32_t (&cur)[16] = (g & 1) ? wb : wa;
+            uint32_t (&nxt)[16] = (g & 1) ? wa : wb;
+            if (g + 1 < 8) tmem_ld16_issue(ta + (uint32_t)((g + 1) * 16), nxt);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              gemv8<NB>(make_uint4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]), u, B, pr,
+                        g * 4 + j);
+            if (g + 1 < 8) tmem_ld16_wait(nxt);
+          }
+        } else {
+          const int itb = (k * nstream + (i - nres)) * nkb;
+          for (int kb = 0; kb < nkb; ++kb) {
+            const int it = itb + kb;
+            ok = ok && mbar_wait_spin(&ringFull[it % S], (uint32_t)(it / S) & 1u);
+          }
+          const uint8_t* stg = sRing + ((itb + kb_l) % S) * kStageBytes;
+          // two halves of 16 rows: the barrier keeps the compiler from
+          // hoisting all 32 shared loads (128 registers) at once
+#pragma unroll
+          for (int rr = 0; rr < 32; ++rr) {
+            if (rr == 16) asm volatile("" ::: "memory");
+            const int m = quarter * 32 + rr;
+            const uint4 q = *reinterpret_cast<const uint4*>(stg + m * 128 + ((j8 ^ (m & 7)) << 4));
+            gemv8<NB>(q, u, B, pr, rr);
+          }
+          __syncwarp();
+          if (lane == 0)
+            for (int kb = 0; kb < nkb; ++kb) mbar_arrive(&ringEmpty[(itb + kb) % S]);
         }
-        const int vl = main_rows + lane;
-        finish_unit(pr, vl, vl < nrows, mainc);
+        // row within the CTA range, its validity and its chunk
+        const int vl = gemv ? i * kTileN + quarter * 32 + lane : main_rows + lane;
+        const bool valid = vl < (gemv ? main_rows : nrows);
+        finish_unit(pr, vl, valid, gemv ? i * 4 + quarter : mainc);
       }
       if (!ok) {
         *s_abort = 1;
@@ -1105,23 +1117,25 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       if (gemv && cw < B) {
         const int b = cw;
         const unsigned long long* cr = rec.cta + (((size_t)par * B + b) * G) * 2;
+        // one warp per CTA polls; a poll is one round of loads (no back-off: the
+        // reads are a few KB per round across the grid)
         const int per = (G + 31) / 32;
         const int c0 = min(lane * per, G), c1 = min(c0 + per, G);
-        float2 q[kPMaxG / 32];
+        float2 q[kGPerLane];
         unsigned pend = 0;
 #pragma unroll
-        for (int i = 0; i < kPMaxG / 32; ++i) {
+        for (int i = 0; i < kGPerLane; ++i) {
           q[i] = make_float2(-CUDART_INF_F, 0.0f);
           if (c0 + i < c1) pend |= 1u << i;
         }
         const uint64_t tstart = global_timer_ns();
         for (;;) {
-          ulonglong2 m[kPMaxG / 32];
+          ulonglong2 m[kGPerLane];
 #pragma unroll
-          for (int i = 0; i < kPMaxG / 32; ++i)
+          for (int i = 0; i < kGPerLane; ++i)
             if (pend & (1u << i)) m[i] = ld_rec2(cr + 2 * (c0 + i));
 #pragma unroll
-          for (int i = 0; i < kPMaxG / 32; ++i) {
+          for (int i = 0; i < kGPerLane; ++i) {
             if ((pend & (1u << i)) && (uint32_t)(m[i].x >> 32) == seq && (uint32_t)(m[i].y >> 32) == seq) {
               q[i] = make_float2(__uint_as_float((uint32_t)m[i].x), __uint_as_float((uint32_t)m[i].y));
               pend &= ~(1u << i);
@@ -1135,15 +1149,14 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             }
             break;
           }
-          __nanosleep(32);
         }
         float mx = -CUDART_INF_F;
 #pragma unroll
-        for (int i = 0; i < kPMaxG / 32; ++i) mx = fmaxf(mx, q[i].x);
+        for (int i = 0; i < kGPerLane; ++i) mx = fmaxf(mx, q[i].x);
         const float M = warp_max(mx);
         double wsum = 0.0;
 #pragma unroll
-        for (int i = 0; i < kPMaxG / 32; ++i) wsum += partial_weight(q[i], M, it2[b]);
+        for (int i = 0; i < kGPerLane; ++i) wsum += partial_weight(q[i], M, it2[b]);
         const double incl = warp_incl_scan_d(wsum);
         const double Z = __shfl_sync(0xffffffffu, incl, 31);
         const double T = (double)p.u_draft[(size_t)b * K + k] * Z;
@@ -1155,7 +1168,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         {
           double cum = start;
 #pragma unroll
-          for (int i = 0; i < kPMaxG / 32; ++i) {
+          for (int i = 0; i < kGPerLane; ++i) {
             const double w = partial_weight(q[i], M, it2[b]);
             if (pick < 0 && w > 0.0) {
               lastp = c0 + i;
@@ -1243,7 +1256,8 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         }
       }
       // one thread per request waits for the token; every warp then loads its U[x] slice
-      if (cw == 0 && lane < B) {
+      // (after the last position nothing waits for it)
+      if (cw == 0 && lane < B && k + 1 < K) {
         unsigned long long v;
         bool to = false;
         backoff_spin_u64(rec.tok + lane, seq, &v, &to);
@@ -1269,7 +1283,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, kPTmemCols);
+  if (warp == 0) tmem_dealloc(tmem, kPTmemCols);
 }
 
 // ---------------------------------------------------------------------------

@@ -13,6 +13,8 @@
 namespace dspark {
 
 constexpr int kPrefixThreads = 1024;
+constexpr int kPrefixThreadsSmall = 128;   // for at most kPrefixSmallCand candidates
+constexpr int kPrefixSmallCand = 1024;
 constexpr int kMaxCand = 8192;
 
 // Piecewise-linear cost (ms) of a verify batch of n tokens, extended
@@ -30,7 +32,8 @@ __device__ __forceinline__ bool cand_before(double sa, int ia, double sb, int ib
   return sa > sb || (sa == sb && ia < ib);
 }
 
-__global__ void __launch_bounds__(kPrefixThreads)
+template <int kT>
+__global__ void __launch_bounds__(kT)
 prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
               const float* __restrict__ cost_tokens, const float* __restrict__ cost_ms, int n_pts,
               int B, int K, int enable, float* __restrict__ c_out, float* __restrict__ s_out,
@@ -47,8 +50,9 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   __shared__ int s_stop;
   const int tid = threadIdx.x;
 
+  if (tid == 0) *flags = 0u;  // status of this call
   // cost table into shared memory; it must be ascending in tokens
-  for (int i = tid; i < n_pts; i += kPrefixThreads) {
+  for (int i = tid; i < n_pts; i += kT) {
     s_xs[i] = cost_tokens[i];
     s_ys[i] = cost_ms[i];
   }
@@ -60,21 +64,26 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     s_stop = n;
   }
 
-  // c = sigmoid(z / T_k) and survival = running product over k, in fp64
-  for (int b = tid; b < B; b += kPrefixThreads) {
+  // c = sigmoid(z / T_k), one candidate per thread, in fp64
+  for (int o = tid; o < n; o += kT) {
+    const int b = o / K, k = o - b * K;
+    const double ck = 1.0 / (1.0 + exp(-(double)z[o] / (double)temps[k]));
+    c_out[o] = (float)ck;
+    key[k * B + b] = ck;
+  }
+  __syncthreads();
+  // survival = running product over k (one thread per request)
+  for (int b = tid; b < B; b += kT) {
     double run = 1.0;
     for (int k = 0; k < K; ++k) {
-      const size_t o = (size_t)b * K + k;
-      const double ck = 1.0 / (1.0 + exp(-(double)z[o] / (double)temps[k]));
-      run *= ck;
-      c_out[o] = (float)ck;
-      s_out[o] = (float)run;
+      run *= key[k * B + b];
+      s_out[(size_t)b * K + k] = (float)run;
       key[k * B + b] = run;
       idx[k * B + b] = k * B + b;
     }
     lcount[b] = 0;
   }
-  for (int i = n + tid; i < npad; i += kPrefixThreads) {
+  for (int i = n + tid; i < npad; i += kT) {
     key[i] = -1.0;  // padding sorts last
     idx[i] = 0x7fffffff;
   }
@@ -82,9 +91,9 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
 
   if (!enable) {
     double e = 0.0;
-    for (int i = tid; i < n; i += kPrefixThreads) e += key[i];
-    const double E = (double)B + block_sum_d<kPrefixThreads>(e, shd);
-    for (int b = tid; b < B; b += kPrefixThreads) verify_len[b] = K;
+    for (int i = tid; i < n; i += kT) e += key[i];
+    const double E = (double)B + block_sum_d<kT>(e, shd);
+    for (int b = tid; b < B; b += kT) verify_len[b] = K;
     if (tid == 0) {
       const double t = cost_at(s_xs, s_ys, n_pts, (double)B + (double)n);
       if (!(t > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
@@ -96,7 +105,7 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   // bitonic sort of (key, idx) in the order of cand_before
   for (int size = 2; size <= npad; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < npad; i += kPrefixThreads) {
+      for (int i = tid; i < npad; i += kT) {
         const int j = i ^ stride;
         if (j > i) {
           const bool up = (i & size) == 0;  // this half sorts in cand_before order
@@ -114,12 +123,12 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   }
 
   // E_i = B + sum of the first i survivals; each thread owns a contiguous run
-  const int per = npad / kPrefixThreads > 0 ? npad / kPrefixThreads : 1;
+  const int per = npad / kT > 0 ? npad / kT : 1;
   const int i0 = tid * per;
   double run = 0.0;
   for (int i = i0; i < i0 + per && i < n; ++i) run += key[i];
   double total;
-  const double excl = block_excl_scan_d<kPrefixThreads>(run, shd, &total);
+  const double excl = block_excl_scan_d<kT>(run, shd, &total);
   // candidate i (0-based) raises the objective iff E_{i+1}/t(B+i+1) > E_i/t(B+i)
   double E = (double)B + excl;
   for (int i = i0; i < i0 + per && i < n; ++i) {
@@ -135,9 +144,9 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   }
   __syncthreads();
   const int n_commit = s_stop;
-  for (int i = tid; i < n_commit; i += kPrefixThreads) atomicAdd(&lcount[idx[i] % B], 1);
+  for (int i = tid; i < n_commit; i += kT) atomicAdd(&lcount[idx[i] % B], 1);
   __syncthreads();
-  for (int b = tid; b < B; b += kPrefixThreads) verify_len[b] = lcount[b];
+  for (int b = tid; b < B; b += kT) verify_len[b] = lcount[b];
   // objective of the committed set: E at n_commit from the owning thread's run
   const bool owner = (n_commit == n) ? (tid == 0) : (n_commit >= i0 && n_commit < i0 + per);
   if (owner) {
