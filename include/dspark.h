@@ -255,18 +255,30 @@ dspark_status dspark_verify_noalloc(
  * to DSPARK_OK / DSPARK_ERR_TIMEOUT / DSPARK_ERR_DEVICE_DATA. */
 dspark_status dspark_get_device_status(const void *workspace, void *stream);
 
-/* Synchronises `stream`; returns the raw DSPARK_FLAG_* bits (or -1 on a
- * CUDA error). */
+/* Synchronises `stream`; returns the status word of the last call made
+ * with this workspace, low 31 bits (the DSPARK_FLAG_* bits), or -1 on a
+ * CUDA error.  A workspace no call has used yet holds no status word: what
+ * this returns for it is meaningless. */
 int dspark_get_device_flags(const void *workspace, void *stream);
 
 /* Static string for a status code. */
 const char *dspark_status_string(dspark_status s);
 
 /* Name of the draft projection path these sizes take:
- * "tcgen05-persistent" (bf16, B <= 16: all K positions in one launch),
- * "tcgen05" (bf16, B > 16: one launch per position) or "cuda-core"
- * (fp32 U/W, or shapes outside the tensor-core paths). */
+ * "persistent-cuda-core" (bf16, r = 256, B <= 2: all K positions in one
+ * launch, GEMV on the CUDA cores), "tcgen05-persistent" (bf16, B <= 16: all
+ * K positions in one launch), "tcgen05" (bf16, B > 16: one launch per
+ * position) or "cuda-core" (fp32 U/W, or shapes outside those paths). */
 const char *dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype);
+
+/* Name of the path dspark_verify takes for these sizes, with (have_bias
+ * != 0) or without the draft's bias rows: "single-launch" (B <= 4, at most
+ * 72 verified rows, bias rows given: one cooperative kernel), "staged-bias"
+ * (four kernels, the residual row rebuilt from the bias rows),
+ * "staged-tcgen05" or "staged-cuda-core" (four kernels, the residual row
+ * re-projected from U and W on the tensor or CUDA cores).  Same results
+ * either way, up to floating-point summation order. */
+const char *dspark_verify_path(int V, int r, int B, int K, dspark_dtype uw_dtype, int have_bias);
 
 /* Library ABI version (major*100 + minor). */
 int dspark_version(void);

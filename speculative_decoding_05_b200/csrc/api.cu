@@ -14,6 +14,7 @@
 #include "draft_persist.cuh"
 #include "sample.cuh"
 #include "verify.cuh"
+#include "verify_fused.cuh"
 
 using namespace dspark;
 
@@ -44,11 +45,15 @@ DraftWs draft_ws(int V, int B) {
 // Workspace of the verify: header, target partials [B*(K+1)][n_segs],
 // ResInfo [B], residual partials [B][n_chunks].
 struct VerifyWs {
-  size_t tpart_off, info_off, rpart_off, total;
+  size_t frec_off, frec_bytes, tpart_off, info_off, rpart_off, total;
 };
+// Header, then the records of the fused small-batch verify (cleared together
+// with the header, one memset), then the buffers of the multi-kernel path.
 VerifyWs verify_ws(int V, int B, int K) {
   VerifyWs w;
-  w.tpart_off = kHeaderBytes;
+  w.frec_off = kHeaderBytes;
+  w.frec_bytes = fused_verify_ok(V, B, K, true) ? align256(fused_rec_bytes(V, B, K)) : 0;
+  w.tpart_off = w.frec_off + w.frec_bytes;
   w.info_off = w.tpart_off + align256((size_t)B * (K + 1) * n_segs_of(V) * sizeof(float2));
   w.rpart_off = w.info_off + align256((size_t)B * sizeof(ResInfo));
   w.total = w.rpart_off + align256((size_t)B * n_chunks_of(V) * sizeof(float2));
@@ -190,7 +195,7 @@ dspark_status draft_impl(const float* base, const void* U, const void* W, dspark
     a.n_tiles = (V + kTileN - 1) / kTileN;
     GemvRecs recs;
     recs.cta = reinterpret_cast<unsigned long long*>(ws + w.rec_off);
-    recs.tok = recs.cta + (size_t)2 * B * kPMaxG * 2;
+    recs.tok = recs.cta + gemv_rec_words_cta(B);
     if (gemv_path(r, B) &&
         cudaMemsetAsync(ws + w.rec_off, 0, gemv_rec_bytes(B), s) != cudaSuccess)
       return DSPARK_ERR_CUDA;
@@ -228,10 +233,56 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
                           int32_t* last, unsigned char* ws, cudaStream_t s) {
   const VerifyWs w = verify_ws(V, B, K);
   unsigned* flags = reinterpret_cast<unsigned*>(ws);
+  const int nc = n_chunks_of(V);
+  const int G = fused_grid(nc);
+  if (dbias != nullptr && w.frec_bytes > 0 && G > 0) {
+    // one cooperative launch; its records are cleared with the status word
+    if (cudaMemsetAsync(ws, 0, kHeaderBytes + w.frec_bytes, s) != cudaSuccess) return DSPARK_ERR_CUDA;
+    FusedArgs a;
+    a.target = target;
+    a.n_rows = n_rows;
+    a.row_start = row_start;
+    a.verify_len = vlen;
+    a.base = base;
+    a.draft_bias = dbias;
+    a.inv_temp = it;
+    a.prev_token = prev;
+    a.tokens = tokens;
+    a.p_tok = p_tok;
+    a.ref_max = rmax;
+    a.ref_sum = rsum;
+    a.u_accept = ua;
+    a.u_res = ur;
+    a.n_accepted = n_acc;
+    a.out_tokens = out;
+    a.last_token = last;
+    a.flags = flags;
+    a.seg_rec = reinterpret_cast<unsigned long long*>(ws + w.frec_off);
+    a.tot_rec = a.seg_rec + fused_seg_words(V, B, K);
+    a.V = V;
+    a.B = B;
+    a.K = K;
+    a.n_seg = fused_n_seg(V);
+    a.n_chunks = nc;
+    a.mstride = fused_mstride(V, B, K, G);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kFThreads);
+    cfg.stream = s;
+    cudaLaunchAttribute attrs[1];
+    attrs[0].id = cudaLaunchAttributeCooperative;
+    attrs[0].val.cooperative = 1;
+    cfg.attrs = attrs;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, verify_fused_kernel, a) != cudaSuccess) return DSPARK_ERR_CUDA;
+    return check_launch();
+  }
+  dspark_status st0 = clear_status(ws, s);
+  if (st0 != DSPARK_OK) return st0;
   float2* tpart = reinterpret_cast<float2*>(ws + w.tpart_off);
   ResInfo* info = reinterpret_cast<ResInfo*>(ws + w.info_off);
   float2* rpart = reinterpret_cast<float2*>(ws + w.rpart_off);
-  const int ns = n_segs_of(V), nc = n_chunks_of(V);
+  const int ns = n_segs_of(V);
   dim3 sgrid(ns, B * (K + 1));
   target_stats_kernel<<<sgrid, kStatsThreads, 0, s>>>(target, n_rows, row_start, vlen, it, V, K,
                                                        tpart, ns, flags);
@@ -314,6 +365,12 @@ const char* dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype)
   return use_tc(V, r, B, uw_dtype) ? "tcgen05" : "cuda-core";
 }
 
+const char* dspark_verify_path(int V, int r, int B, int K, dspark_dtype uw_dtype, int have_bias) {
+  if (fused_verify_ok(V, B, K, have_bias != 0) && fused_grid(n_chunks_of(V)) > 0) return "single-launch";
+  if (have_bias) return "staged-bias";
+  return use_tc(V, r, B, uw_dtype) ? "staged-tcgen05" : "staged-cuda-core";
+}
+
 size_t dspark_draft_workspace_size(int V, int r, int B, int K) {
   (void)r;
   (void)K;
@@ -388,7 +445,7 @@ dspark_status dspark_verify(const float* target_logits, int64_t n_target_rows,
       !aligned(W, 16))
     return DSPARK_ERR_INVALID_ARG;
   if ((long long)B * (K + 1) > (1ll << 31) - 1) return DSPARK_ERR_UNSUPPORTED;
-  if ((st = clear_status(workspace, s)) != DSPARK_OK) return st;
+  // verify_impl clears the status word (and its records) before its kernels
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   if (uw_dtype == DSPARK_BF16)
     return verify_impl<__nv_bfloat16>(target_logits, n_target_rows, row_start, verify_len,
@@ -442,7 +499,7 @@ int dspark_get_device_flags(const void* workspace, void* stream) {
   unsigned h = 0;
   if (cudaMemcpyAsync(&h, workspace, sizeof h, cudaMemcpyDeviceToHost, s) != cudaSuccess) return -1;
   if (cudaStreamSynchronize(s) != cudaSuccess) return -1;
-  return (int)h;
+  return (int)(h & 0x7fffffffu);  // -1 stays reserved for CUDA errors
 }
 
 dspark_status dspark_get_device_status(const void* workspace, void* stream) {

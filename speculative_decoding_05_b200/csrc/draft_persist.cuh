@@ -106,6 +106,10 @@ constexpr int kGTailBytes = kChunk * kGRank * 2;    // 16 KB: the tail chunk's W
 constexpr int kGMaxChunks = 64;                     // chunks of one CTA (two per lane in level 2)
 constexpr int kGPerLane = 5;                        // CTA partials per lane in level 1
 constexpr int kGMaxG = 32 * kGPerLane;              // grid limit of the GEMV variant
+// Each CTA's partial record sits on its own 128-byte line: with 148 pollers
+// reading every record, records that share lines slow the exchange several
+// fold (the writes queue behind the reads of the shared line).
+constexpr int kGRecWords = 16;                      // 8-byte words per record line
 
 // First chunk of CTA c: runs balanced to within one chunk.
 __host__ __device__ inline int gemv_chunk_begin(int cta, int G, int n_chunks) {
@@ -808,8 +812,8 @@ __device__ __forceinline__ void load_u_slice(const __nv_bfloat16* U, const int (
 }
 
 struct GemvRecs {
-  unsigned long long* cta;  // [2][B][G][2]: {M, seq}, {S, seq}
-  unsigned long long* tok;  // [B]: {position + 1, token}
+  unsigned long long* cta;  // [2][B][G][16]: {M, seq}, {S, seq}, then padding to 128 B
+  unsigned long long* tok;  // [B][16]: {position + 1, token}, then padding
 };
 
 __device__ __forceinline__ void backoff_spin_u64(const unsigned long long* p, uint32_t seq,
@@ -874,6 +878,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [kGSlots][kGMaxB]
   float* s_ws = s_wm + kGSlots * kGMaxB;                  // [kGSlots][kGMaxB]
   volatile int* s_i = reinterpret_cast<volatile int*>(s_ws + kGSlots * kGMaxB);  // [4]
+  float* s_ud = const_cast<float*>(reinterpret_cast<volatile float*>(s_i + 4));   // [B][K] draft uniforms
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -981,6 +986,9 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         *reinterpret_cast<uint4*>(sTail + rr * (kGRank * 2) + lane * 16) = val;
       }
     }
+    // the draft uniforms of every position, staged so the sampling step
+    // never waits on a global load
+    for (int i = threadIdx.x - kGTailWarp * 32; i < B * K; i += kGSyncThreads) s_ud[i] = p.u_draft[i];
     // U[prev_token] slice of this lane
     uint32_t u[NB][4];
     {
@@ -1108,7 +1116,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         float M = -CUDART_INF_F, Sm = 0.0f;
         for (int w2 = 0; w2 < kGSlots; ++w2)
           merge_partial(M, Sm, s_wm[w2 * kGMaxB + b], s_ws[w2 * kGMaxB + b], it2[b]);
-        unsigned long long* r0 = rec.cta + (((size_t)par * B + b) * G + cta) * 2;
+        unsigned long long* r0 = rec.cta + (((size_t)par * B + b) * G + cta) * kGRecWords;
         st_rec(r0, __float_as_uint(M), seq);
         st_rec(r0 + 1, __float_as_uint(Sm), seq);
       }
@@ -1116,7 +1124,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       // the CTA that holds the sample resolves chunk and token
       if (gemv && cw < B) {
         const int b = cw;
-        const unsigned long long* cr = rec.cta + (((size_t)par * B + b) * G) * 2;
+        const unsigned long long* cr = rec.cta + (((size_t)par * B + b) * G) * kGRecWords;
         // one warp per CTA polls; a poll is one round of loads (no back-off: the
         // reads are a few KB per round across the grid)
         const int per = (G + 31) / 32;
@@ -1133,7 +1141,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           ulonglong2 m[kGPerLane];
 #pragma unroll
           for (int i = 0; i < kGPerLane; ++i)
-            if (pend & (1u << i)) m[i] = ld_rec2(cr + 2 * (c0 + i));
+            if (pend & (1u << i)) m[i] = ld_rec2(cr + (size_t)kGRecWords * (c0 + i));
 #pragma unroll
           for (int i = 0; i < kGPerLane; ++i) {
             if ((pend & (1u << i)) && (uint32_t)(m[i].x >> 32) == seq && (uint32_t)(m[i].y >> 32) == seq) {
@@ -1159,7 +1167,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         for (int i = 0; i < kGPerLane; ++i) wsum += partial_weight(q[i], M, it2[b]);
         const double incl = warp_incl_scan_d(wsum);
         const double Z = __shfl_sync(0xffffffffu, incl, 31);
-        const double T = (double)p.u_draft[(size_t)b * K + k] * Z;
+        const double T = (double)s_ud[b * K + k] * Z;
         double start = __shfl_up_sync(0xffffffffu, incl, 1);
         if (lane == 0) start = 0.0;
         const unsigned own = __ballot_sync(0xffffffffu, start <= T && T < incl && wsum > 0.0);
@@ -1252,7 +1260,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             }
           }
           // publish {position, token}
-          if (lane == 0) st_rec(rec.tok + b, (uint32_t)x, seq);
+          if (lane == 0) st_rec(rec.tok + (size_t)b * kGRecWords, (uint32_t)x, seq);
         }
       }
       // one thread per request waits for the token; every warp then loads its U[x] slice
@@ -1260,7 +1268,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       if (cw == 0 && lane < B && k + 1 < K) {
         unsigned long long v;
         bool to = false;
-        backoff_spin_u64(rec.tok + lane, seq, &v, &to);
+        backoff_spin_u64(rec.tok + (size_t)lane * kGRecWords, seq, &v, &to);
         if (to) {
           *s_abort = 1;
           raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
@@ -1356,9 +1364,11 @@ inline dspark_status persist_launch(const CUtensorMap& tm_w, PersistArgs a, Gemv
 }
 
 // Bytes of the position records of the GEMV variant (zeroed by the caller
-// before each call): CTA partials [2][B][G][2], token words [B].
+// before each call): CTA partials [2][B][G] and token words [B], one
+// 128-byte line each.
+inline size_t gemv_rec_words_cta(int B) { return (size_t)2 * B * kGMaxG * kGRecWords; }
 inline size_t gemv_rec_bytes(int B) {
-  return (size_t)2 * B * kPMaxG * 2 * 8 + (size_t)B * 8 + 256;
+  return (gemv_rec_words_cta(B) + (size_t)B * kGRecWords) * 8;
 }
 
 }  // namespace dspark

@@ -1,0 +1,534 @@
+// verify_fused.cuh -- the whole rejection-sampling verify of a few requests
+// (B <= 4, at most 72 verified rows) in one cooperative launch, used when the
+// draft's bias rows are kept so the residual needs no projection.
+//
+// Same arithmetic as the multi-kernel path (target_stats_kernel,
+// accept_kernel, residual_bias_kernel, residual_sample_kernel), reorganised
+// so that one launch replaces four and the only grid-wide waits are two
+// rounds of polling on records that carry their own validity word:
+//   phase 1  target-row statistics: every verified row is cut into
+//            1024-element segments, one warp per segment (max, then
+//            sum of 2^((t - max) * log2e / T)); each segment's pair is
+//            stored as two 8-byte words {value, 1}, in a block of lines that
+//            only this CTA writes (records of several CTAs on one line, polled
+//            by every CTA, slow the exchange several fold);
+//   phase 2  every CTA polls all segment pairs, forms each row's
+//            (max, partition sum) and runs the accept scan of every request
+//            itself, so no second exchange is needed for it; CTA 0 writes
+//            n_accepted and the accepted / -1 entries of out_tokens;
+//   phase 3  residual partials max(0, p_t - p_d) (or p_t for a bonus draw)
+//            over this CTA's run of 32-row chunks; per request the CTA's
+//            totals (fp64) are stored as four words {32-bit half, 1} on a
+//            line of their own;
+//   phase 4  the warp of request b polls every CTA's totals, finds the CTA
+//            whose run holds the sample, and only that CTA resolves chunk and
+//            token (two more scans over its own data) and writes the
+//            correction / bonus token.
+// The records are zeroed by the caller before the launch (a record is valid
+// once its high word is 1).  Every wait has the 2 s limit of the library;
+// running out raises DSPARK_FLAG_TIMEOUT and the kernel finishes with
+// whatever it has.
+#pragma once
+
+#include "proj_tc.cuh"
+#include "sample.cuh"
+#include "tc_common.cuh"
+#include "verify.cuh"
+
+namespace dspark {
+
+constexpr int kFThreads = 512;
+constexpr int kFWarps = kFThreads / 32;
+constexpr int kFMaxB = 4;
+constexpr int kFMaxRows = 72;              // B * (K + 1)
+constexpr int kFSeg = 1024;                // target elements of one phase-1 segment (one warp)
+constexpr int kFSegPerLane = 8;            // row statistics: V <= 32 * 8 * 1024
+constexpr int kFPerLane = 5;               // CTA totals per lane: grid <= 160
+constexpr int kFMaxG = 32 * kFPerLane;
+constexpr int kFMaxChunks = 64;            // residual chunks of one CTA (two per lane)
+
+struct FusedArgs {
+  const float* target;
+  long long n_rows;
+  const int64_t* row_start;
+  const int32_t* verify_len;
+  const float* base;
+  const float* draft_bias;
+  const float* inv_temp;
+  const int32_t* prev_token;
+  const int32_t* tokens;
+  const float* p_tok;
+  const float* ref_max;
+  const float* ref_sum;
+  const float* u_accept;
+  const float* u_res;
+  int32_t* n_accepted;
+  int32_t* out_tokens;
+  int32_t* last_token;
+  unsigned* flags;
+  unsigned long long* seg_rec;  // [G][mstride][2]: segment t at (t % G, t / G): {M, 1}, {S, 1}
+  unsigned long long* tot_rec;  // [B][G][16]: halves of Q and P (fp64), each {half, 1}; padding
+  int V, B, K, n_seg, n_chunks;
+  int mstride;                  // record slots per CTA block (a multiple of 8: whole lines)
+};
+
+inline int fused_n_seg(int V) { return (V + kFSeg - 1) / kFSeg; }
+// Record slots per CTA block for a grid of G.
+inline int fused_mstride(int V, int B, int K, int G) {
+  const int n_items = B * (K + 1) * fused_n_seg(V);
+  return ((n_items + G - 1) / G + 7) / 8 * 8;
+}
+// Words of the segment records for any grid up to kFMaxG (G * mstride <=
+// n_items + 8 G), then the totals.
+inline size_t fused_seg_words(int V, int B, int K) {
+  const size_t w = ((size_t)B * (K + 1) * fused_n_seg(V) + 8 * kFMaxG) * 2;
+  return (w + 15) / 16 * 16;  // the totals start on a line boundary
+}
+// Bytes of the records of the fused verify (zeroed before each call).
+inline size_t fused_rec_bytes(int V, int B, int K) {
+  return fused_seg_words(V, B, K) * 8 + (size_t)B * kFMaxG * 128;
+}
+inline bool fused_verify_ok(int V, int B, int K, bool have_bias) {
+  const int n_seg = fused_n_seg(V);
+  return have_bias && B >= 1 && B <= kFMaxB && B * (K + 1) <= kFMaxRows &&
+         n_seg <= 32 * kFSegPerLane;
+}
+
+// Grid of the fused verify (one CTA per SM), or 0 when a CTA's run of
+// chunks would not fit its scan.
+inline int fused_grid(int n_chunks) {
+  int G = num_sms();
+  if (G > kFMaxG) G = kFMaxG;
+  return (n_chunks + G - 1) / G <= kFMaxChunks ? G : 0;
+}
+
+__device__ __forceinline__ void st_pair(unsigned long long* p, uint32_t a, uint32_t b) {
+  const unsigned long long x = (1ull << 32) | a, y = (1ull << 32) | b;
+  asm volatile("st.relaxed.gpu.global.v2.u64 [%0], {%1, %2};" ::"l"(p), "l"(x), "l"(y) : "memory");
+}
+__device__ __forceinline__ ulonglong2 ld_pair(const unsigned long long* p) {
+  ulonglong2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(v.x), "=l"(v.y) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ bool pair_valid(ulonglong2 v) {
+  return (uint32_t)(v.x >> 32) == 1u && (uint32_t)(v.y >> 32) == 1u;
+}
+
+__global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedArgs a) {
+  __shared__ int s_rofs[kFMaxB + 1];  // first flat row of request b; s_rofs[B] = rows
+  __shared__ int s_len[kFMaxB];
+  __shared__ float s_it2[kFMaxB];
+  __shared__ int s_prev[kFMaxB];
+  __shared__ float s_tmax[kFMaxRows];
+  __shared__ double s_tz[kFMaxRows];
+  __shared__ float s_tx[kFMaxRows];    // target logit of the drafted token (p < L)
+  __shared__ int s_tok[kFMaxRows];     // drafted token (p < K)
+  __shared__ float s_pd[kFMaxRows];    // its draft probability
+  __shared__ float s_ua[kFMaxRows];    // its accept uniform
+  __shared__ float s_dmax[kFMaxRows];  // draft reference max / sum of position p
+  __shared__ float s_dsum[kFMaxRows];
+  __shared__ ResInfo s_ri[kFMaxB];
+  __shared__ float2 s_chunk[kFMaxB][kFMaxChunks];
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x, cta = blockIdx.x;
+  const int B = a.B, K = a.K, V = a.V, n_seg = a.n_seg;
+
+  if (tid == 0) {
+    int r = 0;
+    for (int b = 0; b < B; ++b) {
+      const int L = checked_len(a.verify_len, b, K, a.flags);
+      s_rofs[b] = r;
+      s_len[b] = L;
+      s_it2[b] = checked_inv_temp(a.inv_temp, b, a.flags) * kLog2e;
+      s_prev[b] = checked_token(a.prev_token[b], V, true, a.flags);
+      r += L + 1;
+    }
+    s_rofs[B] = r;
+  }
+  __syncthreads();
+  const int R = s_rofs[B];
+  auto row_of = [&](int rho, int* pb) {
+    int b = 0;
+    while (b + 1 < B && rho >= s_rofs[b + 1]) ++b;
+    *pb = b;
+    return rho - s_rofs[b];
+  };
+
+  // per-row inputs of the accept scan, loaded now and stored after phase 1
+  float g_tx = 0.0f, g_pd = 1.0f, g_ua = 0.0f, g_dmax = 0.0f, g_dsum = 1.0f;
+  int g_tok = 0;
+  if (tid < R) {
+    int b;
+    const int p = row_of(tid, &b);
+    if (p < K) {
+      const size_t o = (size_t)b * K + p;
+      g_dmax = a.ref_max[o];
+      g_dsum = a.ref_sum[o];
+      if (p < s_len[b]) {
+        g_tok = checked_token(a.tokens[o], V, false, a.flags);
+        const long long row = checked_row(a.row_start, b, p, a.n_rows, a.flags);
+        g_tx = a.target[(size_t)row * V + g_tok];
+        g_pd = a.p_tok[o];
+        g_ua = a.u_accept[o];
+      }
+    }
+  }
+
+  // ---------------------------------------------------------------- phase 1
+  {
+    const int n_items = R * n_seg;
+    const int stride = G * kFWarps;
+    for (int t0 = cta + G * warp; t0 < n_items; t0 += 2 * stride) {
+      float4 x[2][8];
+      float it2v[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = t0 + h * stride;
+        it2v[h] = kLog2e;
+        if (t < n_items) {
+          const int rho = t / n_seg, s = t - rho * n_seg;
+          int b;
+          const int p = row_of(rho, &b);
+          it2v[h] = s_it2[b];
+          const long long row = checked_row(a.row_start, b, p, a.n_rows, a.flags);
+          const float* trow = a.target + (size_t)row * V;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int e = s * kFSeg + (i * 32 + lane) * 4;
+            x[h][i] = (e < V) ? __ldg(reinterpret_cast<const float4*>(trow + e))
+                              : make_float4(-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F);
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t = t0 + h * stride;
+        if (t >= n_items) break;
+        float m = -CUDART_INF_F;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fmaxf(x[h][i].x, x[h][i].y), fmaxf(x[h][i].z, x[h][i].w)));
+        const float M = warp_max(m);
+        float sl = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          sl += ex2((x[h][i].x - M) * it2v[h]) + ex2((x[h][i].y - M) * it2v[h]) +
+                ex2((x[h][i].z - M) * it2v[h]) + ex2((x[h][i].w - M) * it2v[h]);
+        const double S = warp_sum_d((double)sl);
+        if (lane == 0)
+          st_pair(a.seg_rec + ((size_t)(t % G) * a.mstride + t / G) * 2, __float_as_uint(M),
+                  __float_as_uint((float)S));
+      }
+    }
+  }
+  if (tid < R) {
+    s_tx[tid] = g_tx;
+    s_tok[tid] = g_tok;
+    s_pd[tid] = g_pd;
+    s_ua[tid] = g_ua;
+    s_dmax[tid] = g_dmax;
+    s_dsum[tid] = g_dsum;
+  }
+
+  // ---------------------------------------------------------------- phase 2
+  for (int rho = warp; rho < R; rho += kFWarps) {
+    int b;
+    (void)row_of(rho, &b);
+    const float it2 = s_it2[b];
+    float2 q[kFSegPerLane];
+    unsigned pend = 0;
+#pragma unroll
+    for (int i = 0; i < kFSegPerLane; ++i) {
+      q[i] = make_float2(-CUDART_INF_F, 0.0f);
+      if (lane + 32 * i < n_seg) pend |= 1u << i;
+    }
+    const uint64_t tstart = global_timer_ns();
+    for (;;) {
+      ulonglong2 m[kFSegPerLane];
+#pragma unroll
+      for (int i = 0; i < kFSegPerLane; ++i)
+        if (pend & (1u << i)) {
+          const int t = rho * n_seg + lane + 32 * i;
+          m[i] = ld_pair(a.seg_rec + ((size_t)(t % G) * a.mstride + t / G) * 2);
+        }
+#pragma unroll
+      for (int i = 0; i < kFSegPerLane; ++i) {
+        if ((pend & (1u << i)) && pair_valid(m[i])) {
+          q[i] = make_float2(__uint_as_float((uint32_t)m[i].x), __uint_as_float((uint32_t)m[i].y));
+          pend &= ~(1u << i);
+        }
+      }
+      if (!__any_sync(0xffffffffu, pend != 0)) break;
+      if (__any_sync(0xffffffffu, global_timer_ns() - tstart > kWaitLimitNs)) {
+        if (lane == 0) raise_flag(a.flags, DSPARK_FLAG_TIMEOUT);
+        break;
+      }
+    }
+    float mx = -CUDART_INF_F;
+#pragma unroll
+    for (int i = 0; i < kFSegPerLane; ++i) mx = fmaxf(mx, q[i].x);
+    const float tmax = warp_max(mx);
+    double z = 0.0;
+#pragma unroll
+    for (int i = 0; i < kFSegPerLane; ++i)
+      if (q[i].y > 0.0f) z += (double)q[i].y * (double)ex2((q[i].x - tmax) * it2);
+    const double tz = warp_sum_d(z);
+    if (lane == 0) {
+      if (!(tz > 0.0) || !isfinite(tz)) raise_flag(a.flags, DSPARK_FLAG_NONFINITE);
+      s_tmax[rho] = tmax;
+      s_tz[rho] = tz;
+    }
+  }
+  __syncthreads();
+
+  // accept scan of request b by warp b (every CTA)
+  if (warp < B) {
+    const int b = warp, L = s_len[b], r0 = s_rofs[b];
+    const float it2 = s_it2[b];
+    int n_acc = L;
+    for (int base_p = 0; base_p <= L; base_p += 32) {
+      const int p = base_p + lane;
+      bool reject = false;
+      if (p < L) {
+        const double pt = (double)ex2((s_tx[r0 + p] - s_tmax[r0 + p]) * it2) / s_tz[r0 + p];
+        const double ratio = pt / (double)s_pd[r0 + p];
+        reject = !((double)s_ua[r0 + p] < ratio);
+      }
+      const unsigned rej = __ballot_sync(0xffffffffu, reject);
+      if (rej) {
+        n_acc = base_p + __ffs(rej) - 1;
+        break;
+      }
+    }
+    const int j = n_acc;
+    if (cta == 0) {
+      for (int p = lane; p <= K; p += 32)
+        if (p != j) a.out_tokens[(size_t)b * (K + 1) + p] = (p < n_acc) ? s_tok[r0 + p] : -1;
+      if (lane == 0) a.n_accepted[b] = n_acc;
+    }
+    if (lane == 0) {
+      ResInfo ri;
+      ri.row = checked_row(a.row_start, b, j, a.n_rows, a.flags);
+      ri.j = j;
+      ri.bonus = (j == L) ? 1 : 0;
+      ri.t_max = s_tmax[r0 + j];
+      ri.t_inv_z = (float)(1.0 / s_tz[r0 + j]);
+      ri.x_prev = -1;
+      ri.d_max = 0.0f;
+      ri.d_inv_z = 0.0f;
+      ri.pad = 0.0f;
+      if (!ri.bonus) {
+        ri.x_prev = (j == 0) ? s_prev[b] : s_tok[r0 + j - 1];
+        ri.d_max = s_dmax[r0 + j];
+        const float zs = s_dsum[r0 + j];
+        if (!(zs > 0.0f) || !isfinite(zs)) raise_flag(a.flags, DSPARK_FLAG_NONFINITE);
+        ri.d_inv_z = 1.0f / zs;
+      }
+      s_ri[b] = ri;
+    }
+  }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- phase 3
+  const int c_begin = (int)((long long)cta * a.n_chunks / G);
+  const int nch = (int)((long long)(cta + 1) * a.n_chunks / G) - c_begin;
+  {
+    const int n_pairs = B * nch;
+    for (int q0 = warp; q0 < n_pairs; q0 += 2 * kFWarps) {
+      float t[2], bv[2], bi[2];
+      int bb[2], lc[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int q = q0 + h * kFWarps;
+        t[h] = 0.0f;
+        bv[h] = 0.0f;
+        bi[h] = 0.0f;
+        bb[h] = 0;
+        lc[h] = 0;
+        if (q < n_pairs) {
+          const int b = q / nch;
+          bb[h] = b;
+          lc[h] = q - b * nch;
+          const int v = (c_begin + lc[h]) * kChunk + lane;
+          if (v < V) {
+            const ResInfo& ri = s_ri[b];
+            t[h] = a.target[(size_t)ri.row * V + v];
+            if (!ri.bonus) {
+              const size_t drow = ((size_t)b * K + ri.j) * (size_t)V;
+              bv[h] = a.base[drow + v];
+              bi[h] = a.draft_bias[drow + v];
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int q = q0 + h * kFWarps;
+        if (q >= n_pairs) break;
+        const int b = bb[h];
+        const int v = (c_begin + lc[h]) * kChunk + lane;
+        float qv = 0.0f, pt = 0.0f;
+        if (v < V) qv = residual_q(t[h], bv[h], bi[h], s_ri[b], s_it2[b], &pt);
+        const float Q = warp_sum(qv), P = warp_sum(pt);
+        if (lane == 0) s_chunk[b][lc[h]] = make_float2(Q, P);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp < B) {
+    const int b = warp;
+    const int ca = 2 * lane, cb = ca + 1;
+    const double q = (ca < nch ? (double)s_chunk[b][ca].x : 0.0) + (cb < nch ? (double)s_chunk[b][cb].x : 0.0);
+    const double pp = (ca < nch ? (double)s_chunk[b][ca].y : 0.0) + (cb < nch ? (double)s_chunk[b][cb].y : 0.0);
+    const double Qc = warp_sum_d(q), Pc = warp_sum_d(pp);
+    if (lane == 0) {
+      unsigned long long* r = a.tot_rec + ((size_t)b * G + cta) * 16;
+      const unsigned long long qb = (unsigned long long)__double_as_longlong(Qc);
+      const unsigned long long pb = (unsigned long long)__double_as_longlong(Pc);
+      st_pair(r, (uint32_t)qb, (uint32_t)(qb >> 32));
+      st_pair(r + 2, (uint32_t)pb, (uint32_t)(pb >> 32));
+    }
+  }
+
+  // ---------------------------------------------------------------- phase 4
+  if (warp < B) {
+    const int b = warp;
+    const ResInfo ri = s_ri[b];
+    const unsigned long long* tr = a.tot_rec + (size_t)b * G * 16;
+    const int per = (G + 31) / 32;
+    const int c0 = min(lane * per, G), c1 = min(c0 + per, G);
+    double wq[kFPerLane], wp[kFPerLane];
+    unsigned pend = 0;
+#pragma unroll
+    for (int i = 0; i < kFPerLane; ++i) {
+      wq[i] = 0.0;
+      wp[i] = 0.0;
+      if (c0 + i < c1) pend |= 1u << i;
+    }
+    const uint64_t tstart = global_timer_ns();
+    for (;;) {
+      ulonglong2 mq[kFPerLane], mp[kFPerLane];
+#pragma unroll
+      for (int i = 0; i < kFPerLane; ++i) {
+        if (pend & (1u << i)) {
+          mq[i] = ld_pair(tr + (size_t)(c0 + i) * 16);
+          mp[i] = ld_pair(tr + (size_t)(c0 + i) * 16 + 2);
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < kFPerLane; ++i) {
+        if ((pend & (1u << i)) && pair_valid(mq[i]) && pair_valid(mp[i])) {
+          wq[i] = __longlong_as_double((long long)(((mq[i].y & 0xffffffffull) << 32) | (mq[i].x & 0xffffffffull)));
+          wp[i] = __longlong_as_double((long long)(((mp[i].y & 0xffffffffull) << 32) | (mp[i].x & 0xffffffffull)));
+          pend &= ~(1u << i);
+        }
+      }
+      if (!__any_sync(0xffffffffu, pend != 0)) break;
+      if (__any_sync(0xffffffffu, global_timer_ns() - tstart > kWaitLimitNs)) {
+        if (lane == 0) raise_flag(a.flags, DSPARK_FLAG_TIMEOUT);
+        break;
+      }
+    }
+    // residual mass if any, else the target distribution (bonus: Q = P)
+    double lq = 0.0;
+#pragma unroll
+    for (int i = 0; i < kFPerLane; ++i) lq += wq[i];
+    const double Qtot = warp_sum_d(lq);
+    const bool use_q = Qtot > 0.0 && isfinite(Qtot);
+    double lw = 0.0;
+#pragma unroll
+    for (int i = 0; i < kFPerLane; ++i) lw += use_q ? wq[i] : wp[i];
+    const double incl = warp_incl_scan_d(lw);
+    const double Z = __shfl_sync(0xffffffffu, incl, 31);
+    const double T = (double)a.u_res[b] * Z;
+    double start = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) start = 0.0;
+    const unsigned own = __ballot_sync(0xffffffffu, start <= T && T < incl && lw > 0.0);
+    int pick = -1, lastp = -1;
+    double before = start, lastb = start;
+    {
+      double cum = start;
+#pragma unroll
+      for (int i = 0; i < kFPerLane; ++i) {
+        const double w = use_q ? wq[i] : wp[i];
+        if (pick < 0 && w > 0.0) {
+          lastp = c0 + i;
+          lastb = cum;
+          if (cum + w > T) {
+            pick = c0 + i;
+            before = cum;
+          }
+        }
+        cum += w;
+      }
+    }
+    if (pick < 0) {
+      pick = lastp;
+      before = lastb;
+    }
+    int cstar;
+    if (own) {
+      const int ol = __ffs(own) - 1;
+      cstar = __shfl_sync(0xffffffffu, pick, ol);
+      before = __shfl_sync(0xffffffffu, before, ol);
+    } else {  // no crossing (u*Z rounded to Z): the last CTA with mass
+      const unsigned pos = __ballot_sync(0xffffffffu, lastp >= 0);
+      const int pl = pos ? 31 - __clz(pos) : 0;
+      cstar = __shfl_sync(0xffffffffu, lastp, pl);
+      if (cstar < 0) cstar = 0;
+      before = -CUDART_INF;
+    }
+    if (cstar == cta) {
+      // chunk: this CTA's chunk partials, two per lane
+      const int ca = 2 * lane, cb = ca + 1;
+      const double wA = (ca < nch) ? (double)(use_q ? s_chunk[b][ca].x : s_chunk[b][ca].y) : 0.0;
+      const double wB = (cb < nch) ? (double)(use_q ? s_chunk[b][cb].x : s_chunk[b][cb].y) : 0.0;
+      const double pin = warp_incl_scan_d(wA + wB);
+      double lstart = __shfl_up_sync(0xffffffffu, pin, 1);
+      if (lane == 0) lstart = 0.0;
+      lstart += before;
+      const bool hitA = wA > 0.0 && lstart + wA > T;
+      const bool hitB = wB > 0.0 && lstart + wA + wB > T;
+      const unsigned h = __ballot_sync(0xffffffffu, hitA || hitB);
+      int chunk;
+      double before2;
+      if (h) {
+        const int hl = __ffs(h) - 1;
+        chunk = __shfl_sync(0xffffffffu, hitA ? ca : cb, hl);
+        before2 = __shfl_sync(0xffffffffu, hitA ? lstart : lstart + wA, hl);
+      } else {
+        const unsigned hp = __ballot_sync(0xffffffffu, wA > 0.0 || wB > 0.0);
+        const int hl = hp ? 31 - __clz(hp) : 0;
+        chunk = __shfl_sync(0xffffffffu, (wB > 0.0) ? cb : ca, hl);
+        if (!hp) chunk = 0;
+        before2 = -CUDART_INF;
+      }
+      // token: the chunk's 32 entries, recomputed
+      const int v = (c_begin + chunk) * kChunk + lane;
+      const bool valid = v < V;
+      double e = 0.0;
+      if (valid) {
+        const float t = a.target[(size_t)ri.row * V + v];
+        float bv = 0.0f, bi = 0.0f;
+        if (!ri.bonus) {
+          const size_t drow = ((size_t)b * K + ri.j) * (size_t)V;
+          bv = a.base[drow + v];
+          bi = a.draft_bias[drow + v];
+        }
+        float pt;
+        const float qv = residual_q(t, bv, bi, ri, s_it2[b], &pt);
+        e = (double)(use_q ? qv : pt);
+      }
+      const int pl = pick_lane(e, before2, T);
+      if (lane == pl) {
+        if (!(Z > 0.0) || !isfinite(Z)) raise_flag(a.flags, DSPARK_FLAG_NONFINITE);
+        const int tok = valid ? v : 0;
+        a.out_tokens[(size_t)b * (K + 1) + ri.j] = tok;
+        if (a.last_token != nullptr) a.last_token[b] = tok;
+      }
+    }
+  }
+}
+
+}  // namespace dspark

@@ -40,9 +40,11 @@ class Report:
         return f"checked={self.checked} near_margin={self.near} skipped={self.skipped} failures={len(self.failures)}"
 
 
-def compare_step(oracle, inp, step, enable_prefix, requests=None, rep=None):
+def compare_step(oracle, inp, step, enable_prefix, requests=None, rep=None, verify_len=None):
     """Run the oracle on `requests` (default: all) and compare with the
-    outputs held by `step` (a DSparkStep that has just run on `inp`)."""
+    outputs held by `step` (a DSparkStep that has just run on `inp`).
+    With `verify_len` (the lengths the caller set by hand) the prefix cut is
+    not compared and both sides verify those lengths."""
     rep = rep or Report()
     B, K, V = inp["base"].shape
     if requests is None:
@@ -51,7 +53,9 @@ def compare_step(oracle, inp, step, enable_prefix, requests=None, rep=None):
     idx = torch.as_tensor(requests, device=inp["base"].device)
 
     # ---- prefix cut: on the whole batch (it is global over requests)
-    if K > 0 and B > 0:
+    if verify_len is not None:
+        L_or = np.asarray(verify_len, np.int32)[requests]
+    elif K > 0 and B > 0:
         pr = oracle.prefix(host(inp["z"]), host(inp["temps"]), host(inp["cost_tokens"]),
                            host(inp["cost_ms"]), enable=enable_prefix)
         c_g, s_g = host(step.c), host(step.survival)

@@ -57,6 +57,14 @@ def test_status_strings_and_paths(lib):
     assert D.dspark_draft_path(151936, 256, 64, 8, D.DSPARK_BF16) == "tcgen05"
     assert D.dspark_draft_path(151936, 256, 17, 8, D.DSPARK_BF16) == "tcgen05"
     assert D.dspark_draft_path(1000, 32, 4, 8, D.DSPARK_BF16) == "cuda-core"
+    bf = D.DSPARK_BF16
+    assert D.dspark_verify_path(151936, 256, 1, 16, bf, True) == "single-launch"
+    assert D.dspark_verify_path(151936, 256, 4, 17, bf, True) == "single-launch"   # 72 rows
+    assert D.dspark_verify_path(151936, 256, 4, 18, bf, True) == "staged-bias"     # 76 rows
+    assert D.dspark_verify_path(151936, 256, 5, 8, bf, True) == "staged-bias"
+    assert D.dspark_verify_path(1024, 16, 2, 4, D.DSPARK_F32, True) == "single-launch"
+    assert D.dspark_verify_path(151936, 256, 1, 16, bf, False) == "staged-cuda-core"
+    assert D.dspark_verify_path(151936, 256, 64, 8, bf, False) == "staged-tcgen05"
 
 
 def test_workspace_sizes(lib):
