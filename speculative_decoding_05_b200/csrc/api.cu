@@ -52,7 +52,7 @@ struct VerifyWs {
 VerifyWs verify_ws(int V, int B, int K) {
   VerifyWs w;
   w.frec_off = kHeaderBytes;
-  w.frec_bytes = fused_verify_ok(V, B, K, true) ? align256(fused_rec_bytes(V, B, K)) : 0;
+  w.frec_bytes = fused_verify_ok(B, K, true) ? align256(fused_rec_bytes(B)) : 0;
   w.tpart_off = w.frec_off + w.frec_bytes;
   w.info_off = w.tpart_off + align256((size_t)B * (K + 1) * n_segs_of(V) * sizeof(float2));
   w.rpart_off = w.info_off + align256((size_t)B * sizeof(ResInfo));
@@ -234,7 +234,7 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
   const VerifyWs w = verify_ws(V, B, K);
   unsigned* flags = reinterpret_cast<unsigned*>(ws);
   const int nc = n_chunks_of(V);
-  const int G = fused_grid(nc);
+  const int G = fused_grid(V, B * (K + 1));
   if (dbias != nullptr && w.frec_bytes > 0 && G > 0) {
     // one cooperative launch; its records are cleared with the status word
     if (cudaMemsetAsync(ws, 0, kHeaderBytes + w.frec_bytes, s) != cudaSuccess) return DSPARK_ERR_CUDA;
@@ -258,13 +258,11 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
     a.last_token = last;
     a.flags = flags;
     a.seg_rec = reinterpret_cast<unsigned long long*>(ws + w.frec_off);
-    a.tot_rec = a.seg_rec + fused_seg_words(V, B, K);
+    a.tot_rec = a.seg_rec + kFSegWords;
     a.V = V;
     a.B = B;
     a.K = K;
-    a.n_seg = fused_n_seg(V);
     a.n_chunks = nc;
-    a.mstride = fused_mstride(V, B, K, G);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kFThreads);
@@ -366,7 +364,8 @@ const char* dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype)
 }
 
 const char* dspark_verify_path(int V, int r, int B, int K, dspark_dtype uw_dtype, int have_bias) {
-  if (fused_verify_ok(V, B, K, have_bias != 0) && fused_grid(n_chunks_of(V)) > 0) return "single-launch";
+  if (fused_verify_ok(B, K, have_bias != 0) && fused_grid(V, B * (K + 1)) > 0)
+    return "single-launch";
   if (have_bias) return "staged-bias";
   return use_tc(V, r, B, uw_dtype) ? "staged-tcgen05" : "staged-cuda-core";
 }

@@ -73,6 +73,14 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Merge softmax partial (A, s) into (M, S) (both relative to their own max).
+__device__ __forceinline__ void merge_partial(float& M, float& S, float A, float s, float it2) {
+  if (A == -CUDART_INF_F) return;
+  const float Mn = fmaxf(M, A);
+  S = S * ex2((M - Mn) * it2) + s * ex2((A - Mn) * it2);
+  M = Mn;
+}
+
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));

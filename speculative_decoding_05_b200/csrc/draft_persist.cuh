@@ -169,13 +169,6 @@ __device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
   return v;
 }
 
-// Merge softmax partial (A, s) into (M, S) (both relative to their own max).
-__device__ __forceinline__ void merge_partial(float& M, float& S, float A, float s, float it2) {
-  if (A == -CUDART_INF_F) return;
-  const float Mn = fmaxf(M, A);
-  S = S * ex2((M - Mn) * it2) + s * ex2((A - Mn) * it2);
-  M = Mn;
-}
 
 __device__ __forceinline__ double partial_weight(float2 q, float M, float it2) {
   return (q.x == -CUDART_INF_F) ? 0.0 : (double)(q.y * ex2((q.x - M) * it2));

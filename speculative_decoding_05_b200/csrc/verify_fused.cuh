@@ -6,16 +6,18 @@
 // accept_kernel, residual_bias_kernel, residual_sample_kernel), reorganised
 // so that one launch replaces four and the only grid-wide waits are two
 // rounds of polling on records that carry their own validity word:
-//   phase 1  target-row statistics: every verified row is cut into
-//            1024-element segments, one warp per segment (max, then
-//            sum of 2^((t - max) * log2e / T)); each segment's pair is
-//            stored as two 8-byte words {value, 1}, in a block of lines that
-//            only this CTA writes (records of several CTAs on one line, polled
-//            by every CTA, slow the exchange several fold);
-//   phase 2  every CTA polls all segment pairs, forms each row's
-//            (max, partition sum) and runs the accept scan of every request
-//            itself, so no second exchange is needed for it; CTA 0 writes
-//            n_accepted and the accepted / -1 entries of out_tokens;
+//   phase 1  target-row statistics: the verified rows laid end to end are
+//            cut into one contiguous range per CTA (at most V elements, so
+//            it meets at most two rows); the CTA reduces its part of each row
+//            to (max, sum of 2^((t - max) * log2e / T)) and stores the pairs
+//            as 8-byte words {value, 1} on a line that only it writes
+//            (records of several CTAs on one line, polled by every CTA, slow
+//            the exchange several fold);
+//   phase 2  every CTA polls, for each row, the pairs of the CTAs whose
+//            ranges meet it, forms the row's (max, partition sum) and runs the
+//            accept scan of every request itself, so no second exchange is
+//            needed for it; CTA 0 writes n_accepted and the accepted / -1
+//            entries of out_tokens;
 //   phase 3  residual partials max(0, p_t - p_d) (or p_t for a bonus draw)
 //            over this CTA's run of 32-row chunks; per request the CTA's
 //            totals (fp64) are stored as four words {32-bit half, 1} on a
@@ -41,8 +43,7 @@ constexpr int kFThreads = 512;
 constexpr int kFWarps = kFThreads / 32;
 constexpr int kFMaxB = 4;
 constexpr int kFMaxRows = 72;              // B * (K + 1)
-constexpr int kFSeg = 1024;                // target elements of one phase-1 segment (one warp)
-constexpr int kFSegPerLane = 8;            // row statistics: V <= 32 * 8 * 1024
+constexpr int kFBatch = 12;                // float4 loads per thread in flight in phase 1
 constexpr int kFPerLane = 5;               // CTA totals per lane: grid <= 160
 constexpr int kFMaxG = 32 * kFPerLane;
 constexpr int kFMaxChunks = 64;            // residual chunks of one CTA (two per lane)
@@ -66,40 +67,42 @@ struct FusedArgs {
   int32_t* out_tokens;
   int32_t* last_token;
   unsigned* flags;
-  unsigned long long* seg_rec;  // [G][mstride][2]: segment t at (t % G, t / G): {M, 1}, {S, 1}
+  unsigned long long* seg_rec;  // [G][16]: row statistics of CTA c: {M_A, 1}, {S_A, 1}, {M_B, 1}, {S_B, 1}
   unsigned long long* tot_rec;  // [B][G][16]: halves of Q and P (fp64), each {half, 1}; padding
-  int V, B, K, n_seg, n_chunks;
-  int mstride;                  // record slots per CTA block (a multiple of 8: whole lines)
+  int V, B, K, n_chunks;
 };
 
-inline int fused_n_seg(int V) { return (V + kFSeg - 1) / kFSeg; }
-// Record slots per CTA block for a grid of G.
-inline int fused_mstride(int V, int B, int K, int G) {
-  const int n_items = B * (K + 1) * fused_n_seg(V);
-  return ((n_items + G - 1) / G + 7) / 8 * 8;
-}
-// Words of the segment records for any grid up to kFMaxG (G * mstride <=
-// n_items + 8 G), then the totals.
-inline size_t fused_seg_words(int V, int B, int K) {
-  const size_t w = ((size_t)B * (K + 1) * fused_n_seg(V) + 8 * kFMaxG) * 2;
-  return (w + 15) / 16 * 16;  // the totals start on a line boundary
-}
+// Words of the row-statistics records (one line per CTA), then the totals.
+constexpr size_t kFSegWords = (size_t)kFMaxG * 16;
 // Bytes of the records of the fused verify (zeroed before each call).
-inline size_t fused_rec_bytes(int V, int B, int K) {
-  return fused_seg_words(V, B, K) * 8 + (size_t)B * kFMaxG * 128;
+inline size_t fused_rec_bytes(int B) { return (kFSegWords + (size_t)B * kFMaxG * 16) * 8; }
+inline bool fused_verify_ok(int B, int K, bool have_bias) {
+  return have_bias && B >= 1 && B <= kFMaxB && B * (K + 1) <= kFMaxRows;
 }
-inline bool fused_verify_ok(int V, int B, int K, bool have_bias) {
-  const int n_seg = fused_n_seg(V);
-  return have_bias && B >= 1 && B <= kFMaxB && B * (K + 1) <= kFMaxRows &&
-         n_seg <= 32 * kFSegPerLane;
+
+// First element of CTA c's range of the E = R V concatenated row elements.
+__host__ __device__ inline long long fused_e_begin(int c, int G, long long E) {
+  return E * c / G / 4 * 4;
+}
+// The CTA whose (non-empty) range holds element e.
+__device__ inline int fused_cta_of(long long e, int G, long long E) {
+  int c = (int)(e * G / E);
+  if (c > G - 1) c = G - 1;
+  while (c + 1 < G && fused_e_begin(c + 1, G, E) <= e) ++c;
+  while (c > 0 && fused_e_begin(c, G, E) > e) --c;
+  return c;
 }
 
 // Grid of the fused verify (one CTA per SM), or 0 when a CTA's run of
 // chunks would not fit its scan.
-inline int fused_grid(int n_chunks) {
+// A CTA's range of the verified rows (rows V / G elements, rounded to float4)
+// must stay within V elements, so that it meets at most two rows.
+inline int fused_grid(int V, int rows) {
   int G = num_sms();
   if (G > kFMaxG) G = kFMaxG;
-  return (n_chunks + G - 1) / G <= kFMaxChunks ? G : 0;
+  const bool chunks_fit = (n_chunks_of(V) + G - 1) / G <= kFMaxChunks;
+  const bool ranges_fit = (long long)rows * V + 4ll * G <= (long long)G * V;
+  return (chunks_fit && ranges_fit) ? G : 0;
 }
 
 __device__ __forceinline__ void st_pair(unsigned long long* p, uint32_t a, uint32_t b) {
@@ -130,10 +133,12 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
   __shared__ float s_dsum[kFMaxRows];
   __shared__ ResInfo s_ri[kFMaxB];
   __shared__ float2 s_chunk[kFMaxB][kFMaxChunks];
+  __shared__ float s_wm[2][kFWarps];
+  __shared__ double s_ws[2][kFWarps];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
-  const int B = a.B, K = a.K, V = a.V, n_seg = a.n_seg;
+  const int B = a.B, K = a.K, V = a.V;
 
   if (tid == 0) {
     int r = 0;
@@ -177,49 +182,85 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
   }
 
   // ---------------------------------------------------------------- phase 1
+  // This CTA's range of the R verified rows laid end to end: float4-aligned,
+  // at most V + 4 elements long (R < G), so it meets at most two rows, A and
+  // B = A + 1.  One (max, sum) pair per row it meets goes out on this CTA's
+  // own line.
+  const long long E = (long long)R * V;
+  const long long e0 = fused_e_begin(cta, G, E), e1 = fused_e_begin(cta + 1, G, E);
   {
-    const int n_items = R * n_seg;
-    const int stride = G * kFWarps;
-    for (int t0 = cta + G * warp; t0 < n_items; t0 += 2 * stride) {
-      float4 x[2][8];
-      float it2v[2];
+    const int rowA = (int)min(e0 / V, (long long)max(R - 1, 0));
+    const long long bnd = (long long)(rowA + 1) * V;  // first element of row B
+    int bA, bB = 0;
+    const int pA = row_of(rowA, &bA);
+    const int pB = (rowA + 1 < R) ? row_of(rowA + 1, &bB) : 0;
+    const float it2A = s_it2[bA], it2B = s_it2[bB];
+    const float* tA = a.target + (size_t)checked_row(a.row_start, bA, pA, a.n_rows, a.flags) * V;
+    const float* tB = (rowA + 1 < R)
+                          ? a.target + (size_t)checked_row(a.row_start, bB, pB, a.n_rows, a.flags) * V
+                          : tA;
+    const int n4 = (int)((e1 - e0) / 4);
+    float mA = -CUDART_INF_F, sA = 0.0f, mB = -CUDART_INF_F, sB = 0.0f;
+    for (int j0 = 0; j0 < n4; j0 += kFBatch * kFThreads) {
+      float4 x[kFBatch];
+      bool inB[kFBatch], ok[kFBatch];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int t = t0 + h * stride;
-        it2v[h] = kLog2e;
-        if (t < n_items) {
-          const int rho = t / n_seg, s = t - rho * n_seg;
-          int b;
-          const int p = row_of(rho, &b);
-          it2v[h] = s_it2[b];
-          const long long row = checked_row(a.row_start, b, p, a.n_rows, a.flags);
-          const float* trow = a.target + (size_t)row * V;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int e = s * kFSeg + (i * 32 + lane) * 4;
-            x[h][i] = (e < V) ? __ldg(reinterpret_cast<const float4*>(trow + e))
-                              : make_float4(-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F);
-          }
+      for (int i = 0; i < kFBatch; ++i) {
+        const int j = j0 + i * kFThreads + tid;
+        ok[i] = j < n4;
+        const long long e = e0 + 4ll * j;
+        inB[i] = e >= bnd;
+        if (ok[i]) {
+          const float* src = inB[i] ? tB + (e - bnd) : tA + (e - (long long)rowA * V);
+          x[i] = __ldg(reinterpret_cast<const float4*>(src));
         }
       }
+      float ma = -CUDART_INF_F, mb = -CUDART_INF_F;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int t = t0 + h * stride;
-        if (t >= n_items) break;
-        float m = -CUDART_INF_F;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m = fmaxf(m, fmaxf(fmaxf(x[h][i].x, x[h][i].y), fmaxf(x[h][i].z, x[h][i].w)));
-        const float M = warp_max(m);
-        float sl = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-          sl += ex2((x[h][i].x - M) * it2v[h]) + ex2((x[h][i].y - M) * it2v[h]) +
-                ex2((x[h][i].z - M) * it2v[h]) + ex2((x[h][i].w - M) * it2v[h]);
-        const double S = warp_sum_d((double)sl);
-        if (lane == 0)
-          st_pair(a.seg_rec + ((size_t)(t % G) * a.mstride + t / G) * 2, __float_as_uint(M),
-                  __float_as_uint((float)S));
+      for (int i = 0; i < kFBatch; ++i) {
+        if (!ok[i]) continue;
+        const float m4 = fmaxf(fmaxf(x[i].x, x[i].y), fmaxf(x[i].z, x[i].w));
+        if (inB[i]) mb = fmaxf(mb, m4);
+        else ma = fmaxf(ma, m4);
       }
+      float sa = 0.0f, sb = 0.0f;
+#pragma unroll
+      for (int i = 0; i < kFBatch; ++i) {
+        if (!ok[i]) continue;
+        const float m = inB[i] ? mb : ma, it2 = inB[i] ? it2B : it2A;
+        const float e4 = ex2((x[i].x - m) * it2) + ex2((x[i].y - m) * it2) + ex2((x[i].z - m) * it2) +
+                         ex2((x[i].w - m) * it2);
+        if (inB[i]) sb += e4;
+        else sa += e4;
+      }
+      merge_partial(mA, sA, ma, sa, it2A);
+      merge_partial(mB, sB, mb, sb, it2B);
+    }
+    // warp, then CTA (fp64)
+    const float MwA = warp_max(mA), MwB = warp_max(mB);
+    const double SwA = warp_sum_d(mA == -CUDART_INF_F ? 0.0 : (double)sA * (double)ex2((mA - MwA) * it2A));
+    const double SwB = warp_sum_d(mB == -CUDART_INF_F ? 0.0 : (double)sB * (double)ex2((mB - MwB) * it2B));
+    if (lane == 0) {
+      s_wm[0][warp] = MwA;
+      s_wm[1][warp] = MwB;
+      s_ws[0][warp] = SwA;
+      s_ws[1][warp] = SwB;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      float M[2];
+      double S[2];
+      for (int h = 0; h < 2; ++h) {
+        const float it2 = h ? it2B : it2A;
+        M[h] = -CUDART_INF_F;
+        for (int w2 = 0; w2 < kFWarps; ++w2) M[h] = fmaxf(M[h], s_wm[h][w2]);
+        S[h] = 0.0;
+        for (int w2 = 0; w2 < kFWarps; ++w2)
+          if (s_wm[h][w2] != -CUDART_INF_F) S[h] += s_ws[h][w2] * (double)ex2((s_wm[h][w2] - M[h]) * it2);
+      }
+      unsigned long long* r = a.seg_rec + (size_t)cta * 16;
+      st_pair(r, __float_as_uint(M[0]), __float_as_uint((float)S[0]));
+      st_pair(r + 2, __float_as_uint(M[1]), __float_as_uint((float)S[1]));
     }
   }
   if (tid < R) {
@@ -232,28 +273,33 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
   }
 
   // ---------------------------------------------------------------- phase 2
+  // row rho = the CTAs whose ranges meet it: [cta_of(rho V), cta_of((rho+1) V - 1)]
   for (int rho = warp; rho < R; rho += kFWarps) {
     int b;
     (void)row_of(rho, &b);
     const float it2 = s_it2[b];
-    float2 q[kFSegPerLane];
+    const int c_lo = fused_cta_of((long long)rho * V, G, E);
+    const int c_hi = fused_cta_of((long long)(rho + 1) * V - 1, G, E);
+    float2 q[kFPerLane];
     unsigned pend = 0;
 #pragma unroll
-    for (int i = 0; i < kFSegPerLane; ++i) {
+    for (int i = 0; i < kFPerLane; ++i) {
       q[i] = make_float2(-CUDART_INF_F, 0.0f);
-      if (lane + 32 * i < n_seg) pend |= 1u << i;
+      if (c_lo + lane + 32 * i <= c_hi) pend |= 1u << i;
     }
     const uint64_t tstart = global_timer_ns();
     for (;;) {
-      ulonglong2 m[kFSegPerLane];
+      ulonglong2 m[kFPerLane];
 #pragma unroll
-      for (int i = 0; i < kFSegPerLane; ++i)
+      for (int i = 0; i < kFPerLane; ++i) {
         if (pend & (1u << i)) {
-          const int t = rho * n_seg + lane + 32 * i;
-          m[i] = ld_pair(a.seg_rec + ((size_t)(t % G) * a.mstride + t / G) * 2);
+          const int c = c_lo + lane + 32 * i;
+          const int slot = rho - (int)(fused_e_begin(c, G, E) / V);  // 0 or 1
+          m[i] = ld_pair(a.seg_rec + (size_t)c * 16 + 2 * slot);
         }
+      }
 #pragma unroll
-      for (int i = 0; i < kFSegPerLane; ++i) {
+      for (int i = 0; i < kFPerLane; ++i) {
         if ((pend & (1u << i)) && pair_valid(m[i])) {
           q[i] = make_float2(__uint_as_float((uint32_t)m[i].x), __uint_as_float((uint32_t)m[i].y));
           pend &= ~(1u << i);
@@ -267,11 +313,11 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
     }
     float mx = -CUDART_INF_F;
 #pragma unroll
-    for (int i = 0; i < kFSegPerLane; ++i) mx = fmaxf(mx, q[i].x);
+    for (int i = 0; i < kFPerLane; ++i) mx = fmaxf(mx, q[i].x);
     const float tmax = warp_max(mx);
     double z = 0.0;
 #pragma unroll
-    for (int i = 0; i < kFSegPerLane; ++i)
+    for (int i = 0; i < kFPerLane; ++i)
       if (q[i].y > 0.0f) z += (double)q[i].y * (double)ex2((q[i].x - tmax) * it2);
     const double tz = warp_sum_d(z);
     if (lane == 0) {
