@@ -872,6 +872,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   float* s_ws = s_wm + kGSlots * kGMaxB;                  // [kGSlots][kGMaxB]
   volatile int* s_i = reinterpret_cast<volatile int*>(s_ws + kGSlots * kGMaxB);  // [4]
   float* s_ud = const_cast<float*>(reinterpret_cast<volatile float*>(s_i + 4));   // [B][K] draft uniforms
+  int* s_units = reinterpret_cast<int*>(s_ud + kGMaxB * 64);                      // [2][8] unit -> tile
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -979,6 +980,25 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         *reinterpret_cast<uint4*>(sTail + rr * (kGRank * 2) + lane * 16) = val;
       }
     }
+    // Units of 32 rows: the GEMV warps' tiles of parity h (TMEM-resident and
+    // streamed ones alternating, half 0 starting with a resident tile and
+    // half 1 with a streamed one, so that only four warps read the ring at a
+    // time; each half still takes its streamed tiles in increasing order,
+    // which keeps the ring free of deadlock); the tail warp's single chunk.
+    if (threadIdx.x == kGTailWarp * 32) {
+      for (int h = 0; h < 2; ++h) {
+        const int n_units = (nt - h + 1) / 2;
+        const int n_res = (nres - h + 1) / 2, n_str = n_units - n_res;
+        const int r0 = nres + ((h + nres) & 1);  // first streamed tile of parity h
+        const int m = min(n_res, n_str);
+        for (int n = 0; n < n_units && n < kPMaxTiles / 2; ++n) {
+          int i;
+          if (n < 2 * m) i = (((n & 1) == 0) == (h == 0)) ? h + 2 * (n >> 1) : r0 + 2 * (n >> 1);
+          else i = (n_res > n_str) ? h + 2 * (m + n - 2 * m) : r0 + 2 * (m + n - 2 * m);
+          s_units[h * (kPMaxTiles / 2) + n] = i;
+        }
+      }
+    }
     // the draft uniforms of every position, staged so the sampling step
     // never waits on a global load
     for (int i = threadIdx.x - kGTailWarp * 32; i < B * K; i += kGSyncThreads) s_ud[i] = p.u_draft[i];
@@ -1006,36 +1026,15 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       }
       bool ok = mbar_wait_spin(&baseFull[buf], (uint32_t)(k >> 1) & 1u);
 
-      // per 32-row unit: bias of lane `lane`'s row, its softmax partial, stores
-      auto finish_unit = [&](float (&pr)[NB][32], int vl, bool valid, int chunk) {
-        const int v = v0 + vl;
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-          if (b >= B) break;
-          const float bias = transpose_reduce32(pr[b], lane);
-          const float bv = valid ? bse[(size_t)b * rows_cap + vl] : 0.0f;
-          const float a = valid ? bv + bias : -CUDART_INF_F;
-          const float A = warp_max(a);
-          const float e = valid ? ex2(((bv - A) + bias) * it2[b]) : 0.0f;
-          const float sm2 = warp_sum(e);
-          sBias[(size_t)b * rows_cap + vl] = bias;
-          if (valid) {
-            const size_t row = ((size_t)b * K + k) * (size_t)V;
-            if (p.draft_bias != nullptr) p.draft_bias[row + v] = bias;
-            if (p.draft_logits != nullptr) p.draft_logits[row + v] = a * itv[b];
-          }
-          if (lane == 0) {
-            sPart[(size_t)b * part_cap + chunk] = make_float2(A, sm2);
-            merge_partial(wm[b], ws[b], A, sm2, it2[b]);
-          }
-        }
-      };
-
-      // units of 32 rows: the GEMV warps' tiles i = half, half + 2, ...; the
-      // tail warp's single chunk
       const int n_units = gemv ? (nt - half + 1) / 2 : tail;
+      const int* units = s_units + (gemv ? half : 0) * (kPMaxTiles / 2);
+      auto unit_tile = [&](int n) { return units[n]; };
+      auto unit_row = [&](int i) { return gemv ? i * kTileN + quarter * 32 + lane : main_rows + lane; };
+      auto unit_limit = [&]() { return gemv ? main_rows : nrows; };
+      auto unit_chunk = [&](int i) { return gemv ? i * 4 + quarter : mainc; };
+
       for (int n = 0; n < n_units; ++n) {
-        const int i = half + 2 * n;
+        const int i = gemv ? unit_tile(n) : 0;
         float pr[NB][32];
 #pragma unroll
         for (int b = 0; b < NB; ++b)
@@ -1086,10 +1085,62 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           if (lane == 0)
             for (int kb = 0; kb < nkb; ++kb) mbar_arrive(&ringEmpty[(itb + kb) % S]);
         }
-        // row within the CTA range, its validity and its chunk
-        const int vl = gemv ? i * kTileN + quarter * 32 + lane : main_rows + lane;
-        const bool valid = vl < (gemv ? main_rows : nrows);
-        finish_unit(pr, vl, valid, gemv ? i * 4 + quarter : mainc);
+        // this lane's row: its bias (butterfly), kept in shared memory and,
+        // when asked for, in global memory
+        const int vl = unit_row(i);
+        const bool valid = vl < unit_limit();
+        const int v = v0 + vl;
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b >= B) break;
+          const float bias = transpose_reduce32(pr[b], lane);
+          sBias[(size_t)b * rows_cap + vl] = bias;
+          if (valid) {
+            const size_t row = ((size_t)b * K + k) * (size_t)V;
+            if (p.draft_bias != nullptr) p.draft_bias[row + v] = bias;
+            if (p.draft_logits != nullptr)
+              p.draft_logits[row + v] = (bse[(size_t)b * rows_cap + vl] + bias) * itv[b];
+          }
+        }
+      }
+      // softmax partial of every unit (chunk), four units at a time so that
+      // their shuffle chains overlap
+      __syncwarp();
+      for (int n0 = 0; n0 < n_units; n0 += 4) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+          if (b >= B) break;
+          float bv[4], bi[4], am[4], es[4];
+          bool ok4[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int n = n0 + j;
+            const int vl = unit_row(n < n_units && gemv ? unit_tile(n) : 0);
+            ok4[j] = n < n_units && vl < unit_limit();
+            bv[j] = ok4[j] ? bse[(size_t)b * rows_cap + vl] : 0.0f;
+            bi[j] = ok4[j] ? sBias[(size_t)b * rows_cap + vl] : 0.0f;
+            am[j] = ok4[j] ? bv[j] + bi[j] : -CUDART_INF_F;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) am[j] = fmaxf(am[j], __shfl_xor_sync(0xffffffffu, am[j], o));
+#pragma unroll
+          for (int j = 0; j < 4; ++j) es[j] = ok4[j] ? ex2(((bv[j] - am[j]) + bi[j]) * it2[b]) : 0.0f;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) es[j] += __shfl_xor_sync(0xffffffffu, es[j], o);
+          if (lane == 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int n = n0 + j;
+              if (n >= n_units) break;
+              sPart[(size_t)b * part_cap + unit_chunk(gemv ? unit_tile(n) : 0)] = make_float2(am[j], es[j]);
+              merge_partial(wm[b], ws[b], am[j], es[j], it2[b]);
+            }
+          }
+        }
       }
       if (!ok) {
         *s_abort = 1;
