@@ -110,6 +110,10 @@ constexpr int kGMaxG = 32 * kGPerLane;              // grid limit of the GEMV va
 // reading every record, records that share lines slow the exchange several
 // fold (the writes queue behind the reads of the shared line).
 constexpr int kGRecWords = 16;                      // 8-byte words per record line
+// W chunks (32 rows, 16 KB) kept in shared memory for the whole call, beside
+// the 16 in TMEM; the rest of a CTA's chunks stream through the ring.
+constexpr int kGResChunks = 8;
+constexpr int kGMaxUnits = 12;                      // units per warp and position
 
 // First chunk of CTA c: runs balanced to within one chunk.
 __host__ __device__ inline int gemv_chunk_begin(int cta, int G, int n_chunks) {
@@ -145,8 +149,9 @@ inline PersistLayout persist_layout(int V, int r, int B) {
     gemv_runs(n_chunks, G, &max_chunks, &L.max_nt);
     // tail rows, sBias [B][rows_cap] + sBase [2][B][rows_cap] + sPart [B][part_cap]
     const size_t rows_cap = (size_t)L.max_nt * kTileN + kChunk, part_cap = (size_t)L.max_nt * 4 + 1;
-    L.u_bytes = kGTailBytes;
-    L.base_bytes = (size_t)3 * B * rows_cap * 4 + (size_t)B * part_cap * 8 + 16;
+    L.u_bytes = kGTailBytes + (size_t)kGResChunks * kStageBytes;
+    L.base_bytes = (size_t)3 * B * rows_cap * 4 + (size_t)B * part_cap * 8 + 16 +
+                   (size_t)2 * B * kGMaxChunks * 8;  // + chunk weights and prefix sums (fp64)
   } else {
     L.u_bytes = (size_t)(r / 64) * 2048;
     L.base_bytes = (((size_t)B * L.max_nt * kTileN * 4) + 1023) & ~size_t(1023);
@@ -838,7 +843,6 @@ __global__ void __launch_bounds__(kGThreads, 1)
 draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p, const GemvRecs rec) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int nkb = kGRank / 64;
   const int G = gridDim.x, cta = blockIdx.x;
   const int B = p.B, K = p.K, V = p.V;
   const int S = p.n_stages;
@@ -853,14 +857,19 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   const int rows_cap = p.max_nt * kTileN + kChunk;  // row slots per request in sBias / sBase
   const int part_cap = p.max_nt * 4 + 1;            // chunk slots per request in sPart
   const int nres = min(nt, kGMaxTmemTiles);
-  const int nstream = nt - nres;
+  const int n_tm = min(4 * nres, mainc);             // chunks held in TMEM (tiles 0..nres-1)
+  const int n_res = min(kGResChunks, mainc - n_tm);  // chunks held in shared memory
+  const int n_str = mainc - n_tm - n_res;            // chunks streamed every position
 
   uint8_t* sRing = sm;
   uint8_t* sTail = sRing + S * kStageBytes;                                  // [32 rows][512 B]
-  float* sBias = reinterpret_cast<float*>(sTail + kGTailBytes);              // [B][rows_cap]
+  uint8_t* sRes = sTail + kGTailBytes;                                       // [kGResChunks][16 KB]
+  float* sBias = reinterpret_cast<float*>(sRes + kGResChunks * kStageBytes); // [B][rows_cap]
   float* sBase = sBias + (size_t)B * rows_cap;                               // [2][B][rows_cap]
   float2* sPart = reinterpret_cast<float2*>(sBase + (size_t)2 * B * rows_cap);  // [B][part_cap]
-  uint8_t* misc = reinterpret_cast<uint8_t*>(sPart + (size_t)B * part_cap);
+  // after sPart: the chunk weights and prefix sums (2 B kGMaxChunks doubles,
+  // one float2 slot each), then the barriers and small arrays
+  uint8_t* misc = reinterpret_cast<uint8_t*>(sPart + (size_t)B * part_cap + (size_t)2 * B * kGMaxChunks);
   misc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(misc) + 15) & ~uintptr_t(15));
   uint64_t* ringFull = reinterpret_cast<uint64_t*>(misc);
   uint64_t* ringEmpty = ringFull + kPMaxStages;
@@ -872,14 +881,19 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   float* s_ws = s_wm + kGSlots * kGMaxB;                  // [kGSlots][kGMaxB]
   volatile int* s_i = reinterpret_cast<volatile int*>(s_ws + kGSlots * kGMaxB);  // [4]
   float* s_ud = const_cast<float*>(reinterpret_cast<volatile float*>(s_i + 4));   // [B][K] draft uniforms
-  int* s_units = reinterpret_cast<int*>(s_ud + kGMaxB * 64);                      // [2][8] unit -> tile
+  int* s_units = reinterpret_cast<int*>(s_ud + kGMaxB * 64);  // [9][kGMaxUnits] (type, index, chunk)
+  int* s_nunits = s_units + 9 * kGMaxUnits;                    // [9]
+  float* s_acta = reinterpret_cast<float*>(s_nunits + 12);     // [kGMaxB] CTA max per request
+  // chunk weights relative to the CTA max and their inclusive prefix sums
+  double* s_cw = reinterpret_cast<double*>(sPart + (size_t)B * part_cap);  // [B][kGMaxChunks]
+  double* s_cp = s_cw + (size_t)B * kGMaxChunks;                                     // [B][kGMaxChunks]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&ringFull[i], 1);
-      mbar_init(&ringEmpty[i], 4);
+      mbar_init(&ringEmpty[i], 1);  // one consumer warp per stage
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&baseFull[i], 1);
@@ -896,21 +910,29 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
 
   if (warp == 0) {
     // ------------------------------------------------ W producer (streamed tiles)
-    if (lane == 0 && nstream > 0) {
+    if (lane == 0 && n_str > 0) {
+      // Stage = one streamed chunk, 32 whole W rows (16 KB, contiguous in
+      // global memory): one bulk copy, consumed by one warp.  (A swizzled 2D
+      // box of 128 rows x 128 B per stage arrived several times slower.)
+      // Rows past V are not read.
       const uint64_t pol = policy_evict_last();
       int it = 0;
       for (int k = 0; k < K && !*s_abort; ++k) {
-        for (int i = nres; i < nt && !*s_abort; ++i) {
-          for (int kb = 0; kb < nkb; ++kb) {
-            const int s = it % S;
-            if (!mbar_wait(&ringEmpty[s], ((uint32_t)(it / S) & 1u) ^ 1u)) {
-              *s_abort = 1;
-              raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
-              break;
-            }
-            mbar_arrive_expect_tx(&ringFull[s], kStageBytes);
-            tma_load_2d_hint(sRing + s * kStageBytes, &tm_w, &ringFull[s], kb * 64, v0 + i * kTileN, pol);
-            ++it;
+        for (int sc = 0; sc < n_str && !*s_abort; ++sc, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&ringEmpty[s], ((uint32_t)(it / S) & 1u) ^ 1u)) {
+            *s_abort = 1;
+            raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
+            break;
+          }
+          const int row0 = v0 + (n_tm + n_res + sc) * kChunk;
+          const int nr = max(0, min(kChunk, V - row0));
+          if (nr > 0) {
+            mbar_arrive_expect_tx(&ringFull[s], (uint32_t)nr * (kGRank * 2));
+            bulk_load(sRing + s * kStageBytes, p.W + (size_t)row0 * kGRank, (uint32_t)nr * (kGRank * 2),
+                      &ringFull[s], pol);
+          } else {
+            mbar_arrive(&ringFull[s]);
           }
         }
       }
@@ -944,7 +966,6 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
     const int slot = gemv ? cw : kGSlots - 1;   // this warp's partial slot
     const int half = cw >> 1 >> 1;              // tile parity owned by a GEMV warp
     const int quarter = warp & 3;               // TMEM lane quarter = rows 32q..32q+31 of a tile
-    const int kb_l = lane >> 3, j8 = lane & 7;  // this lane's K slice: k-block, 16-byte chunk
     float it2[NB], itv[NB];
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
@@ -970,6 +991,15 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         }
       }
       tmem_st_wait();
+      // this warp's shared-memory-resident chunks, row-major (512 B per row)
+      for (int j = cw; j < n_res; j += 8) {
+        for (int rr = 0; rr < kChunk; ++rr) {
+          const int row = v0 + (n_tm + j) * kChunk + rr;
+          const uint4 val = (row < V) ? __ldg(reinterpret_cast<const uint4*>(p.W + (size_t)row * kGRank) + lane)
+                                      : make_uint4(0, 0, 0, 0);
+          *reinterpret_cast<uint4*>(sRes + j * kStageBytes + rr * (kGRank * 2) + lane * 16) = val;
+        }
+      }
     } else if (tail) {
       // the tail chunk's W rows -> shared memory, row-major (512 B per row)
       for (int rr = 0; rr < kChunk; ++rr) {
@@ -980,24 +1010,39 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         *reinterpret_cast<uint4*>(sTail + rr * (kGRank * 2) + lane * 16) = val;
       }
     }
-    // Units of 32 rows: the GEMV warps' tiles of parity h (TMEM-resident and
-    // streamed ones alternating, half 0 starting with a resident tile and
-    // half 1 with a streamed one, so that only four warps read the ring at a
-    // time; each half still takes its streamed tiles in increasing order,
-    // which keeps the ring free of deadlock); the tail warp's single chunk.
+    // Units of 32 rows (one chunk each), per warp: its TMEM chunks (rows
+    // 32q..32q+31 of the tiles of parity h), its shared-memory chunks and its
+    // streamed chunks (chunk j of those outside TMEM goes to warp j % 8).
+    // Half 0 takes its streamed chunks first (they were fetched during the
+    // previous exchange; releasing them early lets the rest of this
+    // position's stream land in time), half 1 last.  Each warp takes its
+    // streamed chunks in increasing order, which keeps the ring free of
+    // deadlock.  Entry: (type << 24) | (index << 12) | chunk, type 0 = TMEM
+    // tile, 1 = resident chunk, 2 = stream index, 3 = the tail chunk.
     if (threadIdx.x == kGTailWarp * 32) {
-      for (int h = 0; h < 2; ++h) {
-        const int n_units = (nt - h + 1) / 2;
-        const int n_res = (nres - h + 1) / 2, n_str = n_units - n_res;
-        const int r0 = nres + ((h + nres) & 1);  // first streamed tile of parity h
-        const int m = min(n_res, n_str);
-        for (int n = 0; n < n_units && n < kPMaxTiles / 2; ++n) {
-          int i;
-          if (n < 2 * m) i = (((n & 1) == 0) == (h == 0)) ? h + 2 * (n >> 1) : r0 + 2 * (n >> 1);
-          else i = (n_res > n_str) ? h + 2 * (m + n - 2 * m) : r0 + 2 * (m + n - 2 * m);
-          s_units[h * (kPMaxTiles / 2) + n] = i;
+      for (int w = 0; w < 8; ++w) {
+        const int h = w >> 2, q = (w + kGCompWarp0) & 3;
+        int a_[kGMaxUnits], na = 0, r_[kGMaxUnits], nr_ = 0, st[kGMaxUnits], nst = 0;
+        for (int i = h; i < nres; i += 2)
+          if (4 * i + q < mainc && na < kGMaxUnits) a_[na++] = (i << 12) | (4 * i + q);
+        for (int j = w; j < n_res; j += 8)
+          if (nr_ < kGMaxUnits) r_[nr_++] = (1 << 24) | (j << 12) | (n_tm + j);
+        for (int j = n_res; j < mainc - n_tm; ++j)
+          if (j % 8 == w && nst < kGMaxUnits) st[nst++] = (2 << 24) | ((j - n_res) << 12) | (n_tm + j);
+        int* ul = s_units + w * kGMaxUnits;
+        int n = 0;
+        if (h == 0)
+          for (int t = 0; t < nst && n < kGMaxUnits; ++t) ul[n++] = st[t];
+        for (int t = 0; t < max(na, nr_); ++t) {
+          if (t < na && n < kGMaxUnits) ul[n++] = a_[t];
+          if (t < nr_ && n < kGMaxUnits) ul[n++] = r_[t];
         }
+        if (h == 1)
+          for (int t = 0; t < nst && n < kGMaxUnits; ++t) ul[n++] = st[t];
+        s_nunits[w] = n;
       }
+      s_units[8 * kGMaxUnits] = (3 << 24) | mainc;
+      s_nunits[8] = tail;
     }
     // the draft uniforms of every position, staged so the sampling step
     // never waits on a global load
@@ -1026,31 +1071,20 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       }
       bool ok = mbar_wait_spin(&baseFull[buf], (uint32_t)(k >> 1) & 1u);
 
-      const int n_units = gemv ? (nt - half + 1) / 2 : tail;
-      const int* units = s_units + (gemv ? half : 0) * (kPMaxTiles / 2);
-      auto unit_tile = [&](int n) { return units[n]; };
-      auto unit_row = [&](int i) { return gemv ? i * kTileN + quarter * 32 + lane : main_rows + lane; };
-      auto unit_limit = [&]() { return gemv ? main_rows : nrows; };
-      auto unit_chunk = [&](int i) { return gemv ? i * 4 + quarter : mainc; };
-
+      const int* ul = s_units + (gemv ? cw : 8) * kGMaxUnits;
+      const int n_units = s_nunits[gemv ? cw : 8];
       for (int n = 0; n < n_units; ++n) {
-        const int i = gemv ? unit_tile(n) : 0;
+        const int e = ul[n];
+        const int type = e >> 24, idx = (e >> 12) & 0xfff, c = e & 0xfff;
         float pr[NB][32];
 #pragma unroll
         for (int b = 0; b < NB; ++b)
 #pragma unroll
           for (int j = 0; j < 32; ++j) pr[b][j] = 0.0f;
-        if (!gemv) {
-#pragma unroll
-          for (int rr = 0; rr < 32; ++rr) {
-            if (rr == 16) asm volatile("" ::: "memory");
-            const uint4 q = *reinterpret_cast<const uint4*>(sTail + rr * (kGRank * 2) + lane * 16);
-            gemv8<NB>(q, u, B, pr, rr);
-          }
-        } else if (i < nres) {
+        if (type == 0) {
           // eight 16-column groups (4 rows each), the next group's
           // tcgen05.ld in flight while the current one is multiplied
-          const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(i * 128);
+          const uint32_t ta = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(idx * 128);
           uint32_t wa[16], wb[16];
           tmem_ld16_issue(ta, wa);
           tmem_ld16_wait(wa);
@@ -1066,29 +1100,34 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             if (g + 1 < 8) tmem_ld16_wait(nxt);
           }
         } else {
-          const int itb = (k * nstream + (i - nres)) * nkb;
-          for (int kb = 0; kb < nkb; ++kb) {
-            const int it = itb + kb;
+          // 32 rows of 512 B in shared memory: a resident chunk, a ring
+          // stage or the tail chunk
+          int it = 0;
+          const uint8_t* buf;
+          if (type == 2) {
+            it = k * n_str + idx;
             ok = ok && mbar_wait_spin(&ringFull[it % S], (uint32_t)(it / S) & 1u);
+            buf = sRing + (it % S) * kStageBytes;
+          } else {
+            buf = (type == 1) ? sRes + idx * kStageBytes : sTail;
           }
-          const uint8_t* stg = sRing + ((itb + kb_l) % S) * kStageBytes;
           // two halves of 16 rows: the barrier keeps the compiler from
           // hoisting all 32 shared loads (128 registers) at once
 #pragma unroll
           for (int rr = 0; rr < 32; ++rr) {
             if (rr == 16) asm volatile("" ::: "memory");
-            const int m = quarter * 32 + rr;
-            const uint4 q = *reinterpret_cast<const uint4*>(stg + m * 128 + ((j8 ^ (m & 7)) << 4));
+            const uint4 q = *reinterpret_cast<const uint4*>(buf + rr * (kGRank * 2) + lane * 16);
             gemv8<NB>(q, u, B, pr, rr);
           }
-          __syncwarp();
-          if (lane == 0)
-            for (int kb = 0; kb < nkb; ++kb) mbar_arrive(&ringEmpty[(itb + kb) % S]);
+          if (type == 2) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ringEmpty[it % S]);
+          }
         }
         // this lane's row: its bias (butterfly), kept in shared memory and,
         // when asked for, in global memory
-        const int vl = unit_row(i);
-        const bool valid = vl < unit_limit();
+        const int vl = c * kChunk + lane;
+        const bool valid = vl < nrows;
         const int v = v0 + vl;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
@@ -1115,8 +1154,8 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int n = n0 + j;
-            const int vl = unit_row(n < n_units && gemv ? unit_tile(n) : 0);
-            ok4[j] = n < n_units && vl < unit_limit();
+            const int vl = ((n < n_units) ? (ul[n] & 0xfff) : 0) * kChunk + lane;
+            ok4[j] = n < n_units && vl < nrows;
             bv[j] = ok4[j] ? bse[(size_t)b * rows_cap + vl] : 0.0f;
             bi[j] = ok4[j] ? sBias[(size_t)b * rows_cap + vl] : 0.0f;
             am[j] = ok4[j] ? bv[j] + bi[j] : -CUDART_INF_F;
@@ -1126,7 +1165,12 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
 #pragma unroll
             for (int j = 0; j < 4; ++j) am[j] = fmaxf(am[j], __shfl_xor_sync(0xffffffffu, am[j], o));
 #pragma unroll
-          for (int j = 0; j < 4; ++j) es[j] = ok4[j] ? ex2(((bv[j] - am[j]) + bi[j]) * it2[b]) : 0.0f;
+          for (int j = 0; j < 4; ++j) {
+            es[j] = ok4[j] ? ex2(((bv[j] - am[j]) + bi[j]) * it2[b]) : 0.0f;
+            // from here on the slot holds the row's weight relative to its
+            // chunk's max (the sampling step's last level reads it)
+            if (n0 + j < n_units) sBias[(size_t)b * rows_cap + ((ul[n0 + j] & 0xfff) * kChunk + lane)] = es[j];
+          }
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1)
 #pragma unroll
@@ -1136,7 +1180,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             for (int j = 0; j < 4; ++j) {
               const int n = n0 + j;
               if (n >= n_units) break;
-              sPart[(size_t)b * part_cap + unit_chunk(gemv ? unit_tile(n) : 0)] = make_float2(am[j], es[j]);
+              sPart[(size_t)b * part_cap + (ul[n] & 0xfff)] = make_float2(am[j], es[j]);
               merge_partial(wm[b], ws[b], am[j], es[j], it2[b]);
             }
           }
@@ -1164,8 +1208,29 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         st_rec(r0, __float_as_uint(M), seq);
         st_rec(r0 + 1, __float_as_uint(Sm), seq);
       }
-      // warp b: gathers the partials of request b from every CTA (level 1);
-      // the CTA that holds the sample resolves chunk and token
+      // While warp b polls, warp 2 + b turns this CTA's chunk partials of
+      // request b into weights relative to the CTA's own max and their prefix
+      // sums (fp64), so that the owner's chunk search is one rescale and one
+      // ballot.
+      if (gemv && cw >= 2 && cw - 2 < B) {
+        const int b = cw - 2;
+        float Acta = -CUDART_INF_F;
+        for (int w2 = 0; w2 < kGSlots; ++w2) Acta = fmaxf(Acta, s_wm[w2 * kGMaxB + b]);
+        const float2* lp = sPart + (size_t)b * part_cap;
+        const int ca = 2 * lane, cb = ca + 1;
+        const double wA = (ca < nc && lp[ca].y > 0.0f) ? partial_weight(lp[ca], Acta, it2[b]) : 0.0;
+        const double wB = (cb < nc && lp[cb].y > 0.0f) ? partial_weight(lp[cb], Acta, it2[b]) : 0.0;
+        const double pin = warp_incl_scan_d(wA + wB);
+        s_cw[b * kGMaxChunks + ca] = wA;
+        s_cw[b * kGMaxChunks + cb] = wB;
+        s_cp[b * kGMaxChunks + ca] = pin - wB;
+        s_cp[b * kGMaxChunks + cb] = pin;
+        if (lane == 0) s_acta[b] = Acta;
+      }
+      // warp b: gathers the partials of request b from every CTA (level 1)
+      float M = 0.0f;
+      double Z = 0.0, T = 0.0, before = 0.0;
+      int cstar = -1;
       if (gemv && cw < B) {
         const int b = cw;
         const unsigned long long* cr = rec.cta + (((size_t)par * B + b) * G) * kGRecWords;
@@ -1205,42 +1270,44 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         float mx = -CUDART_INF_F;
 #pragma unroll
         for (int i = 0; i < kGPerLane; ++i) mx = fmaxf(mx, q[i].x);
-        const float M = warp_max(mx);
-        double wsum = 0.0;
+        M = warp_max(mx);
+        double w[kGPerLane], wsum = 0.0;
 #pragma unroll
-        for (int i = 0; i < kGPerLane; ++i) wsum += partial_weight(q[i], M, it2[b]);
+        for (int i = 0; i < kGPerLane; ++i) {
+          w[i] = partial_weight(q[i], M, it2[b]);
+          wsum += w[i];
+        }
         const double incl = warp_incl_scan_d(wsum);
-        const double Z = __shfl_sync(0xffffffffu, incl, 31);
-        const double T = (double)s_ud[b * K + k] * Z;
+        Z = __shfl_sync(0xffffffffu, incl, 31);
+        T = (double)s_ud[b * K + k] * Z;
         double start = __shfl_up_sync(0xffffffffu, incl, 1);
         if (lane == 0) start = 0.0;
         const unsigned own = __ballot_sync(0xffffffffu, start <= T && T < incl && wsum > 0.0);
-        int cstar, pick = -1, lastp = -1;
-        double before = start, lastb = start;
+        int pick = -1, lastp = -1;
+        double bef = start, lastb = start;
         {
           double cum = start;
 #pragma unroll
           for (int i = 0; i < kGPerLane; ++i) {
-            const double w = partial_weight(q[i], M, it2[b]);
-            if (pick < 0 && w > 0.0) {
+            if (pick < 0 && w[i] > 0.0) {
               lastp = c0 + i;
               lastb = cum;
-              if (cum + w > T) {
+              if (cum + w[i] > T) {
                 pick = c0 + i;
-                before = cum;
+                bef = cum;
               }
             }
-            cum += w;
+            cum += w[i];
           }
         }
         if (pick < 0) {
           pick = lastp;
-          before = lastb;
+          bef = lastb;
         }
         if (own) {
           const int ol = __ffs(own) - 1;
           cstar = __shfl_sync(0xffffffffu, pick, ol);
-          before = __shfl_sync(0xffffffffu, before, ol);
+          before = __shfl_sync(0xffffffffu, bef, ol);
         } else {  // no crossing (u*Z rounded to Z): last CTA with mass
           const unsigned pos = __ballot_sync(0xffffffffu, lastp >= 0);
           const int pl = pos ? 31 - __clz(pos) : 0;
@@ -1248,63 +1315,65 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           if (cstar < 0) cstar = 0;
           before = -CUDART_INF;
         }
-        if (cstar == cta) {
-          // level 2: this CTA's chunk partials (shared memory), two per lane
-          const float2* lp = sPart + (size_t)b * part_cap;
-          const int ca = 2 * lane, cb2 = ca + 1;
-          const double wA = (ca < nc) ? partial_weight(lp[ca], M, it2[b]) : 0.0;
-          const double wB = (cb2 < nc) ? partial_weight(lp[cb2], M, it2[b]) : 0.0;
-          const double pin = warp_incl_scan_d(wA + wB);
-          double lstart = __shfl_up_sync(0xffffffffu, pin, 1);
-          if (lane == 0) lstart = 0.0;
-          lstart += before;
-          const bool hitA = wA > 0.0 && lstart + wA > T;
-          const bool hitB = wB > 0.0 && lstart + wA + wB > T;
-          const unsigned h = __ballot_sync(0xffffffffu, hitA || hitB);
-          int chunk;
-          double before2;
-          if (h) {
-            const int hl = __ffs(h) - 1;
-            chunk = __shfl_sync(0xffffffffu, hitA ? ca : cb2, hl);
-            before2 = __shfl_sync(0xffffffffu, hitA ? lstart : lstart + wA, hl);
+      }
+      gemv_sync();  // the chunk weights of every request are in shared memory
+      // the CTA that holds the sample resolves chunk and token; scales: global
+      // = f * (relative to the CTA max) and (relative to the CTA max) = g *
+      // (relative to the chunk max)
+      if (gemv && cw < B && cstar == cta) {
+        const int b = cw;
+        const float Acta = s_acta[b];
+        const double f = (double)ex2((Acta - M) * it2[b]);
+        const double Tp = (T - before) / f;
+        const int ca = 2 * lane, cb = ca + 1;
+        const double wA = s_cw[b * kGMaxChunks + ca], wB = s_cw[b * kGMaxChunks + cb];
+        const double pA = s_cp[b * kGMaxChunks + ca], pB = s_cp[b * kGMaxChunks + cb];
+        const bool hitA = wA > 0.0 && pA > Tp;
+        const bool hitB = wB > 0.0 && pB > Tp;
+        const unsigned h = __ballot_sync(0xffffffffu, hitA || hitB);
+        int chunk;
+        double before2;  // mass before the chunk, relative to the CTA max
+        if (h) {
+          const int hl = __ffs(h) - 1;
+          chunk = __shfl_sync(0xffffffffu, hitA ? ca : cb, hl);
+          before2 = __shfl_sync(0xffffffffu, hitA ? pA - wA : pB - wB, hl);
+        } else {
+          const unsigned hp = __ballot_sync(0xffffffffu, wA > 0.0 || wB > 0.0);
+          const int hl = hp ? 31 - __clz(hp) : 0;
+          chunk = __shfl_sync(0xffffffffu, (wB > 0.0) ? cb : ca, hl);
+          if (!hp) chunk = 0;
+          before2 = -CUDART_INF;
+        }
+        // the chunk's rows: weights relative to the chunk max, kept by the epilogue
+        const double g = (double)ex2((sPart[(size_t)b * part_cap + chunk].x - Acta) * it2[b]);
+        const double Tpp = (Tp - before2) / g;
+        const int vl = chunk * kChunk + lane;
+        const int v = v0 + vl;
+        const bool valid = vl < nrows;
+        const double e = valid ? (double)sBias[(size_t)b * rows_cap + vl] : 0.0;
+        const int pl = pick_lane(e, 0.0, Tpp);
+        const int x = __shfl_sync(0xffffffffu, valid ? v : 0, pl);
+        // start pulling U[x] into L2 for every CTA's next position, publish
+        // {position, token}, then write the outputs
+        if (k + 1 < K && lane < (kGRank * 2) / 128)
+          prefetch_l2(reinterpret_cast<const uint8_t*>(p.U + (size_t)x * kGRank) + lane * 128);
+        if (lane == 0) st_rec(rec.tok + (size_t)b * kGRecWords, (uint32_t)x, seq);
+        if (lane == pl) {
+          const size_t o = (size_t)b * K + k;
+          if (!(Z > 0.0) || !isfinite(Z)) {
+            raise_flag(p.flags, DSPARK_FLAG_NONFINITE);
+            p.tokens[o] = 0;
+            p.p_tok[o] = 0.0f;
+            p.lse[o] = CUDART_NAN_F;
+            p.ref_max[o] = M;
+            p.ref_sum[o] = 1.0f;
           } else {
-            const unsigned hp = __ballot_sync(0xffffffffu, wA > 0.0 || wB > 0.0);
-            const int hl = hp ? 31 - __clz(hp) : 0;
-            chunk = __shfl_sync(0xffffffffu, (wB > 0.0) ? cb2 : ca, hl);
-            if (!hp) chunk = 0;
-            before2 = -CUDART_INF;
+            p.tokens[o] = x;
+            p.p_tok[o] = (float)(f * g * e / Z);
+            p.lse[o] = (float)((double)M * (double)itv[b] + log(Z));
+            p.ref_max[o] = M;
+            p.ref_sum[o] = (float)Z;
           }
-          // level 3: the chunk's rows from shared memory
-          const int vl = chunk * kChunk + lane;
-          const int v = v0 + vl;
-          const bool valid = vl < nrows;
-          float ef = 0.0f;
-          if (valid)
-            ef = ex2(((bse[(size_t)b * rows_cap + vl] - M) + sBias[(size_t)b * rows_cap + vl]) * it2[b]);
-          const int pl = pick_lane((double)ef, before2, T);
-          const int x = __shfl_sync(0xffffffffu, valid ? v : 0, pl);
-          // start pulling U[x] into L2 for every CTA's next position
-          if (k + 1 < K && lane < (kGRank * 2) / 128)
-            prefetch_l2(reinterpret_cast<const uint8_t*>(p.U + (size_t)x * kGRank) + lane * 128);
-          if (lane == pl) {
-            const size_t o = (size_t)b * K + k;
-            if (!(Z > 0.0) || !isfinite(Z)) {
-              raise_flag(p.flags, DSPARK_FLAG_NONFINITE);
-              p.tokens[o] = 0;
-              p.p_tok[o] = 0.0f;
-              p.lse[o] = CUDART_NAN_F;
-              p.ref_max[o] = M;
-              p.ref_sum[o] = 1.0f;
-            } else {
-              p.tokens[o] = x;
-              p.p_tok[o] = (float)((double)ef / Z);
-              p.lse[o] = (float)((double)M * (double)itv[b] + log(Z));
-              p.ref_max[o] = M;
-              p.ref_sum[o] = (float)Z;
-            }
-          }
-          // publish {position, token}
-          if (lane == 0) st_rec(rec.tok + (size_t)b * kGRecWords, (uint32_t)x, seq);
         }
       }
       // one thread per request waits for the token; every warp then loads its U[x] slice
@@ -1350,6 +1419,7 @@ inline bool persist_supported(int V, int r, int B) {
     int max_chunks, max_tiles;
     gemv_runs(n_chunks_of(V), L.G, &max_chunks, &max_tiles);
     if (max_chunks > kGMaxChunks) return false;
+    return L.max_nt <= kPMaxTiles && L.n_stages >= 1;  // any ring depth is deadlock-free
   }
   return L.max_nt <= kPMaxTiles && L.n_stages >= kPMinStages;
 }

@@ -123,6 +123,7 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
   __shared__ int s_len[kFMaxB];
   __shared__ float s_it2[kFMaxB];
   __shared__ int s_prev[kFMaxB];
+  __shared__ long long s_rs[kFMaxB];    // row_start
   __shared__ float s_tmax[kFMaxRows];
   __shared__ double s_tz[kFMaxRows];
   __shared__ float s_tx[kFMaxRows];    // target logit of the drafted token (p < L)
@@ -140,19 +141,34 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
   const int G = gridDim.x, cta = blockIdx.x;
   const int B = a.B, K = a.K, V = a.V;
 
+  // per-request inputs, one thread each (all loads in flight together)
+  if (tid < B) {
+    const int b = tid;
+    s_len[b] = checked_len(a.verify_len, b, K, a.flags);
+    s_it2[b] = checked_inv_temp(a.inv_temp, b, a.flags) * kLog2e;
+    s_prev[b] = checked_token(a.prev_token[b], V, true, a.flags);
+    s_rs[b] = a.row_start[b];
+  }
+  __syncthreads();
   if (tid == 0) {
     int r = 0;
     for (int b = 0; b < B; ++b) {
-      const int L = checked_len(a.verify_len, b, K, a.flags);
       s_rofs[b] = r;
-      s_len[b] = L;
-      s_it2[b] = checked_inv_temp(a.inv_temp, b, a.flags) * kLog2e;
-      s_prev[b] = checked_token(a.prev_token[b], V, true, a.flags);
-      r += L + 1;
+      r += s_len[b] + 1;
     }
     s_rofs[B] = r;
   }
   __syncthreads();
+  // target row of request b, position p (clamped into [0, n_rows), which
+  // raises DSPARK_FLAG_BAD_LENGTH)
+  auto trow_of = [&](int b, int p) {
+    long long row = s_rs[b] + p;
+    if (row < 0 || row >= a.n_rows) {
+      raise_flag(a.flags, DSPARK_FLAG_BAD_LENGTH);
+      row = row < 0 ? 0 : a.n_rows - 1;
+    }
+    return row;
+  };
   const int R = s_rofs[B];
   auto row_of = [&](int rho, int* pb) {
     int b = 0;
@@ -161,20 +177,21 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
     return rho - s_rofs[b];
   };
 
-  // per-row inputs of the accept scan, loaded now and stored after phase 1
-  float g_tx = 0.0f, g_pd = 1.0f, g_ua = 0.0f, g_dmax = 0.0f, g_dsum = 1.0f;
-  int g_tok = 0;
-  if (tid < R) {
-    int b;
-    const int p = row_of(tid, &b);
-    if (p < K) {
-      const size_t o = (size_t)b * K + p;
+  // per-row inputs of the accept scan: loaded now, used after phase 1 (the
+  // target value at the drafted token is gathered after phase 1, once the
+  // token has arrived and the row is in L2)
+  float g_pd = 1.0f, g_ua = 0.0f, g_dmax = 0.0f, g_dsum = 1.0f;
+  int g_tokraw = 0;
+  const bool g_row = tid < R;
+  int g_b = 0, g_p = 0;
+  if (g_row) {
+    g_p = row_of(tid, &g_b);
+    if (g_p < K) {
+      const size_t o = (size_t)g_b * K + g_p;
       g_dmax = a.ref_max[o];
       g_dsum = a.ref_sum[o];
-      if (p < s_len[b]) {
-        g_tok = checked_token(a.tokens[o], V, false, a.flags);
-        const long long row = checked_row(a.row_start, b, p, a.n_rows, a.flags);
-        g_tx = a.target[(size_t)row * V + g_tok];
+      if (g_p < s_len[g_b]) {
+        g_tokraw = a.tokens[o];
         g_pd = a.p_tok[o];
         g_ua = a.u_accept[o];
       }
@@ -195,10 +212,8 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
     const int pA = row_of(rowA, &bA);
     const int pB = (rowA + 1 < R) ? row_of(rowA + 1, &bB) : 0;
     const float it2A = s_it2[bA], it2B = s_it2[bB];
-    const float* tA = a.target + (size_t)checked_row(a.row_start, bA, pA, a.n_rows, a.flags) * V;
-    const float* tB = (rowA + 1 < R)
-                          ? a.target + (size_t)checked_row(a.row_start, bB, pB, a.n_rows, a.flags) * V
-                          : tA;
+    const float* tA = a.target + (size_t)trow_of(bA, pA) * V;
+    const float* tB = (rowA + 1 < R) ? a.target + (size_t)trow_of(bB, pB) * V : tA;
     const int n4 = (int)((e1 - e0) / 4);
     float mA = -CUDART_INF_F, sA = 0.0f, mB = -CUDART_INF_F, sB = 0.0f;
     for (int j0 = 0; j0 < n4; j0 += kFBatch * kFThreads) {
@@ -263,9 +278,15 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
       st_pair(r + 2, __float_as_uint(M[1]), __float_as_uint((float)S[1]));
     }
   }
-  if (tid < R) {
-    s_tx[tid] = g_tx;
-    s_tok[tid] = g_tok;
+  if (g_row) {
+    float tx = 0.0f;
+    int tok = 0;
+    if (g_p < K && g_p < s_len[g_b]) {
+      tok = checked_token(g_tokraw, V, false, a.flags);
+      tx = a.target[(size_t)trow_of(g_b, g_p) * V + tok];
+    }
+    s_tx[tid] = tx;
+    s_tok[tid] = tok;
     s_pd[tid] = g_pd;
     s_ua[tid] = g_ua;
     s_dmax[tid] = g_dmax;
@@ -355,7 +376,7 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
     }
     if (lane == 0) {
       ResInfo ri;
-      ri.row = checked_row(a.row_start, b, j, a.n_rows, a.flags);
+      ri.row = trow_of(b, j);
       ri.j = j;
       ri.bonus = (j == L) ? 1 : 0;
       ri.t_max = s_tmax[r0 + j];
