@@ -778,13 +778,12 @@ __device__ __forceinline__ float fma_bf16_hi(uint32_t w, uint32_t u, float c) {
 }
 
 // pr[b][row] += sum_{e<8} w_e * u_e over the 8 bf16 packed in q and in u[b]
-// (ascending e, one rounding per step)
+// (ascending e, one rounding per step), for all NB requests (the kernel runs
+// with exactly NB requests: no runtime test splits the unrolled FMA stream)
 template <int NB>
-__device__ __forceinline__ void gemv8(uint4 q, const uint32_t (&u)[NB][4], int B, float (&pr)[NB][32],
-                                      int row) {
+__device__ __forceinline__ void gemv8(uint4 q, const uint32_t (&u)[NB][4], float (&pr)[NB][32], int row) {
 #pragma unroll
   for (int b = 0; b < NB; ++b) {
-    if (b >= B) break;
     float a = pr[b][row];
     a = fma_bf16_lo(q.x, u[b][0], a); a = fma_bf16_hi(q.x, u[b][0], a);
     a = fma_bf16_lo(q.y, u[b][1], a); a = fma_bf16_hi(q.y, u[b][1], a);
@@ -844,7 +843,8 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = gridDim.x, cta = blockIdx.x;
-  const int B = p.B, K = p.K, V = p.V;
+  constexpr int B = NB;  // launched with exactly NB requests
+  const int K = p.K, V = p.V;
   const int S = p.n_stages;
   const int c_begin = gemv_chunk_begin(cta, G, p.n_chunks);
   const int nc = gemv_chunk_begin(cta + 1, G, p.n_chunks) - c_begin;  // chunks of this CTA
@@ -1095,8 +1095,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             if (g + 1 < 8) tmem_ld16_issue(ta + (uint32_t)((g + 1) * 16), nxt);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-              gemv8<NB>(make_uint4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]), u, B, pr,
-                        g * 4 + j);
+              gemv8<NB>(make_uint4(cur[4 * j], cur[4 * j + 1], cur[4 * j + 2], cur[4 * j + 3]), u, pr, g * 4 + j);
             if (g + 1 < 8) tmem_ld16_wait(nxt);
           }
         } else {
@@ -1111,13 +1110,13 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           } else {
             buf = (type == 1) ? sRes + idx * kStageBytes : sTail;
           }
-          // two halves of 16 rows: the barrier keeps the compiler from
+          // four groups of 8 rows: the barriers keep the compiler from
           // hoisting all 32 shared loads (128 registers) at once
 #pragma unroll
           for (int rr = 0; rr < 32; ++rr) {
-            if (rr == 16) asm volatile("" ::: "memory");
+            if ((rr & 7) == 0 && rr > 0) asm volatile("" ::: "memory");
             const uint4 q = *reinterpret_cast<const uint4*>(buf + rr * (kGRank * 2) + lane * 16);
-            gemv8<NB>(q, u, B, pr, rr);
+            gemv8<NB>(q, u, pr, rr);
           }
           if (type == 2) {
             __syncwarp();
@@ -1131,7 +1130,6 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
         const int v = v0 + vl;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          if (b >= B) break;
           const float bias = transpose_reduce32(pr[b], lane);
           sBias[(size_t)b * rows_cap + vl] = bias;
           if (valid) {
@@ -1148,7 +1146,6 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
       for (int n0 = 0; n0 < n_units; n0 += 4) {
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-          if (b >= B) break;
           float bv[4], bi[4], am[4], es[4];
           bool ok4[4];
 #pragma unroll
