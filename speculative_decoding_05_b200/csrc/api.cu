@@ -263,9 +263,16 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
     a.B = B;
     a.K = K;
     a.n_chunks = nc;
+    static bool fused_attr = false;
+    if (!fused_attr) {
+      cudaFuncSetAttribute(verify_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kFBufFloats * (int)sizeof(float));
+      fused_attr = true;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kFThreads);
+    cfg.dynamicSmemBytes = kFBufFloats * sizeof(float);
     cfg.stream = s;
     cudaLaunchAttribute attrs[1];
     attrs[0].id = cudaLaunchAttributeCooperative;

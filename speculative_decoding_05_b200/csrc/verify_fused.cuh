@@ -43,7 +43,7 @@ constexpr int kFThreads = 512;
 constexpr int kFWarps = kFThreads / 32;
 constexpr int kFMaxB = 4;
 constexpr int kFMaxRows = 72;              // B * (K + 1)
-constexpr int kFBatch = 12;                // float4 loads per thread in flight in phase 1
+constexpr int kFBufFloats = 24576;         // shared staging buffer (96 KB)
 constexpr int kFPerLane = 5;               // CTA totals per lane: grid <= 160
 constexpr int kFMaxG = 32 * kFPerLane;
 constexpr int kFMaxChunks = 64;            // residual chunks of one CTA (two per lane)
@@ -136,11 +136,18 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
   __shared__ float2 s_chunk[kFMaxB][kFMaxChunks];
   __shared__ float s_wm[2][kFWarps];
   __shared__ double s_ws[2][kFWarps];
+  __shared__ uint64_t s_bar;             // bulk copies into s_buf
+  extern __shared__ __align__(16) float s_buf[];  // kFBufFloats
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int B = a.B, K = a.K, V = a.V;
 
+  if (tid == 0) {
+    mbar_init(&s_bar, 1);
+    fence_barrier_init();
+  }
+  uint32_t bar_phase = 0;
   // per-request inputs, one thread each (all loads in flight together)
   if (tid < B) {
     const int b = tid;
@@ -214,42 +221,45 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
     const float it2A = s_it2[bA], it2B = s_it2[bB];
     const float* tA = a.target + (size_t)trow_of(bA, pA) * V;
     const float* tB = (rowA + 1 < R) ? a.target + (size_t)trow_of(bB, pB) * V : tA;
-    const int n4 = (int)((e1 - e0) / 4);
     float mA = -CUDART_INF_F, sA = 0.0f, mB = -CUDART_INF_F, sB = 0.0f;
-    for (int j0 = 0; j0 < n4; j0 += kFBatch * kFThreads) {
-      float4 x[kFBatch];
-      bool inB[kFBatch], ok[kFBatch];
-#pragma unroll
-      for (int i = 0; i < kFBatch; ++i) {
-        const int j = j0 + i * kFThreads + tid;
-        ok[i] = j < n4;
-        const long long e = e0 + 4ll * j;
-        inB[i] = e >= bnd;
-        if (ok[i]) {
-          const float* src = inB[i] ? tB + (e - bnd) : tA + (e - (long long)rowA * V);
-          x[i] = __ldg(reinterpret_cast<const float4*>(src));
-        }
+    // pieces of at most kFBufFloats: one or two bulk copies each (the part
+    // in row A, the part in row B) into shared memory, then one pass
+    for (long long p0 = e0; p0 < e1; p0 += kFBufFloats) {
+      const long long p1 = min(e1, p0 + kFBufFloats);
+      const long long a1 = min(p1, bnd), b0 = max(p0, bnd);
+      const int nA = (int)max(0ll, a1 - p0), nB = (int)max(0ll, p1 - b0);
+      if (tid == 0) {
+        const uint64_t pol = policy_evict_last();  // row j is read again for the residual
+        fence_proxy_async_smem();  // earlier reads of s_buf before the copies' writes
+        mbar_arrive_expect_tx(&s_bar, (uint32_t)(nA + nB) * 4u);
+        if (nA > 0) bulk_load(s_buf, tA + (p0 - (long long)rowA * V), (uint32_t)nA * 4u, &s_bar, pol);
+        if (nB > 0) bulk_load(s_buf + nA, tB + (b0 - bnd), (uint32_t)nB * 4u, &s_bar, pol);
       }
+      if (!mbar_wait(&s_bar, bar_phase)) {
+        if (tid == 0) raise_flag(a.flags, DSPARK_FLAG_TIMEOUT);
+      }
+      bar_phase ^= 1u;
+      const int n4 = (nA + nB) / 4;
       float ma = -CUDART_INF_F, mb = -CUDART_INF_F;
-#pragma unroll
-      for (int i = 0; i < kFBatch; ++i) {
-        if (!ok[i]) continue;
-        const float m4 = fmaxf(fmaxf(x[i].x, x[i].y), fmaxf(x[i].z, x[i].w));
-        if (inB[i]) mb = fmaxf(mb, m4);
+      for (int j = tid; j < n4; j += kFThreads) {
+        const float4 x = reinterpret_cast<const float4*>(s_buf)[j];
+        const float m4 = fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w));
+        if (4 * j >= nA) mb = fmaxf(mb, m4);
         else ma = fmaxf(ma, m4);
       }
       float sa = 0.0f, sb = 0.0f;
-#pragma unroll
-      for (int i = 0; i < kFBatch; ++i) {
-        if (!ok[i]) continue;
-        const float m = inB[i] ? mb : ma, it2 = inB[i] ? it2B : it2A;
-        const float e4 = ex2((x[i].x - m) * it2) + ex2((x[i].y - m) * it2) + ex2((x[i].z - m) * it2) +
-                         ex2((x[i].w - m) * it2);
-        if (inB[i]) sb += e4;
+      for (int j = tid; j < n4; j += kFThreads) {
+        const float4 x = reinterpret_cast<const float4*>(s_buf)[j];
+        const bool inB = 4 * j >= nA;
+        const float m = inB ? mb : ma, it2 = inB ? it2B : it2A;
+        const float e4 = ex2((x.x - m) * it2) + ex2((x.y - m) * it2) + ex2((x.z - m) * it2) +
+                         ex2((x.w - m) * it2);
+        if (inB) sb += e4;
         else sa += e4;
       }
       merge_partial(mA, sA, ma, sa, it2A);
       merge_partial(mB, sB, mb, sb, it2B);
+      __syncthreads();  // s_buf is refilled by the next piece
     }
     // warp, then CTA (fp64)
     const float MwA = warp_max(mA), MwB = warp_max(mB);
@@ -400,47 +410,46 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
   // ---------------------------------------------------------------- phase 3
   const int c_begin = (int)((long long)cta * a.n_chunks / G);
   const int nch = (int)((long long)(cta + 1) * a.n_chunks / G) - c_begin;
-  {
-    const int n_pairs = B * nch;
-    for (int q0 = warp; q0 < n_pairs; q0 += 2 * kFWarps) {
-      float t[2], bv[2], bi[2];
-      int bb[2], lc[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int q = q0 + h * kFWarps;
-        t[h] = 0.0f;
-        bv[h] = 0.0f;
-        bi[h] = 0.0f;
-        bb[h] = 0;
-        lc[h] = 0;
-        if (q < n_pairs) {
-          const int b = q / nch;
-          bb[h] = b;
-          lc[h] = q - b * nch;
-          const int v = (c_begin + lc[h]) * kChunk + lane;
-          if (v < V) {
-            const ResInfo& ri = s_ri[b];
-            t[h] = a.target[(size_t)ri.row * V + v];
-            if (!ri.bonus) {
-              const size_t drow = ((size_t)b * K + ri.j) * (size_t)V;
-              bv[h] = a.base[drow + v];
-              bi[h] = a.draft_bias[drow + v];
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int q = q0 + h * kFWarps;
-        if (q >= n_pairs) break;
-        const int b = bb[h];
-        const int v = (c_begin + lc[h]) * kChunk + lane;
-        float qv = 0.0f, pt = 0.0f;
-        if (v < V) qv = residual_q(t[h], bv[h], bi[h], s_ri[b], s_it2[b], &pt);
-        const float Q = warp_sum(qv), P = warp_sum(pt);
-        if (lane == 0) s_chunk[b][lc[h]] = make_float2(Q, P);
+  // the residual row's inputs of this CTA's chunk run, per request: target
+  // row j, draft base and bias rows j (bulk copies into s_buf)
+  const int n3 = nch * kChunk;                                  // floats per slice
+  const int len3 = max(0, min(V, (c_begin + nch) * kChunk) - c_begin * kChunk);
+  if (tid == 0 && len3 > 0) {
+    const uint64_t pol = policy_evict_first();
+    uint32_t bytes = 0;
+    for (int b = 0; b < B; ++b) bytes += (s_ri[b].bonus ? 1u : 3u) * (uint32_t)len3 * 4u;
+    fence_proxy_async_smem();  // phase 1's reads of s_buf before the copies' writes
+    mbar_arrive_expect_tx(&s_bar, bytes);
+    for (int b = 0; b < B; ++b) {
+      const ResInfo& ri = s_ri[b];
+      const size_t c0 = (size_t)c_begin * kChunk;
+      bulk_load(s_buf + (b * 3) * n3, a.target + (size_t)ri.row * V + c0, (uint32_t)len3 * 4u, &s_bar, pol);
+      if (!ri.bonus) {
+        const size_t drow = ((size_t)b * K + ri.j) * (size_t)V + c0;
+        bulk_load(s_buf + (b * 3 + 1) * n3, a.base + drow, (uint32_t)len3 * 4u, &s_bar, pol);
+        bulk_load(s_buf + (b * 3 + 2) * n3, a.draft_bias + drow, (uint32_t)len3 * 4u, &s_bar, pol);
       }
     }
+  }
+  if (len3 > 0) {
+    if (!mbar_wait(&s_bar, bar_phase)) {
+      if (tid == 0) raise_flag(a.flags, DSPARK_FLAG_TIMEOUT);
+    }
+    bar_phase ^= 1u;
+  }
+  for (int q = warp; q < B * nch; q += kFWarps) {
+    const int b = q / nch, lc = q - b * nch;
+    const int vl = lc * kChunk + lane;  // element within the run
+    float qv = 0.0f, pt = 0.0f;
+    if (vl < len3) {
+      const ResInfo& ri = s_ri[b];
+      const float t = s_buf[(b * 3) * n3 + vl];
+      const float bv = ri.bonus ? 0.0f : s_buf[(b * 3 + 1) * n3 + vl];
+      const float bi = ri.bonus ? 0.0f : s_buf[(b * 3 + 2) * n3 + vl];
+      qv = residual_q(t, bv, bi, ri, s_it2[b], &pt);
+    }
+    const float Q = warp_sum(qv), P = warp_sum(pt);
+    if (lane == 0) s_chunk[b][lc] = make_float2(Q, P);
   }
   __syncthreads();
   if (warp < B) {
@@ -573,16 +582,13 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
       }
       // token: the chunk's 32 entries, recomputed
       const int v = (c_begin + chunk) * kChunk + lane;
-      const bool valid = v < V;
+      const int vl = chunk * kChunk + lane;
+      const bool valid = vl < len3;
       double e = 0.0;
       if (valid) {
-        const float t = a.target[(size_t)ri.row * V + v];
-        float bv = 0.0f, bi = 0.0f;
-        if (!ri.bonus) {
-          const size_t drow = ((size_t)b * K + ri.j) * (size_t)V;
-          bv = a.base[drow + v];
-          bi = a.draft_bias[drow + v];
-        }
+        const float t = s_buf[(b * 3) * n3 + vl];
+        const float bv = ri.bonus ? 0.0f : s_buf[(b * 3 + 1) * n3 + vl];
+        const float bi = ri.bonus ? 0.0f : s_buf[(b * 3 + 2) * n3 + vl];
         float pt;
         const float qv = residual_q(t, bv, bi, ri, s_it2[b], &pt);
         e = (double)(use_q ? qv : pt);
