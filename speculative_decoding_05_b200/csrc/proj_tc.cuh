@@ -34,9 +34,10 @@ namespace dspark {
 constexpr int kTcThreads = 352;
 constexpr int kBlockM = 128;
 constexpr int kTileN = 128;
-constexpr int kWStages = 4;
+constexpr int kWStagesMax = 12;     // W ring depth: as deep as shared memory allows
 constexpr int kBStages = 5;
 constexpr int kStageBytes = 16384;  // 128 rows x 128 bytes
+constexpr size_t kTcSmemLimit = 232448 - 1024;  // dynamic: 227 KB less the static arrays
 constexpr int kTmemCols = 256;
 
 struct TcPlan {
@@ -47,11 +48,26 @@ struct TcPlan {
   const __nv_bfloat16* U;
   int V, r, B, K;
   int n_tiles, n_bb, ctas_per_bb;
+  int w_stages, base_rows;  // W ring depth, request rows per base box
 };
 
-inline size_t tc_smem_bytes(int r, bool residual) {
-  return 1024 + (size_t)(r / 64) * kStageBytes + (size_t)kWStages * kStageBytes +
-         (residual ? 0 : (size_t)kBStages * kStageBytes) + 256;
+// Request rows of a base-logit box: the batch rounded up to 8 (the 128-byte
+// swizzle repeats every 8 rows), at most one block of kBlockM.  A batch of 64
+// then moves half the bytes of a full 128-row box.
+inline int tc_base_rows(int B) { return B < kBlockM ? (B + 7) / 8 * 8 : kBlockM; }
+// W ring depth: what shared memory holds after operand A and the base ring.
+// With the ring one tile deep, the next tile's W could only start loading
+// once the current tile's MMAs had released it.
+inline int tc_w_stages(int r, int B, bool residual) {
+  const size_t fixed = 1024 + (size_t)(r / 64) * kStageBytes +
+                       (residual ? 0 : (size_t)kBStages * tc_base_rows(B) * 128) + 512;
+  int s = (int)((kTcSmemLimit - fixed) / kStageBytes);
+  if (s > kWStagesMax) s = kWStagesMax;
+  return s;
+}
+inline size_t tc_smem_bytes(int r, int B, bool residual) {
+  return 1024 + (size_t)(r / 64) * kStageBytes + (size_t)tc_w_stages(r, B, residual) * kStageBytes +
+         (residual ? 0 : (size_t)kBStages * tc_base_rows(B) * 128) + 512;
 }
 
 inline bool tc_supported(int V, int r, int B) {
@@ -67,17 +83,18 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                const float* __restrict__ base, const ResInfo* __restrict__ info,
                float* __restrict__ draft_logits, float* __restrict__ draft_bias,
                float2* __restrict__ part, int n_chunks, int n_tiles, int ctas_per_bb,
-               unsigned* flags) {
+               int n_ws, int base_rows, unsigned* flags) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nkb = r >> 6;
   uint8_t* sA = sm;
+  const int bstage = base_rows * 128;  // bytes of one base box
   uint8_t* sW = sA + nkb * kStageBytes;
-  uint8_t* sBase = sW + kWStages * kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + (kRes ? 0 : kBStages * kStageBytes));
+  uint8_t* sBase = sW + n_ws * kStageBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + (kRes ? 0 : kBStages * bstage));
   uint64_t* fullW = bars;
-  uint64_t* emptyW = fullW + kWStages;
-  uint64_t* fullB = emptyW + kWStages;
+  uint64_t* emptyW = fullW + kWStagesMax;
+  uint64_t* fullB = emptyW + kWStagesMax;
   uint64_t* emptyB = fullB + kBStages;
   uint64_t* accFull = emptyB + kBStages;
   uint64_t* accEmpty = accFull + 2;
@@ -90,7 +107,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   const int t1 = (int)((long long)(pi + 1) * n_tiles / ctas_per_bb);
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kWStages; ++i) {
+    for (int i = 0; i < n_ws; ++i) {
       mbar_init(&fullW[i], 1);
       mbar_init(&emptyW[i], 1);
     }
@@ -107,10 +124,13 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
 
-  // operand A: the previous-token rows of U for this block of requests
-  const int cpr = r >> 3;  // 16-byte chunks per row
-  for (int q = threadIdx.x; q < kBlockM * cpr; q += kTcThreads) {
-    const int m = q / cpr, c = q % cpr;
+  // operand A: the previous-token rows of U for this block of requests.  The
+  // 128 token ids go to shared memory first (one round of loads), then every
+  // thread issues all of its U loads before storing any, so the gather costs
+  // two memory round trips rather than one per loop iteration.
+  __shared__ int s_x[kBlockM];
+  if (threadIdx.x < kBlockM) {
+    const int m = threadIdx.x;
     const int b = bb * kBlockM + m;
     int x = -1;
     if (b < B) {
@@ -120,15 +140,36 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       } else {
         x = (k == 0) ? prev_token[b] : tokens[(size_t)b * K + (k - 1)];
         if (x >= V || (k > 0 && x < 0)) {
-          if (c == 0) raise_flag(flags, DSPARK_FLAG_BAD_TOKEN);
+          raise_flag(flags, DSPARK_FLAG_BAD_TOKEN);
           x = (k > 0) ? (x < 0 ? 0 : V - 1) : -1;
         }
       }
     }
-    uint4 val = make_uint4(0, 0, 0, 0);
-    if (x >= 0) val = __ldg(reinterpret_cast<const uint4*>(U + (size_t)x * r) + c);
-    const int kb = c >> 3, j = c & 7;
-    *reinterpret_cast<uint4*>(sA + kb * kStageBytes + m * 128 + ((j ^ (m & 7)) << 4)) = val;
+    s_x[m] = x;
+  }
+  __syncthreads();
+  {
+    const int cpr = r >> 3;  // 16-byte chunks per row
+    constexpr int kPer = (kBlockM * 32 + kTcThreads - 1) / kTcThreads;  // r <= 256: 32 chunks per row
+    uint4 val[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int q = threadIdx.x + i * kTcThreads;
+      val[i] = make_uint4(0, 0, 0, 0);
+      if (q < kBlockM * cpr) {
+        const int x = s_x[q / cpr];
+        if (x >= 0) val[i] = __ldg(reinterpret_cast<const uint4*>(U + (size_t)x * r) + (q % cpr));
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int q = threadIdx.x + i * kTcThreads;
+      if (q < kBlockM * cpr) {
+        const int m = q / cpr, c = q % cpr;
+        const int kb = c >> 3, j = c & 7;
+        *reinterpret_cast<uint4*>(sA + kb * kStageBytes + m * 128 + ((j ^ (m & 7)) << 4)) = val[i];
+      }
+    }
   }
   fence_proxy_async_smem();
   tc_fence_before();
@@ -143,8 +184,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       int it = 0;
       for (int t = t0; t < t1 && !*s_abort; ++t) {
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % kWStages;
-          const uint32_t ph = (uint32_t)(it / kWStages) & 1u;
+          const int s = it % n_ws;
+          const uint32_t ph = (uint32_t)(it / n_ws) & 1u;
           if (!mbar_wait(&emptyW[s], ph ^ 1u)) {
             *s_abort = 1;
             raise_flag(flags, DSPARK_FLAG_TIMEOUT);
@@ -172,8 +213,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         tc_fence_after();
         bool ok = true;
         for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % kWStages;
-          const uint32_t ph = (uint32_t)(it / kWStages) & 1u;
+          const int s = it % n_ws;
+          const uint32_t ph = (uint32_t)(it / n_ws) & 1u;
           if (!mbar_wait(&fullW[s], ph)) {
             ok = false;
             break;
@@ -209,8 +250,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             raise_flag(flags, DSPARK_FLAG_TIMEOUT);
             break;
           }
-          mbar_arrive_expect_tx(&fullB[s], kStageBytes);
-          tma_load_3d_hint(sBase + s * kStageBytes, &tm_base, &fullB[s], t * kTileN + cb * 32, k,
+          mbar_arrive_expect_tx(&fullB[s], (uint32_t)bstage);
+          tma_load_3d_hint(sBase + s * bstage, &tm_base, &fullB[s], t * kTileN + cb * 32, k,
                            bb * kBlockM, pol);
         }
       }
@@ -251,10 +292,13 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             *s_abort = 1;
             raise_flag(flags, DSPARK_FLAG_TIMEOUT);
           }
-          const uint8_t* row = sBase + s * kStageBytes + m * 128;
+          // a box holds base_rows requests: rows past it are not read (their
+          // results are discarded, since base_rows >= the block's requests)
+          const uint8_t* row = sBase + s * bstage + m * 128;
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float4 q4 = *reinterpret_cast<const float4*>(row + ((j ^ (m & 7)) << 4));
+            float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (m < base_rows) q4 = *reinterpret_cast<const float4*>(row + ((j ^ (m & 7)) << 4));
             bv[4 * j] = q4.x; bv[4 * j + 1] = q4.y; bv[4 * j + 2] = q4.z; bv[4 * j + 3] = q4.w;
           }
           __syncwarp();
@@ -383,7 +427,7 @@ inline bool encode_base_map(CUtensorMap* m, const float* base, int V, int K, int
   if (!enc) return false;
   cuuint64_t dims[3] = {(cuuint64_t)V, (cuuint64_t)K, (cuuint64_t)B};
   cuuint64_t strides[2] = {(cuuint64_t)V * 4, (cuuint64_t)K * V * 4};
-  cuuint32_t box[3] = {32, 1, (cuuint32_t)kBlockM};
+  cuuint32_t box[3] = {32, 1, (cuuint32_t)tc_base_rows(B)};
   cuuint32_t es[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box,
              es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -408,6 +452,8 @@ inline dspark_status tc_plan_draft(TcPlan& p, const float* base, const void* U, 
   if (!encode_w_map(&p.tm_w, W, V, r) || !encode_base_map(&p.tm_base, base, V, K, B))
     return DSPARK_ERR_CUDA;
   tc_grid(p);
+  p.w_stages = tc_w_stages(r, B, false);
+  p.base_rows = tc_base_rows(B);
   return DSPARK_OK;
 }
 
@@ -420,6 +466,8 @@ inline dspark_status tc_plan_residual(TcPlan& p, const float* target, const floa
   if (!encode_w_map(&p.tm_w, W, V, r)) return DSPARK_ERR_CUDA;
   p.tm_base = p.tm_w;  // unused in residual mode
   tc_grid(p);
+  p.w_stages = tc_w_stages(r, B, true);
+  p.base_rows = tc_base_rows(B);
   return DSPARK_OK;
 }
 
@@ -428,7 +476,7 @@ inline void tc_set_attr() {
   static bool done = false;
   if (!done) {
     cudaFuncSetAttribute(proj_tc_kernel<kRes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)tc_smem_bytes(256, kRes));
+                         (int)kTcSmemLimit);
     done = true;
   }
 }
@@ -437,17 +485,17 @@ inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const i
                             const float* it, float* dl, float* dbias, float2* part,
                             unsigned* flags, cudaStream_t s) {
   tc_set_attr<false>();
-  proj_tc_kernel<false><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, false), s>>>(
+  proj_tc_kernel<false><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, false), s>>>(
       p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, k, prev, tokens, it, nullptr, p.base, nullptr,
-      dl, dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, flags);
+      dl, dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.base_rows, flags);
 }
 
 inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,
                                float2* rpart, unsigned* flags, cudaStream_t s) {
   tc_set_attr<true>();
-  proj_tc_kernel<true><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, true), s>>>(
+  proj_tc_kernel<true><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, true), s>>>(
       p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, 0, nullptr, nullptr, it, p.target, p.base, info,
-      nullptr, nullptr, rpart, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, flags);
+      nullptr, nullptr, rpart, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.base_rows, flags);
 }
 
 }  // namespace dspark
