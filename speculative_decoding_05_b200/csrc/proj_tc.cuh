@@ -35,7 +35,7 @@ constexpr int kTcThreads = 352;
 constexpr int kBlockM = 128;
 constexpr int kTileN = 128;
 constexpr int kWStagesMax = 12;     // W ring depth: as deep as shared memory allows
-constexpr int kBStages = 5;
+constexpr int kBStagesMax = 16;     // base ring depth (draft): likewise
 constexpr int kStageBytes = 16384;  // 128 rows x 128 bytes
 constexpr size_t kTcSmemLimit = 232448 - 1024;  // dynamic: 227 KB less the static arrays
 constexpr int kTmemCols = 256;
@@ -48,26 +48,34 @@ struct TcPlan {
   const __nv_bfloat16* U;
   int V, r, B, K;
   int n_tiles, n_bb, ctas_per_bb;
-  int w_stages, base_rows;  // W ring depth, request rows per base box
+  int w_stages, b_stages, base_rows;  // ring depths, request rows per base box
 };
 
 // Request rows of a base-logit box: the batch rounded up to 8 (the 128-byte
 // swizzle repeats every 8 rows), at most one block of kBlockM.  A batch of 64
 // then moves half the bytes of a full 128-row box.
 inline int tc_base_rows(int B) { return B < kBlockM ? (B + 7) / 8 * 8 : kBlockM; }
-// W ring depth: what shared memory holds after operand A and the base ring.
-// With the ring one tile deep, the next tile's W could only start loading
-// once the current tile's MMAs had released it.
+// Ring depths.  Draft: W gets one tile (r / 64 stages) and the base ring the
+// rest -- every base box is B separate 128-byte rows from DRAM (one per
+// request), so the base stream needs many boxes in flight.  Residual: no
+// base ring; W takes what operand A leaves.
+inline int tc_b_stages(int r, int B, bool residual) {
+  if (residual) return 0;
+  const size_t fixed = 1024 + (size_t)(r / 64) * kStageBytes * 2 + 512;
+  int s = (int)((kTcSmemLimit - fixed) / ((size_t)tc_base_rows(B) * 128));
+  if (s > kBStagesMax) s = kBStagesMax;
+  return s;
+}
 inline int tc_w_stages(int r, int B, bool residual) {
   const size_t fixed = 1024 + (size_t)(r / 64) * kStageBytes +
-                       (residual ? 0 : (size_t)kBStages * tc_base_rows(B) * 128) + 512;
+                       (size_t)tc_b_stages(r, B, residual) * tc_base_rows(B) * 128 + 512;
   int s = (int)((kTcSmemLimit - fixed) / kStageBytes);
   if (s > kWStagesMax) s = kWStagesMax;
   return s;
 }
 inline size_t tc_smem_bytes(int r, int B, bool residual) {
   return 1024 + (size_t)(r / 64) * kStageBytes + (size_t)tc_w_stages(r, B, residual) * kStageBytes +
-         (residual ? 0 : (size_t)kBStages * tc_base_rows(B) * 128) + 512;
+         (size_t)tc_b_stages(r, B, residual) * tc_base_rows(B) * 128 + 512;
 }
 
 inline bool tc_supported(int V, int r, int B) {
@@ -83,7 +91,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                const float* __restrict__ base, const ResInfo* __restrict__ info,
                float* __restrict__ draft_logits, float* __restrict__ draft_bias,
                float2* __restrict__ part, int n_chunks, int n_tiles, int ctas_per_bb,
-               int n_ws, int base_rows, unsigned* flags) {
+               int n_ws, int n_bs, int base_rows, unsigned* flags) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nkb = r >> 6;
@@ -91,12 +99,12 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   const int bstage = base_rows * 128;  // bytes of one base box
   uint8_t* sW = sA + nkb * kStageBytes;
   uint8_t* sBase = sW + n_ws * kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + (kRes ? 0 : kBStages * bstage));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + (kRes ? 0 : n_bs * bstage));
   uint64_t* fullW = bars;
   uint64_t* emptyW = fullW + kWStagesMax;
   uint64_t* fullB = emptyW + kWStagesMax;
-  uint64_t* emptyB = fullB + kBStages;
-  uint64_t* accFull = emptyB + kBStages;
+  uint64_t* emptyB = fullB + kBStagesMax;
+  uint64_t* accFull = emptyB + kBStagesMax;
   uint64_t* accEmpty = accFull + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accEmpty + 2);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -111,7 +119,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       mbar_init(&fullW[i], 1);
       mbar_init(&emptyW[i], 1);
     }
-    for (int i = 0; i < kBStages; ++i) {
+    for (int i = 0; i < n_bs; ++i) {
       mbar_init(&fullB[i], 1);
       mbar_init(&emptyB[i], 4);
     }
@@ -243,8 +251,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       int it = 0;
       for (int t = t0; t < t1 && !*s_abort; ++t) {
         for (int cb = 0; cb < kTileN / 32; ++cb, ++it) {
-          const int s = it % kBStages;
-          const uint32_t ph = (uint32_t)(it / kBStages) & 1u;
+          const int s = it % n_bs;
+          const uint32_t ph = (uint32_t)(it / n_bs) & 1u;
           if (!mbar_wait(&emptyB[s], ph ^ 1u)) {
             *s_abort = 1;
             raise_flag(flags, DSPARK_FLAG_TIMEOUT);
@@ -263,6 +271,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const int m = quarter * 32 + lane;
     const int b = bb * kBlockM + m;
     const bool bval = b < B;
+    // a warp whose 32 requests are all past the batch only keeps the
+    // pipeline moving (its arrivals), without loading or reducing anything
+    const bool wval = bb * kBlockM + quarter * 32 < B;
     const float it = bval ? checked_inv_temp(inv_temp, b, flags) : 1.0f;
     const float it2 = it * kLog2e;
     ResInfo ri{};
@@ -282,12 +293,12 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       for (int ci = 0; ci < 2; ++ci) {
         const int cb = 2 * eg + ci;
         float d[32], bv[32];
-        tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
+        if (wval) tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
         const int v0 = t * kTileN + cb * 32;
         if (!kRes) {
           const int itB = (t - t0) * (kTileN / 32) + cb;
-          const int s = itB % kBStages;
-          const uint32_t ph = (uint32_t)(itB / kBStages) & 1u;
+          const int s = itB % n_bs;
+          const uint32_t ph = (uint32_t)(itB / n_bs) & 1u;
           if (!mbar_wait(&fullB[s], ph)) {
             *s_abort = 1;
             raise_flag(flags, DSPARK_FLAG_TIMEOUT);
@@ -295,23 +306,29 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           // a box holds base_rows requests: rows past it are not read (their
           // results are discarded, since base_rows >= the block's requests)
           const uint8_t* row = sBase + s * bstage + m * 128;
+          if (wval) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (m < base_rows) q4 = *reinterpret_cast<const float4*>(row + ((j ^ (m & 7)) << 4));
-            bv[4 * j] = q4.x; bv[4 * j + 1] = q4.y; bv[4 * j + 2] = q4.z; bv[4 * j + 3] = q4.w;
+            for (int j = 0; j < 8; ++j) {
+              float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (m < base_rows) q4 = *reinterpret_cast<const float4*>(row + ((j ^ (m & 7)) << 4));
+              bv[4 * j] = q4.x; bv[4 * j + 1] = q4.y; bv[4 * j + 2] = q4.z; bv[4 * j + 3] = q4.w;
+            }
           }
           __syncwarp();
           if (lane == 0) mbar_arrive(&emptyB[s]);
-          float A = -CUDART_INF_F;
+          if (!wval) continue;
+          // four independent max and sum chains (the 32-long serial ones
+          // bounded the epilogue)
+          float A4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (v0 + j < V) A = fmaxf(A, bv[j] + d[j]);
-          float sum = 0.0f;
+            if (v0 + j < V) A4[j & 3] = fmaxf(A4[j & 3], bv[j] + d[j]);
+          const float A = fmaxf(fmaxf(A4[0], A4[1]), fmaxf(A4[2], A4[3]));
+          float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
           for (int j = 0; j < 32; ++j)
-            if (v0 + j < V) sum += ex2(((bv[j] - A) + d[j]) * it2);
-          pp[ci] = make_float2(A, sum);
+            if (v0 + j < V) s4[j & 3] += ex2(((bv[j] - A) + d[j]) * it2);
+          pp[ci] = make_float2(A, (s4[0] + s4[1]) + (s4[2] + s4[3]));
           if (draft_bias != nullptr && bval) {
             float* dst = draft_bias + ((size_t)b * K + k) * (size_t)V + v0;
 #pragma unroll
@@ -344,18 +361,18 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
               bv[j] = b4.x; bv[j + 1] = b4.y; bv[j + 2] = b4.z; bv[j + 3] = b4.w;
             }
           }
-          float qs = 0.0f, ps = 0.0f;
+          float qs4[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
           if (bval) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (v0 + j < V) {
                 float pt;
-                qs += residual_q(tq[j], bv[j], d[j], ri, it2, &pt);
-                ps += pt;
+                qs4[j & 3] += residual_q(tq[j], bv[j], d[j], ri, it2, &pt);
+                ps4[j & 3] += pt;
               }
             }
           }
-          pp[ci] = make_float2(qs, ps);
+          pp[ci] = make_float2((qs4[0] + qs4[1]) + (qs4[2] + qs4[3]), (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
         }
       }
       tc_fence_before();
@@ -453,6 +470,7 @@ inline dspark_status tc_plan_draft(TcPlan& p, const float* base, const void* U, 
     return DSPARK_ERR_CUDA;
   tc_grid(p);
   p.w_stages = tc_w_stages(r, B, false);
+  p.b_stages = tc_b_stages(r, B, false);
   p.base_rows = tc_base_rows(B);
   return DSPARK_OK;
 }
@@ -467,6 +485,7 @@ inline dspark_status tc_plan_residual(TcPlan& p, const float* target, const floa
   p.tm_base = p.tm_w;  // unused in residual mode
   tc_grid(p);
   p.w_stages = tc_w_stages(r, B, true);
+  p.b_stages = 0;
   p.base_rows = tc_base_rows(B);
   return DSPARK_OK;
 }
@@ -487,7 +506,7 @@ inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const i
   tc_set_attr<false>();
   proj_tc_kernel<false><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, false), s>>>(
       p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, k, prev, tokens, it, nullptr, p.base, nullptr,
-      dl, dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.base_rows, flags);
+      dl, dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, flags);
 }
 
 inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,
@@ -495,7 +514,7 @@ inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float
   tc_set_attr<true>();
   proj_tc_kernel<true><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, true), s>>>(
       p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, 0, nullptr, nullptr, it, p.target, p.base, info,
-      nullptr, nullptr, rpart, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.base_rows, flags);
+      nullptr, nullptr, rpart, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, flags);
 }
 
 }  // namespace dspark
