@@ -216,6 +216,10 @@ dspark_status draft_impl(const float* base, const void* U, const void* W, dspark
     } else {
       draft_proj_simt<TW>(nb, base, U, W, V, r, B, K, k, prev, tokens, it, dl, dbias, part, flags, s);
     }
+    // A plain launch: started early behind the projection, the sampler's
+    // small CTAs crowd onto the first SMs the projection frees (several per
+    // SM) and the position gets slower; launched after it, they spread one
+    // per SM.  The next projection still starts early, behind the sampler.
     draft_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
         base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, k, prev, tokens, it,
         ud, part, nc, dbias, p_tok, lse, rmax, rsum, flags);

@@ -10,6 +10,15 @@
 
 namespace dspark {
 
+// Programmatic dependent launch.  wait: block until the kernel this one was
+// launched behind has finished and its writes are visible (returns at once
+// when the launch carried no programmatic dependency).  launch_dependents:
+// let the kernel launched behind this one start its own prologue.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // sizes and workspace layout
 // ---------------------------------------------------------------------------

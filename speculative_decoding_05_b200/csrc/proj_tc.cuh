@@ -4,13 +4,26 @@
 // Each CTA owns a block of kBlockM = 128 requests (MMA M; rows past B are
 // zero) and a contiguous range of vocabulary tiles of kTileN = 128 rows
 // (MMA N); K = r (64..256).  The gathered U rows (operand A) are written to
-// shared memory once per launch in the 128-byte-swizzled K-major layout;
+// shared memory once per launch in the 128-byte-swizzled K-major layout,
+// only as many rows as the block has requests (rounded up to 8): the MMA
+// still reads 128 rows, and the ones past them fall on whatever bytes follow
+// in shared memory.  Row m of the product depends on row m of A alone, so
+// those rows only reach TMEM lanes of requests past the batch, which no
+// epilogue warp reads;
 // W tiles (operand B) stream through a TMA ring and the accumulator lives
 // in TMEM (two 128-column buffers, so the epilogue of tile t overlaps the
 // MMAs of tile t+1).  The epilogue thread of request b reads its TMEM row
 // (tcgen05.ld) and reduces every 32-row chunk of its row to a softmax
 // partial locally -- no cross-thread reduction, because the request is the
 // TMEM lane.
+//
+// In the draft the projection of position k >= 1 is launched while the
+// sampler of position k - 1 runs (programmatic dependent launch), and its two
+// producer warps start filling the W and base rings at once: neither depends
+// on the sampled tokens, and both inputs were complete before the call's
+// first projection got past its own wait (which its producers take too).
+// The other warps wait for the sampler to finish before reading tokens;
+// every write of the kernel comes after that wait.
 //
 //   warp 0       W producer (TMA, evict-last: W is re-read every position)
 //   warp 1       TMEM allocator + MMA issuer (one thread)
@@ -55,27 +68,43 @@ struct TcPlan {
 // swizzle repeats every 8 rows), at most one block of kBlockM.  A batch of 64
 // then moves half the bytes of a full 128-row box.
 inline int tc_base_rows(int B) { return B < kBlockM ? (B + 7) / 8 * 8 : kBlockM; }
-// Ring depths.  Draft: W gets one tile (r / 64 stages) and the base ring the
-// rest -- every base box is B separate 128-byte rows from DRAM (one per
-// request), so the base stream needs many boxes in flight.  Residual: no
-// base ring; W takes what operand A leaves.
-inline int tc_b_stages(int r, int B, bool residual) {
-  if (residual) return 0;
-  const size_t fixed = 1024 + (size_t)(r / 64) * kStageBytes * 2 + 512;
-  int s = (int)((kTcSmemLimit - fixed) / ((size_t)tc_base_rows(B) * 128));
-  if (s > kBStagesMax) s = kBStagesMax;
-  return s;
+// Bytes of one k-block of operand A (and of one base box): the block's
+// request rows, 128 bytes each.  A multiple of 1024, the swizzle atom.
+inline size_t tc_a_stage_bytes(int B) { return (size_t)tc_base_rows(B) * 128; }
+// Shared memory left for the two rings once operand A (r / 64 k-blocks)
+// and the barriers are placed.
+inline size_t tc_ring_bytes(int r, int B) {
+  return kTcSmemLimit - 1024 - (size_t)(r / 64) * tc_a_stage_bytes(B) - 512;
 }
+// Ring depths.  Each copy in flight waits about the same time for its
+// bytes, so the rings get shared memory in proportion to what they move per
+// tile: W r / 64 stages of 16 KB, base kTileN / 32 boxes of base_rows rows.
+// W keeps at least one tile.  Residual: no base ring; W takes it all.
 inline int tc_w_stages(int r, int B, bool residual) {
-  const size_t fixed = 1024 + (size_t)(r / 64) * kStageBytes +
-                       (size_t)tc_b_stages(r, B, residual) * tc_base_rows(B) * 128 + 512;
-  int s = (int)((kTcSmemLimit - fixed) / kStageBytes);
+  const size_t ring = tc_ring_bytes(r, B);
+  const int nkb = r / 64;
+  size_t wb = ring;
+  if (!residual) {
+    const size_t w_tile = (size_t)nkb * kStageBytes;
+    const size_t b_tile = (size_t)(kTileN / 32) * tc_a_stage_bytes(B);
+    wb = ring * w_tile / (w_tile + b_tile);
+  }
+  int s = (int)(wb / kStageBytes);
+  if (s < nkb) s = nkb;
   if (s > kWStagesMax) s = kWStagesMax;
   return s;
 }
+inline int tc_b_stages(int r, int B, bool residual) {
+  if (residual) return 0;
+  const size_t left = tc_ring_bytes(r, B) - (size_t)tc_w_stages(r, B, false) * kStageBytes;
+  int s = (int)(left / tc_a_stage_bytes(B));
+  if (s > kBStagesMax) s = kBStagesMax;
+  return s;
+}
 inline size_t tc_smem_bytes(int r, int B, bool residual) {
-  return 1024 + (size_t)(r / 64) * kStageBytes + (size_t)tc_w_stages(r, B, residual) * kStageBytes +
-         (size_t)tc_b_stages(r, B, residual) * tc_base_rows(B) * 128 + 512;
+  return 1024 + (size_t)(r / 64) * tc_a_stage_bytes(B) +
+         (size_t)tc_w_stages(r, B, residual) * kStageBytes +
+         (size_t)tc_b_stages(r, B, residual) * tc_a_stage_bytes(B) + 512;
 }
 
 inline bool tc_supported(int V, int r, int B) {
@@ -96,8 +125,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nkb = r >> 6;
   uint8_t* sA = sm;
-  const int bstage = base_rows * 128;  // bytes of one base box
-  uint8_t* sW = sA + nkb * kStageBytes;
+  const int bstage = base_rows * 128;  // bytes of one base box and of one k-block of A
+  uint8_t* sW = sA + nkb * bstage;
   uint8_t* sBase = sW + n_ws * kStageBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + (kRes ? 0 : n_bs * bstage));
   uint64_t* fullW = bars;
@@ -131,14 +160,26 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tmem_slot, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  // operand A: the previous-token rows of U for this block of requests.  The
-  // 128 token ids go to shared memory first (one round of loads), then every
-  // thread issues all of its U loads before storing any, so the gather costs
-  // two memory round trips rather than one per loop iteration.
+  // Producers (warps 0 and 2) read only W and base; at k = 0 they too wait
+  // for the kernel before the call, which may have written either.
+  const bool producer = warp == 0 || warp == 2;
+  if (!producer || k == 0) grid_dep_wait();
+
+  // operand A: the previous-token rows of U for this block of requests,
+  // gathered by the nine non-producer warps.  The 128 token ids go to shared
+  // memory first (one round of loads), then every thread issues all of its U
+  // loads before storing any, so the gather costs two memory round trips
+  // rather than one per loop iteration.
+  constexpr int kGather = kTcThreads - 64;
+  const int gtid = warp == 1 ? lane : threadIdx.x - 64;  // 0..kGather-1 off the producers
   __shared__ int s_x[kBlockM];
-  if (threadIdx.x < kBlockM) {
-    const int m = threadIdx.x;
+  if (!producer && gtid < kBlockM) {
+    const int m = gtid;
     const int b = bb * kBlockM + m;
     int x = -1;
     if (b < B) {
@@ -155,35 +196,33 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
     s_x[m] = x;
   }
-  __syncthreads();
-  {
+  if (!producer) {
+    named_sync(1, kGather);
     const int cpr = r >> 3;  // 16-byte chunks per row
-    constexpr int kPer = (kBlockM * 32 + kTcThreads - 1) / kTcThreads;  // r <= 256: 32 chunks per row
+    constexpr int kPer = (kBlockM * 32 + kGather - 1) / kGather;  // r <= 256: 32 chunks per row
     uint4 val[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-      const int q = threadIdx.x + i * kTcThreads;
+      const int q = gtid + i * kGather;
       val[i] = make_uint4(0, 0, 0, 0);
-      if (q < kBlockM * cpr) {
+      if (q < base_rows * cpr) {
         const int x = s_x[q / cpr];
         if (x >= 0) val[i] = __ldg(reinterpret_cast<const uint4*>(U + (size_t)x * r) + (q % cpr));
       }
     }
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
-      const int q = threadIdx.x + i * kTcThreads;
-      if (q < kBlockM * cpr) {
+      const int q = gtid + i * kGather;
+      if (q < base_rows * cpr) {
         const int m = q / cpr, c = q % cpr;
         const int kb = c >> 3, j = c & 7;
-        *reinterpret_cast<uint4*>(sA + kb * kStageBytes + m * 128 + ((j ^ (m & 7)) << 4)) = val[i];
+        *reinterpret_cast<uint4*>(sA + kb * bstage + m * 128 + ((j ^ (m & 7)) << 4)) = val[i];
       }
     }
+    fence_proxy_async_smem();
+    named_sync(1, kGather);
+    grid_dep_launch();
   }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
     // ---------------- W producer
@@ -230,7 +269,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc_sw128(a0 + kb * kStageBytes + kk * 32);
+            const uint64_t ad = sdesc_sw128(a0 + kb * bstage + kk * 32);
             const uint64_t bd = sdesc_sw128(w0 + s * kStageBytes + kk * 32);
             mma_bf16_ss(tmem + a * kTileN, ad, bd, idesc, (kb | kk) != 0);
           }
@@ -500,13 +539,33 @@ inline void tc_set_attr() {
   }
 }
 
+// Launch configuration with programmatic stream serialisation: the kernel
+// may start while the one before it in the stream is still running, and
+// orders itself behind it with griddepcontrol.wait.
+struct PdlLaunch {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  PdlLaunch(unsigned grid, unsigned block, size_t smem, cudaStream_t s) {
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+};
+
 inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const int32_t* tokens,
                             const float* it, float* dl, float* dbias, float2* part,
                             unsigned* flags, cudaStream_t s) {
   tc_set_attr<false>();
-  proj_tc_kernel<false><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, false), s>>>(
-      p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, k, prev, tokens, it, nullptr, p.base, nullptr,
-      dl, dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, flags);
+  PdlLaunch L(p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, false), s);
+  cudaLaunchKernelEx(&L.cfg, proj_tc_kernel<false>, p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, k,
+                     prev, tokens, it, (const float*)nullptr, p.base, (const ResInfo*)nullptr, dl,
+                     dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages,
+                     p.b_stages, p.base_rows, flags);
 }
 
 inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,

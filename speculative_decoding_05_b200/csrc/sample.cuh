@@ -124,6 +124,11 @@ draft_sample_kernel(const float* __restrict__ base, const TW* __restrict__ U,
                     float* __restrict__ ref_sum, unsigned* flags) {
   __shared__ __align__(16) float u_s[kMaxRank];
   __shared__ float shf[32];
+  // The next position's projection is launched behind this kernel with a
+  // programmatic dependency; let it start its prologue once this kernel is
+  // running (the wait is a no-op for a plain launch).
+  grid_dep_wait();
+  grid_dep_launch();
   const int b = blockIdx.x;
   const float it = checked_inv_temp(inv_temp, b, flags);
   const float it2 = it * kLog2e;

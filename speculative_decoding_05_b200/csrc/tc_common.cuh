@@ -139,6 +139,10 @@ __device__ __forceinline__ uint64_t policy_evict_last() {
   return pol;
 }
 // Make generic-proxy shared-memory writes visible to the async proxy (MMA).
+// Named barrier over `count` threads (a multiple of 32), id 1..15.
+__device__ __forceinline__ void named_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
