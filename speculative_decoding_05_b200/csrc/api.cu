@@ -304,7 +304,7 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
                                                 flags);
   } else if (use_tc(V, r, B, dt)) {
     TcPlan plan;
-    dspark_status st = tc_plan_residual(plan, target, base, U, W, V, r, B, K);
+    dspark_status st = tc_plan_residual(plan, target, n_rows, base, U, W, V, r, B, K);
     if (st != DSPARK_OK) return st;
     tc_launch_residual(plan, info, it, rpart, flags, s);
   } else {

@@ -28,13 +28,21 @@
 //   warp 0       W producer (TMA, evict-last: W is re-read every position)
 //   warp 1       TMEM allocator + MMA issuer (one thread)
 //   warp 2       base-logit producer (TMA 3-D boxes, evict-first)   [draft]
+//                target / base row-segment producer (TMA gather4)   [residual]
 //   warps 3..10  epilogue: two warpgroups of 128 threads (= 128 requests),
 //                each taking half of every tile's 32-column chunks
 //
 // Draft mode streams base[b, k, v0:v0+32] boxes through a second TMA ring.
-// Residual mode reads the per-request rows base[b, j_b, :] and
-// target[row_b, :] directly (each thread owns one request's contiguous
-// row segment), since j_b differs between requests.
+// Residual mode needs the per-request rows target[row_b, :] and
+// base[b, j_b, :] (j_b differs between requests): warp 2 fetches each
+// request's 128-byte segment of every 32-column chunk with TMA tile::gather4
+// loads (four rows of a one-row-high box per instruction) into a second
+// ring, unswizzled (rows at a 128-byte stride).  A gather through the
+// load/store units instead (per-thread loads, or 16-byte cp.async copies)
+// was capped near 5 GB/s per SM by the SM's outstanding misses.  The
+// epilogue thread of request m reads its row's 16-byte chunks starting at
+// chunk m & 7, so the eight lanes of a shared-memory phase meet eight
+// different bank groups, and rotates its TMEM values to the same order.
 #pragma once
 
 #include <cudaTypedefs.h>
@@ -55,7 +63,8 @@ constexpr int kTmemCols = 256;
 
 struct TcPlan {
   CUtensorMap tm_w;
-  CUtensorMap tm_base;
+  CUtensorMap tm_base;  // draft: [B, K, V] boxes; residual: [B * K, V] rows
+  CUtensorMap tm_tgt;   // residual: target rows [n_rows, V]
   const float* base;
   const float* target;
   const __nv_bfloat16* U;
@@ -71,40 +80,41 @@ inline int tc_base_rows(int B) { return B < kBlockM ? (B + 7) / 8 * 8 : kBlockM;
 // Bytes of one k-block of operand A (and of one base box): the block's
 // request rows, 128 bytes each.  A multiple of 1024, the swizzle atom.
 inline size_t tc_a_stage_bytes(int B) { return (size_t)tc_base_rows(B) * 128; }
-// Shared memory left for the two rings once operand A (r / 64 k-blocks)
-// and the barriers are placed.
-inline size_t tc_ring_bytes(int r, int B) {
-  return kTcSmemLimit - 1024 - (size_t)(r / 64) * tc_a_stage_bytes(B) - 512;
+// One stage of the second ring, per 32-column chunk: the base box (draft),
+// or the target and base segments of every request (residual).
+inline size_t tc_r_stage_bytes(int B, bool residual) {
+  return (residual ? 2 : 1) * tc_a_stage_bytes(B);
+}
+// Alignment slack, operand A (r / 64 k-blocks) and the barriers.
+inline size_t tc_fixed_bytes(int r, int B, bool residual) {
+  (void)residual;
+  return 1024 + (size_t)(r / 64) * tc_a_stage_bytes(B) + 512;
 }
 // Ring depths.  Each copy in flight waits about the same time for its
-// bytes, so the rings get shared memory in proportion to what they move per
-// tile: W r / 64 stages of 16 KB, base kTileN / 32 boxes of base_rows rows.
-// W keeps at least one tile.  Residual: no base ring; W takes it all.
+// bytes, so the two rings share what is left in proportion to what they
+// move per tile: W r / 64 stages of 16 KB, the second ring kTileN / 32
+// stages.  W keeps at least two stages (a ring shorter than a tile still
+// flows: the MMAs free its stages in order).
 inline int tc_w_stages(int r, int B, bool residual) {
-  const size_t ring = tc_ring_bytes(r, B);
+  const size_t ring = kTcSmemLimit - tc_fixed_bytes(r, B, residual);
   const int nkb = r / 64;
-  size_t wb = ring;
-  if (!residual) {
-    const size_t w_tile = (size_t)nkb * kStageBytes;
-    const size_t b_tile = (size_t)(kTileN / 32) * tc_a_stage_bytes(B);
-    wb = ring * w_tile / (w_tile + b_tile);
-  }
-  int s = (int)(wb / kStageBytes);
-  if (s < nkb) s = nkb;
+  const size_t w_tile = (size_t)nkb * kStageBytes;
+  const size_t b_tile = (size_t)(kTileN / 32) * tc_r_stage_bytes(B, residual);
+  int s = (int)(ring * w_tile / (w_tile + b_tile) / kStageBytes);
+  if (s < 2) s = 2;
   if (s > kWStagesMax) s = kWStagesMax;
   return s;
 }
 inline int tc_b_stages(int r, int B, bool residual) {
-  if (residual) return 0;
-  const size_t left = tc_ring_bytes(r, B) - (size_t)tc_w_stages(r, B, false) * kStageBytes;
-  int s = (int)(left / tc_a_stage_bytes(B));
+  const size_t left = kTcSmemLimit - tc_fixed_bytes(r, B, residual) -
+                      (size_t)tc_w_stages(r, B, residual) * kStageBytes;
+  int s = (int)(left / tc_r_stage_bytes(B, residual));
   if (s > kBStagesMax) s = kBStagesMax;
   return s;
 }
 inline size_t tc_smem_bytes(int r, int B, bool residual) {
-  return 1024 + (size_t)(r / 64) * tc_a_stage_bytes(B) +
-         (size_t)tc_w_stages(r, B, residual) * kStageBytes +
-         (size_t)tc_b_stages(r, B, residual) * tc_a_stage_bytes(B) + 512;
+  return tc_fixed_bytes(r, B, residual) + (size_t)tc_w_stages(r, B, residual) * kStageBytes +
+         (size_t)tc_b_stages(r, B, residual) * tc_r_stage_bytes(B, residual);
 }
 
 inline bool tc_supported(int V, int r, int B) {
@@ -114,7 +124,7 @@ inline bool tc_supported(int V, int r, int B) {
 template <bool kRes>
 __global__ void __launch_bounds__(kTcThreads, 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_base,
-               const __nv_bfloat16* __restrict__ U, int V, int r, int B, int K, int k,
+               const __grid_constant__ CUtensorMap tm_tgt, const __nv_bfloat16* __restrict__ U, int V, int r, int B, int K, int k,
                const int32_t* __restrict__ prev_token, const int32_t* __restrict__ tokens,
                const float* __restrict__ inv_temp, const float* __restrict__ target,
                const float* __restrict__ base, const ResInfo* __restrict__ info,
@@ -128,7 +138,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   const int bstage = base_rows * 128;  // bytes of one base box and of one k-block of A
   uint8_t* sW = sA + nkb * bstage;
   uint8_t* sBase = sW + n_ws * kStageBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + (kRes ? 0 : n_bs * bstage));
+  const int rstage = (kRes ? 2 : 1) * bstage;  // one stage of the second ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + n_bs * rstage);
   uint64_t* fullW = bars;
   uint64_t* emptyW = fullW + kWStagesMax;
   uint64_t* fullB = emptyW + kWStagesMax;
@@ -283,6 +294,51 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         mma_commit(&accFull[a]);
       }
     }
+  } else if (warp == 2 && kRes) {
+    // ---------------- target / base row producer (residual)
+    // lane g gathers requests 4g..4g+3: their target rows and base rows
+    // (row 0 stands in for a request past the batch, or for the base row of
+    // a bonus request; neither is read)
+    const int groups = base_rows >> 2;
+    int trow[4] = {0, 0, 0, 0}, brow[4] = {0, 0, 0, 0};
+    if (lane < groups) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int b = bb * kBlockM + 4 * lane + i;
+        if (b < B) {
+          const ResInfo& ri = info[b];
+          trow[i] = (int)ri.row;
+          if (!ri.bonus) brow[i] = b * K + ri.j;
+        }
+      }
+    }
+    const uint64_t pol = policy_evict_first();
+    int it = 0;
+    for (int t = t0; t < t1 && !*s_abort; ++t) {
+      bool ok = true;
+      for (int cb = 0; cb < kTileN / 32; ++cb, ++it) {
+        const int s = it % n_bs;
+        const uint32_t ph = (uint32_t)(it / n_bs) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_wait(&emptyB[s], ph ^ 1u))) {
+          ok = false;
+          break;
+        }
+        if (lane == 0) mbar_arrive_expect_tx(&fullB[s], (uint32_t)(2 * groups * 512));
+        __syncwarp();
+        if (lane < groups) {
+          const int v0 = t * kTileN + cb * 32;
+          uint8_t* st = sBase + s * rstage + lane * 512;
+          tma_gather4_hint(st, &tm_tgt, &fullB[s], v0, trow[0], trow[1], trow[2], trow[3], pol);
+          tma_gather4_hint(st + bstage, &tm_base, &fullB[s], v0, brow[0], brow[1], brow[2], brow[3],
+                           pol);
+        }
+      }
+      if (!ok) {
+        *s_abort = 1;
+        raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+        break;
+      }
+    }
   } else if (warp == 2) {
     // ---------------- base-logit producer (draft only)
     if (!kRes && lane == 0) {
@@ -317,7 +373,6 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const float it2 = it * kLog2e;
     ResInfo ri{};
     if (kRes && bval) ri = info[b];
-    const uint64_t pol = policy_evict_first();
     for (int t = t0; t < t1; ++t) {
       const int a = (t - t0) & 1;
       const uint32_t aph = (uint32_t)((t - t0) >> 1) & 1u;
@@ -385,29 +440,49 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                                 (bv[j + 2] + d[j + 2]) * it, (bv[j + 3] + d[j + 3]) * it);
           }
         } else {
-          float tq[32];
+          const int itB = (t - t0) * (kTileN / 32) + cb;
+          const int s = itB % n_bs;
+          const uint32_t ph = (uint32_t)(itB / n_bs) & 1u;
+          if (!mbar_wait(&fullB[s], ph)) {
+            *s_abort = 1;
+            raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+          }
+          // this request's segments, staged by warp 2 (m < base_rows when
+          // bval): slot j holds chunk (j + rot) & 7, and the TMEM values are
+          // rotated to match (three select stages, static register indices)
+          const int rot = lane & 7;
+          float tq[32], dr[32];
           if (bval) {
-            const float* trow = target + (size_t)ri.row * V + v0;
-            const float* brow = base + ((size_t)b * K + (ri.bonus ? 0 : ri.j)) * (size_t)V + v0;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
+            for (int x = 0; x < 32; ++x) dr[x] = (rot & 1) ? d[(x + 4) & 31] : d[x];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) d[x] = (rot & 2) ? dr[(x + 8) & 31] : dr[x];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) dr[x] = (rot & 4) ? d[(x + 16) & 31] : d[x];
+            const uint8_t* trow = sBase + s * rstage + m * 128;
+            const uint8_t* brow = trow + bstage;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int c = (j + rot) & 7;
               float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f), b4 = t4;
-              if (v0 + j < V) {
-                t4 = ld_stream4(trow + j, pol);
-                if (!ri.bonus) b4 = ld_stream4(brow + j, pol);
+              if (v0 + 4 * c < V) {
+                t4 = *reinterpret_cast<const float4*>(trow + c * 16);
+                if (!ri.bonus) b4 = *reinterpret_cast<const float4*>(brow + c * 16);
               }
-              tq[j] = t4.x; tq[j + 1] = t4.y; tq[j + 2] = t4.z; tq[j + 3] = t4.w;
-              bv[j] = b4.x; bv[j + 1] = b4.y; bv[j + 2] = b4.z; bv[j + 3] = b4.w;
+              tq[4 * j] = t4.x; tq[4 * j + 1] = t4.y; tq[4 * j + 2] = t4.z; tq[4 * j + 3] = t4.w;
+              bv[4 * j] = b4.x; bv[4 * j + 1] = b4.y; bv[4 * j + 2] = b4.z; bv[4 * j + 3] = b4.w;
             }
           }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&emptyB[s]);
           float qs4[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
           if (bval) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (v0 + j < V) {
+            for (int x = 0; x < 32; ++x) {
+              if (v0 + 4 * ((x / 4 + rot) & 7) < V) {
                 float pt;
-                qs4[j & 3] += residual_q(tq[j], bv[j], d[j], ri, it2, &pt);
-                ps4[j & 3] += pt;
+                qs4[x & 3] += residual_q(tq[x], bv[x], dr[x], ri, it2, &pt);
+                ps4[x & 3] += pt;
               }
             }
           }
@@ -477,6 +552,20 @@ inline bool encode_w_map(CUtensorMap* m, const void* W, int V, int r) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// rows [n, V] fp32 as 32 x 1 boxes (one row's 128-byte segment), no swizzle:
+// the box of a tile::gather4 load, which takes four rows at once.
+inline bool encode_rows_map(CUtensorMap* m, const float* p, int V, long long rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)V, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)V * 4};
+  cuuint32_t box[2] = {32, 1};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // base [B, K, V] fp32 as 32 (v) x 1 (k) x 128 (b) boxes, 128-byte swizzle.
 inline bool encode_base_map(CUtensorMap* m, const float* base, int V, int K, int B) {
   auto enc = tensor_map_encoder();
@@ -507,6 +596,7 @@ inline dspark_status tc_plan_draft(TcPlan& p, const float* base, const void* U, 
   p.U = static_cast<const __nv_bfloat16*>(U);
   if (!encode_w_map(&p.tm_w, W, V, r) || !encode_base_map(&p.tm_base, base, V, K, B))
     return DSPARK_ERR_CUDA;
+  p.tm_tgt = p.tm_w;  // unused in draft mode
   tc_grid(p);
   p.w_stages = tc_w_stages(r, B, false);
   p.b_stages = tc_b_stages(r, B, false);
@@ -514,17 +604,19 @@ inline dspark_status tc_plan_draft(TcPlan& p, const float* base, const void* U, 
   return DSPARK_OK;
 }
 
-inline dspark_status tc_plan_residual(TcPlan& p, const float* target, const float* base,
-                                      const void* U, const void* W, int V, int r, int B, int K) {
+inline dspark_status tc_plan_residual(TcPlan& p, const float* target, long long n_rows,
+                                      const float* base, const void* U, const void* W, int V,
+                                      int r, int B, int K) {
   p.V = V; p.r = r; p.B = B; p.K = K;
   p.base = base;
   p.target = target;
   p.U = static_cast<const __nv_bfloat16*>(U);
-  if (!encode_w_map(&p.tm_w, W, V, r)) return DSPARK_ERR_CUDA;
-  p.tm_base = p.tm_w;  // unused in residual mode
+  if (!encode_w_map(&p.tm_w, W, V, r) || !encode_rows_map(&p.tm_tgt, target, V, n_rows) ||
+      !encode_rows_map(&p.tm_base, base, V, (long long)B * K))
+    return DSPARK_ERR_CUDA;
   tc_grid(p);
   p.w_stages = tc_w_stages(r, B, true);
-  p.b_stages = 0;
+  p.b_stages = tc_b_stages(r, B, true);
   p.base_rows = tc_base_rows(B);
   return DSPARK_OK;
 }
@@ -562,7 +654,8 @@ inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const i
                             unsigned* flags, cudaStream_t s) {
   tc_set_attr<false>();
   PdlLaunch L(p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, false), s);
-  cudaLaunchKernelEx(&L.cfg, proj_tc_kernel<false>, p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, k,
+  cudaLaunchKernelEx(&L.cfg, proj_tc_kernel<false>, p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r,
+                     p.B, p.K, k,
                      prev, tokens, it, (const float*)nullptr, p.base, (const ResInfo*)nullptr, dl,
                      dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages,
                      p.b_stages, p.base_rows, flags);
@@ -572,7 +665,7 @@ inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float
                                float2* rpart, unsigned* flags, cudaStream_t s) {
   tc_set_attr<true>();
   proj_tc_kernel<true><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, true), s>>>(
-      p.tm_w, p.tm_base, p.U, p.V, p.r, p.B, p.K, 0, nullptr, nullptr, it, p.target, p.base, info,
+      p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r, p.B, p.K, 0, nullptr, nullptr, it, p.target, p.base, info,
       nullptr, nullptr, rpart, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, flags);
 }
 
