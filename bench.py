@@ -87,13 +87,32 @@ def whole_job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
 
 # ---------------------------------------------------------------- traffic --
 
-def source_digest() -> str:
-    """Hash of the CUDA sources: a stored DRAM-traffic figure is only valid
-    for the kernels it was measured on."""
+def source_digest(root: str | None = None) -> str:
+    """Hash of the CUDA sources a stored DRAM-traffic figure depends on: the
+    kernel's header and every file it includes, transitively (launch
+    configuration included: each kernel's header holds its launcher), or all
+    sources when no header is named.  A figure is only valid for the kernel
+    code it was measured on."""
     import glob
     import hashlib
+    import re
+    csrc = os.path.join(ROOT, "speculative_decoding_05_b200", "csrc")
+    if root is None:
+        files = sorted(glob.glob(os.path.join(csrc, "*")))
+    else:
+        seen, todo = set(), [os.path.join(csrc, root)]
+        while todo:
+            f = os.path.normpath(todo.pop())
+            if f in seen or not os.path.exists(f):
+                continue
+            seen.add(f)
+            for line in open(f):
+                m = re.match(r'\s*#include\s+"([^"]+)"', line)
+                if m:
+                    todo.append(os.path.join(os.path.dirname(f), m.group(1)))
+        files = sorted(seen)
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "speculative_decoding_05_b200", "csrc", "*"))):
+    for f in files:
         h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 
@@ -120,7 +139,7 @@ def measured_traffic(kernel: str, workload: str):
         d = json.load(open(p)).get(f"{kernel}|{workload}")
     except ValueError:
         return None
-    if not d or d.get("source_digest") != source_digest():
+    if not d or d.get("source_digest") != source_digest(d.get("root")):
         return None
     return d.get("dram_bytes_per_launch")
 
