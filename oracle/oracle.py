@@ -59,6 +59,8 @@ def _load():
                                           i32, i32, i32, i32, P, P, P, P, P, P,
                                           P, P, P, P]
             lib.oracle_verify.restype = i32
+            lib.oracle_sts_fit.argtypes = [P, P, ctypes.c_long, i32, P, P, P]
+            lib.oracle_sts_fit.restype = i32
             lib.oracle_num_threads.argtypes = []
             lib.oracle_num_threads.restype = i32
             _lib = lib
@@ -180,3 +182,22 @@ def verify(target, row_start, verify_len, base, U, W, prev_token, tokens, p_d,
     if rc != 0:
         raise ValueError(f"oracle_verify rejected its arguments (rc={rc})")
     return dict(n_acc=n_acc, out_tokens=out, accept_margin=am, res_margin=rm)
+
+
+def sts_fit(z, n_accepted):
+    """Sequential temperature scaling: per-position temperatures fitted by
+    likelihood on the sequences that reached each position, and the pooled
+    expected calibration error before and after."""
+    lib = _load()
+    z = _c(z, np.float32)
+    N, K = z.shape
+    n_acc = _c(n_accepted, np.int32)
+    if n_acc.shape != (N,):
+        raise ValueError("n_accepted must be [N]")
+    temps = np.empty(K, np.float64)
+    ece = np.empty(2, np.float64)
+    count = np.empty(K, np.int64)
+    rc = lib.oracle_sts_fit(_p(z), _p(n_acc), N, K, _p(temps), _p(ece), _p(count))
+    if rc != 0:
+        raise ValueError(f"oracle_sts_fit rejected its arguments (rc={rc})")
+    return dict(temps=temps, ece_before=float(ece[0]), ece_after=float(ece[1]), count=count)
