@@ -474,14 +474,18 @@ int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
  * c = 1 / (1 + exp(-z / T_j)); positions are taken left to right, each on
  * the sequences that reached it.
  *
- * Procedure.  With theta = 1/T the likelihood is convex in theta and its
- * derivative g(theta) = sum (sigma(theta z) - y) z is non-decreasing.
- * theta is kept in [1/T_MAX, 1/T_MIN]: a derivative >= 0 at the lower bound
- * or <= 0 at the upper bound puts the minimiser on that bound; otherwise the
- * root of g is bisected STS_ITERS times in log(theta) and theta is the
- * midpoint of the last bracket.  A position with no observed sample, or with
- * only z = 0 (every temperature fits equally), gets T = 1.  Samples whose z
- * is not finite are left out.
+ * Procedure.  With theta = 1/T the likelihood is convex in theta: its
+ * derivative g(theta) = sum (sigma(theta z) - y) z is non-decreasing, with
+ * slope h(theta) = sum sigma(theta z) (1 - sigma(theta z)) z^2 >= 0.  theta
+ * is kept in [1/T_MAX, 1/T_MIN]: g >= 0 at the lower bound or <= 0 at the
+ * upper bound puts the minimiser on that bound.  Otherwise, from theta = 1,
+ * each step evaluates g and h, narrows the bracket (in log theta) by the
+ * sign of g, and takes the Newton step theta - g/h, or the bracket's
+ * log-midpoint when h is not positive or the step leaves the bracket; the
+ * search ends when g = 0, when a step moves theta by at most STS_TOL
+ * relative, or after STS_ITERS steps.  A position with no observed sample,
+ * or with only z = 0 (every temperature fits equally), gets T = 1.
+ * Samples whose z is not finite are left out.
  *
  * ECE: observed (n, j) pairs pooled, STS_BINS equal-width bins of c on
  * [0, 1] (bin = floor(c * STS_BINS), the top edge in the last bin);
@@ -489,17 +493,18 @@ int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
  * ------------------------------------------------------------------------ */
 #define STS_T_MIN 0.05
 #define STS_T_MAX 20.0
-#define STS_ITERS 60
+#define STS_ITERS 40
+#define STS_TOL 1e-13
 #define STS_BINS 15
 
 static double logistic(double x) { return 1.0 / (1.0 + exp(-x)); }
 
-/* derivative of the position-j likelihood at theta; also the number of
- * observed samples and whether any observed z is non-zero */
+/* derivative (and its slope) of the position-j likelihood at theta; also
+ * the number of observed samples and whether any observed z is non-zero */
 static double sts_grad(const float *z, const int32_t *n_acc, long N, int K, int j,
-                       double theta, long *count, int *nonzero)
+                       double theta, double *slope, long *count, int *nonzero)
 {
-    double g = 0.0;
+    double g = 0.0, h = 0.0;
     long c = 0;
     int nz = 0;
     for (long n = 0; n < N; ++n) {
@@ -509,10 +514,14 @@ static double sts_grad(const float *z, const int32_t *n_acc, long N, int K, int 
         if (!isfinite(zz))
             continue;
         const double y = n_acc[n] > j ? 1.0 : 0.0;
-        g += (logistic(theta * zz) - y) * zz;
+        const double s = logistic(theta * zz);
+        g += (s - y) * zz;
+        h += s * (1.0 - s) * zz * zz;
         ++c;
         nz |= zz != 0.0;
     }
+    if (slope)
+        *slope = h;
     if (count)
         *count = c;
     if (nonzero)
@@ -563,24 +572,33 @@ int oracle_sts_fit(const float *z, const int32_t *n_acc_in, long N, int K, doubl
         long c = 0;
         int nz = 0;
         double lo = log(1.0 / STS_T_MAX), hi = log(1.0 / STS_T_MIN);
-        const double g_lo = sts_grad(z, n_acc, N, K, j, exp(lo), &c, &nz);
-        const double g_hi = sts_grad(z, n_acc, N, K, j, exp(hi), NULL, NULL);
+        const double g_lo = sts_grad(z, n_acc, N, K, j, exp(lo), NULL, &c, &nz);
         double th;
         if (c == 0 || !nz) {
             th = 1.0;
         } else if (g_lo >= 0.0) {
             th = exp(lo);
-        } else if (g_hi <= 0.0) {
+        } else if (sts_grad(z, n_acc, N, K, j, exp(hi), NULL, NULL, NULL) <= 0.0) {
             th = exp(hi);
         } else {
+            th = 1.0;
             for (int it = 0; it < STS_ITERS; ++it) {
-                const double mid = 0.5 * (lo + hi);
-                if (sts_grad(z, n_acc, N, K, j, exp(mid), NULL, NULL) < 0.0)
-                    lo = mid;
+                double h;
+                const double g = sts_grad(z, n_acc, N, K, j, th, &h, NULL, NULL);
+                if (g == 0.0)
+                    break;
+                if (g < 0.0)
+                    lo = log(th);
                 else
-                    hi = mid;
+                    hi = log(th);
+                double next = th - g / h;
+                if (!(h > 0.0) || !(next > exp(lo)) || !(next < exp(hi)))
+                    next = exp(0.5 * (lo + hi));
+                const int done = fabs(next - th) <= STS_TOL * th;
+                th = next;
+                if (done)
+                    break;
             }
-            th = exp(0.5 * (lo + hi));
         }
         theta[j] = th;
         temps[j] = 1.0 / th;
