@@ -479,11 +479,12 @@ int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
  * slope h(theta) = sum sigma(theta z) (1 - sigma(theta z)) z^2 >= 0.  theta
  * is kept in [1/T_MAX, 1/T_MIN]: g >= 0 at the lower bound or <= 0 at the
  * upper bound puts the minimiser on that bound.  Otherwise, from theta = 1,
- * each step evaluates g and h, narrows the bracket (in log theta) by the
- * sign of g, and takes the Newton step theta - g/h, or the bracket's
- * log-midpoint when h is not positive or the step leaves the bracket; the
- * search ends when g = 0, when a step moves theta by at most STS_TOL
- * relative, or after STS_ITERS steps.  A position with no observed sample,
+ * each step evaluates g and h and narrows the bracket [lo, hi] (values of
+ * theta) by the sign of g.  The search ends when g = 0, when the Newton
+ * step -g/h moves theta by at most STS_TOL relative (the step is then
+ * taken), or after STS_ITERS steps; otherwise theta becomes theta - g/h, or
+ * the bracket's geometric midpoint sqrt(lo * hi) when h is not positive or
+ * the step leaves the bracket.  A position with no observed sample,
  * or with only z = 0 (every temperature fits equally), gets T = 1.
  * Samples whose z is not finite are left out.
  *
@@ -571,15 +572,15 @@ int oracle_sts_fit(const float *z, const int32_t *n_acc_in, long N, int K, doubl
     for (int j = 0; j < K; ++j) {
         long c = 0;
         int nz = 0;
-        double lo = log(1.0 / STS_T_MAX), hi = log(1.0 / STS_T_MIN);
-        const double g_lo = sts_grad(z, n_acc, N, K, j, exp(lo), NULL, &c, &nz);
+        double lo = 1.0 / STS_T_MAX, hi = 1.0 / STS_T_MIN;
+        const double g_lo = sts_grad(z, n_acc, N, K, j, lo, NULL, &c, &nz);
         double th;
         if (c == 0 || !nz) {
             th = 1.0;
         } else if (g_lo >= 0.0) {
-            th = exp(lo);
-        } else if (sts_grad(z, n_acc, N, K, j, exp(hi), NULL, NULL, NULL) <= 0.0) {
-            th = exp(hi);
+            th = lo;
+        } else if (sts_grad(z, n_acc, N, K, j, hi, NULL, NULL, NULL) <= 0.0) {
+            th = hi;
         } else {
             th = 1.0;
             for (int it = 0; it < STS_ITERS; ++it) {
@@ -588,16 +589,15 @@ int oracle_sts_fit(const float *z, const int32_t *n_acc_in, long N, int K, doubl
                 if (g == 0.0)
                     break;
                 if (g < 0.0)
-                    lo = log(th);
+                    lo = th;
                 else
-                    hi = log(th);
-                double next = th - g / h;
-                if (!(h > 0.0) || !(next > exp(lo)) || !(next < exp(hi)))
-                    next = exp(0.5 * (lo + hi));
-                const int done = fabs(next - th) <= STS_TOL * th;
-                th = next;
-                if (done)
+                    hi = th;
+                const double newton = th - g / h;
+                if (h > 0.0 && fabs(newton - th) <= STS_TOL * th) {
+                    th = newton;
                     break;
+                }
+                th = (h > 0.0 && newton > lo && newton < hi) ? newton : sqrt(lo * hi);
             }
         }
         theta[j] = th;
