@@ -297,12 +297,195 @@ def cpu_baseline(w, inp_dev, seconds):
 
 # ----------------------------------------------------------------- main --
 
+STS_METRIC = ("calibration score entries fitted per second (sequential temperature "
+              "scaling of the confidence head, N x K per fit)")
+STS_UNIT = "entries/s"
+STS_LAUNCHES = 1 + 2 * 42 + 4  # init, (derivative + update) x (2 bounds + 40 steps), ECE
+
+
+def sts_alg_bytes(c, passes: int) -> int:
+    """Bytes one fit reads: each of its passes reads all scores and accepted
+    lengths once (the fit reports how many passes its search took)."""
+    return passes * (c.N * c.K * 4 + c.N * 4)
+
+
+def sts_oracle_sample(c, z, n_acc, seconds: float):
+    """The oracle on the leading sequences of the set, sized to about
+    ``seconds`` of CPU work: (entries/s, sequences, seconds of the fit)."""
+    from oracle import oracle
+    n = min(c.N, 20_000)
+    t0 = time.perf_counter()
+    oracle.sts_fit(z[:n], n_acc[:n])
+    dt = time.perf_counter() - t0
+    n2 = min(c.N, int(n * seconds / max(dt, 1e-3)))
+    if n2 > n:
+        t0 = time.perf_counter()
+        oracle.sts_fit(z[:n2], n_acc[:n2])
+        dt, n = time.perf_counter() - t0, n2
+    return n * c.K / dt, n, dt
+
+
+def run_calibration(args, c, rank, world):
+    """Bench line of the temperature fit on one calibration set per rank."""
+    import torch
+    import torch.distributed as dist
+    from speculative_decoding_05_b200 import build as BLD
+    from speculative_decoding_05_b200 import dspark as D
+    from speculative_decoding_05_b200 import workloads as WL
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        from oracle import oracle
+        d = WL.make_calibration(c, device="cpu")
+        z, n_acc = d["z"].numpy(), d["n_acc"].numpy()
+        n_ref = min(c.N, int(os.environ.get("DSPARK_REF_SEQUENCES", "50000")))
+        for _ in range(args.warmup):
+            oracle.sts_fit(z[:n_ref], n_acc[:n_ref])
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            oracle.sts_fit(z[:n_ref], n_acc[:n_ref])
+        dt = (time.perf_counter() - t0) / args.steps
+        value = n_ref * c.K / dt
+        sample = f"{n_ref} of {c.N} sequences of the {c.name} set per fit (K={c.K})"
+        print(json.dumps({
+            "impl": "reference", "metric": STS_METRIC, "value": value, "unit": STS_UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded)",
+            "config": {"workload": c.name, "N": c.N, "K": c.K, "requests": n_ref},
+            "cpu_baseline": {"value": value, "unit": STS_UNIT, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": STS_UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}), flush=True)
+        return
+
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    if rank == 0:
+        BLD.build()
+    if world > 1:
+        dist.barrier()
+    D.load()
+    d = WL.make_calibration(c, device=dev, seed=c.seed + 1000 * rank)
+    z, n_acc = d["z"], d["n_acc"]
+    ws = torch.zeros(D.dspark_sts_workspace_size(c.N, c.K), dtype=torch.uint8, device=dev)
+    temps = torch.empty(c.K, dtype=torch.float32, device=dev)
+    ece = torch.empty(2, dtype=torch.float32, device=dev)
+    passes = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def fit():
+        D.dspark_sts_fit(z, n_acc, temps, ece, ws, passes=passes, stream=stream)
+
+    with torch.cuda.stream(stream):
+        fit()
+    torch.cuda.synchronize()
+    flags = D.dspark_get_device_flags(ws, stream)
+    if flags:
+        raise RuntimeError(f"device status flags after warm-up: {flags}")
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fit()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    dev_id = os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[local_rank] \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else str(local_rank)
+    clocks = ClockSampler(dev_id)
+    clocks.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            g.replay()
+            ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in ev), dev)
+    units = c.N * c.K
+    value = whole_job_rate(units, world, ms)
+    pk = peaks()
+    n_pass = int(passes.item())
+    alg = sts_alg_bytes(c, n_pass)
+    achieved = alg / (ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": pk["hbm"], "unit": "GB/s",
+                "frac": achieved / pk["hbm"], "traffic": None,
+                "kernel": f"sts_grad_kernel + sts_update_kernel ({n_pass - 2} passes), "
+                          "sts_ece_kernel (2 passes)",
+                "call": "dspark_sts_fit", "peak_source": pk["src"] + " (burst copy)",
+                "algorithmic_bytes_per_launch": alg}
+
+    host_z = z.cpu().pin_memory()
+    host_n = n_acc.cpu().pin_memory()
+    host_t = torch.empty(c.K, dtype=torch.float32, pin_memory=True)
+    host_e = torch.empty(2, dtype=torch.float32, pin_memory=True)
+    n_e2e = max(1, min(args.e2e_steps, args.steps))
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_e2e)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(n_e2e):
+            flush.zero_()
+            e2e_ev[i][0].record(stream)
+            z.copy_(host_z, non_blocking=True)
+            n_acc.copy_(host_n, non_blocking=True)
+            g.replay()
+            host_t.copy_(temps, non_blocking=True)
+            host_e.copy_(ece, non_blocking=True)
+            e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in e2e_ev), dev)
+    e2e = {"value": whole_job_rate(units, world, e2e_ms), "unit": STS_UNIT,
+           "h2d_bytes_per_step": host_z.numel() * 4 + host_n.numel() * 4,
+           "d2h_bytes_per_step": c.K * 4 + 8, "ms_per_step": e2e_ms}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, dt = sts_oracle_sample(c, host_z.numpy(), host_n.numpy(), args.cpu_seconds)
+        cpu = {"value": v, "unit": STS_UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"one fit on the first {n} of {c.N} sequences (K={c.K}), {dt:.2f} s"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    print(json.dumps({
+        "metric": STS_METRIC, "value": value, "unit": STS_UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": c.name, "N": c.N, "K": c.K,
+                   "l2": "flushed by a 256 MB write between steps",
+                   "parallelism": f"replicas x{world}", "graphs": True},
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": STS_LAUNCHES * args.steps, "clocks": clk, "passes": n_pass,
+        "temps": [round(float(t), 4) for t in temps.cpu()],
+        "ece_before_after": [float(e) for e in ece.cpu()]}), flush=True)
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     from speculative_decoding_05_b200 import workloads as WL
+    if args.config in WL.CALIBRATIONS:
+        run_calibration(args, WL.CALIBRATIONS[args.config], rank, world)
+        return
     w = WL.get(args.config)
 
     if args.impl == "reference":

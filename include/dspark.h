@@ -131,6 +131,54 @@ dspark_status dspark_draft_markov(
     void *stream);
 
 /* ---------------------------------------------------------------------- */
+/* 1b. Sequential temperature scaling of the confidence head (offline)     */
+/* ---------------------------------------------------------------------- */
+
+/* Largest K dspark_sts_fit takes. */
+#define DSPARK_STS_MAX_K 32
+
+/* Workspace bytes dspark_sts_fit needs (0 for sizes it does not take). */
+size_t dspark_sts_workspace_size(long long N, int K);
+
+/*
+ * Fits the per-position temperatures T_k that dspark_confidence_prefix
+ * divides the head's scores by (freeaitool 4.1: the head's raw scores are
+ * over-confident and are calibrated after training, position by position
+ * from left to right; yage.ai scheduler paragraph: on an offline set, so
+ * that the probabilities match the observed acceptance rates).
+ *
+ * Calibration set: N sequences with head scores z[n, k] and the accepted
+ * prefix length n_accepted[n] of a full-block verify (what dspark_verify
+ * writes).  Position k (0-based) of sequence n is observed when
+ * n_accepted[n] >= k and accepted when n_accepted[n] > k.  T_k minimises
+ * the Bernoulli negative log-likelihood of the observed labels under
+ * c = 1 / (1 + exp(-z / T_k)).  Search, the same for every position:
+ * theta = 1/T in [1/20, 1/0.05]; the likelihood's derivative in theta at
+ * both bounds (a sign that puts the minimiser on a bound settles it), then
+ * from theta = 1 Newton steps on the derivative kept inside a bracket of
+ * theta (its geometric midpoint when a step leaves it), until a step moves
+ * theta by at most 1e-13 relative or after 40 steps.  A position nobody
+ * reached, or with only z = 0, gets T = 1.  Sums are fp64 in a fixed
+ * order (run-to-run identical).
+ *
+ * ece[0], ece[1]: expected calibration error before (every T = 1) and
+ * after the fit: observed pairs pooled into 15 equal-width bins of c,
+ * sum over bins of |accepted count - sum of c| / number of pairs.
+ *
+ * Inputs   z [N,K] fp32 (non-finite scores are left out and flagged),
+ *          n_accepted [N] int32 in [0,K] (clamped and flagged otherwise)
+ * Outputs  temps [K] fp32, ece [2] fp32, passes [1] int32 or NULL: the
+ *          passes over the data the fit made (derivative evaluations of
+ *          the longest search, plus two for the ECE)
+ * Errors   K > DSPARK_STS_MAX_K: DSPARK_ERR_UNSUPPORTED.  At most 2 + 40
+ *          derivative passes (a pass with nothing left to search returns
+ *          at once), 89 launches, no host sync.
+ */
+dspark_status dspark_sts_fit(const float *z, const int32_t *n_accepted, long long N, int K,
+                             float *temps, float *ece, int32_t *passes, void *workspace,
+                             size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
 /* 2. Confidence-scheduled prefix cut                                      */
 /* ---------------------------------------------------------------------- */
 

@@ -15,6 +15,7 @@
 #include "sample.cuh"
 #include "verify.cuh"
 #include "verify_fused.cuh"
+#include "sts.cuh"
 
 using namespace dspark;
 
@@ -500,6 +501,66 @@ dspark_status dspark_confidence_prefix(const float* z, const float* temps,
     prefix_kernel<kPrefixThreads><<<1, kPrefixThreads, smem, s>>>(
         z, temps, cost_tokens, cost_ms, n_pts, B, K, enable, c, survival, verify_len, objective,
         static_cast<unsigned*>(workspace));
+  return check_launch();
+}
+
+// Workspace of the temperature fit: header, search state per position and
+// the active count, derivative partials [G][K][4], calibration-error
+// partials [G][31].
+struct StsWs {
+  size_t pos_off, part_off, bpart_off, total;
+};
+StsWs sts_ws(long long N, int K) {
+  const int G = sts_grid(N);
+  StsWs w;
+  w.pos_off = kHeaderBytes;
+  w.part_off = w.pos_off + align256(kStsPosBytes);
+  w.bpart_off = w.part_off + align256((size_t)G * K * kStsPart * sizeof(double));
+  w.total = w.bpart_off + align256((size_t)G * kStsBinVals * sizeof(double));
+  return w;
+}
+
+size_t dspark_sts_workspace_size(long long N, int K) {
+  if (N < 0 || K < 1 || K > kStsMaxK) return 0;
+  return sts_ws(N, K).total;
+}
+
+dspark_status dspark_sts_fit(const float* z, const int32_t* n_accepted, long long N, int K,
+                             float* temps, float* ece, int32_t* passes, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  if (N < 0 || K < 1) return DSPARK_ERR_INVALID_ARG;
+  if (K > kStsMaxK) return DSPARK_ERR_UNSUPPORTED;
+  if (!temps || !ece || (N > 0 && (!z || !n_accepted))) return DSPARK_ERR_INVALID_ARG;
+  if (!workspace || !aligned(workspace, 256) || ws_bytes < sts_ws(N, K).total)
+    return DSPARK_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  dspark_status st = clear_status(workspace, s);
+  if (st != DSPARK_OK) return st;
+  const StsWs w = sts_ws(N, K);
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  unsigned* flags = reinterpret_cast<unsigned*>(ws);
+  StsPos* pos = reinterpret_cast<StsPos*>(ws + w.pos_off);
+  int* n_active = reinterpret_cast<int*>(ws + w.pos_off + sizeof(StsPos) * kStsMaxK);
+  double* part = reinterpret_cast<double*>(ws + w.part_off);
+  double* bpart = reinterpret_cast<double*>(ws + w.bpart_off);
+  const int G = sts_grid(N);
+  sts_init_kernel<<<1, 32, 0, s>>>(pos, n_active, K);
+  // bounds at steps 0 and 1, then Newton steps; a pass with nothing left to
+  // search returns at once
+  const int last = 1 + kStsIters;
+  for (int step = 0; step <= last; ++step) {
+    if (step == 0)
+      sts_grad_kernel<true><<<G, kStsThreads, 0, s>>>(z, n_accepted, N, K, pos, n_active, part,
+                                                       flags);
+    else
+      sts_grad_kernel<false><<<G, kStsThreads, 0, s>>>(z, n_accepted, N, K, pos, n_active, part,
+                                                        flags);
+    sts_update_kernel<<<1, 32 * K, 0, s>>>(part, G, K, pos, n_active, step, last, temps, passes);
+  }
+  for (int fitted = 0; fitted < 2; ++fitted) {
+    sts_ece_kernel<<<G, kStsThreads, 0, s>>>(z, n_accepted, N, K, pos, !fitted, bpart, flags);
+    sts_ece_final_kernel<<<1, 32 * kStsBinVals, 0, s>>>(bpart, G, ece + fitted);
+  }
   return check_launch();
 }
 

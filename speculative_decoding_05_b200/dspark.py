@@ -37,6 +37,8 @@ SYMBOLS = [
     "dspark_get_device_status", "dspark_get_device_flags",
     "dspark_status_string", "dspark_draft_path", "dspark_verify_path", "dspark_version",
     "dspark_verify_noalloc",
+    "dspark_sts_workspace_size",
+    "dspark_sts_fit",
 ]
 
 
@@ -76,6 +78,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.dspark_verify_noalloc.restype = I
     lib.dspark_confidence_prefix.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P, S, P]
     lib.dspark_confidence_prefix.restype = I
+    lib.dspark_sts_workspace_size.argtypes = [L, I]
+    lib.dspark_sts_workspace_size.restype = S
+    lib.dspark_sts_fit.argtypes = [P, P, L, I, P, P, P, P, S, P]
+    lib.dspark_sts_fit.restype = I
     lib.dspark_get_device_status.argtypes = [P, P]
     lib.dspark_get_device_status.restype = I
     lib.dspark_get_device_flags.argtypes = [P, P]
@@ -219,3 +225,17 @@ def dspark_get_device_flags(workspace, stream=None) -> int:
 
 def dspark_get_device_status(workspace, stream=None) -> int:
     return int(load().dspark_get_device_status(_ptr(workspace), _stream(stream)))
+
+
+def dspark_sts_workspace_size(N, K) -> int:
+    return int(load().dspark_sts_workspace_size(int(N), int(K)))
+
+
+def dspark_sts_fit(z, n_accepted, temps, ece, workspace, passes=None, stream=None):
+    """Per-position temperatures of the confidence head fitted on a
+    calibration set (z [N,K] fp32, n_accepted [N] int32); writes temps [K],
+    ece [2] (before, after) and, if given, passes [1] int32."""
+    N, K = z.shape
+    rc = load().dspark_sts_fit(_ptr(z), _ptr(n_accepted), N, K, _ptr(temps), _ptr(ece),
+                               _ptr(passes), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("dspark_sts_fit", rc)

@@ -197,3 +197,50 @@ def host_uw(t: torch.Tensor):
     if t.dtype == torch.bfloat16:
         return t.view(torch.int16).numpy().view("uint16")
     return t.numpy()
+
+
+# ---------------------------------------------------------------------------
+# Calibration set for the sequential temperature fit
+# ---------------------------------------------------------------------------
+
+@dataclass(frozen=True)
+class Calibration:
+    """An offline calibration set: N sequences of K head scores and the
+    accepted-prefix length of a full-block verify of each."""
+    name: str
+    N: int
+    K: int
+    seed: int = 5
+
+
+CALIBRATIONS = {
+    # one million logged sequences at the Stress draft length
+    "calibration": Calibration("calibration", N=1_000_000, K=16),
+    # a smaller set that the oracle fits in well under a second per position
+    "calibration_small": Calibration("calibration_small", N=50_003, K=16, seed=6),
+}
+
+
+def make_calibration(c: Calibration, device="cpu", seed: int | None = None) -> dict:
+    """Head scores z [N,K] f32 ~ N(1.5, 1.5^2) and accepted lengths n_acc [N]
+    i32 in [0, K].
+
+    Ground truth of the synthetic head: given every earlier token was
+    accepted, position k (1-based) is accepted with probability
+    Phi(z * 0.588 / (1.2 + 0.05 k)), Phi the standard normal CDF.  This is a
+    probit link, not the logistic form the fit assumes; 0.588 z is close to
+    the logistic scale, so the raw scores read as over-confident by a factor
+    of about 1.2 + 0.05 k, as the pages describe the head.  The first
+    rejected position ends the prefix."""
+    device = torch.device(device)
+    g = torch.Generator(device=device)
+    g.manual_seed(c.seed if seed is None else seed)
+    z = torch.randn(c.N, c.K, generator=g, device=device, dtype=torch.float32).mul_(1.5).add_(1.5)
+    u = torch.rand(c.N, c.K, generator=g, device=device, dtype=torch.float32)
+    k = torch.arange(1, c.K + 1, device=device, dtype=torch.float32)
+    scale = 0.588 / (1.2 + 0.05 * k)
+    accepted = u < torch.special.ndtr(z * scale)
+    rejected = ~accepted
+    first = rejected.to(torch.int32).argmax(dim=1).to(torch.int32)
+    n_acc = torch.where(rejected.any(dim=1), first, torch.full_like(first, c.K))
+    return dict(z=z, n_acc=n_acc.contiguous())

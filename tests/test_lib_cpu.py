@@ -104,6 +104,17 @@ def test_argument_validation_before_launch(lib):
     # prefix: too many candidates, bad table size
     assert lib.dspark_confidence_prefix(p, p, p, p, 16, 1024, 9, 1, p, p, p, p, ws, 256, None) == 4
     assert lib.dspark_confidence_prefix(p, p, p, p, 1, 4, 4, 1, p, p, p, p, ws, 256, None) == 1
+    # temperature fit: bad K, K past the limit, missing outputs, short or misaligned workspace
+    sb = lib.dspark_sts_workspace_size(1000, 16)
+    assert sb > 0 and lib.dspark_sts_workspace_size(1000, 33) == 0
+    assert lib.dspark_sts_workspace_size(-1, 4) == 0
+    assert lib.dspark_sts_fit(p, p, 1000, 0, p, p, None, ws, sb, None) == 1
+    assert lib.dspark_sts_fit(p, p, 1000, 33, p, p, None, ws, sb, None) == 4
+    assert lib.dspark_sts_fit(p, p, 1000, 16, None, p, None, ws, sb, None) == 1
+    assert lib.dspark_sts_fit(None, p, 1000, 16, p, p, None, ws, sb, None) == 1
+    assert lib.dspark_sts_fit(p, p, -5, 16, p, p, None, ws, sb, None) == 1
+    assert lib.dspark_sts_fit(p, p, 1000, 16, p, p, None, ws, sb - 8, None) == 6
+    assert lib.dspark_sts_fit(p, p, 1000, 16, p, p, None, P((1 << 24) + 8), sb, None) == 6
     # verify: missing target
     vb = lib.dspark_verify_workspace_size(1024, 16, 2, 3)
     assert lib.dspark_verify(None, 10, p, p, p, p, p, 1, 1024, 16, 2, 3, p, None, p, p, p, p, None,
