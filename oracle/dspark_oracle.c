@@ -233,6 +233,31 @@ double oracle_cost_ms(const float *xs, const float *ys, int n, double tokens)
     return y0 + (y1 - y0) * (tokens - x0) / (x1 - x0);
 }
 
+/*
+ * Staircase reading of the same table ([yage], engineering paragraph: the
+ * real throughput curve SPS(B) jumps in steps, because of tensor-core
+ * alignment and cache limits): a batch of n tokens costs the entry of the
+ * smallest profiled size that holds it, ys[i] for the first i with
+ * xs[i] >= n (ys[0] at or below xs[0]); past the last entry the cost grows
+ * along the last segment's slope.
+ */
+double oracle_cost_stair_ms(const float *xs, const float *ys, int n, double tokens)
+{
+    if (tokens > (double)xs[n - 1])
+        return ys[n - 1] + ((double)ys[n - 1] - ys[n - 2]) * (tokens - xs[n - 1]) /
+                               ((double)xs[n - 1] - xs[n - 2]);
+    int i = 0;
+    while ((double)xs[i] < tokens)
+        ++i;
+    return ys[i];
+}
+
+static double cost_mode(const float *xs, const float *ys, int n, int staircase, double tokens)
+{
+    return staircase ? oracle_cost_stair_ms(xs, ys, n, tokens)
+                     : oracle_cost_ms(xs, ys, n, tokens);
+}
+
 typedef struct {
     double s;
     int k;
@@ -270,11 +295,22 @@ static int cand_cmp(const void *pa, const void *pb)
  * outputs: c, S [B, K]; L [B] = committed positions per request;
  * objective = E / t(N) of the committed set; margin = relative objective
  * gap at the stopping decision (+inf when every candidate was taken).
+ *
+ * Asynchronous budget ([yage], engineering paragraph): the number of
+ * tokens a step verifies is decided from the confidences of two steps
+ * back, while which tokens fill it is decided by the current confidences.
+ * With budget >= 0 (verify tokens N, one per request included) the first
+ * budget - B candidates of the current order are committed (clamped to
+ * [0, B*K]); the order is survival-descending and survival never rises
+ * along k, so the set is a prefix of every request's draft.  margin is
+ * then the relative survival gap at the cut.  n_greedy always returns N of
+ * the greedy scan on the current confidences: the budget for two steps
+ * later.  staircase selects the cost reading (see oracle_cost_stair_ms).
  */
-int oracle_prefix(const float *z, const float *temps, const float *cost_tokens,
-                  const float *cost_ms, int n_pts, int B, int K, int enable,
-                  double *c, double *S, int32_t *L, double *objective,
-                  double *margin)
+int oracle_prefix_async(const float *z, const float *temps, const float *cost_tokens,
+                        const float *cost_ms, int n_pts, int staircase, int B, int K,
+                        int enable, int budget, double *c, double *S, int32_t *L,
+                        double *objective, double *margin, int *n_greedy)
 {
     if (B < 0 || K < 0 || n_pts < 2)
         return 1;
@@ -294,9 +330,10 @@ int oracle_prefix(const float *z, const float *temps, const float *cost_tokens,
             E += S[o];
         for (int b = 0; b < B; ++b)
             L[b] = K;
-        *objective = E / oracle_cost_ms(cost_tokens, cost_ms, n_pts,
-                                        (double)B + (double)B * K);
+        *objective = E / cost_mode(cost_tokens, cost_ms, n_pts, staircase,
+                                   (double)B + (double)B * K);
         *margin = INFINITY;
+        *n_greedy = B + B * K;
         return 0;
     }
     size_t n = (size_t)B * K;
@@ -309,26 +346,52 @@ int oracle_prefix(const float *z, const float *temps, const float *cost_tokens,
             cand[o].b = b;
         }
     qsort(cand, n, sizeof(cand_t), cand_cmp);
-    for (int b = 0; b < B; ++b)
-        L[b] = 0;
+    /* the greedy scan: commit while the objective strictly rises */
     double E = B, N = B;
-    double obj = E / oracle_cost_ms(cost_tokens, cost_ms, n_pts, N);
-    *margin = INFINITY;
+    double obj = E / cost_mode(cost_tokens, cost_ms, n_pts, staircase, N);
+    double gmargin = INFINITY;
+    size_t stop = n;
     for (size_t i = 0; i < n; ++i) {
         double E2 = E + cand[i].s, N2 = N + 1.0;
-        double obj2 = E2 / oracle_cost_ms(cost_tokens, cost_ms, n_pts, N2);
+        double obj2 = E2 / cost_mode(cost_tokens, cost_ms, n_pts, staircase, N2);
         if (!(obj2 > obj)) {
-            *margin = fabs(obj2 - obj) / obj;
+            gmargin = fabs(obj2 - obj) / obj;
+            stop = i;
             break;
         }
-        L[cand[i].b] += 1;
         E = E2;
         N = N2;
         obj = obj2;
     }
-    *objective = obj;
+    *n_greedy = B + (int)stop;
+    size_t m = stop;
+    *margin = gmargin;
+    if (budget >= 0) {
+        long want = (long)budget - B;
+        m = want < 0 ? 0 : ((size_t)want > n ? n : (size_t)want);
+        *margin = (m == 0 || m == n) ? INFINITY
+                                     : (cand[m - 1].s - cand[m].s) / cand[m - 1].s;
+    }
+    for (int b = 0; b < B; ++b)
+        L[b] = 0;
+    double Em = B;
+    for (size_t i = 0; i < m; ++i) {
+        L[cand[i].b] += 1;
+        Em += cand[i].s;
+    }
+    *objective = Em / cost_mode(cost_tokens, cost_ms, n_pts, staircase, (double)B + (double)m);
     free(cand);
     return 0;
+}
+
+int oracle_prefix(const float *z, const float *temps, const float *cost_tokens,
+                  const float *cost_ms, int n_pts, int B, int K, int enable,
+                  double *c, double *S, int32_t *L, double *objective,
+                  double *margin)
+{
+    int n_greedy;
+    return oracle_prefix_async(z, temps, cost_tokens, cost_ms, n_pts, 0, B, K, enable, -1, c, S,
+                               L, objective, margin, &n_greedy);
 }
 
 /* ------------------------------------------------------------------ */

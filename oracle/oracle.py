@@ -55,6 +55,11 @@ def _load():
             lib.oracle_prefix.restype = i32
             lib.oracle_cost_ms.argtypes = [P, P, i32, f64]
             lib.oracle_cost_ms.restype = f64
+            lib.oracle_cost_stair_ms.argtypes = [P, P, i32, f64]
+            lib.oracle_cost_stair_ms.restype = f64
+            lib.oracle_prefix_async.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, i32, P, P, P,
+                                                P, P, P]
+            lib.oracle_prefix_async.restype = i32
             lib.oracle_verify.argtypes = [P, ctypes.c_int64, P, P, P, P, P, i32,
                                           i32, i32, i32, i32, P, P, P, P, P, P,
                                           P, P, P, P]
@@ -201,3 +206,38 @@ def sts_fit(z, n_accepted):
     if rc != 0:
         raise ValueError(f"oracle_sts_fit rejected its arguments (rc={rc})")
     return dict(temps=temps, ece_before=float(ece[0]), ece_after=float(ece[1]), count=count)
+
+
+def cost_stair_ms(cost_tokens, cost_ms_, n_tokens: float) -> float:
+    """Staircase reading of the cost table: the entry of the smallest
+    profiled size that holds n_tokens."""
+    lib = _load()
+    xs = _c(cost_tokens, np.float32)
+    ys = _c(cost_ms_, np.float32)
+    return float(lib.oracle_cost_stair_ms(_p(xs), _p(ys), len(xs), float(n_tokens)))
+
+
+def prefix_async(z, temps, cost_tokens, cost_ms_, staircase: bool = False, enable: bool = True,
+                 budget: int | None = None):
+    """Prefix cut with the cost table read as a staircase or piecewise
+    linear, optionally against a budget of verify tokens decided earlier;
+    also returns n_greedy, the greedy N of the current confidences."""
+    lib = _load()
+    z = _c(z, np.float32)
+    B, K = z.shape
+    temps = _c(temps, np.float32)
+    xs = _c(cost_tokens, np.float32)
+    ys = _c(cost_ms_, np.float32)
+    c = np.empty((B, K), np.float64)
+    S = np.empty((B, K), np.float64)
+    L = np.empty(B, np.int32)
+    obj = np.empty(1, np.float64)
+    mg = np.empty(1, np.float64)
+    ng = np.empty(1, np.int32)
+    rc = lib.oracle_prefix_async(_p(z), _p(temps), _p(xs), _p(ys), len(xs), int(bool(staircase)),
+                                 B, K, int(bool(enable)), -1 if budget is None else int(budget),
+                                 _p(c), _p(S), _p(L), _p(obj), _p(mg), _p(ng))
+    if rc != 0:
+        raise ValueError(f"oracle_prefix_async rejected its arguments (rc={rc})")
+    return dict(c=c, S=S, L=L, objective=float(obj[0]), margin=float(mg[0]),
+                n_greedy=int(ng[0]))
