@@ -207,6 +207,42 @@ dspark_status dspark_confidence_prefix(
     float *c, float *survival, int32_t *verify_len, float *objective,
     void *workspace, size_t ws_bytes, void *stream);
 
+/* Cost-table readings for dspark_confidence_prefix_async. */
+#define DSPARK_COST_LINEAR 0    /* piecewise-linear interpolation (as above) */
+#define DSPARK_COST_STAIRCASE 1 /* a batch of N tokens costs the entry of the
+                                   smallest profiled size >= N; past the last
+                                   entry, the last segment's slope */
+
+/*
+ * The prefix cut with the asynchronous budget (yage.ai, engineering
+ * paragraph: the number of tokens a step verifies is decided from the
+ * confidences of two steps back, so the decision never waits for the
+ * current step; which tokens fill it is still decided by the current,
+ * calibrated confidences) and a choice of cost-table reading (the same
+ * paragraph: the measured throughput curve jumps in steps).
+ *
+ *   staircase   DSPARK_COST_LINEAR or DSPARK_COST_STAIRCASE
+ *   budget_in   [1] int32 device, or NULL: verify tokens N (one per request
+ *               included) decided earlier; the first N - B candidates of
+ *               the current order are committed (N clamped to [B, B + B*K]).
+ *               NULL, or a negative value: the greedy cut of
+ *               dspark_confidence_prefix.
+ *   budget_out  [1] int32 device, or NULL: N of the greedy cut on this
+ *               step's confidences (B + B*K when enable = 0), the budget
+ *               for two steps later.  May be the same word as budget_in:
+ *               the budget is read before the new one is written, so a
+ *               two-slot ring (step t uses slot t % 2) replays in a graph.
+ * Everything else as for dspark_confidence_prefix, which is this call
+ * with DSPARK_COST_LINEAR and no budgets.  The candidate order makes every
+ * budget cut a prefix of each request's draft (survival never rises along
+ * k; equal survivals go to the earlier position).
+ */
+dspark_status dspark_confidence_prefix_async(
+    const float *z, const float *temps, const float *cost_tokens, const float *cost_ms,
+    int n_pts, int staircase, int B, int K, int enable, const int32_t *budget_in,
+    float *c, float *survival, int32_t *verify_len, float *objective, int32_t *budget_out,
+    void *workspace, size_t ws_bytes, void *stream);
+
 /* ---------------------------------------------------------------------- */
 /* 3. Rejection-sampling verify                                            */
 /* ---------------------------------------------------------------------- */

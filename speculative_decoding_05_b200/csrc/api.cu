@@ -470,12 +470,15 @@ dspark_status dspark_verify(const float* target_logits, int64_t n_target_rows,
                             last_token, ws, s);
 }
 
-dspark_status dspark_confidence_prefix(const float* z, const float* temps,
-                                       const float* cost_tokens, const float* cost_ms, int n_pts,
-                                       int B, int K, int enable, float* c, float* survival,
-                                       int32_t* verify_len, float* objective, void* workspace,
-                                       size_t ws_bytes, void* stream) {
-  if (B < 0 || K < 0 || n_pts < 2 || n_pts > 64) return DSPARK_ERR_INVALID_ARG;
+dspark_status dspark_confidence_prefix_async(const float* z, const float* temps,
+                                             const float* cost_tokens, const float* cost_ms,
+                                             int n_pts, int staircase, int B, int K, int enable,
+                                             const int32_t* budget_in, float* c, float* survival,
+                                             int32_t* verify_len, float* objective,
+                                             int32_t* budget_out, void* workspace,
+                                             size_t ws_bytes, void* stream) {
+  if (B < 0 || K < 0 || n_pts < 2 || n_pts > 64 || (staircase != 0 && staircase != 1))
+    return DSPARK_ERR_INVALID_ARG;
   if ((long long)B * K > kMaxCand) return DSPARK_ERR_UNSUPPORTED;
   if (!workspace || !aligned(workspace, 256) || ws_bytes < dspark_prefix_workspace_size(B, K, n_pts))
     return DSPARK_ERR_WORKSPACE;
@@ -495,13 +498,23 @@ dspark_status dspark_confidence_prefix(const float* z, const float* temps,
   // the kernel clears the status word itself (one CTA: before any flag is raised)
   if (npad <= kPrefixSmallCand)
     prefix_kernel<kPrefixThreadsSmall><<<1, kPrefixThreadsSmall, smem, s>>>(
-        z, temps, cost_tokens, cost_ms, n_pts, B, K, enable, c, survival, verify_len, objective,
-        static_cast<unsigned*>(workspace));
+        z, temps, cost_tokens, cost_ms, n_pts, staircase, B, K, enable, budget_in, c, survival,
+        verify_len, objective, budget_out, static_cast<unsigned*>(workspace));
   else
     prefix_kernel<kPrefixThreads><<<1, kPrefixThreads, smem, s>>>(
-        z, temps, cost_tokens, cost_ms, n_pts, B, K, enable, c, survival, verify_len, objective,
-        static_cast<unsigned*>(workspace));
+        z, temps, cost_tokens, cost_ms, n_pts, staircase, B, K, enable, budget_in, c, survival,
+        verify_len, objective, budget_out, static_cast<unsigned*>(workspace));
   return check_launch();
+}
+
+dspark_status dspark_confidence_prefix(const float* z, const float* temps,
+                                       const float* cost_tokens, const float* cost_ms, int n_pts,
+                                       int B, int K, int enable, float* c, float* survival,
+                                       int32_t* verify_len, float* objective, void* workspace,
+                                       size_t ws_bytes, void* stream) {
+  return dspark_confidence_prefix_async(z, temps, cost_tokens, cost_ms, n_pts, 0, B, K, enable,
+                                        nullptr, c, survival, verify_len, objective, nullptr,
+                                        workspace, ws_bytes, stream);
 }
 
 // Workspace of the temperature fit: header, search state per position and

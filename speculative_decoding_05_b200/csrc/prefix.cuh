@@ -6,6 +6,16 @@
 // candidate index k*B + b ascending, i.e. position then request), the
 // expected-emitted-token prefix sums are a block scan in fp64, and the
 // early stop is the first index where E/t(N) does not increase.
+//
+// Asynchronous budget (yage.ai, engineering paragraph: how many tokens a
+// step verifies is decided from the confidences of two steps back, which
+// tokens fill that budget from the current ones): with a budget of N verify
+// tokens the first N - B candidates of the current order are committed;
+// the greedy N of the current confidences is returned either way, to be the
+// budget two steps later.  The budget is read before the new one is
+// written, so the two may share one device word.  The cost table can be
+// read piecewise-linearly or as a staircase (the same page: the measured
+// throughput curve jumps in steps).
 #pragma once
 
 #include "common.cuh"
@@ -27,6 +37,25 @@ __device__ __forceinline__ double cost_at(const float* __restrict__ xs, const fl
   return y0 + (y1 - y0) * (tokens - x0) / (x1 - x0);
 }
 
+// Staircase reading: the entry of the smallest profiled size that holds the
+// batch; past the table, the last segment's slope.
+__device__ __forceinline__ double cost_stair_at(const float* __restrict__ xs,
+                                                const float* __restrict__ ys, int n,
+                                                double tokens) {
+  if (tokens > (double)xs[n - 1])
+    return (double)ys[n - 1] + ((double)ys[n - 1] - (double)ys[n - 2]) *
+                                   (tokens - (double)xs[n - 1]) /
+                                   ((double)xs[n - 1] - (double)xs[n - 2]);
+  int i = 0;
+  while ((double)xs[i] < tokens) ++i;
+  return ys[i];
+}
+
+__device__ __forceinline__ double cost_of(const float* __restrict__ xs, const float* __restrict__ ys,
+                                          int n, int staircase, double tokens) {
+  return staircase ? cost_stair_at(xs, ys, n, tokens) : cost_at(xs, ys, n, tokens);
+}
+
 // key order: larger survival first; equal survival: smaller index first
 __device__ __forceinline__ bool cand_before(double sa, int ia, double sb, int ib) {
   return sa > sb || (sa == sb && ia < ib);
@@ -36,8 +65,10 @@ template <int kT>
 __global__ void __launch_bounds__(kT)
 prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
               const float* __restrict__ cost_tokens, const float* __restrict__ cost_ms, int n_pts,
-              int B, int K, int enable, float* __restrict__ c_out, float* __restrict__ s_out,
-              int32_t* __restrict__ verify_len, float* __restrict__ objective, unsigned* flags) {
+              int staircase, int B, int K, int enable, const int32_t* budget_in,
+              float* __restrict__ c_out, float* __restrict__ s_out,
+              int32_t* __restrict__ verify_len, float* __restrict__ objective,
+              int32_t* budget_out, unsigned* flags) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int n = B * K;
   int npad = 1;
@@ -47,10 +78,13 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   int* lcount = idx + npad;                                     // [B]
   __shared__ float s_xs[64], s_ys[64];
   __shared__ double shd[32];
-  __shared__ int s_stop;
+  __shared__ int s_stop, s_budget;
   const int tid = threadIdx.x;
 
-  if (tid == 0) *flags = 0u;  // status of this call
+  if (tid == 0) {
+    *flags = 0u;  // status of this call
+    s_budget = budget_in != nullptr ? *budget_in : -1;  // read before budget_out is written
+  }
   // cost table into shared memory; it must be ascending in tokens
   for (int i = tid; i < n_pts; i += kT) {
     s_xs[i] = cost_tokens[i];
@@ -95,9 +129,10 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     const double E = (double)B + block_sum_d<kT>(e, shd);
     for (int b = tid; b < B; b += kT) verify_len[b] = K;
     if (tid == 0) {
-      const double t = cost_at(s_xs, s_ys, n_pts, (double)B + (double)n);
+      const double t = cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)n);
       if (!(t > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
       objective[0] = (float)(E / t);
+      if (budget_out != nullptr) *budget_out = B + n;
     }
     return;
   }
@@ -132,8 +167,8 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   // candidate i (0-based) raises the objective iff E_{i+1}/t(B+i+1) > E_i/t(B+i)
   double E = (double)B + excl;
   for (int i = i0; i < i0 + per && i < n; ++i) {
-    const double t0 = cost_at(s_xs, s_ys, n_pts, (double)B + (double)i);
-    const double t1 = cost_at(s_xs, s_ys, n_pts, (double)B + (double)i + 1.0);
+    const double t0 = cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)i);
+    const double t1 = cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)i + 1.0);
     const double E1 = E + key[i];
     if (!(t0 > 0.0) || !(t1 > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
     if (!(E1 / t1 > E / t0)) {
@@ -143,7 +178,13 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     E = E1;
   }
   __syncthreads();
-  const int n_commit = s_stop;
+  // the greedy cut, or the budget's (clamped to [0, n])
+  int n_commit = s_stop;
+  if (s_budget >= 0) {
+    const long long want = (long long)s_budget - B;
+    n_commit = want < 0 ? 0 : (want > n ? n : (int)want);
+  }
+  if (tid == 0 && budget_out != nullptr) *budget_out = B + s_stop;
   for (int i = tid; i < n_commit; i += kT) atomicAdd(&lcount[idx[i] % B], 1);
   __syncthreads();
   for (int b = tid; b < B; b += kT) verify_len[b] = lcount[b];
@@ -155,7 +196,7 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
       Ec = (double)B + excl;
       for (int i = i0; i < n_commit; ++i) Ec += key[i];
     }
-    objective[0] = (float)(Ec / cost_at(s_xs, s_ys, n_pts, (double)B + (double)n_commit));
+    objective[0] = (float)(Ec / cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)n_commit));
   }
 }
 

@@ -39,6 +39,7 @@ SYMBOLS = [
     "dspark_verify_noalloc",
     "dspark_sts_workspace_size",
     "dspark_sts_fit",
+    "dspark_confidence_prefix_async",
 ]
 
 
@@ -78,6 +79,9 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.dspark_verify_noalloc.restype = I
     lib.dspark_confidence_prefix.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P, S, P]
     lib.dspark_confidence_prefix.restype = I
+    lib.dspark_confidence_prefix_async.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P,
+                                                   S, P]
+    lib.dspark_confidence_prefix_async.restype = I
     lib.dspark_sts_workspace_size.argtypes = [L, I]
     lib.dspark_sts_workspace_size.restype = S
     lib.dspark_sts_fit.argtypes = [P, P, L, I, P, P, P, P, S, P]
@@ -239,3 +243,21 @@ def dspark_sts_fit(z, n_accepted, temps, ece, workspace, passes=None, stream=Non
     rc = load().dspark_sts_fit(_ptr(z), _ptr(n_accepted), N, K, _ptr(temps), _ptr(ece),
                                _ptr(passes), _ptr(workspace), workspace.numel(), _stream(stream))
     _check("dspark_sts_fit", rc)
+
+
+COST_LINEAR, COST_STAIRCASE = 0, 1
+
+
+def dspark_confidence_prefix_async(z, temps, cost_tokens, cost_ms, enable, c, survival, verify_len,
+                                   objective, workspace, staircase=False, budget_in=None,
+                                   budget_out=None, stream=None):
+    """The prefix cut with an optional budget decided earlier (budget_in
+    [1] int32) and the greedy N of this step written to budget_out [1]
+    (the two may be the same tensor); staircase selects the cost reading."""
+    B, K = z.shape
+    rc = load().dspark_confidence_prefix_async(
+        _ptr(z), _ptr(temps), _ptr(cost_tokens), _ptr(cost_ms), cost_tokens.numel(),
+        COST_STAIRCASE if staircase else COST_LINEAR, B, K, int(bool(enable)), _ptr(budget_in),
+        _ptr(c), _ptr(survival), _ptr(verify_len), _ptr(objective), _ptr(budget_out),
+        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("dspark_confidence_prefix_async", rc)

@@ -104,6 +104,11 @@ def test_argument_validation_before_launch(lib):
     # prefix: too many candidates, bad table size
     assert lib.dspark_confidence_prefix(p, p, p, p, 16, 1024, 9, 1, p, p, p, p, ws, 256, None) == 4
     assert lib.dspark_confidence_prefix(p, p, p, p, 1, 4, 4, 1, p, p, p, p, ws, 256, None) == 1
+    # asynchronous prefix: bad cost reading, too many candidates
+    assert lib.dspark_confidence_prefix_async(p, p, p, p, 16, 2, 4, 4, 1, None, p, p, p, p, None,
+                                              ws, 256, None) == 1
+    assert lib.dspark_confidence_prefix_async(p, p, p, p, 16, 1, 1024, 9, 1, None, p, p, p, p,
+                                              None, ws, 256, None) == 4
     # temperature fit: bad K, K past the limit, missing outputs, short or misaligned workspace
     sb = lib.dspark_sts_workspace_size(1000, 16)
     assert sb > 0 and lib.dspark_sts_workspace_size(1000, 33) == 0
