@@ -84,17 +84,6 @@ __global__ void sts_init_kernel(StsPos* __restrict__ pos, int* __restrict__ n_ac
   }
 }
 
-// Clamped accepted length of sequence n (flags a value outside [0, K]).
-__device__ __forceinline__ int sts_nacc(const int32_t* __restrict__ n_acc, long long n, int K,
-                                        unsigned* flags, bool check) {
-  int na = n_acc[n];
-  if (na < 0 || na > K) {
-    if (check) raise_flag(flags, DSPARK_FLAG_BAD_LENGTH);
-    na = na < 0 ? 0 : K;
-  }
-  return na;
-}
-
 // Derivative and slope of every position's likelihood at its current theta
 // (the first pass also counts the observed samples and notes any non-zero
 // score): part [gridDim.x][K][kStsPart].
