@@ -87,32 +87,35 @@ def whole_job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
 
 # ---------------------------------------------------------------- traffic --
 
-def source_digest(root: str | None = None) -> str:
-    """Hash of the CUDA sources a stored DRAM-traffic figure depends on: the
-    kernel's header and every file it includes, transitively (launch
-    configuration included: each kernel's header holds its launcher), or all
-    sources when no header is named.  A figure is only valid for the kernel
-    code it was measured on."""
+def source_closure(root: str | None = None) -> list:
+    """The CUDA sources a kernel is built from: its header and every file it
+    includes, transitively (each kernel's header also holds its launcher);
+    every source when no header is named."""
     import glob
-    import hashlib
     import re
     csrc = os.path.join(ROOT, "speculative_decoding_05_b200", "csrc")
     if root is None:
-        files = sorted(glob.glob(os.path.join(csrc, "*")))
-    else:
-        seen, todo = set(), [os.path.join(csrc, root)]
-        while todo:
-            f = os.path.normpath(todo.pop())
-            if f in seen or not os.path.exists(f):
-                continue
-            seen.add(f)
-            for line in open(f):
-                m = re.match(r'\s*#include\s+"([^"]+)"', line)
-                if m:
-                    todo.append(os.path.join(os.path.dirname(f), m.group(1)))
-        files = sorted(seen)
+        return sorted(glob.glob(os.path.join(csrc, "*")))
+    seen, todo = set(), [os.path.join(csrc, root)]
+    while todo:
+        f = os.path.normpath(todo.pop())
+        if f in seen or not os.path.exists(f):
+            continue
+        seen.add(f)
+        for line in open(f):
+            m = re.match(r'\s*#include\s+"([^"]+)"', line)
+            if m:
+                todo.append(os.path.join(os.path.dirname(f), m.group(1)))
+    return sorted(seen)
+
+
+def source_digest(root: str | None = None) -> str:
+    """Hash of the sources a stored DRAM-traffic figure depends on (see
+    source_closure).  A figure is only valid for the kernel code it was
+    measured on."""
+    import hashlib
     h = hashlib.sha256()
-    for f in files:
+    for f in source_closure(root):
         h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 

@@ -124,3 +124,17 @@ def test_argument_validation_before_launch(lib):
     vb = lib.dspark_verify_workspace_size(1024, 16, 2, 3)
     assert lib.dspark_verify(None, 10, p, p, p, p, p, 1, 1024, 16, 2, 3, p, None, p, p, p, p, None,
                              p, p, p, p, None, ws, vb, None) == 1
+
+
+def test_traffic_hash_covers_the_draft_kernels_sources():
+    """The stored DRAM traffic of the persistent draft is keyed to the files
+    that kernel is built from, not to every source of the library."""
+    import os
+    import bench
+    names = {os.path.basename(f) for f in bench.source_closure("draft_persist.cuh")}
+    assert {"draft_persist.cuh", "proj_tc.cuh", "tc_common.cuh", "common.cuh", "sample.cuh",
+            "proj_simt.cuh", "dspark.h"} <= names
+    assert not names & {"prefix.cuh", "sts.cuh", "verify.cuh", "verify_fused.cuh", "api.cu"}
+    assert bench.source_digest("draft_persist.cuh") != bench.source_digest()
+    # the committed figure matches the current sources
+    assert bench.measured_traffic("draft_gemv_kernel<1>", "single") is not None
