@@ -137,20 +137,21 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     return;
   }
 
-  // bitonic sort of (key, idx) in the order of cand_before
+  // bitonic sort of (key, idx) in the order of cand_before; each stage walks
+  // the npad / 2 compare-exchange pairs (i, i + stride), i with bit `stride`
+  // clear: pair p puts a zero bit into p at that position
   for (int size = 2; size <= npad; size <<= 1) {
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < npad; i += kT) {
-        const int j = i ^ stride;
-        if (j > i) {
-          const bool up = (i & size) == 0;  // this half sorts in cand_before order
-          const double ki = key[i], kj = key[j];
-          const int ii = idx[i], ij = idx[j];
-          const bool jfirst = cand_before(kj, ij, ki, ii);
-          if (jfirst == up) {
-            key[i] = kj; key[j] = ki;
-            idx[i] = ij; idx[j] = ii;
-          }
+      for (int p = tid; p < (npad >> 1); p += kT) {
+        const int i = (p & (stride - 1)) | ((p & ~(stride - 1)) << 1);
+        const int j = i + stride;
+        const bool up = (i & size) == 0;  // this half sorts in cand_before order
+        const double ki = key[i], kj = key[j];
+        const int ii = idx[i], ij = idx[j];
+        const bool jfirst = cand_before(kj, ij, ki, ii);
+        if (jfirst == up) {
+          key[i] = kj; key[j] = ki;
+          idx[i] = ij; idx[j] = ii;
         }
       }
       __syncthreads();

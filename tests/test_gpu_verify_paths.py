@@ -58,6 +58,8 @@ def test_single_launch_verify_twice_in_a_row(oracle_mod):
     inp = WL.make_inputs(w, device="cuda")
     step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype, keep_bias=True)
     step.draft(inp)
+    torch.cuda.synchronize()
+    assert step.flags()["draft"] == 0, step.flags()  # a timed-out exchange would show here
     step.verify_len.fill_(w.K)
     outs = []
     for seed in (1, 2):
