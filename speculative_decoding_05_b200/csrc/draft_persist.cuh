@@ -201,11 +201,11 @@ __device__ __forceinline__ bool persist_grid_barrier(unsigned* counter, int k, i
   const unsigned target = (unsigned)(k + 1) * (unsigned)G;
   const uint64_t tstart = global_timer_ns();
   bool ok = true;
-  for (;;) {
+  for (uint32_t polls = 1;; ++polls) {
     unsigned seen;
     asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(counter) : "memory");
     if (seen >= target) break;
-    if (global_timer_ns() - tstart > kWaitLimitNs) {
+    if (wait_expired(tstart, polls)) {
       raise_flag(flags, DSPARK_FLAG_TIMEOUT);
       ok = false;
       break;
@@ -816,13 +816,13 @@ struct GemvRecs {
 __device__ __forceinline__ void backoff_spin_u64(const unsigned long long* p, uint32_t seq,
                                                  unsigned long long* out, bool* timed_out) {
   const uint64_t tstart = global_timer_ns();
-  for (;;) {
+  for (uint32_t polls = 1;; ++polls) {
     const unsigned long long v = ld_rec(p);
     if ((uint32_t)(v >> 32) == seq) {
       *out = v;
       return;
     }
-    if (global_timer_ns() - tstart > kWaitLimitNs) {
+    if (wait_expired(tstart, polls)) {
       *timed_out = true;
       *out = 0;
       return;
@@ -1243,7 +1243,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           if (c0 + i < c1) pend |= 1u << i;
         }
         const uint64_t tstart = global_timer_ns();
-        for (;;) {
+        for (uint32_t polls = 1;; ++polls) {
           ulonglong2 m[kGPerLane];
 #pragma unroll
           for (int i = 0; i < kGPerLane; ++i)
@@ -1256,7 +1256,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             }
           }
           if (!__any_sync(0xffffffffu, pend != 0)) break;
-          if (__any_sync(0xffffffffu, global_timer_ns() - tstart > kWaitLimitNs)) {
+          if (__any_sync(0xffffffffu, wait_expired(tstart, polls))) {
             if (lane == 0) {
               *s_abort = 1;
               raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);

@@ -33,6 +33,15 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 // Upper bound of every device-side wait (a correct pipeline never gets
 // close; a stuck one gives up, raises DSPARK_FLAG_TIMEOUT and unwinds).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kWaitMinPolls = 4096;
+// Whether a wait that started at t0 and has polled `polls` times gives up:
+// only after kWaitMinPolls polls and kWaitLimitNs of elapsed time, the
+// difference taken signed, so that a timer read that steps back counts as
+// no time elapsed and one odd timer value cannot end a wait early.
+__device__ __forceinline__ bool wait_expired(uint64_t t0, uint32_t polls) {
+  return polls >= kWaitMinPolls &&
+         (long long)(global_timer_ns() - t0) > (long long)kWaitLimitNs;
+}
 
 // ---------------------------------------------------------------------------
 // mbarrier
@@ -70,7 +79,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if ((i & 255u) == 0 && wait_expired(t0, i)) return false;
   }
 }
 
@@ -91,7 +100,7 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_test_wait(bar, parity)) return true;
-    if ((i & 1023u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if ((i & 1023u) == 0 && wait_expired(t0, i)) return false;
   }
 }
 

@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
       if (c_lo + lane + 32 * i <= c_hi) pend |= 1u << i;
     }
     const uint64_t tstart = global_timer_ns();
-    for (;;) {
+    for (uint32_t polls = 1;; ++polls) {
       ulonglong2 m[kFPerLane];
 #pragma unroll
       for (int i = 0; i < kFPerLane; ++i) {
@@ -337,7 +337,7 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
         }
       }
       if (!__any_sync(0xffffffffu, pend != 0)) break;
-      if (__any_sync(0xffffffffu, global_timer_ns() - tstart > kWaitLimitNs)) {
+      if (__any_sync(0xffffffffu, wait_expired(tstart, polls))) {
         if (lane == 0) raise_flag(a.flags, DSPARK_FLAG_TIMEOUT);
         break;
       }
@@ -483,7 +483,7 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
       if (c0 + i < c1) pend |= 1u << i;
     }
     const uint64_t tstart = global_timer_ns();
-    for (;;) {
+    for (uint32_t polls = 1;; ++polls) {
       ulonglong2 mq[kFPerLane], mp[kFPerLane];
 #pragma unroll
       for (int i = 0; i < kFPerLane; ++i) {
@@ -501,7 +501,7 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
         }
       }
       if (!__any_sync(0xffffffffu, pend != 0)) break;
-      if (__any_sync(0xffffffffu, global_timer_ns() - tstart > kWaitLimitNs)) {
+      if (__any_sync(0xffffffffu, wait_expired(tstart, polls))) {
         if (lane == 0) raise_flag(a.flags, DSPARK_FLAG_TIMEOUT);
         break;
       }
