@@ -120,6 +120,16 @@ def source_digest(root: str | None = None) -> str:
     return h.hexdigest()[:16]
 
 
+def launches_per_step(draft_path: str, verify_path: str, K: int) -> int:
+    """Kernels one step launches: the draft (one persistent launch, else a
+    projection and a sampler per position), the prefix cut (one), the verify
+    (one single-launch kernel, else statistics, accept, residual and
+    sample)."""
+    draft = 1 if draft_path.startswith(("persistent", "tcgen05-persistent")) else 2 * K
+    verify = 1 if verify_path == "single-launch" else 4
+    return draft + 1 + verify
+
+
 def kernel_name(path: str, call: str, w) -> str:
     if call != "dspark_draft_markov":
         return "dspark_verify kernels"
@@ -645,10 +655,8 @@ def main():
         e2e = {"value": whole_job_rate(units_per_rank, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    # kernels of one step: persistent draft = 1 launch, otherwise 2 per
-    # position; prefix 1; verify 4 (statistics, accept, residual, sample)
-    launches_per_step = (1 if step.path.startswith(("persistent", "tcgen05-persistent"))
-                         else 2 * w.K) + 1 + 4
+    vpath = D.dspark_verify_path(w.V, w.r, w.B, w.K, inp["U"].dtype, step.draft_bias is not None)
+    n_launch = launches_per_step(step.path, vpath, w.K)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, args.cpu_seconds)
@@ -667,7 +675,7 @@ def main():
                    "draft_path": step.path, "l2": "flushed by a 256 MB write between steps",
                    "parallelism": f"replicas x{world}", "graphs": True},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": n_launch * args.steps,
         "clocks": clk,
         "breakdown_ms": {"draft": md, "prefix": statistics.mean(t_prefix), "verify": mv,
                          "note": "separate graphs per call, untimed pass"},

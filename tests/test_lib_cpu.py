@@ -136,3 +136,19 @@ def test_traffic_hash_covers_the_draft_kernels_sources():
             "proj_simt.cuh", "dspark.h"} <= names
     assert not names & {"prefix.cuh", "sts.cuh", "verify.cuh", "verify_fused.cuh", "api.cu"}
     assert bench.source_digest("draft_persist.cuh") != bench.source_digest()
+
+
+def test_bench_launch_count_follows_the_paths():
+    """The bench's gpu_launches claim: three kernels per step on the single
+    workload (persistent draft, prefix, single-launch verify), 2K + 5 on the
+    tensor-core path with the staged verify."""
+    import torch
+    import bench
+    d = D.dspark_draft_path(151936, 256, 1, 16, D.DSPARK_BF16)
+    v = D.dspark_verify_path(151936, 256, 1, 16, torch.bfloat16, True)
+    assert (d, v) == ("persistent-cuda-core", "single-launch")
+    assert bench.launches_per_step(d, v, 16) == 3
+    d = D.dspark_draft_path(129280, 256, 256, 6, D.DSPARK_BF16)
+    v = D.dspark_verify_path(129280, 256, 256, 6, torch.bfloat16, False)
+    assert (d, v) == ("tcgen05", "staged-tcgen05")
+    assert bench.launches_per_step(d, v, 6) == 2 * 6 + 1 + 4
