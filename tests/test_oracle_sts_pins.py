@@ -12,7 +12,8 @@ What each test fixes, and which plausible mistake it catches:
   reached and a position with z = 0 only get T = 1 (bound handling);
 - a position's fit ignores the scores of sequences that never reached it
   (the conditional set of "every earlier token accepted");
-- the ECE of a hand-worked sample, and the ECE falls after the fit.
+- the ECE of hand-worked samples (two bins; two confidences sharing one
+  bin of width 1/15), and the ECE falls after the fit.
 """
 import numpy as np
 import pytest
@@ -114,6 +115,18 @@ def test_ece_hand_worked(oracle_mod):
     c = 1.0 / (1.0 + np.exp(-np.float64(np.float32(np.log(3.0)))))  # z is stored in fp32
     assert r["ece_before"] == pytest.approx(abs(2.0 - 2 * c) / 4.0, abs=1e-15)
     assert r["ece_before"] == pytest.approx(0.125, abs=1e-7)
+
+
+def test_ece_shares_a_bin_one_fifteenth_wide(oracle_mod):
+    # c = 0.62 and 0.66 (T = 1) share bin 9 of 15 ([0.6, 0.6667)), so their
+    # label and confidence sums meet in one |sum y - sum c|; with any other
+    # bin count near 15 they would fall apart (14 bins: bins 8 and 9)
+    z = np.array([[np.log(0.62 / 0.38)], [np.log(0.66 / 0.34)]], np.float32)
+    n_acc = np.array([1, 0], np.int32)  # the first accepted, the second rejected
+    c = 1.0 / (1.0 + np.exp(-z[:, 0].astype(np.float64)))
+    assert np.all(np.floor(c * 15) == 9) and np.floor(c[0] * 14) != np.floor(c[1] * 14)
+    r = oracle_mod.sts_fit(z, n_acc)
+    assert r["ece_before"] == pytest.approx(abs(1.0 - c.sum()) / 2.0, abs=1e-15)
 
 
 def test_fit_lowers_ece_on_an_overconfident_head(oracle_mod):
