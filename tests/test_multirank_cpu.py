@@ -4,7 +4,8 @@ The path partitions by request: every rank runs its own replica of the
 workload and the only cross-rank step is the timing reduction (max over
 ranks) and the whole-job rate.  Two spawned ranks check that both see the
 same maximum, that the rate counts every rank's units over the slowest
-rank's time, and that the reference arm runs on rank 0 only.
+rank's time, and that the reference arm (of the step metric and of the
+calibration fit) runs and prints on rank 0 only.
 """
 import multiprocessing
 import os
@@ -40,7 +41,18 @@ def _worker(rank, world, port, q):
         steps, warmup = 1, 0
 
     ref = bench.run_reference(Args, WL.get("tiny"), rank, world)
-    q.put((rank, mx, rate, ref is None))
+
+    class CalArgs:
+        impl, steps, warmup = "reference", 1, 0
+
+    os.environ["DSPARK_REF_SEQUENCES"] = "2000"
+    import contextlib
+    import io
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.run_calibration(CalArgs, WL.CALIBRATIONS["calibration_small"], rank, world)
+    cal_lines = [l for l in buf.getvalue().splitlines() if l.startswith("{")]
+    q.put((rank, mx, rate, ref is None, len(cal_lines)))
     dist.barrier()
     dist.destroy_process_group()
 
@@ -60,10 +72,11 @@ def test_two_rank_timing_reduction_and_reference_arm():
     assert not alive, "a rank hung"
     assert all(p.exitcode == 0 for p in procs)
     res = sorted(q.get(timeout=5) for _ in range(2))
-    for rank, mx, rate, ref_none in res:
+    for rank, mx, rate, ref_none, n_cal in res:
         assert mx == 3.5
         assert rate == pytest.approx(16 * 2 / 3.5e-3)
         assert ref_none == (rank != 0)  # rank 0 alone runs the reference arm
+        assert n_cal == (1 if rank == 0 else 0)  # also for the calibration line
 
 
 def test_single_process_identity():
