@@ -4,8 +4,14 @@
  *
  * Three calls make one decode step, in this order on one stream:
  *   1. dspark_draft_markov       the semi-autoregressive Markov-head draft
- *   2. dspark_confidence_prefix  the confidence-scheduled prefix cut
+ *   2. dspark_confidence_prefix  the confidence-scheduled prefix cut (or
+ *      dspark_confidence_prefix_async: against a verify budget decided two
+ *      steps earlier, with a staircase or piecewise-linear cost table)
  *   3. dspark_verify             the lossless rejection-sampling verify
+ * and one offline call calibrates the confidence head that step 2 reads:
+ *   dspark_sts_fit               per-position temperatures fitted on a
+ *                                calibration set (sequential temperature
+ *                                scaling) and the calibration error
  *
  * Sources (page title, section):
  *   yage.ai "DSpark speculative decoding hardware scheduling": the
@@ -15,8 +21,11 @@
  *     sampling paragraph (the draft must give the exact single-step
  *     p_d(x_k)); the SPS(B) scheduler paragraph (rank every draft token of
  *     the batch by calibrated survival, add the most probable first, stop
- *     before the throughput curve turns down); the variable-length verify
- *     paragraph (verify rows flattened into one tensor, no padding).
+ *     before the throughput curve turns down; STS on an offline set); the
+ *     engineering paragraph (a staircase throughput curve; the budget from
+ *     the confidences of two steps back, the selection from the current
+ *     ones); the variable-length verify paragraph (verify rows flattened
+ *     into one tensor, no padding).
  *   freeaitool.com "DeepSeek DSpark complete guide": 3.1 (Markov head,
  *     rank 256), 4.1 (confidence c_k, sequential temperature scaling),
  *     4.2 (greedy ordering with early stop against a profiled curve).
