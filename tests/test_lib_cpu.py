@@ -152,3 +152,35 @@ def test_bench_launch_count_follows_the_paths():
     v = D.dspark_verify_path(129280, 256, 256, 6, torch.bfloat16, False)
     assert (d, v) == ("tcgen05", "staged-tcgen05")
     assert bench.launches_per_step(d, v, 6) == 2 * 6 + 1 + 4
+
+
+def test_temperature_fit_workspace_is_bounded(lib):
+    """The fit's workspace does not grow with the calibration set past its
+    grid cap: header, 32 search states, per-CTA partials (at most 1184 CTAs)."""
+    small = lib.dspark_sts_workspace_size(1000, 16)
+    big = lib.dspark_sts_workspace_size(10 ** 8, 16)
+    assert 2048 < small <= big < 1.3e6
+    assert lib.dspark_sts_workspace_size(10 ** 8, 32) > big  # partials grow with K
+    assert lib.dspark_sts_workspace_size(10 ** 8, 32) % 256 == 0
+
+
+def test_binding_raises_on_refused_calls(lib):
+    """Argument errors come back from the library before any launch and the
+    binding raises them (a stream handle is passed explicitly: without CUDA
+    the binding cannot ask torch for the current stream)."""
+    import types
+
+    import torch
+    s0 = types.SimpleNamespace(cuda_stream=0)
+    z = torch.zeros(10, 33)
+    n = torch.zeros(10, dtype=torch.int32)
+    t = torch.zeros(33)
+    e = torch.zeros(2)
+    ws = torch.zeros(4096, dtype=torch.uint8)
+    with pytest.raises(D.DSparkError) as err:
+        D.dspark_sts_fit(z, n, t, e, ws, stream=s0)  # K = 33 > DSPARK_STS_MAX_K
+    assert err.value.code == 4
+    z = torch.zeros(10, 16)
+    with pytest.raises(D.DSparkError) as err:
+        D.dspark_sts_fit(z, n, torch.zeros(16), e, ws, stream=s0)  # workspace far too small
+    assert err.value.code == 6
