@@ -181,6 +181,7 @@ def test_binding_raises_on_refused_calls(lib):
         D.dspark_sts_fit(z, n, t, e, ws, stream=s0)  # K = 33 > DSPARK_STS_MAX_K
     assert err.value.code == 4
     z = torch.zeros(10, 16)
+    assert lib.dspark_sts_workspace_size(10, 16) > 1024
     with pytest.raises(D.DSparkError) as err:
-        D.dspark_sts_fit(z, n, torch.zeros(16), e, ws, stream=s0)  # workspace far too small
+        D.dspark_sts_fit(z, n, torch.zeros(16), e, ws[:1024], stream=s0)  # workspace too small
     assert err.value.code == 6
