@@ -76,7 +76,7 @@ typedef enum {
     DSPARK_ERR_INVALID_ARG = 1,  /* bad argument, reported before any launch */
     DSPARK_ERR_CUDA = 2,         /* a CUDA runtime call failed */
     DSPARK_ERR_TIMEOUT = 3,      /* a bounded device-side wait gave up */
-    DSPARK_ERR_UNSUPPORTED = 4,  /* sizes outside what this build supports */
+    DSPARK_ERR_UNSUPPORTED = 4,  /* sizes outside what this library supports */
     DSPARK_ERR_DEVICE_DATA = 5,  /* device found bad data (see status flags) */
     DSPARK_ERR_WORKSPACE = 6     /* workspace missing, misaligned or too small */
 } dspark_status;

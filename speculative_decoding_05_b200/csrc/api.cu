@@ -361,7 +361,7 @@ const char* dspark_status_string(dspark_status s) {
     case DSPARK_ERR_INVALID_ARG: return "invalid argument";
     case DSPARK_ERR_CUDA: return "CUDA runtime error";
     case DSPARK_ERR_TIMEOUT: return "device wait timed out";
-    case DSPARK_ERR_UNSUPPORTED: return "sizes not supported by this build";
+    case DSPARK_ERR_UNSUPPORTED: return "sizes not supported by this library";
     case DSPARK_ERR_DEVICE_DATA: return "device found invalid data";
     case DSPARK_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
   }

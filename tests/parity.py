@@ -1,6 +1,6 @@
 """Compare one GPU step with the oracle on the same seeded inputs.
 
-Rules (tolerances of the benchmark spec):
+Rules (the tolerances every comparison uses):
   * sampled / accepted tokens and prefix lengths bit-exact, except where the
     oracle's margin of that decision is below 1e-6; such cases are counted
     and reported, and the rest of that request's draft is not compared
