@@ -29,22 +29,28 @@
  * probabilities and needs the exact p_d.
  *
  * Parity status (what pins each function; the tests live in
- * tests/test_oracle_pins.py):
+ * tests/test_oracle_pins.py, tests/test_oracle_sts_pins.py and
+ * tests/test_oracle_async_pins.py):
  *   oracle_draft_row / oracle_draft : pinned (W=0 reduces to independent
  *       categorical sampling checked against numpy searchsorted; a
  *       constructed deterministic transition chain; exact enumeration of
  *       the Markov chain on V=4, K=3 against a 10^6-sample histogram; a
- *       hand-worked V=4 example under tests/golden/).
+ *       hand-worked V=4 inverse CDF).
  *   oracle_prefix : pinned (flat / steep cost limits, T_k=1 reduces to the
  *       logistic function, prefix property, linear cost without knee equals
  *       the argmax over prefix lengths of the sorted survival list).
  *   oracle_verify : pinned (p_d = p_t accepts everything, E[accept] =
  *       1 - TV, chi-square losslessness on V=8 at positions 1 and 2, exact
  *       E[n_acc] by enumeration).
+ *   oracle_prefix_async / oracle_cost_stair_ms : pinned (hand lookups on
+ *       a staircase table; a budget commits exactly the top candidates of a
+ *       numpy lexsort of the survival order; the greedy N as budget
+ *       reproduces the greedy cut; clamping; a stair-edge stop).
  *   oracle_sts_fit : pinned (recovers the temperature that generated
  *       logistic labels on a large sample; agrees with a dense grid search
  *       of the likelihood; z -> a*z gives T -> a*T; separable data ends on
- *       the temperature bounds; ECE of a hand-worked sample).
+ *       the temperature bounds; unreached positions do not move the fit;
+ *       hand-worked ECEs).
  *
  * Numerical conventions (stated once, used everywhere):
  *   - inputs are read exactly (fp32 and bf16 values are exact in double);
