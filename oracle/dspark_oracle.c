@@ -29,8 +29,8 @@
  * probabilities and needs the exact p_d.
  *
  * Parity status (what pins each function; the tests live in
- * tests/test_oracle_pins.py, tests/test_oracle_sts_pins.py and
- * tests/test_oracle_async_pins.py):
+ * tests/test_oracle_pins.py, tests/test_oracle_sts_pins.py,
+ * tests/test_oracle_async_pins.py and tests/test_oracle_lmhead_pins.py):
  *   oracle_draft_row / oracle_draft : pinned (W=0 reduces to independent
  *       categorical sampling checked against numpy searchsorted; a
  *       constructed deterministic transition chain; exact enumeration of
@@ -42,6 +42,10 @@
  *   oracle_verify : pinned (p_d = p_t accepts everything, E[accept] =
  *       1 - TV, chi-square losslessness on V=8 at positions 1 and 2, exact
  *       E[n_acc] by enumeration).
+ *   oracle_verify_lmhead : pinned (an identity head reproduces the verify
+ *       on the hidden rows; small-integer hidden states and head make the
+ *       product exact, and the result equals the verify on it bit for bit,
+ *       in fp32 and in bf16, and under H*2, E/2).
  *   oracle_prefix_async / oracle_cost_stair_ms : pinned (hand lookups on
  *       a staircase table; a budget commits exactly the top candidates of a
  *       numpy lexsort of the survival order; the greedy N as budget
@@ -429,14 +433,49 @@ int oracle_prefix(const float *z, const float *temps, const float *cost_tokens,
  *   over the tested positions (+inf if none); res_margin [B] = CDF margin
  *   of the correction/bonus draw.
  */
-int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
-                  const int32_t *verify_len, const float *base, const void *U,
-                  const void *W, int uw_bf16, int V, int r, int B, int K,
-                  const int32_t *prev_token, const float *inv_temp,
-                  const int32_t *tokens, const double *p_d,
-                  const float *u_accept, const float *u_res, int32_t *n_acc,
-                  int32_t *out_tokens, double *accept_margin,
-                  double *res_margin)
+/*
+ * Where the verify's target logits come from: stored rows [n_rows, V], or
+ * the target model's final hidden states [n_rows, dm] times its LM head
+ * [V, dm] (row v of the head gives vocabulary entry v), accumulated in fp64
+ * from the exact stored values.  [freeaitool] 6.3: the target's last hidden
+ * state is passed on instead of its vocabulary-sized distribution and the
+ * LM-head projection is done locally, O(hidden) instead of O(vocab); here
+ * the same projection is applied to the verify's flattened rows ([yage],
+ * variable-length verify paragraph), so the logit rows need not exist in
+ * memory.  Either way the row is scaled by 1/T after it is formed.
+ */
+typedef struct {
+    const float *logits;   /* [n_rows, V], or NULL */
+    const void *hidden;    /* [n_rows, dm] */
+    const void *lm_head;   /* [V, dm] */
+    int dm, bf16;
+} target_src_t;
+
+static void target_row(const target_src_t *t, int64_t row, int V, double it, double *lt)
+{
+    if (t->logits) {
+        const float *trow = t->logits + (size_t)row * (size_t)V;
+        for (int v = 0; v < V; ++v)
+            lt[v] = (double)trow[v] * it;
+        return;
+    }
+    for (int v = 0; v < V; ++v) {
+        double acc = 0.0;
+        for (int i = 0; i < t->dm; ++i)
+            acc += mat_at(t->hidden, t->bf16, t->dm, (long)row, i) *
+                   mat_at(t->lm_head, t->bf16, t->dm, (long)v, i);
+        lt[v] = acc * it;
+    }
+}
+
+static int verify_core(const target_src_t *src, int64_t n_rows, const int64_t *row_start,
+                       const int32_t *verify_len, const float *base, const void *U,
+                       const void *W, int uw_bf16, int V, int r, int B, int K,
+                       const int32_t *prev_token, const float *inv_temp,
+                       const int32_t *tokens, const double *p_d,
+                       const float *u_accept, const float *u_res, int32_t *n_acc,
+                       int32_t *out_tokens, double *accept_margin,
+                       double *res_margin)
 {
     for (int b = 0; b < B; ++b) {
         int L = verify_len[b];
@@ -455,9 +494,7 @@ int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
         int n = 0, rejected = 0;
         double amg = INFINITY;
         for (int p = 0; p < L; ++p) {
-            const float *trow = target + (size_t)(row_start[b] + p) * (size_t)V;
-            for (int v = 0; v < V; ++v)
-                lt[v] = (double)trow[v] * it;
+            target_row(src, row_start[b] + p, V, it, lt);
             double m;
             double zt = softmax_weights(lt, V, pt, &m);
             int x = tokens[(size_t)b * K + p];
@@ -478,9 +515,7 @@ int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
             }
         }
         int j = n; /* position of the correction (or bonus) token */
-        const float *trow = target + (size_t)(row_start[b] + j) * (size_t)V;
-        for (int v = 0; v < V; ++v)
-            lt[v] = (double)trow[v] * it;
+        target_row(src, row_start[b] + j, V, it, lt);
         double m;
         double zt = softmax_weights(lt, V, pt, &m);
         for (int v = 0; v < V; ++v)
@@ -522,6 +557,42 @@ int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
         free(pd);
     }
     return bad ? 3 : 0;
+}
+
+int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
+                  const int32_t *verify_len, const float *base, const void *U,
+                  const void *W, int uw_bf16, int V, int r, int B, int K,
+                  const int32_t *prev_token, const float *inv_temp,
+                  const int32_t *tokens, const double *p_d,
+                  const float *u_accept, const float *u_res, int32_t *n_acc,
+                  int32_t *out_tokens, double *accept_margin,
+                  double *res_margin)
+{
+    target_src_t src = {target, NULL, NULL, 0, 0};
+    return verify_core(&src, n_rows, row_start, verify_len, base, U, W, uw_bf16, V, r, B, K,
+                       prev_token, inv_temp, tokens, p_d, u_accept, u_res, n_acc, out_tokens,
+                       accept_margin, res_margin);
+}
+
+/* The verify with the target logits formed from hidden states and the LM
+ * head (see target_src_t); hidden [n_rows, dm] and lm_head [V, dm] are both
+ * bf16 (hm_bf16 = 1, uint16 bit patterns) or both fp32. */
+int oracle_verify_lmhead(const void *hidden, const void *lm_head, int dm, int hm_bf16,
+                         int64_t n_rows, const int64_t *row_start,
+                         const int32_t *verify_len, const float *base, const void *U,
+                         const void *W, int uw_bf16, int V, int r, int B, int K,
+                         const int32_t *prev_token, const float *inv_temp,
+                         const int32_t *tokens, const double *p_d,
+                         const float *u_accept, const float *u_res, int32_t *n_acc,
+                         int32_t *out_tokens, double *accept_margin,
+                         double *res_margin)
+{
+    if (dm < 1)
+        return 1;
+    target_src_t src = {NULL, hidden, lm_head, dm, hm_bf16};
+    return verify_core(&src, n_rows, row_start, verify_len, base, U, W, uw_bf16, V, r, B, K,
+                       prev_token, inv_temp, tokens, p_d, u_accept, u_res, n_acc, out_tokens,
+                       accept_margin, res_margin);
 }
 
 

@@ -64,6 +64,10 @@ def _load():
                                           i32, i32, i32, i32, P, P, P, P, P, P,
                                           P, P, P, P]
             lib.oracle_verify.restype = i32
+            lib.oracle_verify_lmhead.argtypes = [P, P, i32, i32, ctypes.c_int64, P, P, P, P, P,
+                                                 i32, i32, i32, i32, i32, P, P, P, P, P, P, P,
+                                                 P, P, P]
+            lib.oracle_verify_lmhead.restype = i32
             lib.oracle_sts_fit.argtypes = [P, P, ctypes.c_long, i32, P, P, P]
             lib.oracle_sts_fit.restype = i32
             lib.oracle_num_threads.argtypes = []
@@ -186,6 +190,43 @@ def verify(target, row_start, verify_len, base, U, W, prev_token, tokens, p_d,
                            _p(rm))
     if rc != 0:
         raise ValueError(f"oracle_verify rejected its arguments (rc={rc})")
+    return dict(n_acc=n_acc, out_tokens=out, accept_margin=am, res_margin=rm)
+
+
+def verify_lmhead(hidden, lm_head, row_start, verify_len, base, U, W, prev_token, tokens, p_d,
+                  u_accept, u_res, inv_temp=None):
+    """The verify with target logits formed as hidden [n_rows, dm] times
+    lm_head [V, dm] transposed (both fp32, or both bf16 as uint16 bit
+    patterns) instead of read from stored rows."""
+    lib = _load()
+    Ha, hb = _uw(hidden)
+    Ea, eb = _uw(lm_head)
+    if hb != eb or Ha.shape[1] != Ea.shape[1]:
+        raise ValueError("hidden and lm_head must share dtype and width")
+    n_rows, dm = Ha.shape
+    V = Ea.shape[0]
+    base = _c(base, np.float32)
+    B, K, _ = base.shape
+    Ua, bf = _uw(U)
+    Wa, _ = _uw(W)
+    r = Wa.shape[1]
+    rs = _c(row_start, np.int64)
+    vl = _c(verify_len, np.int32)
+    prev = _c(prev_token, np.int32)
+    toks = _c(tokens, np.int32).reshape(B, K)
+    pd = _c(p_d, np.float64).reshape(B, K)
+    ua = _c(u_accept, np.float32).reshape(B, K)
+    ur = _c(u_res, np.float32)
+    it = None if inv_temp is None else _c(inv_temp, np.float32)
+    n_acc = np.empty(B, np.int32)
+    out = np.empty((B, K + 1), np.int32)
+    am = np.empty(B, np.float64)
+    rm = np.empty(B, np.float64)
+    rc = lib.oracle_verify_lmhead(_p(Ha), _p(Ea), dm, hb, n_rows, _p(rs), _p(vl), _p(base),
+                                  _p(Ua), _p(Wa), bf, V, r, B, K, _p(prev), _p(it), _p(toks),
+                                  _p(pd), _p(ua), _p(ur), _p(n_acc), _p(out), _p(am), _p(rm))
+    if rc != 0:
+        raise ValueError(f"oracle_verify_lmhead rejected its arguments (rc={rc})")
     return dict(n_acc=n_acc, out_tokens=out, accept_margin=am, res_margin=rm)
 
 
