@@ -30,7 +30,8 @@
  *
  * Parity status (what pins each function; the tests live in
  * tests/test_oracle_pins.py, tests/test_oracle_sts_pins.py,
- * tests/test_oracle_async_pins.py and tests/test_oracle_lmhead_pins.py):
+ * tests/test_oracle_async_pins.py, tests/test_oracle_lmhead_pins.py and
+ * tests/test_oracle_rnn_pins.py):
  *   oracle_draft_row / oracle_draft : pinned (W=0 reduces to independent
  *       categorical sampling checked against numpy searchsorted; a
  *       constructed deterministic transition chain; exact enumeration of
@@ -46,6 +47,11 @@
  *       on the hidden rows; small-integer hidden states and head make the
  *       product exact, and the result equals the verify on it bit for bit,
  *       in fp32 and in bf16, and under H*2, E/2).
+ *   oracle_draft_rnn / oracle_verify_rnn : pinned (R = 0 reduces the head
+ *       to the Markov head on tanh(U); at small amplitude the logits equal
+ *       the linear recurrence's to third order; the state carries the token
+ *       before the previous one exactly when R != 0; equal target and draft
+ *       rows accept everything; chi-square losslessness of the verify).
  *   oracle_prefix_async / oracle_cost_stair_ms : pinned (hand lookups on
  *       a staircase table; a budget commits exactly the top candidates of a
  *       numpy lexsort of the survival order; the greedy N as budget
@@ -220,6 +226,115 @@ int oracle_draft(const float *base, const void *U, const void *W, int uw_bf16,
         }
         free(l);
         free(w);
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* RNN sequential head                                                 */
+/* ------------------------------------------------------------------ */
+
+/*
+ * [freeaitool 3.1] names two sequential heads on top of the parallel
+ * backbone: the Markov head above, which sees only the previous token, and
+ * an optional RNN head that keeps a recurrent state and so captures longer
+ * dependencies.  The page gives no formula for it.  Reading taken: the
+ * plainest recurrent state in the same rank-r space as the Markov head's
+ * lookup (Elman form), whose previous-token input is that lookup:
+ *     s_{-1} = h0[b]            (zeros when h0 is NULL)
+ *     x_{-1} = prev_token[b]
+ *     s_k    = tanh(R s_{k-1} + U[x_{k-1}])   (U[x] left out when x < 0)
+ *     l_v    = (base[b, k, v] + s_k . W[v]) * inv_temp
+ * and softmax and inverse-CDF sampling exactly as in the Markov head.
+ * p_d(x_k | x_{<k}) is still one softmax over the vocabulary, so it is
+ * exact, as the rejection-sampling verify needs ([yage, rejection-sampling
+ * paragraph]); the state is a deterministic function of the sampled
+ * prefix.  With R = 0 and h0 = 0 the head is the Markov head on tanh(U).
+ *
+ *   R  [r, r] in the dtype of U and W; (R s)_i = sum_j R[i, j] s_j
+ *   h0 [B, r] fp32 or NULL
+ * outputs as oracle_draft, plus states [B, K, r] (s_k) when not NULL.
+ */
+static void rnn_step(const void *U, const void *R, int uw_bf16, int r, int x_prev,
+                     const double *s_prev, double *s_out)
+{
+    for (int i = 0; i < r; ++i) {
+        double acc = 0.0;
+        for (int j = 0; j < r; ++j)
+            acc += mat_at(R, uw_bf16, r, i, j) * s_prev[j];
+        if (x_prev >= 0)
+            acc += mat_at(U, uw_bf16, r, x_prev, i);
+        s_out[i] = tanh(acc);
+    }
+}
+
+/* one draft row of the RNN head from its state: (base_v + s . W[v]) / T */
+static void rnn_row(const float *base_row, const void *W, int uw_bf16, int V, int r,
+                    const double *s, double inv_temp, double *logits)
+{
+    for (int v = 0; v < V; ++v) {
+        double bias = 0.0;
+        for (int i = 0; i < r; ++i)
+            bias += s[i] * mat_at(W, uw_bf16, r, v, i);
+        logits[v] = ((double)base_row[v] + bias) * inv_temp;
+    }
+}
+
+/* the state before position j: s_{j} from h0, prev_token and x_0..x_{j-1} */
+static void rnn_state_at(const void *U, const void *R, int uw_bf16, int r, const float *h0b,
+                         int x_prev0, const int32_t *toks, int j, double *s, double *tmp)
+{
+    for (int i = 0; i < r; ++i)
+        tmp[i] = h0b ? (double)h0b[i] : 0.0;
+    int x = x_prev0;
+    for (int p = 0; p <= j; ++p) {
+        rnn_step(U, R, uw_bf16, r, x, tmp, s);
+        memcpy(tmp, s, sizeof(double) * (size_t)r);
+        if (p < j)
+            x = toks[p];
+    }
+}
+
+int oracle_draft_rnn(const float *base, const void *U, const void *W, const void *R,
+                     int uw_bf16, int V, int r, int B, int K, const int32_t *prev_token,
+                     const float *h0, const float *inv_temp, const float *u_draft,
+                     int32_t *tokens, double *p_tok, double *lse, double *margin,
+                     double *states)
+{
+    if (V <= 0 || r <= 0 || B < 0 || K < 0 || !R)
+        return 1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int b = 0; b < B; ++b) {
+        double *l = (double *)malloc(sizeof(double) * (size_t)V);
+        double *w = (double *)malloc(sizeof(double) * (size_t)V);
+        double *sp = (double *)malloc(sizeof(double) * (size_t)r);
+        double *sn = (double *)malloc(sizeof(double) * (size_t)r);
+        double it = inv_temp ? (double)inv_temp[b] : 1.0;
+        for (int i = 0; i < r; ++i)
+            sp[i] = h0 ? (double)h0[(size_t)b * r + i] : 0.0;
+        int x = prev_token[b];
+        for (int k = 0; k < K; ++k) {
+            rnn_step(U, R, uw_bf16, r, x, sp, sn);
+            if (states)
+                memcpy(states + ((size_t)b * K + k) * (size_t)r, sn, sizeof(double) * (size_t)r);
+            const float *brow = base + ((size_t)b * K + k) * (size_t)V;
+            rnn_row(brow, W, uw_bf16, V, r, sn, it, l);
+            double m;
+            double z = softmax_weights(l, V, w, &m);
+            double mg;
+            int xk = inverse_cdf(w, V, z, (double)u_draft[(size_t)b * K + k], &mg);
+            size_t o = (size_t)b * K + k;
+            tokens[o] = xk;
+            p_tok[o] = w[xk] / z;
+            lse[o] = m + log(z);
+            margin[o] = mg;
+            x = xk;
+            memcpy(sp, sn, sizeof(double) * (size_t)r);
+        }
+        free(l);
+        free(w);
+        free(sp);
+        free(sn);
     }
     return 0;
 }
@@ -468,7 +583,16 @@ static void target_row(const target_src_t *t, int64_t row, int V, double it, dou
     }
 }
 
-static int verify_core(const target_src_t *src, int64_t n_rows, const int64_t *row_start,
+/* Where the verify's draft row at the rejected position comes from: the
+ * Markov head (R NULL: U[x_{j-1}] . W) or the RNN head (its state s_j,
+ * rebuilt from h0, the previous token and the drafted tokens before j). */
+typedef struct {
+    const void *R;    /* [r, r] or NULL */
+    const float *h0;  /* [B, r] or NULL */
+} draft_src_t;
+
+static int verify_core(const target_src_t *src, const draft_src_t *dsrc, int64_t n_rows,
+                       const int64_t *row_start,
                        const int32_t *verify_len, const float *base, const void *U,
                        const void *W, int uw_bf16, int V, int r, int B, int K,
                        const int32_t *prev_token, const float *inv_temp,
@@ -526,7 +650,16 @@ static int verify_core(const target_src_t *src, int64_t n_rows, const int64_t *r
         if (rejected) {
             int xp = (j == 0) ? prev_token[b] : tokens[(size_t)b * K + j - 1];
             const float *brow = base + ((size_t)b * K + j) * (size_t)V;
-            oracle_draft_row(brow, U, W, uw_bf16, V, r, xp, it, ld);
+            if (dsrc && dsrc->R) {
+                double *st = (double *)malloc(sizeof(double) * (size_t)r * 2);
+                rnn_state_at(U, dsrc->R, uw_bf16, r,
+                             dsrc->h0 ? dsrc->h0 + (size_t)b * r : NULL, prev_token[b],
+                             tokens + (size_t)b * K, j, st, st + r);
+                rnn_row(brow, W, uw_bf16, V, r, st, it, ld);
+                free(st);
+            } else {
+                oracle_draft_row(brow, U, W, uw_bf16, V, r, xp, it, ld);
+            }
             double md;
             double zd = softmax_weights(ld, V, pd, &md);
             double q = 0.0;
@@ -569,7 +702,7 @@ int oracle_verify(const float *target, int64_t n_rows, const int64_t *row_start,
                   double *res_margin)
 {
     target_src_t src = {target, NULL, NULL, 0, 0};
-    return verify_core(&src, n_rows, row_start, verify_len, base, U, W, uw_bf16, V, r, B, K,
+    return verify_core(&src, NULL, n_rows, row_start, verify_len, base, U, W, uw_bf16, V, r, B, K,
                        prev_token, inv_temp, tokens, p_d, u_accept, u_res, n_acc, out_tokens,
                        accept_margin, res_margin);
 }
@@ -590,11 +723,30 @@ int oracle_verify_lmhead(const void *hidden, const void *lm_head, int dm, int hm
     if (dm < 1)
         return 1;
     target_src_t src = {NULL, hidden, lm_head, dm, hm_bf16};
-    return verify_core(&src, n_rows, row_start, verify_len, base, U, W, uw_bf16, V, r, B, K,
+    return verify_core(&src, NULL, n_rows, row_start, verify_len, base, U, W, uw_bf16, V, r, B, K,
                        prev_token, inv_temp, tokens, p_d, u_accept, u_res, n_acc, out_tokens,
                        accept_margin, res_margin);
 }
 
+
+/* The verify of an RNN-head draft: the draft row at the rejected position
+ * is the RNN head's (its state rebuilt from h0 and the drafted prefix). */
+int oracle_verify_rnn(const float *target, int64_t n_rows, const int64_t *row_start,
+                      const int32_t *verify_len, const float *base, const void *U,
+                      const void *W, const void *R, int uw_bf16, int V, int r, int B, int K,
+                      const int32_t *prev_token, const float *h0, const float *inv_temp,
+                      const int32_t *tokens, const double *p_d, const float *u_accept,
+                      const float *u_res, int32_t *n_acc, int32_t *out_tokens,
+                      double *accept_margin, double *res_margin)
+{
+    if (!R)
+        return 1;
+    target_src_t src = {target, NULL, NULL, 0, 0};
+    draft_src_t dsrc = {R, h0};
+    return verify_core(&src, &dsrc, n_rows, row_start, verify_len, base, U, W, uw_bf16, V, r, B,
+                       K, prev_token, inv_temp, tokens, p_d, u_accept, u_res, n_acc, out_tokens,
+                       accept_margin, res_margin);
+}
 
 /* ------------------------------------------------------------------------
  * Sequential temperature scaling of the confidence head

@@ -68,6 +68,12 @@ def _load():
                                                  i32, i32, i32, i32, i32, P, P, P, P, P, P, P,
                                                  P, P, P]
             lib.oracle_verify_lmhead.restype = i32
+            lib.oracle_draft_rnn.argtypes = [P, P, P, P, i32, i32, i32, i32, i32, P, P, P, P, P,
+                                             P, P, P, P]
+            lib.oracle_draft_rnn.restype = i32
+            lib.oracle_verify_rnn.argtypes = [P, ctypes.c_int64, P, P, P, P, P, P, i32, i32, i32,
+                                              i32, i32, P, P, P, P, P, P, P, P, P, P, P]
+            lib.oracle_verify_rnn.restype = i32
             lib.oracle_sts_fit.argtypes = [P, P, ctypes.c_long, i32, P, P, P]
             lib.oracle_sts_fit.restype = i32
             lib.oracle_num_threads.argtypes = []
@@ -132,6 +138,71 @@ def draft(base, U, W, prev_token, u_draft, inv_temp=None):
     if rc != 0:
         raise ValueError(f"oracle_draft rejected its arguments (rc={rc})")
     return dict(tokens=tokens, p_tok=p_tok, lse=lse, margin=margin)
+
+
+def draft_rnn(base, U, W, R, prev_token, u_draft, h0=None, inv_temp=None, states=False):
+    """RNN-head draft: state s_k = tanh(R s_{k-1} + U[x_{k-1}]) from h0
+    (zeros if None), logits (base + s_k . W^T) / T.  U, W [V,r] and R [r,r]
+    share one dtype (fp32, or uint16 bf16 bit patterns)."""
+    lib = _load()
+    base = _c(base, np.float32)
+    B, K, V = base.shape
+    Ua, bf = _uw(U)
+    Wa, _ = _uw(W)
+    Ra, rb = _uw(R)
+    r = Wa.shape[1]
+    assert Ra.shape == (r, r) and rb == bf and Ua.shape == (V, r)
+    prev = _c(prev_token, np.int32)
+    ud = _c(u_draft, np.float32).reshape(B, K)
+    hh = None if h0 is None else _c(h0, np.float32).reshape(B, r)
+    it = None if inv_temp is None else _c(inv_temp, np.float32)
+    tokens = np.empty((B, K), np.int32)
+    p_tok = np.empty((B, K), np.float64)
+    lse = np.empty((B, K), np.float64)
+    margin = np.empty((B, K), np.float64)
+    st = np.empty((B, K, r), np.float64) if states else None
+    rc = lib.oracle_draft_rnn(_p(base), _p(Ua), _p(Wa), _p(Ra), bf, V, r, B, K, _p(prev), _p(hh),
+                              _p(it), _p(ud), _p(tokens), _p(p_tok), _p(lse), _p(margin), _p(st))
+    if rc != 0:
+        raise ValueError(f"oracle_draft_rnn rejected its arguments (rc={rc})")
+    out = dict(tokens=tokens, p_tok=p_tok, lse=lse, margin=margin)
+    if states:
+        out["states"] = st
+    return out
+
+
+def verify_rnn(target, row_start, verify_len, base, U, W, R, prev_token, tokens, p_d, u_accept,
+               u_res, h0=None, inv_temp=None):
+    """The verify of an RNN-head draft (the rejected position's draft row
+    is the RNN head's)."""
+    lib = _load()
+    target = _c(target, np.float32)
+    n_rows, V = target.shape
+    base = _c(base, np.float32)
+    B, K, _ = base.shape
+    Ua, bf = _uw(U)
+    Wa, _ = _uw(W)
+    Ra, _ = _uw(R)
+    r = Wa.shape[1]
+    rs = _c(row_start, np.int64)
+    vl = _c(verify_len, np.int32)
+    prev = _c(prev_token, np.int32)
+    hh = None if h0 is None else _c(h0, np.float32).reshape(B, r)
+    toks = _c(tokens, np.int32).reshape(B, K)
+    pd = _c(p_d, np.float64).reshape(B, K)
+    ua = _c(u_accept, np.float32).reshape(B, K)
+    ur = _c(u_res, np.float32)
+    it = None if inv_temp is None else _c(inv_temp, np.float32)
+    n_acc = np.empty(B, np.int32)
+    out = np.empty((B, K + 1), np.int32)
+    am = np.empty(B, np.float64)
+    rm = np.empty(B, np.float64)
+    rc = lib.oracle_verify_rnn(_p(target), n_rows, _p(rs), _p(vl), _p(base), _p(Ua), _p(Wa),
+                               _p(Ra), bf, V, r, B, K, _p(prev), _p(hh), _p(it), _p(toks), _p(pd),
+                               _p(ua), _p(ur), _p(n_acc), _p(out), _p(am), _p(rm))
+    if rc != 0:
+        raise ValueError(f"oracle_verify_rnn rejected its arguments (rc={rc})")
+    return dict(n_acc=n_acc, out_tokens=out, accept_margin=am, res_margin=rm)
 
 
 def cost_ms(cost_tokens, cost_ms_, n_tokens: float) -> float:
