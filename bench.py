@@ -9,9 +9,18 @@ is no data-path collective, so scaling is weak).
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
     python bench.py --impl reference ...   # the CPU oracle on host cores
 
+The default workload is stress (V=151936, r=256, B=512, K=16, scheduler on),
+the largest configuration at the metric's vocabulary.  Its steps are
+sequential decode steps: each step draws fresh uniforms (the run's per-step
+sets, copied into the step's input buffers before its timed region) and
+takes as previous token the token the step before emitted last, copied on
+the device inside the step's graph.  The logits stay fixed for the run.
+
 Timing: every step is replayed from CUDA graphs and timed with CUDA events
 on the launching stream; a 256 MB scratch write between steps flushes L2
-(outside the timed events).  Prints one JSON line (rank 0).
+(outside the timed events).  Prints one JSON line (rank 0).  With --gpus N
+and no launcher environment (WORLD_SIZE unset) the script starts N ranks
+itself through torch.distributed.run.
 """
 from __future__ import annotations
 
@@ -28,7 +37,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "draft+verify tokens/s (B×K per step) at V=151936; % of HBM / tensor roofline"
 UNIT = "tokens/s"
-DEFAULT_CONFIG = "single"
+DEFAULT_CONFIG = "stress"
 
 
 def parse():
@@ -41,7 +50,19 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    # smaller shapes of a workload (profiling captures, parity spot checks);
+    # the line's config reports the sizes that ran
+    ap.add_argument("--B", type=int, default=0)
+    ap.add_argument("--K", type=int, default=0)
+    ap.add_argument("--V", type=int, default=0)
     return ap.parse_args()
+
+
+def workload_of(args):
+    """The workload named by --config with any --B / --K / --V override."""
+    from speculative_decoding_05_b200 import workloads as WL
+    over = {k: v for k, v in (("B", args.B), ("K", args.K), ("V", args.V)) if v}
+    return WL.get(args.config, **over)
 
 
 def peaks():
@@ -54,14 +75,20 @@ def peaks():
     return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, src="fallback")
 
 
-def algorithmic(w, L):
-    """Algorithmic bytes / flops of one step (W counted once per step)."""
+def algorithmic(w, L, reproject: bool = True):
+    """Algorithmic bytes / flops of one step (W counted once per step).
+
+    The verify reads every verified target row and, per request, one more
+    row of draft logits for the residual; W (and the residual's flops) only
+    when it re-projects that row (without the draft's bias rows)."""
     V, r, B, K = w.V, w.r, w.B, w.K
     uw = 2 if w.uw_bf16 else 4
     draft_bytes = uw * r * V + B * K * 4 * V + B * K * uw * r
-    verify_bytes = sum(int(l) + 1 for l in L) * 4 * V + B * 4 * V + uw * r * V
+    verify_bytes = sum(int(l) + 1 for l in L) * 4 * V + B * 4 * V
+    if reproject:
+        verify_bytes += uw * r * V
     draft_flops = 2.0 * B * K * r * V
-    verify_flops = 2.0 * B * r * V
+    verify_flops = 2.0 * B * r * V if reproject else 0.0
     return dict(draft_bytes=draft_bytes, verify_bytes=verify_bytes,
                 step_bytes=draft_bytes + verify_bytes, draft_flops=draft_flops,
                 verify_flops=verify_flops)
@@ -310,6 +337,21 @@ def cpu_baseline(w, inp_dev, seconds):
 
 # ----------------------------------------------------------------- main --
 
+def step_uniform_sets(w, inp, rank: int = 0):
+    """The uniforms of every step of one run of the workload, stacked on the
+    device: step 0 takes the workload's own draw (already in `inp`), step
+    s > 0 the fresh set WL.step_uniforms draws for it.  A one-step workload
+    has one set."""
+    import torch
+    from speculative_decoding_05_b200 import workloads as WL
+    dev = inp["u_draft"].device
+    sets = [dict(u_draft=inp["u_draft"].clone(), u_accept=inp["u_accept"].clone(),
+                 u_res=inp["u_res"].clone())]
+    for s in range(1, max(1, w.steps)):
+        sets.append(WL.step_uniforms(w, s, device=dev, seed=w.seed + 1000 * rank))
+    return {k: torch.stack([d[k] for d in sets]) for k in ("u_draft", "u_accept", "u_res")}
+
+
 STS_METRIC = ("calibration score entries fitted per second (sequential temperature "
               "scaling of the confidence head, N x K per fit)")
 STS_UNIT = "entries/s"
@@ -490,16 +532,41 @@ def run_calibration(args, c, rank, world):
         "ece_before_after": [float(e) for e in ece.cpu()]}), flush=True)
 
 
+def launcher_argv(n: int, argv: list, port: int) -> list:
+    """The command that runs this script as n ranks on one node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def check_world(gpus: int, env) -> int:
+    """World size of this process; --gpus must match the launcher's."""
+    world = int(env.get("WORLD_SIZE", "1"))
+    if world != gpus:
+        raise SystemExit(f"bench.py: --gpus {gpus} but the launcher started {world} rank(s)")
+    return world
+
+
 def main():
     args = parse()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # no launcher: start the ranks here (one process per GPU), with a
+        # bound on the whole run
+        import socket
+        import subprocess
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        rc = subprocess.call(launcher_argv(args.gpus, sys.argv[1:], port))
+        sys.exit(rc)
     rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    world = check_world(args.gpus, os.environ)
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     from speculative_decoding_05_b200 import workloads as WL
     if args.config in WL.CALIBRATIONS:
         run_calibration(args, WL.CALIBRATIONS[args.config], rank, world)
         return
-    w = WL.get(args.config)
+    w = workload_of(args)
 
     if args.impl == "reference":
         out = run_reference(args, w, rank, world)
@@ -530,6 +597,11 @@ def main():
     step = DSparkStep(w.V, w.r, w.B, w.K, n_rows, inp["U"].dtype, dev)
     stream = torch.cuda.Stream(dev)
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    uni = step_uniform_sets(w, inp, rank)
+    # the inputs are drawn on the default stream and the steps run on
+    # `stream`: finish the draws (and the allocator's reuse of the blocks
+    # they freed) before the first step
+    torch.cuda.synchronize()
 
     # eager warm-up (sets kernel attributes), then capture each call in a graph
     with torch.cuda.stream(stream):
@@ -546,14 +618,25 @@ def main():
         with torch.cuda.graph(g, stream=stream):
             fn()
         graphs.append(g)
-    # timed: the draft call and the rest of the step (prefix + verify) as two
+    # timed: the draft call and the rest of the step (prefix + verify, then
+    # the emitted last token copied into prev_token for the next step) as two
     # graphs, so the draft's own time comes from the same timed region
     g_draft = graphs[0]
     g_rest = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_rest, stream=stream):
         step.prefix(inp, w.scheduler)
         step.verify(inp)
+        if w.steps > 1:
+            inp["prev_token"].copy_(step.last_token)
     torch.cuda.synchronize()
+    n_set = [0]
+
+    def next_uniforms():
+        """Copy the next step's uniforms into the captured input buffers."""
+        i = n_set[0] % len(uni["u_draft"])
+        n_set[0] += 1
+        for k in ("u_draft", "u_accept", "u_res"):
+            inp[k].copy_(uni[k][i], non_blocking=True)
 
     def replay():
         g_draft.replay()
@@ -562,6 +645,7 @@ def main():
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
             flush.zero_()
+            next_uniforms()
             replay()
     torch.cuda.synchronize()
 
@@ -577,6 +661,7 @@ def main():
     with torch.cuda.stream(stream):
         for i in range(args.steps):
             flush.zero_()
+            next_uniforms()
             ev[i][0].record(stream)
             g_draft.replay()
             ev[i][1].record(stream)
@@ -610,7 +695,7 @@ def main():
 
     L = step.verify_len.cpu().tolist()
     na = step.n_accepted.cpu()
-    alg = algorithmic(w, L)
+    alg = algorithmic(w, L, reproject=step.draft_bias is None)
     pk = peaks()
     md, mv = statistics.mean(t_draft_timed), statistics.mean(t_verify)
     # dominant part: the draft call (K projection + sampler launches) or the verify call
@@ -626,15 +711,22 @@ def main():
                 "algorithmic_bytes_per_launch": dom_bytes,
                 "step_frac": alg["step_bytes"] / (ms * 1e-3) / 1e9 / pk["hbm"]}
 
-    # end to end: inputs from pinned host memory, outputs back, every step
+    # end to end: every step copies its inputs in from pinned host memory
+    # (the logits, temperatures, confidences and row offsets, and that step's
+    # uniforms) and its results out; the previous token of a multi-step run
+    # stays on the device (the graph carries it), that of a one-step run is
+    # copied in too
     e2e = None
     if rank == 0 or world > 1:
-        names_in = ["base", "target", "prev_token", "inv_temp", "u_draft", "u_accept", "u_res",
-                    "z", "row_start"]
+        names_in = ["base", "target", "inv_temp", "z", "row_start"]
+        if w.steps <= 1:
+            names_in.append("prev_token")
         host_in = {k: inp[k].cpu().pin_memory() for k in names_in}
+        host_uni = {k: v.cpu().pin_memory() for k, v in uni.items()}
         outs = [step.n_accepted, step.out_tokens, step.last_token]
         host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+        h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + \
+            sum(t[0].numel() * t.element_size() for t in host_uni.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out)
         n_e2e = max(1, min(args.e2e_steps, args.steps))
         e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -643,9 +735,12 @@ def main():
         with torch.cuda.stream(stream):
             for i in range(n_e2e):
                 flush.zero_()
+                j = i % host_uni["u_draft"].shape[0]
                 e2e_ev[i][0].record(stream)
                 for k in names_in:
                     inp[k].copy_(host_in[k], non_blocking=True)
+                for k, v in host_uni.items():
+                    inp[k].copy_(v[j], non_blocking=True)
                 replay()
                 for o, ho in zip(outs, host_out):
                     ho.copy_(o, non_blocking=True)
@@ -654,6 +749,7 @@ def main():
         e2e_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in e2e_ev), dev)
         e2e = {"value": whole_job_rate(units_per_rank, world, e2e_ms), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        del host_in, host_uni
 
     vpath = D.dspark_verify_path(w.V, w.r, w.B, w.K, inp["U"].dtype, step.draft_bias is not None)
     n_launch = launches_per_step(step.path, vpath, w.K)
@@ -673,7 +769,11 @@ def main():
         "config": {"workload": w.name, "V": w.V, "r": w.r, "B": w.B, "K": w.K,
                    "uw": "bf16" if w.uw_bf16 else "f32", "scheduler": w.scheduler,
                    "draft_path": step.path, "l2": "flushed by a 256 MB write between steps",
-                   "parallelism": f"replicas x{world}", "graphs": True},
+                   "parallelism": f"replicas x{world}", "graphs": True,
+                   "steps_per_run": w.steps,
+                   "sequential": ("fresh uniforms every step; prev_token = the previous step's "
+                                  "last emitted token, carried on the device")
+                   if w.steps > 1 else "one step replayed"},
         "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
         "gpu_launches": n_launch * args.steps,
         "clocks": clk,

@@ -1,4 +1,4 @@
-"""Compare one GPU step with the oracle on the same seeded inputs.
+"""Compare GPU steps with the oracle on the same seeded inputs.
 
 Rules (the tolerances every comparison uses):
   * sampled / accepted tokens and prefix lengths bit-exact, except where the
@@ -32,60 +32,72 @@ class Report:
         self.near = dict(draft=0, prefix=0, accept=0, residual=0)
         self.skipped = 0
         self.failures = []
+        # request -> the token the oracle emitted last (its next prev_token),
+        # for requests whose whole step was compared
+        self.oracle_last = {}
 
     def fail(self, msg):
         self.failures.append(msg)
+
+    def merge(self, other):
+        for k in self.checked:
+            self.checked[k] += other.checked[k]
+            self.near[k] += other.near[k]
+        self.skipped += other.skipped
+        self.failures += other.failures
 
     def __repr__(self):
         return f"checked={self.checked} near_margin={self.near} skipped={self.skipped} failures={len(self.failures)}"
 
 
-def compare_step(oracle, inp, step, enable_prefix, requests=None, rep=None, verify_len=None):
-    """Run the oracle on `requests` (default: all) and compare with the
-    outputs held by `step` (a DSparkStep that has just run on `inp`).
-    With `verify_len` (the lengths the caller set by hand) the prefix cut is
-    not compared and both sides verify those lengths."""
-    rep = rep or Report()
-    B, K, V = inp["base"].shape
-    if requests is None:
-        requests = np.arange(B)
+def host_inputs(inp, requests):
+    """Host copies of one step's inputs for `requests`: the per-request
+    logit rows (base [n,K,V], target rows [n][L+1 <= K+1, V] are taken from
+    row_start), U, W, inverse temperatures, uniforms and prev_token."""
     requests = np.asarray(requests)
-    idx = torch.as_tensor(requests, device=inp["base"].device)
+    dev = inp["base"].device
+    idx = torch.as_tensor(requests, device=dev)
+    K = inp["base"].shape[1]
+    rs = host(inp["row_start"])
+    rows = np.concatenate([np.arange(rs[b], rs[b] + K + 1) for b in requests]) if len(requests) \
+        else np.zeros(0, np.int64)
+    tgt = host(inp["target"].index_select(0, torch.as_tensor(rows, device=dev)))
+    return dict(requests=requests, base=host(inp["base"].index_select(0, idx)),
+                target=tgt.reshape(len(requests), K + 1, -1),
+                U=host_uw(inp["U"]), W=host_uw(inp["W"]),
+                inv_temp=host(inp["inv_temp"].index_select(0, idx)),
+                prev_token=host(inp["prev_token"].index_select(0, idx)),
+                u_draft=host(inp["u_draft"].index_select(0, idx)),
+                u_accept=host(inp["u_accept"].index_select(0, idx)),
+                u_res=host(inp["u_res"].index_select(0, idx)))
 
-    # ---- prefix cut: on the whole batch (it is global over requests)
-    if verify_len is not None:
-        L_or = np.asarray(verify_len, np.int32)[requests]
-    elif K > 0 and B > 0:
-        pr = oracle.prefix(host(inp["z"]), host(inp["temps"]), host(inp["cost_tokens"]),
-                           host(inp["cost_ms"]), enable=enable_prefix)
-        c_g, s_g = host(step.c), host(step.survival)
-        if np.abs(c_g - pr["c"]).max() > P_ATOL or np.abs(s_g - pr["S"]).max() > P_ATOL:
-            rep.fail("prefix: c / survival outside 1e-5")
-        L_g = host(step.verify_len)
-        rep.checked["prefix"] += 1
-        if not np.array_equal(L_g, pr["L"]):
-            if pr["margin"] < MARGIN:
-                rep.near["prefix"] += 1
-            else:
-                rep.fail(f"prefix: verify_len differs (margin {pr['margin']:.3g})")
-        elif abs(float(host(step.objective)[0]) - pr["objective"]) > 1e-5 * abs(pr["objective"]):
-            rep.fail("prefix: objective outside 1e-5 relative")
-        L_or = pr["L"][requests]
-    else:
-        L_or = np.zeros(len(requests), np.int32)
-    L_gpu = host(step.verify_len)[requests] if B > 0 else L_or
 
-    # ---- draft on the sampled requests
-    U, W = host_uw(inp["U"]), host_uw(inp["W"])
-    base = host(inp["base"].index_select(0, idx))
-    prev = host(inp["prev_token"].index_select(0, idx))
-    it = host(inp["inv_temp"].index_select(0, idx))
-    d = oracle.draft(base, U, W, prev, host(inp["u_draft"].index_select(0, idx)), inv_temp=it)
-    tok_g = host(step.tokens.index_select(0, idx))
-    p_g = host(step.p_tok.index_select(0, idx))
-    lse_g = host(step.lse.index_select(0, idx))
-    match_len = np.full(len(requests), K)
-    for i in range(len(requests)):
+def gpu_outputs(step, requests):
+    """Host copies of the outputs a DSparkStep holds, for `requests`."""
+    idx = torch.as_tensor(np.asarray(requests), device=step.tokens.device)
+    pick = lambda t: host(t.index_select(0, idx))
+    return dict(tokens=pick(step.tokens), p_tok=pick(step.p_tok), lse=pick(step.lse),
+                verify_len=pick(step.verify_len), n_accepted=pick(step.n_accepted),
+                out_tokens=pick(step.out_tokens), last_token=pick(step.last_token))
+
+
+def compare_requests(oracle, h, g, L_or, rep=None):
+    """Oracle draft and verify of the requests in `h` (host inputs, see
+    host_inputs) against the GPU outputs `g` (see gpu_outputs), both sides
+    verifying the oracle's lengths L_or where the GPU's agree."""
+    rep = rep or Report()
+    requests = h["requests"]
+    n = len(requests)
+    if n == 0:
+        return rep
+    K = h["base"].shape[1]
+    L_or = np.asarray(L_or, np.int32)
+    L_gpu = g["verify_len"]
+    d = oracle.draft(h["base"], h["U"], h["W"], h["prev_token"], h["u_draft"],
+                     inv_temp=h["inv_temp"])
+    tok_g, p_g, lse_g = g["tokens"], g["p_tok"], g["lse"]
+    match_len = np.full(n, K)
+    for i in range(n):
         for k in range(K):
             rep.checked["draft"] += 1
             if tok_g[i, k] != d["tokens"][i, k]:
@@ -101,30 +113,20 @@ def compare_step(oracle, inp, step, enable_prefix, requests=None, rep=None, veri
             if abs(lse_g[i, k] - d["lse"][i, k]) > LSE_RTOL * max(1.0, abs(d["lse"][i, k])):
                 rep.fail(f"draft b={requests[i]} k={k}: lse {lse_g[i, k]} vs {d['lse'][i, k]}")
 
-    # ---- verify: requests whose verified draft prefix and L agree
-    keep = [i for i in range(len(requests))
-            if match_len[i] >= L_or[i] and L_or[i] == L_gpu[i]]
-    rep.skipped += len(requests) - len(keep)
-    if not keep:
+    # verify: requests whose verified draft prefix and L agree
+    keep = np.asarray([i for i in range(n) if match_len[i] >= L_or[i] and L_or[i] == L_gpu[i]],
+                      dtype=np.int64)
+    rep.skipped += n - len(keep)
+    if len(keep) == 0:
         return rep
-    keep = np.asarray(keep)
-    sub = requests[keep]
-    sidx = torch.as_tensor(sub, device=inp["base"].device)
-    rows = []
-    rs_all = host(inp["row_start"])
-    for b, L in zip(sub, L_or[keep]):
-        rows.append(np.arange(rs_all[b], rs_all[b] + L + 1))
-    row_ids = np.concatenate(rows)
-    tgt = host(inp["target"].index_select(0, torch.as_tensor(row_ids, device=inp["base"].device)))
-    rs_sub = np.concatenate([[0], np.cumsum([len(x) for x in rows])[:-1]]).astype(np.int64)
-    v = oracle.verify(tgt, rs_sub, L_or[keep].astype(np.int32), base[keep], U, W, prev[keep],
-                      d["tokens"][keep], d["p_tok"][keep],
-                      host(inp["u_accept"].index_select(0, sidx)),
-                      host(inp["u_res"].index_select(0, sidx)), inv_temp=it[keep])
-    na_g = host(step.n_accepted.index_select(0, sidx))
-    out_g = host(step.out_tokens.index_select(0, sidx))
-    last_g = host(step.last_token.index_select(0, sidx))
-    for i, b in enumerate(sub):
+    Lk = L_or[keep]
+    tgt = np.concatenate([h["target"][i, :L + 1] for i, L in zip(keep, Lk)])
+    rs_sub = np.concatenate([[0], np.cumsum(Lk + 1)[:-1]]).astype(np.int64)
+    v = oracle.verify(tgt, rs_sub, Lk, h["base"][keep], h["U"], h["W"], h["prev_token"][keep],
+                      d["tokens"][keep], d["p_tok"][keep], h["u_accept"][keep],
+                      h["u_res"][keep], inv_temp=h["inv_temp"][keep])
+    na_g, out_g, last_g = g["n_accepted"][keep], g["out_tokens"][keep], g["last_token"][keep]
+    for i, b in enumerate(requests[keep]):
         rep.checked["accept"] += 1
         if na_g[i] != v["n_acc"][i]:
             if v["accept_margin"][i] < MARGIN:
@@ -135,14 +137,58 @@ def compare_step(oracle, inp, step, enable_prefix, requests=None, rep=None, veri
             continue
         rep.checked["residual"] += 1
         if not np.array_equal(out_g[i], v["out_tokens"][i]):
-            n = v["n_acc"][i]
-            same_prefix = np.array_equal(out_g[i, :n], v["out_tokens"][i, :n]) and \
-                np.all(out_g[i, n + 1:] == -1)
+            na = v["n_acc"][i]
+            same_prefix = np.array_equal(out_g[i, :na], v["out_tokens"][i, :na]) and \
+                np.all(out_g[i, na + 1:] == -1)
             if same_prefix and v["res_margin"][i] < MARGIN:
                 rep.near["residual"] += 1
             else:
                 rep.fail(f"verify b={b}: out {out_g[i].tolist()} != {v['out_tokens'][i].tolist()} "
                          f"(margin {v['res_margin'][i]:.3g})")
-        elif last_g[i] != v["out_tokens"][i, v["n_acc"][i]]:
+            continue
+        if last_g[i] != v["out_tokens"][i, v["n_acc"][i]]:
             rep.fail(f"verify b={b}: last_token {last_g[i]}")
+            continue
+        rep.oracle_last[int(b)] = int(v["out_tokens"][i, v["n_acc"][i]])
     return rep
+
+
+def compare_prefix(oracle, inp, step, enable_prefix, rep):
+    """The prefix cut over the whole batch (it is global over requests);
+    returns the oracle's verify lengths."""
+    pr = oracle.prefix(host(inp["z"]), host(inp["temps"]), host(inp["cost_tokens"]),
+                       host(inp["cost_ms"]), enable=enable_prefix)
+    c_g, s_g = host(step.c), host(step.survival)
+    if np.abs(c_g - pr["c"]).max() > P_ATOL or np.abs(s_g - pr["S"]).max() > P_ATOL:
+        rep.fail("prefix: c / survival outside 1e-5")
+    L_g = host(step.verify_len)
+    rep.checked["prefix"] += 1
+    if not np.array_equal(L_g, pr["L"]):
+        if pr["margin"] < MARGIN:
+            rep.near["prefix"] += 1
+        else:
+            rep.fail(f"prefix: verify_len differs (margin {pr['margin']:.3g})")
+    elif abs(float(host(step.objective)[0]) - pr["objective"]) > 1e-5 * abs(pr["objective"]):
+        rep.fail("prefix: objective outside 1e-5 relative")
+    return pr["L"]
+
+
+def compare_step(oracle, inp, step, enable_prefix, requests=None, rep=None, verify_len=None):
+    """Run the oracle on `requests` (default: all) and compare with the
+    outputs held by `step` (a DSparkStep that has just run on `inp`).
+    With `verify_len` (the lengths the caller set by hand) the prefix cut is
+    not compared and both sides verify those lengths."""
+    rep = rep or Report()
+    B, K, V = inp["base"].shape
+    if requests is None:
+        requests = np.arange(B)
+    requests = np.asarray(requests)
+    if verify_len is not None:
+        L_all = np.asarray(verify_len, np.int32)
+    elif K > 0 and B > 0:
+        L_all = compare_prefix(oracle, inp, step, enable_prefix, rep)
+    else:
+        L_all = np.zeros(B, np.int32)
+    h = host_inputs(inp, requests)
+    g = gpu_outputs(step, requests)
+    return compare_requests(oracle, h, g, L_all[requests], rep)

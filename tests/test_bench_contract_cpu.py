@@ -46,3 +46,11 @@ def test_reference_arm_calibration_fit():
     check_reference_line(d, 1, 0)
     assert d["unit"] == "entries/s" and d["config"]["N"] == 50_003 and d["config"]["K"] == 16
     assert d["config"]["requests"] == 5000
+
+
+def test_gpus_two_without_launcher_starts_two_ranks():
+    """`bench.py --gpus 2` with no launcher starts two ranks itself; the
+    reference arm prints its one line on rank 0 and reports both ranks."""
+    d = run_bench("--impl", "reference", "--gpus", "2", "--config", "tiny", "--steps", "1",
+                  "--warmup", "0")
+    assert d["impl"] == "reference" and d["n_gpus"] == 2

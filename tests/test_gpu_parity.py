@@ -151,37 +151,6 @@ def test_full_size(oracle_mod, name):
     torch.cuda.empty_cache()
 
 
-def test_stress_sequential_steps(oracle_mod):
-    """Three sequential steps; each side feeds its own last emitted token
-    into the next step (the oracle never reads the GPU's tokens)."""
-    w = WL.get("stress", V=8192, r=256, B=32, K=16, seed=21)
-    inp = WL.make_inputs(w, device="cuda")
-    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
-    req = np.arange(w.B)
-    prev_gpu = inp["prev_token"].clone()
-    prev_or = host(inp["prev_token"]).copy()
-    for s in range(3):
-        if s > 0:
-            inp.update(WL.step_uniforms(w, s, device="cuda"))
-        step.run(inp, enable_prefix=True, prev_token=prev_gpu)
-        torch.cuda.synchronize()
-        oinp = dict(inp)
-        oinp["prev_token"] = torch.as_tensor(prev_or, device="cuda")
-        rep = compare_step(oracle_mod, oinp, step, True, requests=req)
-        _assert_ok(rep)
-        # next step: GPU uses its own last token, the oracle its own
-        prev_gpu = step.last_token.clone()
-        pr = oracle_mod.prefix(host(inp["z"]), host(inp["temps"]), host(inp["cost_tokens"]),
-                               host(inp["cost_ms"]))
-        d = oracle_mod.draft(host(inp["base"]), WL.host_uw(inp["U"]), WL.host_uw(inp["W"]), prev_or,
-                             host(inp["u_draft"]), inv_temp=host(inp["inv_temp"]))
-        v = oracle_mod.verify(host(inp["target"]), host(inp["row_start"]), pr["L"], host(inp["base"]),
-                              WL.host_uw(inp["U"]), WL.host_uw(inp["W"]), prev_or, d["tokens"],
-                              d["p_tok"], host(inp["u_accept"]), host(inp["u_res"]),
-                              inv_temp=host(inp["inv_temp"]))
-        prev_or = v["out_tokens"][np.arange(w.B), v["n_acc"]].astype(np.int32)
-
-
 def test_edge_cases(oracle_mod):
     # B = 1, K = 1, every verify length 0 and K
     for L in (0, 1):

@@ -84,3 +84,21 @@ def test_single_process_identity():
     import bench
     assert bench.reduce_max(1.25) == 1.25
     assert bench.whole_job_rate(16, 1, 2.0) == pytest.approx(8000.0)
+
+
+def test_launcher_for_gpus_n():
+    """--gpus N without a launcher re-runs the script as N ranks through
+    torch.distributed.run on 127.0.0.1; under a launcher --gpus must match
+    its world size."""
+    sys.path.insert(0, ROOT)
+    import bench
+    argv = bench.launcher_argv(4, ["--gpus", "4", "--steps", "3"], 29512)
+    assert argv[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in argv and "--master-addr=127.0.0.1" in argv
+    assert "--master-port=29512" in argv and argv[-4:] == ["--gpus", "4", "--steps", "3"]
+    assert bench.check_world(2, {"WORLD_SIZE": "2"}) == 2
+    assert bench.check_world(1, {}) == 1
+    with pytest.raises(SystemExit):
+        bench.check_world(4, {"WORLD_SIZE": "2"})
+    with pytest.raises(SystemExit):
+        bench.check_world(2, {"WORLD_SIZE": "1"})
