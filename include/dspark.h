@@ -188,6 +188,45 @@ dspark_status dspark_sts_fit(const float *z, const int32_t *n_accepted, long lon
                              size_t ws_bytes, void *stream);
 
 /* ---------------------------------------------------------------------- */
+/* 1c. RNN sequential head                                                 */
+/* ---------------------------------------------------------------------- */
+
+size_t dspark_draft_rnn_workspace_size(int V, int r, int B, int K);
+
+/*
+ * The draft with the optional RNN head in place of the Markov head
+ * (freeaitool.com "DeepSeek DSpark complete guide" 3.1: the sequential head
+ * is the Markov head by default, or an RNN head that keeps a recurrent state
+ * to capture longer dependencies; the page gives no formula, the one below
+ * is this library's reading):
+ *     s_{-1} = h0[b] (zeros if h0 is NULL),  x_{-1} = prev_token[b]
+ *     s_k    = tanh(R s_{k-1} + U[x_{k-1}])     (no U term when x < 0)
+ *     p(x_k | x_<k) = softmax((base_logits[b,k,:] + s_k . W^T) * inv_temp[b])
+ * sampled by inverse CDF with u_draft[b,k] exactly as dspark_draft_markov
+ * (same outputs: tokens, p_tok, lse, ref_max, ref_sum).  p_d stays one
+ * exact softmax per position, as the rejection-sampling verify needs.
+ *
+ * Inputs beyond dspark_draft_markov's
+ *   R [r, r] bf16, row-major, (R s)_i = sum_j R[i, j] s_j
+ *   h0 [B, r] fp32 or NULL: the state before position 1
+ * Outputs beyond dspark_draft_markov's
+ *   states [B, K, r] fp32 or NULL: s_k of every position (the caller keeps
+ *       the one after the last accepted token for the next step)
+ *   draft_bias [B, K, V] fp32 or NULL: s_k . W^T.  The verify of an RNN
+ *       draft needs it (pass it to dspark_verify): the verify's own
+ *       re-projection of a rejected row is the Markov lookup.
+ * Sizes: bf16 only, r a multiple of 64 up to 256, V >= 128; any B.  The
+ * state is fp32; the projection multiplies W by its bf16 high and low parts
+ * (about 2^-17 relative).  Errors as for dspark_draft_markov.
+ */
+dspark_status dspark_draft_rnn(
+    const float *base_logits, const void *U, const void *W, const void *R,
+    dspark_dtype uw_dtype, int V, int r, int B, int K, const int32_t *prev_token,
+    const float *h0, const float *inv_temp, const float *u_draft, int32_t *tokens,
+    float *p_tok, float *lse, float *ref_max, float *ref_sum, float *states,
+    float *draft_logits, float *draft_bias, void *workspace, size_t ws_bytes, void *stream);
+
+/* ---------------------------------------------------------------------- */
 /* 2. Confidence-scheduled prefix cut                                      */
 /* ---------------------------------------------------------------------- */
 
@@ -300,15 +339,60 @@ dspark_status dspark_verify(
     int32_t *out_tokens, int32_t *last_token, void *workspace, size_t ws_bytes,
     void *stream);
 
+/* ---------------------------------------------------------------------- */
+/* 3b. Verify with the target's LM head projected on chip                  */
+/* ---------------------------------------------------------------------- */
+
+size_t dspark_verify_lmhead_workspace_size(int V, int r, int B, int K, int dm,
+                                           int64_t n_target_rows);
+
+/*
+ * The verify of dspark_verify with the target logits formed from the target
+ * model's final hidden states instead of read from stored rows:
+ *     target logit (row, v) = hidden[row, :] . lm_head[v, :]
+ * (then scaled by inv_temp[b] like a stored row).  freeaitool.com "DeepSeek
+ * DSpark complete guide" 6.3 passes the target's last hidden state and
+ * projects it through the LM head locally, so O(vocab) rows need not move;
+ * yage.ai "DSpark speculative decoding hardware scheduling" (variable-length
+ * verify paragraph) lays the verified tokens of all requests out flat.
+ * Here the projection runs on the tensor cores and its rows are reduced on
+ * chip: no logit row of a verified position is ever written to memory.
+ * Only the one correction / bonus row of each request ([B, V] fp32) lands
+ * in the workspace, for the residual draw.
+ *
+ * Inputs
+ *   hidden [n_target_rows, dm] bf16: the flattened verified positions'
+ *       final hidden states (after the target's last normalisation);
+ *       request b uses rows row_start[b] .. row_start[b] + L_b, and these
+ *       row sets must be disjoint (a row claimed twice raises
+ *       DSPARK_FLAG_BAD_LENGTH);
+ *   lm_head [V, dm] bf16: the target's output projection (no bias);
+ *   dm: a multiple of 64, at most 16384;
+ *   everything else exactly as for dspark_verify (target_logits replaced by
+ *   hidden and lm_head).
+ * Outputs, ownership, status word: as for dspark_verify.  Rows of hidden
+ * that no request verifies are projected too (their results are dropped):
+ * pass only the verified positions' states.  The head is read once per
+ * 2048 hidden rows.
+ */
+dspark_status dspark_verify_lmhead(
+    const void *hidden, const void *lm_head, int dm, int64_t n_target_rows,
+    const int64_t *row_start, const int32_t *verify_len, const float *base_logits,
+    const void *U, const void *W, dspark_dtype uw_dtype, int V, int r, int B, int K,
+    const int32_t *prev_token, const float *inv_temp, const int32_t *tokens,
+    const float *p_tok, const float *ref_max, const float *ref_sum, const float *draft_bias,
+    const float *u_accept, const float *u_resample, int32_t *n_accepted, int32_t *out_tokens,
+    int32_t *last_token, void *workspace, size_t ws_bytes, void *stream);
+
 /*
  * dspark_verify without a workspace argument (the pages have no counterpart;
  * this is a convenience of this library).
  *
- * Who needs it: callers that cannot call cudaMalloc -- code that runs while
- * another component captures a CUDA graph in global capture mode (device
- * allocation is illegal there), plugins whose host application owns every
- * device allocation, runtimes with a fixed device-memory budget.  They still
- * own and pass all inputs and outputs; only the scratch is provided here.
+ * Who needs it: callers that cannot call cudaMalloc -- plugins whose host
+ * application owns every device allocation and hands out no scratch, and
+ * runtimes that run under a fixed device-memory budget decided before the
+ * first step.  They still own and pass all inputs and outputs; only the
+ * scratch is provided here.
  *
  * Scratch: a fixed 2 MiB array inside the library image, held by every GPU
  * that loads the library until the process exits.  Problems whose
@@ -325,8 +409,8 @@ dspark_status dspark_verify(
  * contents behind; each call clears the part that must start at zero (the
  * status word).  Calls whose kernels overlap on the GPU (different streams
  * without ordering) race on the array and give wrong results; order them.
- * Device-side data checks still clamp bad values, but their status word
- * lives in the shared array and is not reported through this entry point.
+ * Device-side data checks clamp bad values and record them in a status
+ * word inside the array: dspark_verify_noalloc_status reads it.
  *
  * Arguments and results: exactly those of dspark_verify, minus workspace and
  * ws_bytes.
@@ -339,6 +423,14 @@ dspark_status dspark_verify_noalloc(
     const float *p_tok, const float *ref_max, const float *ref_sum,
     const float *draft_bias, const float *u_accept, const float *u_resample,
     int32_t *n_accepted, int32_t *out_tokens, int32_t *last_token, void *stream);
+
+/* Status of the last dspark_verify_noalloc call on the current device:
+ * synchronises `stream` (the stream that call used) and maps the status
+ * word of the built-in scratch like dspark_get_device_status:
+ * DSPARK_OK, DSPARK_ERR_TIMEOUT (a device wait ran out) or
+ * DSPARK_ERR_DEVICE_DATA (bad token ids, lengths, rows or temperatures were
+ * clamped).  The next call on the device overwrites the word. */
+dspark_status dspark_verify_noalloc_status(void *stream);
 
 /* ---------------------------------------------------------------------- */
 /* status                                                                  */
@@ -353,6 +445,17 @@ dspark_status dspark_get_device_status(const void *workspace, void *stream);
  * CUDA error.  A workspace no call has used yet holds no status word: what
  * this returns for it is meaningless. */
 int dspark_get_device_flags(const void *workspace, void *stream);
+
+/* Test hook of the timeout path (no counterpart on the pages).  With
+ * skew != 0 the first record exchange of the persistent draft for one or
+ * two requests ("persistent-cuda-core") and the record exchange of the
+ * single-launch verify wait for records that never arrive: their bounded
+ * waits run out (after 2 s and at least 4096 polls), the call sets
+ * DSPARK_FLAG_TIMEOUT in its status word, finishes its work with
+ * meaningless outputs and leaves the device usable.  skew = 0, the default,
+ * restores normal operation.  Synchronises the current device and sets it
+ * for that device only. */
+dspark_status dspark_test_set_exchange_skew(int skew);
 
 /* Static string for a status code. */
 const char *dspark_status_string(dspark_status s);

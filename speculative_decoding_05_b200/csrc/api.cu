@@ -16,6 +16,8 @@
 #include "verify.cuh"
 #include "verify_fused.cuh"
 #include "sts.cuh"
+#include "lmhead.cuh"
+#include "rnn.cuh"
 
 using namespace dspark;
 
@@ -27,8 +29,11 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Workspace of the draft: header (status word at 0, eight grid-barrier
 // counters 128 bytes apart from byte 128), chunk partials [B][n_chunks],
-// then (persistent path) per-CTA partials [B][<=1024] and bias rows [B][V].
+// per-CTA partials [B][<=1024] (persistent paths: one per CTA; tensor-core
+// path: one per CTA of the request's block and epilogue warpgroup), then
+// (persistent paths) bias rows [B][V] and exchange records.
 constexpr size_t kCounterOff = 128;
+static_assert(kTcMaxCtasPerBlock * kS2Parts <= 1024, "per-CTA partials per request");
 struct DraftWs {
   size_t part_off, cta_off, bias_off, rec_off, total;
 };
@@ -37,7 +42,7 @@ DraftWs draft_ws(int V, int B) {
   const int Bp = B <= kPMaxB ? B : 0;  // persistent paths only
   w.part_off = kHeaderBytes;
   w.cta_off = w.part_off + align256((size_t)B * n_chunks_of(V) * sizeof(float2));
-  w.bias_off = w.cta_off + align256((size_t)Bp * 1024 * sizeof(float2));
+  w.bias_off = w.cta_off + align256((size_t)B * 1024 * sizeof(float2));
   w.rec_off = w.bias_off + align256((size_t)Bp * V * sizeof(float));
   w.total = w.rec_off + align256(Bp ? gemv_rec_bytes(Bp) : 0);
   return w;
@@ -93,12 +98,8 @@ void launch_draft_proj_simt(const float* base, const void* U, const void* W, int
                             unsigned* flags, cudaStream_t s) {
   const int nc = n_chunks_of(V);
   const size_t smem = (size_t)NB * r * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(draft_proj_simt_kernel<TW, NB>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, NB * kMaxRank * 4);
-    attr = true;
-  }
+  static DeviceOnce once;
+  set_smem_once(once, draft_proj_simt_kernel<TW, NB>, NB * kMaxRank * 4);
   dim3 grid((nc + 7) / 8, (B + NB - 1) / NB);
   draft_proj_simt_kernel<TW, NB><<<grid, 256, smem, s>>>(
       base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, B, K, k, prev, tokens, it,
@@ -111,12 +112,8 @@ void launch_res_proj_simt(const float* target, const float* base, const void* U,
                           float2* rpart, unsigned* flags, cudaStream_t s) {
   const int nc = n_chunks_of(V);
   const size_t smem = (size_t)NB * r * sizeof(float);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(residual_proj_simt_kernel<TW, NB>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize, NB * kMaxRank * 4);
-    attr = true;
-  }
+  static DeviceOnce once;
+  set_smem_once(once, residual_proj_simt_kernel<TW, NB>, NB * kMaxRank * 4);
   dim3 grid((nc + 7) / 8, (B + NB - 1) / NB);
   residual_proj_simt_kernel<TW, NB><<<grid, 256, smem, s>>>(
       target, base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, B, K, info, it,
@@ -211,20 +208,54 @@ dspark_status draft_impl(const float* base, const void* U, const void* W, dspark
     if (st != DSPARK_OK) return st;
   }
   const int nb = simt_group(B);
+  float2* cta_part = reinterpret_cast<float2*>(ws + w.cta_off);
   for (int k = 0; k < K; ++k) {
+    // The samplers are plain launches: started early behind the projection,
+    // their small CTAs would crowd onto the first SMs the projection frees.
+    // The next projection still starts early, behind the sampler.
     if (tc) {
-      tc_launch_draft(plan, k, prev, tokens, it, dl, dbias, part, flags, s);
+      tc_launch_draft(plan, k, prev, tokens, it, dl, dbias, part, cta_part, flags, s);
+      // two-level sampler over the projection's CTA partials, a warp per request
+      draft_sample2_kernel<TW><<<(B + kS2Warps - 1) / kS2Warps, kS2Warps * 32, 0, s>>>(
+          base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, B, K, k, prev,
+          tokens, it, ud, part, nc, cta_part, plan.ctas_per_bb, plan.n_tiles, dbias, p_tok, lse,
+          rmax, rsum, flags);
     } else {
       draft_proj_simt<TW>(nb, base, U, W, V, r, B, K, k, prev, tokens, it, dl, dbias, part, flags, s);
+      draft_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
+          base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, k, prev, tokens,
+          it, ud, part, nc, dbias, p_tok, lse, rmax, rsum, flags);
     }
-    // A plain launch: started early behind the projection, the sampler's
-    // small CTAs crowd onto the first SMs the projection frees (several per
-    // SM) and the position gets slower; launched after it, they spread one
-    // per SM.  The next projection still starts early, behind the sampler.
-    draft_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
-        base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, k, prev, tokens, it,
-        ud, part, nc, dbias, p_tok, lse, rmax, rsum, flags);
   }
+  return check_launch();
+}
+
+// The verify's last two stages, shared by the stored-logits and the LM-head
+// verify: residual partials of every request's correction / bonus row (from
+// the draft's bias rows, or re-projected on the tensor or CUDA cores), then
+// the draw.  `target` holds that row of request b at info[b].row.
+template <typename TW>
+dspark_status residual_tail(const float* target, long long n_rows, const float* base,
+                            const void* U, const void* W, dspark_dtype dt, int V, int r, int B,
+                            int K, const float* it, const float* ur, const ResInfo* info,
+                            float2* rpart, const float* dbias, int32_t* out, int32_t* last,
+                            unsigned* flags, cudaStream_t s) {
+  const int nc = n_chunks_of(V);
+  if (dbias != nullptr) {
+    dim3 rgrid((nc + 7) / 8, B);
+    residual_bias_kernel<<<rgrid, 256, 0, s>>>(target, base, dbias, V, K, info, it, rpart, nc,
+                                                flags);
+  } else if (use_tc(V, r, B, dt)) {
+    TcPlan plan;
+    dspark_status st = tc_plan_residual(plan, target, n_rows, base, U, W, V, r, B, K);
+    if (st != DSPARK_OK) return st;
+    tc_launch_residual(plan, info, it, rpart, flags, s);
+  } else {
+    res_proj_simt<TW>(simt_group(B), target, base, U, W, V, r, B, K, info, it, rpart, flags, s);
+  }
+  residual_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
+      target, base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, it, ur, info,
+      rpart, nc, dbias, out, last, flags);
   return check_launch();
 }
 
@@ -268,12 +299,8 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
     a.B = B;
     a.K = K;
     a.n_chunks = nc;
-    static bool fused_attr = false;
-    if (!fused_attr) {
-      cudaFuncSetAttribute(verify_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           kFBufFloats * (int)sizeof(float));
-      fused_attr = true;
-    }
+    static DeviceOnce once;
+    set_smem_once(once, verify_fused_kernel, kFBufFloats * (int)sizeof(float));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(G);
     cfg.blockDim = dim3(kFThreads);
@@ -299,22 +326,109 @@ dspark_status verify_impl(const float* target, long long n_rows, const int64_t* 
   accept_kernel<<<(B + 3) / 4, 128, 0, s>>>(target, n_rows, row_start, vlen, it, V, B, K, prev,
                                             tokens, p_tok, rmax, rsum, ua, tpart, ns, n_acc, out,
                                             info, flags);
-  if (dbias != nullptr) {
-    dim3 rgrid((nc + 7) / 8, B);
-    residual_bias_kernel<<<rgrid, 256, 0, s>>>(target, base, dbias, V, K, info, it, rpart, nc,
-                                                flags);
-  } else if (use_tc(V, r, B, dt)) {
-    TcPlan plan;
-    dspark_status st = tc_plan_residual(plan, target, n_rows, base, U, W, V, r, B, K);
-    if (st != DSPARK_OK) return st;
-    tc_launch_residual(plan, info, it, rpart, flags, s);
-  } else {
-    res_proj_simt<TW>(simt_group(B), target, base, U, W, V, r, B, K, info, it, rpart, flags, s);
+  return residual_tail<TW>(target, n_rows, base, U, W, dt, V, r, B, K, it, ur, info, rpart, dbias,
+                           out, last, flags, s);
+}
+
+// ---------------------------------------------------------------------------
+// Verify with the target logits formed from hidden states and the LM head
+// ---------------------------------------------------------------------------
+// Workspace: header, the row map (request and position of every hidden row),
+// the drafted tokens' raw logits, per-CTA partials of every verified row,
+// ResInfo, the correction rows' hidden states [B, dm] and logits [B, V], the
+// residual partials.
+constexpr int kLhMaxG = 256;
+constexpr int kLhMaxDm = 16384;
+struct LmWs {
+  size_t map_off, pos_off, tok_off, tpart_off, info_off, rows_off, logits_off, rpart_off, total;
+};
+LmWs lm_ws(int V, int B, int K, int dm, long long n_rows) {
+  LmWs w;
+  w.map_off = kHeaderBytes;
+  w.pos_off = w.map_off + align256((size_t)n_rows * 4);
+  w.tok_off = w.pos_off + align256((size_t)n_rows * 4);
+  w.tpart_off = w.tok_off + align256((size_t)n_rows * 4);
+  w.info_off = w.tpart_off + align256((size_t)B * (K + 1) * kLhMaxG * sizeof(float2));
+  w.rows_off = w.info_off + align256((size_t)B * sizeof(ResInfo));
+  w.logits_off = w.rows_off + align256((size_t)B * dm * 2);
+  w.rpart_off = w.logits_off + align256((size_t)B * V * 4);
+  w.total = w.rpart_off + align256((size_t)B * n_chunks_of(V) * sizeof(float2));
+  return w;
+}
+
+template <typename TW>
+dspark_status verify_lmhead_impl(const void* hidden, const void* head, int dm, long long n_rows,
+                                 const int64_t* row_start, const int32_t* vlen, const float* base,
+                                 const void* U, const void* W, dspark_dtype dt, int V, int r,
+                                 int B, int K, const int32_t* prev, const float* it,
+                                 const int32_t* tokens, const float* p_tok, const float* rmax,
+                                 const float* rsum, const float* dbias, const float* ua,
+                                 const float* ur, int32_t* n_acc, int32_t* out, int32_t* last,
+                                 unsigned char* ws, cudaStream_t s) {
+  const LmWs w = lm_ws(V, B, K, dm, n_rows);
+  unsigned* flags = reinterpret_cast<unsigned*>(ws);
+  int* row_req = reinterpret_cast<int*>(ws + w.map_off);
+  int* row_pos = reinterpret_cast<int*>(ws + w.pos_off);
+  float* tok_logit = reinterpret_cast<float*>(ws + w.tok_off);
+  float2* tpart = reinterpret_cast<float2*>(ws + w.tpart_off);
+  ResInfo* info = reinterpret_cast<ResInfo*>(ws + w.info_off);
+  __nv_bfloat16* rows = reinterpret_cast<__nv_bfloat16*>(ws + w.rows_off);
+  float* logits = reinterpret_cast<float*>(ws + w.logits_off);
+  float2* rpart = reinterpret_cast<float2*>(ws + w.rpart_off);
+  const int G = lh_grid(V);
+  if (G > kLhMaxG) return DSPARK_ERR_UNSUPPORTED;
+  dspark_status st = clear_status(ws, s);
+  if (st != DSPARK_OK) return st;
+  if (cudaMemsetAsync(row_req, 0xFF, (size_t)n_rows * 4, s) != cudaSuccess) return DSPARK_ERR_CUDA;
+  lm_row_map_kernel<<<(B + 3) / 4, 128, 0, s>>>(row_start, vlen, tokens, V, B, K, n_rows, row_req,
+                                                row_pos, flags);
+  CUtensorMap tm_e;
+  if (!encode_lh_map(&tm_e, head, V, dm)) return DSPARK_ERR_CUDA;
+  const __nv_bfloat16* H = static_cast<const __nv_bfloat16*>(hidden);
+  LhArgs a = {};
+  a.dm = dm;
+  a.V = V;
+  a.n_tiles = (V + kTileN - 1) / kTileN;
+  a.row_req = row_req;
+  a.row_pos = row_pos;
+  a.inv_temp = it;
+  a.tokens = tokens;
+  a.verify_len = vlen;
+  a.K = K;
+  a.tpart = tpart;
+  a.tok_logit = tok_logit;
+  a.flags = flags;
+  // 1. softmax partials of every verified row (and the drafted tokens'
+  //    logits), up to 2048 hidden rows per launch
+  constexpr long long kRowsPerLaunch = (long long)kLhMaxBlocks * 128;
+  for (long long r0 = 0; r0 < n_rows; r0 += kRowsPerLaunch) {
+    const long long nr = n_rows - r0 < kRowsPerLaunch ? n_rows - r0 : kRowsPerLaunch;
+    CUtensorMap tm_h;
+    if (!encode_lh_map(&tm_h, H + (size_t)r0 * dm, nr, dm)) return DSPARK_ERR_CUDA;
+    a.n_rows = (int)nr;
+    a.row0 = r0;
+    a.n_blocks = (int)((nr + 127) / 128);
+    if ((st = lh_launch<kLhStats>(tm_h, tm_e, a, s)) != DSPARK_OK) return st;
   }
-  residual_sample_kernel<TW><<<B, kSampleThreads, 0, s>>>(
-      target, base, static_cast<const TW*>(U), static_cast<const TW*>(W), V, r, K, it, ur, info,
-      rpart, nc, dbias, out, last, flags);
-  return check_launch();
+  // 2. accept scan on those partials
+  accept_kernel<<<(B + 3) / 4, 128, 0, s>>>(nullptr, n_rows, row_start, vlen, it, V, B, K, prev,
+                                            tokens, p_tok, rmax, rsum, ua, tpart, G, n_acc, out,
+                                            info, flags, tok_logit);
+  // 3. the logits of every request's correction / bonus row, to scratch
+  lm_gather_rows_kernel<<<B, 128, 0, s>>>(H, dm, info, rows, B);
+  for (long long r0 = 0; r0 < B; r0 += kRowsPerLaunch) {
+    const long long nr = B - r0 < kRowsPerLaunch ? B - r0 : kRowsPerLaunch;
+    CUtensorMap tm_h;
+    if (!encode_lh_map(&tm_h, rows + (size_t)r0 * dm, nr, dm)) return DSPARK_ERR_CUDA;
+    a.n_rows = (int)nr;
+    a.row0 = 0;
+    a.n_blocks = (int)((nr + 127) / 128);
+    a.logits = logits + (size_t)r0 * V;
+    if ((st = lh_launch<kLhLogits>(tm_h, tm_e, a, s)) != DSPARK_OK) return st;
+  }
+  // 4. residual and draw, as in the stored-logits verify
+  return residual_tail<TW>(logits, B, base, U, W, dt, V, r, B, K, it, ur, info, rpart, dbias, out,
+                           last, flags, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -485,18 +599,15 @@ dspark_status dspark_confidence_prefix_async(const float* z, const float* temps,
   if (!cost_tokens || !cost_ms || !verify_len || !objective) return DSPARK_ERR_INVALID_ARG;
   if (B * K > 0 && (!z || !temps || !c || !survival)) return DSPARK_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int npad = 1;
-  while (npad < B * K) npad <<= 1;
-  const size_t smem = (size_t)npad * (sizeof(double) + sizeof(int)) + (size_t)B * sizeof(int);
-  static bool attr = false;
-  if (!attr) {
-    cudaFuncSetAttribute(prefix_kernel<kPrefixThreads>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kMaxCand * 12 + 8192 * 4);
-    attr = true;
-  }
-  if (smem > (size_t)kMaxCand * 12 + 8192 * 4) return DSPARK_ERR_UNSUPPORTED;
+  // survivals (fp64), two order buffers of the merge and the per-request counts
+  const int n = B * K;
+  const size_t smem = (size_t)n * (sizeof(double) + 2 * sizeof(int)) + (size_t)B * sizeof(int);
+  constexpr int kPrefixSmemMax = kMaxCand * 16 + kMaxCand * 4;
+  static DeviceOnce once;
+  set_smem_once(once, prefix_kernel<kPrefixThreads>, kPrefixSmemMax);
+  if (smem > (size_t)kPrefixSmemMax) return DSPARK_ERR_UNSUPPORTED;
   // the kernel clears the status word itself (one CTA: before any flag is raised)
-  if (npad <= kPrefixSmallCand)
+  if (n <= kPrefixSmallCand)
     prefix_kernel<kPrefixThreadsSmall><<<1, kPrefixThreadsSmall, smem, s>>>(
         z, temps, cost_tokens, cost_ms, n_pts, staircase, B, K, enable, budget_in, c, survival,
         verify_len, objective, budget_out, static_cast<unsigned*>(workspace));
@@ -615,6 +726,130 @@ dspark_status dspark_verify_noalloc(const float* target_logits, int64_t n_target
                        uw_dtype, V, r, B, K, prev_token, inv_temp, tokens, p_tok, ref_max, ref_sum,
                        draft_bias, u_accept, u_resample, n_accepted, out_tokens, last_token, scratch,
                        kNoAllocScratchBytes, stream);
+}
+
+size_t dspark_draft_rnn_workspace_size(int V, int r, int B, int K) {
+  (void)K;
+  if (V <= 0 || r <= 0 || B < 0) return 0;
+  return draft_ws(V, B).total + align256((size_t)B * r * 4) + align256((size_t)B * 2 * r * 2);
+}
+
+dspark_status dspark_draft_rnn(const float* base_logits, const void* U, const void* W,
+                               const void* R, dspark_dtype uw_dtype, int V, int r, int B, int K,
+                               const int32_t* prev_token, const float* h0, const float* inv_temp,
+                               const float* u_draft, int32_t* tokens, float* p_tok, float* lse,
+                               float* ref_max, float* ref_sum, float* states,
+                               float* draft_logits, float* draft_bias, void* workspace,
+                               size_t ws_bytes, void* stream) {
+  dspark_status st = check_shapes(V, r, B, K, uw_dtype);
+  if (st != DSPARK_OK) return st;
+  // the state's projection runs on the tensor cores: bf16 factors, r a
+  // multiple of 64 up to 256, one full vocabulary tile at least
+  if (uw_dtype != DSPARK_BF16 || r % 64 != 0 || r > 256 || V < kTileN)
+    return DSPARK_ERR_UNSUPPORTED;
+  if (!workspace || !aligned(workspace, 256) ||
+      ws_bytes < dspark_draft_rnn_workspace_size(V, r, B, K))
+    return DSPARK_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 0 || K == 0) return clear_status(workspace, s);
+  if (!base_logits || !U || !W || !R || !prev_token || !u_draft || !tokens || !p_tok || !lse ||
+      !ref_max || !ref_sum)
+    return DSPARK_ERR_INVALID_ARG;
+  if (!aligned(base_logits, 16) || !aligned(U, 16) || !aligned(W, 16) || !aligned(R, 16) ||
+      (draft_logits && !aligned(draft_logits, 16)) || (draft_bias && !aligned(draft_bias, 16)))
+    return DSPARK_ERR_INVALID_ARG;
+  if ((st = clear_status(workspace, s)) != DSPARK_OK) return st;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  const DraftWs w = draft_ws(V, B);
+  unsigned* flags = reinterpret_cast<unsigned*>(ws);
+  float2* part = reinterpret_cast<float2*>(ws + w.part_off);
+  float2* cta_part = reinterpret_cast<float2*>(ws + w.cta_off);
+  float* state = reinterpret_cast<float*>(ws + w.total);
+  __nv_bfloat16* a_rows =
+      reinterpret_cast<__nv_bfloat16*>(ws + w.total + align256((size_t)B * r * 4));
+  TcPlan plan;
+  if ((st = tc_plan_draft(plan, base_logits, U, W, V, r, B, K, a_rows)) != DSPARK_OK) return st;
+  const __nv_bfloat16* Ub = static_cast<const __nv_bfloat16*>(U);
+  const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
+  const __nv_bfloat16* Rb = static_cast<const __nv_bfloat16*>(R);
+  const int nc = n_chunks_of(V);
+  for (int k = 0; k < K; ++k) {
+    // state, then the projection of the state (launched early behind it:
+    // its W and base producers do not depend on the state), then the draw
+    rnn_state_kernel<__nv_bfloat16><<<B, kRnnThreads, (size_t)r * sizeof(float), s>>>(
+        Ub, Rb, V, r, K, k, prev_token, tokens, h0, state, a_rows, states, flags);
+    tc_launch_draft(plan, k, prev_token, tokens, inv_temp, draft_logits, draft_bias, part,
+                    cta_part, flags, s);
+    draft_sample2_kernel<__nv_bfloat16><<<(B + kS2Warps - 1) / kS2Warps, kS2Warps * 32, 0, s>>>(
+        base_logits, Ub, Wb, V, r, B, K, k, prev_token, tokens, inv_temp, u_draft, part, nc,
+        cta_part, plan.ctas_per_bb, plan.n_tiles, draft_bias, p_tok, lse, ref_max, ref_sum, flags,
+        state);
+  }
+  return check_launch();
+}
+
+size_t dspark_verify_lmhead_workspace_size(int V, int r, int B, int K, int dm,
+                                           int64_t n_target_rows) {
+  (void)r;
+  if (V <= 0 || B < 0 || K < 0 || dm <= 0 || n_target_rows < 0) return 0;
+  return lm_ws(V, B, K, dm, n_target_rows).total;
+}
+
+dspark_status dspark_verify_lmhead(const void* hidden, const void* lm_head, int dm,
+                                   int64_t n_target_rows, const int64_t* row_start,
+                                   const int32_t* verify_len, const float* base_logits,
+                                   const void* U, const void* W, dspark_dtype uw_dtype, int V,
+                                   int r, int B, int K, const int32_t* prev_token,
+                                   const float* inv_temp, const int32_t* tokens,
+                                   const float* p_tok, const float* ref_max, const float* ref_sum,
+                                   const float* draft_bias, const float* u_accept,
+                                   const float* u_resample, int32_t* n_accepted,
+                                   int32_t* out_tokens, int32_t* last_token, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  dspark_status st = check_shapes(V, r, B, K, uw_dtype);
+  if (st != DSPARK_OK) return st;
+  if (dm <= 0 || n_target_rows < 0) return DSPARK_ERR_INVALID_ARG;
+  if (dm % 64 != 0 || dm > kLhMaxDm) return DSPARK_ERR_UNSUPPORTED;
+  if (!workspace || !aligned(workspace, 256) ||
+      ws_bytes < dspark_verify_lmhead_workspace_size(V, r, B, K, dm, n_target_rows))
+    return DSPARK_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (B == 0) return clear_status(workspace, s);
+  if (!hidden || !lm_head || n_target_rows <= 0 || !row_start || !verify_len || !base_logits ||
+      !U || !W || !prev_token || !u_resample || !n_accepted || !out_tokens)
+    return DSPARK_ERR_INVALID_ARG;
+  if (K > 0 && (!tokens || !p_tok || !ref_max || !ref_sum || !u_accept))
+    return DSPARK_ERR_INVALID_ARG;
+  if (!aligned(hidden, 16) || !aligned(lm_head, 16) || !aligned(base_logits, 16) ||
+      !aligned(U, 16) || !aligned(W, 16) || (draft_bias && !aligned(draft_bias, 16)))
+    return DSPARK_ERR_INVALID_ARG;
+  if ((long long)B * (K + 1) > (1ll << 31) - 1 || n_target_rows > (1ll << 31) - 1)
+    return DSPARK_ERR_UNSUPPORTED;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  if (uw_dtype == DSPARK_BF16)
+    return verify_lmhead_impl<__nv_bfloat16>(hidden, lm_head, dm, n_target_rows, row_start,
+                                             verify_len, base_logits, U, W, uw_dtype, V, r, B, K,
+                                             prev_token, inv_temp, tokens, p_tok, ref_max, ref_sum,
+                                             draft_bias, u_accept, u_resample, n_accepted,
+                                             out_tokens, last_token, ws, s);
+  return verify_lmhead_impl<float>(hidden, lm_head, dm, n_target_rows, row_start, verify_len,
+                                   base_logits, U, W, uw_dtype, V, r, B, K, prev_token, inv_temp,
+                                   tokens, p_tok, ref_max, ref_sum, draft_bias, u_accept,
+                                   u_resample, n_accepted, out_tokens, last_token, ws, s);
+}
+
+dspark_status dspark_test_set_exchange_skew(int skew) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return DSPARK_ERR_CUDA;
+  return cudaMemcpyToSymbol(g_test_exchange_skew, &skew, sizeof(int)) == cudaSuccess
+             ? DSPARK_OK
+             : DSPARK_ERR_CUDA;
+}
+
+dspark_status dspark_verify_noalloc_status(void* stream) {
+  void* scratch = nullptr;
+  const dspark_status st = noalloc_scratch(&scratch);
+  if (st != DSPARK_OK) return st;
+  return dspark_get_device_status(scratch, stream);
 }
 
 }  // extern "C"

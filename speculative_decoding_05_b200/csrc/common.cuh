@@ -6,9 +6,46 @@
 #include <math_constants.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/dspark.h"
 
 namespace dspark {
+
+// ---------------------------------------------------------------------------
+// host: per-device set-up
+// ---------------------------------------------------------------------------
+
+// Kernel attributes (the dynamic shared-memory limit) and device properties
+// belong to one device: a process that drives several GPUs, or several host
+// threads, must set them for every device it launches on, once.
+constexpr int kMaxDevices = 64;
+using DeviceOnce = std::once_flag[kMaxDevices];
+
+inline int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) d = 0;
+  return d;
+}
+
+// Runs f() once per device (the current one), thread-safe.
+template <typename F>
+inline void once_per_device(DeviceOnce& once, F&& f) {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) {
+    f();
+    return;
+  }
+  std::call_once(once[d], f);
+}
+
+// Maximum dynamic shared memory of a kernel, set once per device.
+template <typename Kern>
+inline void set_smem_once(DeviceOnce& once, Kern* kern, int bytes) {
+  once_per_device(once, [&] {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  });
+}
 
 // Programmatic dependent launch.  wait: block until the kernel this one was
 // launched behind has finished and its writes are visible (returns at once
@@ -36,6 +73,13 @@ constexpr float kLog2e = 1.4426950408889634f;
 __host__ __device__ inline int n_chunks_of(int V) { return (V + kChunk - 1) / kChunk; }
 __host__ __device__ inline int n_segs_of(int V) { return (V + kSeg - 1) / kSeg; }
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Test hook of the timeout path (set by dspark_test_set_exchange_skew, 0
+// in normal operation): when non-zero, the first record exchange of the
+// persistent draft for one or two requests, and the partial-record exchange
+// of the single-launch verify, wait for records that never arrive, so their
+// bounded waits run out.  Read once per CTA.
+static __device__ int g_test_exchange_skew;
 
 // ---------------------------------------------------------------------------
 // status word
@@ -80,6 +124,23 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Softmax partial of a 32-row chunk of one request: A = max_j (bv_j + d_j),
+// s = sum_j 2^(((bv_j - A) + d_j) * it2) (0 when every row is -inf), in four
+// interleaved chains (row j in chain j % 4), combined as (c0 + c1) + (c2 + c3).
+// bv - A is exact for the rows that carry the mass (Sterbenz).
+__device__ __forceinline__ float2 chunk_partial32(const float (&bv)[32], const float (&d)[32],
+                                                  float it2) {
+  float A4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+  for (int j = 0; j < 32; ++j) A4[j & 3] = fmaxf(A4[j & 3], bv[j] + d[j]);
+  const float A = fmaxf(fmaxf(A4[0], A4[1]), fmaxf(A4[2], A4[3]));
+  float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int j = 0; j < 32; ++j) s4[j & 3] += ex2(((bv[j] - A) + d[j]) * it2);
+  const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+  return make_float2(A, A == -CUDART_INF_F ? 0.0f : sum);
 }
 
 // Merge softmax partial (A, s) into (M, S) (both relative to their own max).

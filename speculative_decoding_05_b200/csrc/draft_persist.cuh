@@ -168,9 +168,6 @@ __device__ __forceinline__ void epi_sync() {
   asm volatile("bar.sync 1, %0;" ::"r"(kPEpiThreads) : "memory");
 }
 
-__device__ __forceinline__ double partial_weight(float2 q, float M, float it2) {
-  return (q.x == -CUDART_INF_F) ? 0.0 : (double)(q.y * ex2((q.x - M) * it2));
-}
 
 // Write U[x] (or zeros) into row n of the 128-byte swizzled K-major B
 // operand, one 16-byte chunk per lane step.
@@ -365,7 +362,8 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
   uint64_t* uReady = dEmpty + kPDSlots;
   uint64_t* baseFull = uReady + 1;
   uint64_t* baseEmpty = baseFull + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(baseEmpty + 1);
+  uint64_t* mmaDrain = baseEmpty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mmaDrain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_wm = reinterpret_cast<float*>(tmem_slot + 2);  // [4][kPMaxB]
   float* s_ws = s_wm + 4 * kPMaxB;                        // [4][kPMaxB]
@@ -384,6 +382,7 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
     mbar_init(uReady, 1);
     mbar_init(baseFull, 1);
     mbar_init(baseEmpty, 1);
+    mbar_init(mmaDrain, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -457,6 +456,11 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
           }
         }
       }
+      // tail: the MMAs' release of the last stages is an asynchronous arrive
+      // on this CTA's barriers; wait for it before the CTA may exit (after
+      // an abort: for the copies still in flight)
+      if (!*s_abort) wait_ring_released(ringEmpty, S, it, p.flags);
+      else drain_ring_loads(ringFull, S, it);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer
@@ -526,6 +530,7 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
         *s_abort = 1;
         raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
       }
+      drain_mma(mmaDrain);
     }
   } else if (warp == 2) {
     // ------------------------------------------------ base producer
@@ -534,6 +539,7 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
       const int v0 = t0 * kTileN;
       const int nval = min(nt * kTileN, V - v0);
       const uint32_t bytes = (uint32_t)nval * 4u;
+      int last = -1;  // last position whose rows were requested
       for (int k = 0; k < K && !*s_abort; ++k) {
         if (!mbar_wait(baseEmpty, ((uint32_t)k & 1u) ^ 1u)) {
           *s_abort = 1;
@@ -544,7 +550,10 @@ draft_persist_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs
         for (int b = 0; b < B; ++b)
           bulk_load(sBase + (size_t)b * base_stride, p.base + ((size_t)b * K + k) * (size_t)V + v0,
                     bytes, baseFull, pol);
+        last = k;
       }
+      // after an abort the last rows may still be landing
+      if (*s_abort && last >= 0) mbar_wait(baseFull, (uint32_t)last & 1u);
     }
   } else if (warp >= kPEpiWarp0) {
     // ------------------------------------------------ epilogue + sampler
@@ -823,17 +832,12 @@ __device__ __forceinline__ void backoff_spin_u64(const unsigned long long* p, ui
   }
 }
 
-// Bounded wait, at the end of the call, for the copies a producer issued:
-// the last issue into each of the n_slots slots of a ring of `issued` issues.
-__device__ __forceinline__ void drain_ring(uint64_t* full, int n_slots, int issued) {
-  for (int j = max(0, issued - n_slots); j < issued; ++j)
-    (void)mbar_wait(&full[j % n_slots], (uint32_t)(j / n_slots) & 1u);
-}
 
 template <int NB>
 __global__ void __launch_bounds__(kGThreads, 1)
 draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p, const GemvRecs rec) {
   extern __shared__ uint8_t smem_raw[];
+  const uint32_t test_skew = (uint32_t)g_test_exchange_skew;
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int G = gridDim.x, cta = blockIdx.x;
   constexpr int B = NB;  // launched with exactly NB requests
@@ -929,7 +933,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           }
         }
       }
-      drain_ring(ringFull, S, it);
+      drain_ring_loads(ringFull, S, it);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ base producer (double-buffered)
@@ -950,7 +954,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
                     p.base + ((size_t)b * K + k) * (size_t)V + v0, bytes, &baseFull[buf], pol);
         ++issued;
       }
-      drain_ring(baseFull, 2, issued);
+      drain_ring_loads(baseFull, 2, issued);
     }
   } else if (warp >= kGTailWarp) {
     // ------------------------------------------------ GEMV, epilogue, sampling
@@ -1243,7 +1247,9 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             if (pend & (1u << i)) m[i] = ld_rec2(cr + (size_t)kGRecWords * (c0 + i));
 #pragma unroll
           for (int i = 0; i < kGPerLane; ++i) {
-            if ((pend & (1u << i)) && (uint32_t)(m[i].x >> 32) == seq && (uint32_t)(m[i].y >> 32) == seq) {
+            // (a test skew makes the first position wait for a later one)
+            const uint32_t want = seq + (k == 0 ? test_skew : 0u);
+            if ((pend & (1u << i)) && (uint32_t)(m[i].x >> 32) == want && (uint32_t)(m[i].y >> 32) == want) {
               q[i] = make_float2(__uint_as_float((uint32_t)m[i].x), __uint_as_float((uint32_t)m[i].y));
               pend &= ~(1u << i);
             }
@@ -1433,16 +1439,15 @@ inline dspark_status persist_launch_kernel(Kern kern, int threads, const CUtenso
 
 inline dspark_status persist_launch(const CUtensorMap& tm_w, PersistArgs a, GemvRecs recs,
                                     cudaStream_t s) {
-  static bool attr = false;
-  if (!attr) {
+  static DeviceOnce once;
+  once_per_device(once, [] {
     cudaFuncSetAttribute(draft_persist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kPSmemLimit);
     cudaFuncSetAttribute(draft_gemv_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kPSmemLimit);
     cudaFuncSetAttribute(draft_gemv_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          kPSmemLimit);
-    attr = true;
-  }
+  });
   const PersistLayout L = persist_layout(a.V, a.r, a.B);
   a.max_nt = L.max_nt;
   a.n_stages = L.n_stages;

@@ -1,11 +1,15 @@
 // prefix.cuh -- sequential temperature scaling, survival and the greedy
 // hardware-aware prefix cut, in one CTA.
 //
-// The whole batch has at most kMaxCand = 8192 candidates (B*K); they are
-// sorted in shared memory (bitonic, key = survival descending, ties by
-// candidate index k*B + b ascending, i.e. position then request), the
-// expected-emitted-token prefix sums are a block scan in fp64, and the
-// early stop is the first index where E/t(N) does not increase.
+// The whole batch has at most kMaxCand = 8192 candidates (B*K), ordered by
+// survival descending, ties by candidate index k*B + b ascending (position
+// then request).  Survival never rises along a request's positions (each
+// step multiplies by c in (0, 1]), so each request's K candidates are
+// already a sorted run: the order is a merge of B runs, done as a merge tree
+// in shared memory (log2 B levels; each thread finds its output chunk's
+// split by a merge-path binary search, then merges it sequentially).  The
+// expected-emitted-token prefix sums are a block scan in fp64, and the early
+// stop is the first index where E/t(N) does not increase.
 //
 // Asynchronous budget (yage.ai, engineering paragraph: how many tokens a
 // step verifies is decided from the confidences of two steps back, which
@@ -71,11 +75,10 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
               int32_t* budget_out, unsigned* flags) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int n = B * K;
-  int npad = 1;
-  while (npad < n) npad <<= 1;
-  double* key = reinterpret_cast<double*>(smem_raw);           // [npad]
-  int* idx = reinterpret_cast<int*>(key + npad);               // [npad]
-  int* lcount = idx + npad;                                     // [B]
+  double* surv = reinterpret_cast<double*>(smem_raw);          // [n], candidate k*B + b
+  int* ordA = reinterpret_cast<int*>(surv + n);                 // [n] candidate order
+  int* ordB = ordA + n;                                         // [n] merge buffer
+  int* lcount = ordB + n;                                       // [B]
   __shared__ float s_xs[64], s_ys[64];
   __shared__ double shd[32];
   __shared__ int s_stop, s_budget;
@@ -103,29 +106,26 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     const int b = o / K, k = o - b * K;
     const double ck = 1.0 / (1.0 + exp(-(double)z[o] / (double)temps[k]));
     c_out[o] = (float)ck;
-    key[k * B + b] = ck;
+    surv[k * B + b] = ck;
   }
   __syncthreads();
-  // survival = running product over k (one thread per request)
+  // survival = running product over k (one thread per request); request b's
+  // run of the merge starts at b * K
   for (int b = tid; b < B; b += kT) {
     double run = 1.0;
     for (int k = 0; k < K; ++k) {
-      run *= key[k * B + b];
+      run *= surv[k * B + b];
       s_out[(size_t)b * K + k] = (float)run;
-      key[k * B + b] = run;
-      idx[k * B + b] = k * B + b;
+      surv[k * B + b] = run;
+      ordA[b * K + k] = k * B + b;
     }
     lcount[b] = 0;
-  }
-  for (int i = n + tid; i < npad; i += kT) {
-    key[i] = -1.0;  // padding sorts last
-    idx[i] = 0x7fffffff;
   }
   __syncthreads();
 
   if (!enable) {
     double e = 0.0;
-    for (int i = tid; i < n; i += kT) e += key[i];
+    for (int i = tid; i < n; i += kT) e += surv[i];
     const double E = (double)B + block_sum_d<kT>(e, shd);
     for (int b = tid; b < B; b += kT) verify_len[b] = K;
     if (tid == 0) {
@@ -137,32 +137,52 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     return;
   }
 
-  // bitonic sort of (key, idx) in the order of cand_before; each stage walks
-  // the npad / 2 compare-exchange pairs (i, i + stride), i with bit `stride`
-  // clear: pair p puts a zero bit into p at that position
-  for (int size = 2; size <= npad; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int p = tid; p < (npad >> 1); p += kT) {
-        const int i = (p & (stride - 1)) | ((p & ~(stride - 1)) << 1);
-        const int j = i + stride;
-        const bool up = (i & size) == 0;  // this half sorts in cand_before order
-        const double ki = key[i], kj = key[j];
-        const int ii = idx[i], ij = idx[j];
-        const bool jfirst = cand_before(kj, ij, ki, ii);
-        if (jfirst == up) {
-          key[i] = kj; key[j] = ki;
-          idx[i] = ij; idx[j] = ii;
+  // merge tree: runs of width w = K, 2K, 4K, ...; each level merges pairs
+  // of neighbouring runs from src into dst (an unpaired last run is copied)
+  auto before = [&](int ia, int ib) { return cand_before(surv[ia], ia, surv[ib], ib); };
+  int* src = ordA;
+  int* dst = ordB;
+  const int chunk = (n + kT - 1) / kT;  // outputs per thread and level
+  for (long long w = K; w < n; w <<= 1) {
+    const int o0 = min(tid * chunk, n), o1 = min(o0 + chunk, n);
+    int i = 0, j = 0, a1 = 0, b1 = 0;  // cursors into the current pair's two runs
+    int pair_end = -1;
+    for (int o = o0; o < o1; ++o) {
+      if (o >= pair_end) {
+        // first output of this thread in a pair: merge-path split
+        const long long p0 = (o / (2 * w)) * (2 * w);
+        const int a0 = (int)p0;
+        a1 = (int)min(p0 + w, (long long)n);
+        const int b0 = a1;
+        b1 = (int)min(p0 + 2 * w, (long long)n);
+        pair_end = b1;
+        const int q = o - a0;
+        int lo = max(0, q - (b1 - b0)), hi = min(q, a1 - a0);
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          // does A[mid] come before B[q - mid - 1]?  then more of A is in
+          if (before(src[a0 + mid], src[b0 + q - mid - 1])) lo = mid + 1;
+          else hi = mid;
         }
+        i = a0 + lo;
+        j = b0 + (q - lo);
       }
-      __syncthreads();
+      if (j >= b1 || (i < a1 && before(src[i], src[j]))) dst[o] = src[i++];
+      else dst[o] = src[j++];
     }
+    __syncthreads();
+    int* t = src;
+    src = dst;
+    dst = t;
   }
+  const int* idx = src;  // candidates in order
+  auto key = [&](int i) { return surv[idx[i]]; };
 
   // E_i = B + sum of the first i survivals; each thread owns a contiguous run
-  const int per = npad / kT > 0 ? npad / kT : 1;
+  const int per = chunk;
   const int i0 = tid * per;
   double run = 0.0;
-  for (int i = i0; i < i0 + per && i < n; ++i) run += key[i];
+  for (int i = i0; i < i0 + per && i < n; ++i) run += key(i);
   double total;
   const double excl = block_excl_scan_d<kT>(run, shd, &total);
   // candidate i (0-based) raises the objective iff E_{i+1}/t(B+i+1) > E_i/t(B+i)
@@ -170,7 +190,7 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   for (int i = i0; i < i0 + per && i < n; ++i) {
     const double t0 = cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)i);
     const double t1 = cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)i + 1.0);
-    const double E1 = E + key[i];
+    const double E1 = E + key(i);
     if (!(t0 > 0.0) || !(t1 > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
     if (!(E1 / t1 > E / t0)) {
       atomicMin(&s_stop, i);
@@ -195,7 +215,7 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     double Ec = (double)B + total;
     if (n_commit < n) {
       Ec = (double)B + excl;
-      for (int i = i0; i < n_commit; ++i) Ec += key[i];
+      for (int i = i0; i < n_commit; ++i) Ec += key(i);
     }
     objective[0] = (float)(Ec / cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)n_commit));
   }

@@ -52,8 +52,15 @@
 
 namespace dspark {
 
-constexpr int kTcThreads = 352;
 constexpr int kBlockM = 128;
+// Epilogue warpgroups (128 threads = 128 requests each), two chunks of every
+// tile each.  Four warpgroups of one chunk each (608 threads) measured
+// slower at B = 512 (0.127 against 0.102 ms per position): the register cap
+// of the larger block spilled the 64 accumulator and base values.
+template <bool kRes>
+__host__ __device__ constexpr int tc_epi_groups() { return 2; }
+template <bool kRes>
+__host__ __device__ constexpr int tc_threads() { return 96 + 128 * tc_epi_groups<kRes>(); }
 constexpr int kTileN = 128;
 constexpr int kWStagesMax = 12;     // W ring depth: as deep as shared memory allows
 constexpr int kBStagesMax = 16;     // base ring depth (draft): likewise
@@ -71,6 +78,8 @@ struct TcPlan {
   int V, r, B, K;
   int n_tiles, n_bb, ctas_per_bb;
   int w_stages, b_stages, base_rows;  // ring depths, request rows per base box
+  const __nv_bfloat16* a_rows;        // draft: per-request A rows (split state) or NULL
+  int a_split;                         // 1: a_rows hold 2r columns (high, low halves)
 };
 
 // Request rows of a base-logit box: the batch rounded up to 8 (the 128-byte
@@ -85,18 +94,19 @@ inline size_t tc_a_stage_bytes(int B) { return (size_t)tc_base_rows(B) * 128; }
 inline size_t tc_r_stage_bytes(int B, bool residual) {
   return (residual ? 2 : 1) * tc_a_stage_bytes(B);
 }
-// Alignment slack, operand A (r / 64 k-blocks) and the barriers.
-inline size_t tc_fixed_bytes(int r, int B, bool residual) {
+// Alignment slack, operand A (ra / 64 k-blocks, ra = r or a split state's
+// 2r columns) and the barriers.
+inline size_t tc_fixed_bytes(int ra, int B, bool residual) {
   (void)residual;
-  return 1024 + (size_t)(r / 64) * tc_a_stage_bytes(B) + 512;
+  return 1024 + (size_t)(ra / 64) * tc_a_stage_bytes(B) + 512;
 }
 // Ring depths.  Each copy in flight waits about the same time for its
 // bytes, so the two rings share what is left in proportion to what they
 // move per tile: W r / 64 stages of 16 KB, the second ring kTileN / 32
 // stages.  W keeps at least two stages (a ring shorter than a tile still
 // flows: the MMAs free its stages in order).
-inline int tc_w_stages(int r, int B, bool residual) {
-  const size_t ring = kTcSmemLimit - tc_fixed_bytes(r, B, residual);
+inline int tc_w_stages(int r, int B, bool residual, int a_split = 0) {
+  const size_t ring = kTcSmemLimit - tc_fixed_bytes(r << a_split, B, residual);
   const int nkb = r / 64;
   const size_t w_tile = (size_t)nkb * kStageBytes;
   const size_t b_tile = (size_t)(kTileN / 32) * tc_r_stage_bytes(B, residual);
@@ -105,16 +115,17 @@ inline int tc_w_stages(int r, int B, bool residual) {
   if (s > kWStagesMax) s = kWStagesMax;
   return s;
 }
-inline int tc_b_stages(int r, int B, bool residual) {
-  const size_t left = kTcSmemLimit - tc_fixed_bytes(r, B, residual) -
-                      (size_t)tc_w_stages(r, B, residual) * kStageBytes;
+inline int tc_b_stages(int r, int B, bool residual, int a_split = 0) {
+  const size_t left = kTcSmemLimit - tc_fixed_bytes(r << a_split, B, residual) -
+                      (size_t)tc_w_stages(r, B, residual, a_split) * kStageBytes;
   int s = (int)(left / tc_r_stage_bytes(B, residual));
   if (s > kBStagesMax) s = kBStagesMax;
   return s;
 }
-inline size_t tc_smem_bytes(int r, int B, bool residual) {
-  return tc_fixed_bytes(r, B, residual) + (size_t)tc_w_stages(r, B, residual) * kStageBytes +
-         (size_t)tc_b_stages(r, B, residual) * tc_r_stage_bytes(B, residual);
+inline size_t tc_smem_bytes(int r, int B, bool residual, int a_split = 0) {
+  return tc_fixed_bytes(r << a_split, B, residual) +
+         (size_t)tc_w_stages(r, B, residual, a_split) * kStageBytes +
+         (size_t)tc_b_stages(r, B, residual, a_split) * tc_r_stage_bytes(B, residual);
 }
 
 inline bool tc_supported(int V, int r, int B) {
@@ -122,21 +133,28 @@ inline bool tc_supported(int V, int r, int B) {
 }
 
 template <bool kRes>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(tc_threads<kRes>(), 1)
 proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_base,
                const __grid_constant__ CUtensorMap tm_tgt, const __nv_bfloat16* __restrict__ U, int V, int r, int B, int K, int k,
                const int32_t* __restrict__ prev_token, const int32_t* __restrict__ tokens,
                const float* __restrict__ inv_temp, const float* __restrict__ target,
                const float* __restrict__ base, const ResInfo* __restrict__ info,
                float* __restrict__ draft_logits, float* __restrict__ draft_bias,
-               float2* __restrict__ part, int n_chunks, int n_tiles, int ctas_per_bb,
-               int n_ws, int n_bs, int base_rows, unsigned* flags) {
+               float2* __restrict__ part, float2* __restrict__ cta_part, int n_chunks,
+               int n_tiles, int ctas_per_bb, int n_ws, int n_bs, int base_rows,
+               const __nv_bfloat16* __restrict__ a_rows, int a_split, unsigned* flags) {
+  constexpr int kEpi = tc_epi_groups<kRes>();
+  constexpr int kCpg = (kTileN / 32) / kEpi;  // chunks of a tile per epilogue warpgroup
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int nkb = r >> 6;
+  // operand A: U[x] (r columns), or with a_rows (draft only) the request's
+  // row of a_rows, r << a_split columns: a state split into bf16 high and
+  // low parts, both multiplied by the same W block and accumulated
+  const int ra = r << a_split;
   uint8_t* sA = sm;
   const int bstage = base_rows * 128;  // bytes of one base box and of one k-block of A
-  uint8_t* sW = sA + nkb * bstage;
+  uint8_t* sW = sA + (ra >> 6) * bstage;
   uint8_t* sBase = sW + n_ws * kStageBytes;
   const int rstage = (kRes ? 2 : 1) * bstage;  // one stage of the second ring
   uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + n_bs * rstage);
@@ -146,13 +164,19 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   uint64_t* emptyB = fullB + kBStagesMax;
   uint64_t* accFull = emptyB + kBStagesMax;
   uint64_t* accEmpty = accFull + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accEmpty + 2);
+  uint64_t* mmaDrain = accEmpty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mmaDrain + 1);
   volatile int* s_abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bb = blockIdx.x / ctas_per_bb, pi = blockIdx.x % ctas_per_bb;
   const int t0 = (int)((long long)pi * n_tiles / ctas_per_bb);
   const int t1 = (int)((long long)(pi + 1) * n_tiles / ctas_per_bb);
+  const int nt = t1 - t0;
+  // Odd draft positions walk the range backwards, so a position starts on
+  // the W tiles the one before it read last (the likeliest still in L2).
+  const bool rev = !kRes && (k & 1);
+  auto tile_at = [&](int i) { return rev ? t1 - 1 - i : t0 + i; };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < n_ws; ++i) {
@@ -165,8 +189,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accFull[i], 1);
-      mbar_init(&accEmpty[i], 8);
+      mbar_init(&accEmpty[i], 4 * kEpi);
     }
+    mbar_init(mmaDrain, 1);
     *s_abort = 0;
     fence_barrier_init();
   }
@@ -182,11 +207,11 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   if (!producer || k == 0) grid_dep_wait();
 
   // operand A: the previous-token rows of U for this block of requests,
-  // gathered by the nine non-producer warps.  The 128 token ids go to shared
+  // gathered by the non-producer warps.  The 128 token ids go to shared
   // memory first (one round of loads), then every thread issues all of its U
   // loads before storing any, so the gather costs two memory round trips
   // rather than one per loop iteration.
-  constexpr int kGather = kTcThreads - 64;
+  constexpr int kGather = tc_threads<kRes>() - 64;
   const int gtid = warp == 1 ? lane : threadIdx.x - 64;  // 0..kGather-1 off the producers
   __shared__ int s_x[kBlockM];
   if (!producer && gtid < kBlockM) {
@@ -197,6 +222,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       if (kRes) {
         const ResInfo& ri = info[b];
         x = ri.bonus ? -1 : ri.x_prev;
+      } else if (a_rows != nullptr) {
+        x = b;
       } else {
         x = (k == 0) ? prev_token[b] : tokens[(size_t)b * K + (k - 1)];
         if (x >= V || (k > 0 && x < 0)) {
@@ -209,25 +236,28 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   }
   if (!producer) {
     named_sync(1, kGather);
-    const int cpr = r >> 3;  // 16-byte chunks per row
-    constexpr int kPer = (kBlockM * 32 + kGather - 1) / kGather;  // r <= 256: 32 chunks per row
-    uint4 val[kPer];
+    const int cpr = ra >> 3;  // 16-byte chunks per row
+    const __nv_bfloat16* src = a_rows != nullptr ? a_rows : U;
+    constexpr int kPer = (kBlockM * 32 + kGather - 1) / kGather;  // 256 columns per pass
+    for (int q0 = 0; q0 < base_rows * cpr; q0 += kPer * kGather) {
+      uint4 val[kPer];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int q = gtid + i * kGather;
-      val[i] = make_uint4(0, 0, 0, 0);
-      if (q < base_rows * cpr) {
-        const int x = s_x[q / cpr];
-        if (x >= 0) val[i] = __ldg(reinterpret_cast<const uint4*>(U + (size_t)x * r) + (q % cpr));
+      for (int i = 0; i < kPer; ++i) {
+        const int q = q0 + gtid + i * kGather;
+        val[i] = make_uint4(0, 0, 0, 0);
+        if (q < base_rows * cpr) {
+          const int x = s_x[q / cpr];
+          if (x >= 0) val[i] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)x * ra) + (q % cpr));
+        }
       }
-    }
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int q = gtid + i * kGather;
-      if (q < base_rows * cpr) {
-        const int m = q / cpr, c = q % cpr;
-        const int kb = c >> 3, j = c & 7;
-        *reinterpret_cast<uint4*>(sA + kb * bstage + m * 128 + ((j ^ (m & 7)) << 4)) = val[i];
+      for (int i = 0; i < kPer; ++i) {
+        const int q = q0 + gtid + i * kGather;
+        if (q < base_rows * cpr) {
+          const int m = q / cpr, c = q % cpr;
+          const int kb = c >> 3, j = c & 7;
+          *reinterpret_cast<uint4*>(sA + kb * bstage + m * 128 + ((j ^ (m & 7)) << 4)) = val[i];
+        }
       }
     }
     fence_proxy_async_smem();
@@ -240,7 +270,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
       int it = 0;
-      for (int t = t0; t < t1 && !*s_abort; ++t) {
+      for (int i = 0; i < nt && !*s_abort; ++i) {
+        const int t = tile_at(i);
         for (int kb = 0; kb < nkb; ++kb, ++it) {
           const int s = it % n_ws;
           const uint32_t ph = (uint32_t)(it / n_ws) & 1u;
@@ -253,6 +284,13 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           tma_load_2d_hint(sW + s * kStageBytes, &tm_w, &fullW[s], kb * 64, t * kTileN, pol);
         }
       }
+      // Tail: a stage is released by a commit of the MMAs that read it, an
+      // arrive the tensor core makes on this CTA's barrier when they
+      // complete.  Wait for the releases of the last stages filled, so the
+      // CTA never exits with such an arrive still in flight; after an abort,
+      // wait for the copies still in flight instead.
+      if (!*s_abort) wait_ring_released(emptyW, n_ws, it, flags);
+      else drain_ring_loads(fullW, n_ws, it);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
@@ -260,9 +298,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       const uint32_t idesc = idesc_bf16(kBlockM, kTileN);
       const uint32_t a0 = smem_u32(sA), w0 = smem_u32(sW);
       int it = 0;
-      for (int t = t0; t < t1 && !*s_abort; ++t) {
-        const int a = (t - t0) & 1;
-        const uint32_t aph = (uint32_t)((t - t0) >> 1) & 1u;
+      for (int i = 0; i < nt && !*s_abort; ++i) {
+        const int a = i & 1;
+        const uint32_t aph = (uint32_t)(i >> 1) & 1u;
         if (!mbar_wait(&accEmpty[a], aph ^ 1u)) {
           *s_abort = 1;
           raise_flag(flags, DSPARK_FLAG_TIMEOUT);
@@ -278,11 +316,13 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             break;
           }
           tc_fence_after();
+          for (int h = 0; h <= a_split; ++h) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = sdesc_sw128(a0 + kb * bstage + kk * 32);
-            const uint64_t bd = sdesc_sw128(w0 + s * kStageBytes + kk * 32);
-            mma_bf16_ss(tmem + a * kTileN, ad, bd, idesc, (kb | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sdesc_sw128(a0 + (h * nkb + kb) * bstage + kk * 32);
+              const uint64_t bd = sdesc_sw128(w0 + s * kStageBytes + kk * 32);
+              mma_bf16_ss(tmem + a * kTileN, ad, bd, idesc, (kb | kk | h) != 0);
+            }
           }
           mma_commit(&emptyW[s]);
         }
@@ -293,6 +333,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         }
         mma_commit(&accFull[a]);
       }
+      drain_mma(mmaDrain);
     }
   } else if (warp == 2 && kRes) {
     // ---------------- target / base row producer (residual)
@@ -314,7 +355,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
     const uint64_t pol = policy_evict_first();
     int it = 0;
-    for (int t = t0; t < t1 && !*s_abort; ++t) {
+    for (int i = 0; i < nt && !*s_abort; ++i) {
+      const int t = tile_at(i);
       bool ok = true;
       for (int cb = 0; cb < kTileN / 32; ++cb, ++it) {
         const int s = it % n_bs;
@@ -339,12 +381,14 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         break;
       }
     }
+    if (*s_abort && lane == 0) drain_ring_loads(fullB, n_bs, it);
   } else if (warp == 2) {
     // ---------------- base-logit producer (draft only)
     if (!kRes && lane == 0) {
       const uint64_t pol = policy_evict_first();
       int it = 0;
-      for (int t = t0; t < t1 && !*s_abort; ++t) {
+      for (int i = 0; i < nt && !*s_abort; ++i) {
+        const int t = tile_at(i);
         for (int cb = 0; cb < kTileN / 32; ++cb, ++it) {
           const int s = it % n_bs;
           const uint32_t ph = (uint32_t)(it / n_bs) & 1u;
@@ -358,10 +402,11 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                            bb * kBlockM, pol);
         }
       }
+      if (*s_abort) drain_ring_loads(fullB, n_bs, it);
     }
   } else {
     // ---------------- epilogue: thread = request (TMEM lane)
-    const int eg = (warp - 3) >> 2;  // warpgroup: chunks 2*eg, 2*eg+1 of every tile
+    const int eg = (warp - 3) >> 2;  // warpgroup: chunks eg * kCpg .. of every tile
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
     const int b = bb * kBlockM + m;
@@ -373,24 +418,29 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     const float it2 = it * kLog2e;
     ResInfo ri{};
     if (kRes && bval) ri = info[b];
-    for (int t = t0; t < t1; ++t) {
-      const int a = (t - t0) & 1;
-      const uint32_t aph = (uint32_t)((t - t0) >> 1) & 1u;
+    // draft: this warpgroup's partial over all of its chunks of the range
+    float Mr = -CUDART_INF_F, Sr = 0.0f;
+    for (int i = 0; i < nt; ++i) {
+      const int t = tile_at(i);
+      const int a = i & 1;
+      const uint32_t aph = (uint32_t)(i >> 1) & 1u;
       if (*s_abort || !mbar_wait(&accFull[a], aph)) {
         *s_abort = 1;
         raise_flag(flags, DSPARK_FLAG_TIMEOUT);
         break;
       }
       tc_fence_after();
-      float2 pp[2];
+      float2 pp[kCpg];
+      if constexpr (!kRes) {
+        // ---- draft: softmax partial of every 32-row chunk of the tile
 #pragma unroll 1
-      for (int ci = 0; ci < 2; ++ci) {
-        const int cb = 2 * eg + ci;
-        float d[32], bv[32];
-        if (wval) tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
-        const int v0 = t * kTileN + cb * 32;
-        if (!kRes) {
-          const int itB = (t - t0) * (kTileN / 32) + cb;
+        for (int ci = 0; ci < kCpg; ++ci) {
+          const int cb = eg * kCpg + ci;
+          float d[32];
+          if (wval) tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
+          float bv[32];
+          const int v0 = t * kTileN + cb * 32;
+          const int itB = i * (kTileN / 32) + cb;
           const int s = itB % n_bs;
           const uint32_t ph = (uint32_t)(itB / n_bs) & 1u;
           if (!mbar_wait(&fullB[s], ph)) {
@@ -411,18 +461,17 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           __syncwarp();
           if (lane == 0) mbar_arrive(&emptyB[s]);
           if (!wval) continue;
-          // four independent max and sum chains (the 32-long serial ones
-          // bounded the epilogue)
-          float A4[4] = {-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F};
+          if (v0 + 32 > V) {
+            // the ragged end of the vocabulary: rows past V carry no mass
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (v0 + j < V) A4[j & 3] = fmaxf(A4[j & 3], bv[j] + d[j]);
-          const float A = fmaxf(fmaxf(A4[0], A4[1]), fmaxf(A4[2], A4[3]));
-          float s4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if (v0 + j < V) s4[j & 3] += ex2(((bv[j] - A) + d[j]) * it2);
-          pp[ci] = make_float2(A, (s4[0] + s4[1]) + (s4[2] + s4[3]));
+            for (int j = 0; j < 32; ++j)
+              if (v0 + j >= V) {
+                bv[j] = -CUDART_INF_F;
+                d[j] = 0.0f;
+              }
+          }
+          pp[ci] = chunk_partial32(bv, d, it2);
+          merge_partial(Mr, Sr, pp[ci].x, pp[ci].y, it2);
           if (draft_bias != nullptr && bval) {
             float* dst = draft_bias + ((size_t)b * K + k) * (size_t)V + v0;
 #pragma unroll
@@ -439,8 +488,16 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                     make_float4((bv[j] + d[j]) * it, (bv[j + 1] + d[j + 1]) * it,
                                 (bv[j + 2] + d[j + 2]) * it, (bv[j + 3] + d[j + 3]) * it);
           }
-        } else {
-          const int itB = (t - t0) * (kTileN / 32) + cb;
+        }
+      } else {
+        // ---- residual: sums of max(0, p_t - p_d) and of p_t per chunk
+#pragma unroll 1
+        for (int ci = 0; ci < kCpg; ++ci) {
+          const int cb = eg * kCpg + ci;
+          float d[32], bv[32];
+          if (wval) tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
+          const int v0 = t * kTileN + cb * 32;
+          const int itB = i * (kTileN / 32) + cb;
           const int s = itB % n_bs;
           const uint32_t ph = (uint32_t)(itB / n_bs) & 1u;
           if (!mbar_wait(&fullB[s], ph)) {
@@ -493,16 +550,16 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       __syncwarp();
       if (lane == 0) mbar_arrive(&accEmpty[a]);
       if (bval) {
-        const int c0 = t * (kTileN / 32) + 2 * eg;
-        float2* dst = part + (size_t)b * n_chunks + c0;
-        if (c0 + 1 < n_chunks) {
-          dst[0] = pp[0];
-          dst[1] = pp[1];
-        } else if (c0 < n_chunks) {
-          dst[0] = pp[0];
+        float2* dst = part + (size_t)b * n_chunks;
+#pragma unroll
+        for (int ci = 0; ci < kCpg; ++ci) {
+          const int c = t * (kTileN / 32) + eg * kCpg + ci;
+          if (c < n_chunks) dst[c] = pp[ci];
         }
       }
     }
+    if (!kRes && bval && cta_part != nullptr)
+      cta_part[((size_t)b * ctas_per_bb + pi) * kEpi + eg] = make_float2(Mr, Sr);
   }
 
   tc_fence_before();
@@ -516,27 +573,37 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
 // ---------------------------------------------------------------------------
 
 inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
+  // a driver entry point: the same for every device; looked up once,
+  // thread-safe (function-local static)
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return (PFN_cuTensorMapEncodeTiled_v12000) nullptr;
+  }();
   return fn;
 }
 
+// SM count of the current device, looked up once per device.
 inline int num_sms() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (n <= 0) n = 148;
+  static DeviceOnce once;
+  static int n[kMaxDevices];
+  const int dev = current_device();
+  int v = 0;
+  if (dev >= 0 && dev < kMaxDevices) {
+    std::call_once(once[dev], [&] {
+      int c = 0;
+      if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) c = 0;
+      n[dev] = c > 0 ? c : 148;
+    });
+    v = n[dev];
+  } else if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    v = 0;
   }
-  return n;
+  return v > 0 ? v : 148;
 }
 
 // W [V, r] bf16 as 64 x 128 boxes (128-byte rows), 128-byte swizzle.
@@ -579,18 +646,26 @@ inline bool encode_base_map(CUtensorMap* m, const float* base, int V, int K, int
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// CTAs per request block, at most this many (the workspace holds this many
+// partials per request and epilogue warpgroup).
+constexpr int kTcMaxCtasPerBlock = 256;
+
 inline void tc_grid(TcPlan& p) {
   p.n_tiles = (p.V + kTileN - 1) / kTileN;
   p.n_bb = (p.B + kBlockM - 1) / kBlockM;
   int per = num_sms() / p.n_bb;
   if (per < 1) per = 1;
   if (per > p.n_tiles) per = p.n_tiles;
+  if (per > kTcMaxCtasPerBlock) per = kTcMaxCtasPerBlock;
   p.ctas_per_bb = per;
 }
 
 inline dspark_status tc_plan_draft(TcPlan& p, const float* base, const void* U, const void* W,
-                                   int V, int r, int B, int K) {
+                                   int V, int r, int B, int K,
+                                   const __nv_bfloat16* a_rows = nullptr) {
   p.V = V; p.r = r; p.B = B; p.K = K;
+  p.a_rows = a_rows;
+  p.a_split = a_rows != nullptr ? 1 : 0;
   p.base = base;
   p.target = nullptr;
   p.U = static_cast<const __nv_bfloat16*>(U);
@@ -598,8 +673,8 @@ inline dspark_status tc_plan_draft(TcPlan& p, const float* base, const void* U, 
     return DSPARK_ERR_CUDA;
   p.tm_tgt = p.tm_w;  // unused in draft mode
   tc_grid(p);
-  p.w_stages = tc_w_stages(r, B, false);
-  p.b_stages = tc_b_stages(r, B, false);
+  p.w_stages = tc_w_stages(r, B, false, p.a_split);
+  p.b_stages = tc_b_stages(r, B, false, p.a_split);
   p.base_rows = tc_base_rows(B);
   return DSPARK_OK;
 }
@@ -608,6 +683,8 @@ inline dspark_status tc_plan_residual(TcPlan& p, const float* target, long long 
                                       const float* base, const void* U, const void* W, int V,
                                       int r, int B, int K) {
   p.V = V; p.r = r; p.B = B; p.K = K;
+  p.a_rows = nullptr;
+  p.a_split = 0;
   p.base = base;
   p.target = target;
   p.U = static_cast<const __nv_bfloat16*>(U);
@@ -623,12 +700,8 @@ inline dspark_status tc_plan_residual(TcPlan& p, const float* target, long long 
 
 template <bool kRes>
 inline void tc_set_attr() {
-  static bool done = false;
-  if (!done) {
-    cudaFuncSetAttribute(proj_tc_kernel<kRes>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kTcSmemLimit);
-    done = true;
-  }
+  static DeviceOnce once;
+  set_smem_once(once, proj_tc_kernel<kRes>, (int)kTcSmemLimit);
 }
 
 // Launch configuration with programmatic stream serialisation: the kernel
@@ -651,22 +724,25 @@ struct PdlLaunch {
 
 inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const int32_t* tokens,
                             const float* it, float* dl, float* dbias, float2* part,
-                            unsigned* flags, cudaStream_t s) {
+                            float2* cta_part, unsigned* flags, cudaStream_t s) {
   tc_set_attr<false>();
-  PdlLaunch L(p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, false), s);
+  PdlLaunch L(p.n_bb * p.ctas_per_bb, tc_threads<false>(),
+              tc_smem_bytes(p.r, p.B, false, p.a_split), s);
   cudaLaunchKernelEx(&L.cfg, proj_tc_kernel<false>, p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r,
-                     p.B, p.K, k,
-                     prev, tokens, it, (const float*)nullptr, p.base, (const ResInfo*)nullptr, dl,
-                     dbias, part, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages,
-                     p.b_stages, p.base_rows, flags);
+                     p.B, p.K, k, prev, tokens, it, (const float*)nullptr, p.base,
+                     (const ResInfo*)nullptr, dl, dbias, part, cta_part, n_chunks_of(p.V),
+                     p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, p.a_rows,
+                     p.a_split, flags);
 }
 
 inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,
                                float2* rpart, unsigned* flags, cudaStream_t s) {
   tc_set_attr<true>();
-  proj_tc_kernel<true><<<p.n_bb * p.ctas_per_bb, kTcThreads, tc_smem_bytes(p.r, p.B, true), s>>>(
-      p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r, p.B, p.K, 0, nullptr, nullptr, it, p.target, p.base, info,
-      nullptr, nullptr, rpart, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, flags);
+  proj_tc_kernel<true><<<p.n_bb * p.ctas_per_bb, tc_threads<true>(), tc_smem_bytes(p.r, p.B, true),
+                         s>>>(p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r, p.B, p.K, 0, nullptr,
+                              nullptr, it, p.target, p.base, info, nullptr, nullptr, rpart,
+                              nullptr, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages,
+                              p.b_stages, p.base_rows, (const __nv_bfloat16*)nullptr, 0, flags);
 }
 
 }  // namespace dspark

@@ -104,6 +104,31 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Producer tail of a ring of `n` stages whose stage it % n was filled for
+// uses it = 0 .. issued - 1 and is released by a tcgen05.commit arrive on
+// empty[it % n]: waits until the last min(n, issued) uses are released.
+// Returns false (DSPARK_FLAG_TIMEOUT raised) if a release never comes.
+__device__ __forceinline__ bool wait_ring_released(uint64_t* empty, int n, int issued,
+                                                   unsigned* flags) {
+  for (int j = issued > n ? issued - n : 0; j < issued; ++j) {
+    if (!mbar_wait(&empty[j % n], (uint32_t)(j / n) & 1u)) {
+      raise_flag(flags, DSPARK_FLAG_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Drain of a ring's loads: waits until the copies of the last min(n, issued)
+// uses have landed (use it fills stage it % n and completes phase it / n of
+// full[it % n]).  On the normal path every one has been consumed and this
+// returns at once; after an abort it keeps the CTA from exiting while a copy
+// still writes its shared memory.  Bounded like every wait.
+__device__ __forceinline__ void drain_ring_loads(uint64_t* full, int n, int issued) {
+  for (int j = issued > n ? issued - n : 0; j < issued; ++j)
+    if (!mbar_wait(&full[j % n], (uint32_t)(j / n) & 1u)) return;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (no multicast anywhere in this library)
 // ---------------------------------------------------------------------------
@@ -241,24 +266,15 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
-
-// 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
-  uint32_t r[32];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+// Drain of the MMAs: one more commit, to a barrier used for nothing else
+// (initialised with count 1, phase 0), and a bounded wait for it, so every
+// tcgen05 operation this thread issued has completed before the CTA frees
+// its tensor memory -- on the normal path and after an abort alike.
+__device__ __forceinline__ void drain_mma(uint64_t* bar) {
+  mma_commit(bar);
+  mbar_wait(bar, 0u);
 }
+
 // Split form of tmem_ld32 for software pipelining: the load is issued by
 // tmem_ld32_issue and the registers may be read only after
 // tmem_ld32_wait(r), which names them as read-write operands so the
@@ -304,17 +320,21 @@ __device__ __forceinline__ void tmem_ld16_wait(uint32_t (&r)[16]) {
                :
                : "memory");
 }
+// 32 lanes x 32 consecutive 32-bit columns -> 32 registers per thread.  The
+// wait names the destination registers, so no use of them can be scheduled
+// above it.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  tmem_ld32_issue(taddr, r);
+  tmem_ld32_wait(r);
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
 // 32 lanes x 16 consecutive 32-bit columns -> 16 registers per thread.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+  tmem_ld16_issue(taddr, r);
+  tmem_ld16_wait(r);
 #pragma unroll
   for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }

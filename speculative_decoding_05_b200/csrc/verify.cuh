@@ -95,7 +95,8 @@ accept_kernel(const float* __restrict__ target, long long n_rows,
               const float* __restrict__ p_tok, const float* __restrict__ ref_max,
               const float* __restrict__ ref_sum, const float* __restrict__ u_accept,
               const float2* __restrict__ tpart, int n_segs, int32_t* __restrict__ n_accepted,
-              int32_t* __restrict__ out_tokens, ResInfo* __restrict__ info, unsigned* flags) {
+              int32_t* __restrict__ out_tokens, ResInfo* __restrict__ info, unsigned* flags,
+              const float* __restrict__ tok_logit = nullptr) {
   const int lane = threadIdx.x & 31;
   const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (b >= B) return;
@@ -122,7 +123,9 @@ accept_kernel(const float* __restrict__ target, long long n_rows,
       if (!(tz > 0.0) || !isfinite(tz)) raise_flag(flags, DSPARK_FLAG_NONFINITE);
       if (p < L) {
         const int x = checked_token(tokens[(size_t)b * K + p], V, false, flags);
-        const float tx = target[(size_t)row * V + x];
+        // the drafted token's raw target logit: from the stored row, or
+        // (LM-head verify) as the statistics pass recorded it
+        const float tx = tok_logit != nullptr ? tok_logit[row] : target[(size_t)row * V + x];
         const double pt = (double)ex2((tx - tmax) * it2) / tz;
         const double pd = (double)p_tok[(size_t)b * K + p];
         // accept iff u < p_t / p_d (p_t >= p_d always accepts; p_d = 0 gives +inf)

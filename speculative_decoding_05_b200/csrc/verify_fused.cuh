@@ -119,6 +119,7 @@ __device__ __forceinline__ bool pair_valid(ulonglong2 v) {
 }
 
 __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedArgs a) {
+  const bool test_skew = g_test_exchange_skew != 0;  // see common.cuh
   __shared__ int s_rofs[kFMaxB + 1];  // first flat row of request b; s_rofs[B] = rows
   __shared__ int s_len[kFMaxB];
   __shared__ float s_it2[kFMaxB];
@@ -331,7 +332,7 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
       }
 #pragma unroll
       for (int i = 0; i < kFPerLane; ++i) {
-        if ((pend & (1u << i)) && pair_valid(m[i])) {
+        if ((pend & (1u << i)) && pair_valid(m[i]) && !test_skew) {
           q[i] = make_float2(__uint_as_float((uint32_t)m[i].x), __uint_as_float((uint32_t)m[i].y));
           pend &= ~(1u << i);
         }

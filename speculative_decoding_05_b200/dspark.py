@@ -37,6 +37,12 @@ SYMBOLS = [
     "dspark_get_device_status", "dspark_get_device_flags",
     "dspark_status_string", "dspark_draft_path", "dspark_verify_path", "dspark_version",
     "dspark_verify_noalloc",
+    "dspark_verify_noalloc_status",
+    "dspark_verify_lmhead_workspace_size",
+    "dspark_verify_lmhead",
+    "dspark_draft_rnn_workspace_size",
+    "dspark_draft_rnn",
+    "dspark_test_set_exchange_skew",
     "dspark_sts_workspace_size",
     "dspark_sts_fit",
     "dspark_confidence_prefix_async",
@@ -77,6 +83,20 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.dspark_verify_noalloc.argtypes = [P, L, P, P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P,
                                           P, P, P, P, P, P]
     lib.dspark_verify_noalloc.restype = I
+    lib.dspark_verify_noalloc_status.argtypes = [P]
+    lib.dspark_verify_noalloc_status.restype = I
+    lib.dspark_verify_lmhead_workspace_size.argtypes = [I, I, I, I, I, L]
+    lib.dspark_verify_lmhead_workspace_size.restype = S
+    lib.dspark_verify_lmhead.argtypes = [P, P, I, L, P, P, P, P, P, I, I, I, I, I, P, P, P, P, P,
+                                         P, P, P, P, P, P, P, P, S, P]
+    lib.dspark_verify_lmhead.restype = I
+    lib.dspark_draft_rnn_workspace_size.argtypes = [I, I, I, I]
+    lib.dspark_draft_rnn_workspace_size.restype = S
+    lib.dspark_draft_rnn.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P, P,
+                                     P, P, S, P]
+    lib.dspark_draft_rnn.restype = I
+    lib.dspark_test_set_exchange_skew.argtypes = [I]
+    lib.dspark_test_set_exchange_skew.restype = I
     lib.dspark_confidence_prefix.argtypes = [P, P, P, P, I, I, I, I, P, P, P, P, P, S, P]
     lib.dspark_confidence_prefix.restype = I
     lib.dspark_confidence_prefix_async.argtypes = [P, P, P, P, I, I, I, I, I, P, P, P, P, P, P, P,
@@ -218,6 +238,60 @@ def dspark_verify_noalloc(target_logits, row_start, verify_len, base_logits, U, 
         _ptr(tokens), _ptr(p_tok), _ptr(ref_max), _ptr(ref_sum), _ptr(draft_bias), _ptr(u_accept),
         _ptr(u_resample), _ptr(n_accepted), _ptr(out_tokens), _ptr(last_token), _stream(stream))
     _check("dspark_verify_noalloc", rc)
+
+
+def dspark_draft_rnn_workspace_size(V, r, B, K) -> int:
+    return int(load().dspark_draft_rnn_workspace_size(V, r, B, K))
+
+
+def dspark_draft_rnn(base_logits, U, W, R, prev_token, h0, inv_temp, u_draft, tokens, p_tok, lse,
+                     ref_max, ref_sum, workspace, states=None, draft_logits=None, draft_bias=None,
+                     stream=None):
+    """The draft with the RNN head: state s_k = tanh(R s_{k-1} + U[x_{k-1}])
+    from h0 (None: zeros), bias s_k . W^T."""
+    B, K, V = base_logits.shape
+    r = W.shape[1]
+    rc = load().dspark_draft_rnn(
+        _ptr(base_logits), _ptr(U), _ptr(W), _ptr(R), _dtype_code(U), V, r, B, K,
+        _ptr(prev_token), _ptr(h0), _ptr(inv_temp), _ptr(u_draft), _ptr(tokens), _ptr(p_tok),
+        _ptr(lse), _ptr(ref_max), _ptr(ref_sum), _ptr(states), _ptr(draft_logits),
+        _ptr(draft_bias), _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("dspark_draft_rnn", rc)
+
+
+def dspark_verify_lmhead_workspace_size(V, r, B, K, dm, n_rows) -> int:
+    return int(load().dspark_verify_lmhead_workspace_size(V, r, B, K, dm, int(n_rows)))
+
+
+def dspark_verify_lmhead(hidden, lm_head, row_start, verify_len, base_logits, U, W, prev_token,
+                         inv_temp, tokens, p_tok, ref_max, ref_sum, u_accept, u_resample,
+                         n_accepted, out_tokens, workspace, last_token=None, draft_bias=None,
+                         stream=None):
+    """dspark_verify with target logits hidden [n_rows, dm] . lm_head [V, dm]^T
+    (both bf16) formed on chip instead of read from stored rows."""
+    n_rows, dm = hidden.shape
+    V = lm_head.shape[0]
+    B, K = tokens.shape
+    r = W.shape[1]
+    rc = load().dspark_verify_lmhead(
+        _ptr(hidden), _ptr(lm_head), dm, n_rows, _ptr(row_start), _ptr(verify_len),
+        _ptr(base_logits), _ptr(U), _ptr(W), _dtype_code(U), V, r, B, K, _ptr(prev_token),
+        _ptr(inv_temp), _ptr(tokens), _ptr(p_tok), _ptr(ref_max), _ptr(ref_sum), _ptr(draft_bias),
+        _ptr(u_accept), _ptr(u_resample), _ptr(n_accepted), _ptr(out_tokens), _ptr(last_token),
+        _ptr(workspace), workspace.numel(), _stream(stream))
+    _check("dspark_verify_lmhead", rc)
+
+
+def dspark_test_set_exchange_skew(skew: int) -> None:
+    """Test hook: non-zero makes the persistent draft's and the
+    single-launch verify's record exchanges time out (see the header)."""
+    _check("dspark_test_set_exchange_skew", load().dspark_test_set_exchange_skew(int(skew)))
+
+
+def dspark_verify_noalloc_status(stream=None) -> int:
+    """Status code of the last dspark_verify_noalloc call on this device
+    (synchronises the stream)."""
+    return int(load().dspark_verify_noalloc_status(_stream(stream)))
 
 
 def dspark_get_device_flags(workspace, stream=None) -> int:

@@ -1,0 +1,46 @@
+"""Repeated persistent draft calls: every call identical to the first.
+
+The B <= 2 draft is one persistent launch whose CTAs exchange partial
+softmax records and sampled tokens through the workspace on every one of
+the K positions.  A record read before it is written, or a stale record of
+the previous call or position taken for the current one, changes a p_tok or
+a token.  200 back-to-back calls of the full-size single-request workload
+(V = 151936, K = 16) at B = 1 and B = 2, with fresh status flags each call,
+must give bit-identical outputs, and the first call must match the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from speculative_decoding_05_b200 import dspark as D
+from speculative_decoding_05_b200 import workloads as WL
+from speculative_decoding_05_b200.step import DSparkStep
+
+from tests.parity import compare_step
+
+pytestmark = pytest.mark.gpu
+
+N_CALLS = 200
+
+
+@pytest.mark.parametrize("B", [1, 2])
+def test_persistent_draft_repeats_bit_identically(oracle_mod, B):
+    w = WL.get("single", B=B, seed=80 + B)
+    inp = WL.make_inputs(w, device="cuda")
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+    assert step.path == "persistent-cuda-core"
+    step.run(inp, enable_prefix=False)
+    torch.cuda.synchronize()
+    assert all(f == 0 for f in step.flags().values())
+    rep = compare_step(oracle_mod, inp, step, False)
+    assert not rep.failures, rep.failures[:5]
+    first = [t.clone() for t in (step.tokens, step.p_tok, step.lse, step.ref_max, step.ref_sum)]
+    bad = []
+    for i in range(N_CALLS):
+        step.draft(inp)
+        f = D.dspark_get_device_flags(step.ws_draft)  # synchronises
+        same = all(torch.equal(a, b) for a, b in
+                   zip(first, (step.tokens, step.p_tok, step.lse, step.ref_max, step.ref_sum)))
+        if f != 0 or not same:
+            bad.append((i, f, same))
+    assert not bad, bad[:10]

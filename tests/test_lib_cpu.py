@@ -124,6 +124,28 @@ def test_argument_validation_before_launch(lib):
     vb = lib.dspark_verify_workspace_size(1024, 16, 2, 3)
     assert lib.dspark_verify(None, 10, p, p, p, p, p, 1, 1024, 16, 2, 3, p, None, p, p, p, p, None,
                              p, p, p, p, None, ws, vb, None) == 1
+    # LM-head verify: width not a multiple of 64 or too large, missing hidden
+    # states, short workspace, misaligned head
+    lb = lib.dspark_verify_lmhead_workspace_size(1024, 16, 2, 3, 256, 10)
+    assert lb > 0 and lib.dspark_verify_lmhead_workspace_size(1024, 16, 2, 3, 0, 10) == 0
+
+    def lm(hidden=p, head=p, dm=256, ws_bytes=lb):
+        return lib.dspark_verify_lmhead(hidden, head, dm, 10, p, p, p, p, p, 1, 1024, 16, 2, 3, p,
+                                        None, p, p, p, p, None, p, p, p, p, None, ws, ws_bytes,
+                                        None)
+    # RNN draft: fp32 factors, r not a multiple of 64, short workspace
+    rb = lib.dspark_draft_rnn_workspace_size(1024, 64, 4, 3)
+    assert rb > lib.dspark_draft_workspace_size(1024, 64, 4, 3)
+
+    def rnn(dt=D.DSPARK_BF16, r=64, ws_bytes=rb):
+        return lib.dspark_draft_rnn(p, p, p, p, dt, 1024, r, 4, 3, p, None, None, p, p, p, p, p,
+                                    p, None, None, None, ws, ws_bytes, None)
+    assert rnn(dt=D.DSPARK_F32) == 4 and rnn(r=72) == 4 and rnn(r=320) == 4
+    assert rnn(ws_bytes=rb - 256) == 6
+    assert lm(dm=100) == 4 and lm(dm=32768) == 4 and lm(dm=-64) == 1
+    assert lm(hidden=None) == 1
+    assert lm(ws_bytes=lb - 256) == 6
+    assert lm(head=P((1 << 23) + 8)) == 1
 
 
 def test_traffic_hash_covers_the_draft_kernels_sources():

@@ -1,17 +1,18 @@
 """dspark_verify_noalloc against dspark_verify.
 
-Some callers cannot call cudaMalloc: code running while another component
-captures a CUDA graph in global mode, plugins whose host application owns
-every device allocation, runtimes with a fixed device-memory budget.  For
-them the library offers dspark_verify_noalloc, whose scratch is a fixed 2 MiB
-array inside the library image instead of a caller-provided workspace.
+Some callers cannot call cudaMalloc: plugins whose host application owns
+every device allocation and hands out no scratch, runtimes that run under a
+fixed device-memory budget decided before the first step.  For them the
+library offers dspark_verify_noalloc, whose scratch is a fixed 2 MiB array
+inside the library image instead of a caller-provided workspace.
 
 These tests check that it returns exactly what the regular verify returns
 (integer outputs, so bit for bit), on two calls in a row with different
 uniforms (the second call finds the first call's leftovers in the shared
-scratch), and that a problem too large for the scratch is refused before
-anything is enqueued.  This file sorts last so that a run stopping at the
-first failure has already run every other test.
+scratch), that its status query reports the device's data checks, and that a
+problem too large for the scratch is refused before anything is enqueued.
+This file sorts last so that a run stopping at the first failure has already
+run every other test.
 """
 import ctypes
 
@@ -58,6 +59,26 @@ def test_noalloc_verify_matches_workspace_verify(name, over):
         torch.cuda.synchronize()
         for a, b in zip(ref, got):
             assert torch.equal(a, b), (name, call)
+        assert D.dspark_verify_noalloc_status() == 0
+
+
+def test_noalloc_status_reports_bad_data():
+    """Out-of-range token ids and verify lengths are clamped on the device
+    and reported through the status query; a clean call clears it again."""
+    w = WL.get("single", V=1024, r=16, B=4, K=3, seed=40)
+    inp = WL.make_inputs(w, device="cuda")
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+    step.draft(inp)
+    step.prefix(inp, enable=False)
+    good_tokens, good_len = step.tokens.clone(), step.verify_len.clone()
+    step.tokens[1, 0] = w.V + 7
+    step.verify_len[2] = w.K + 5
+    _noalloc(inp, step, inp["u_accept"], inp["u_res"])
+    assert D.dspark_verify_noalloc_status() == 5  # DSPARK_ERR_DEVICE_DATA
+    step.tokens.copy_(good_tokens)
+    step.verify_len.copy_(good_len)
+    _noalloc(inp, step, inp["u_accept"], inp["u_res"])
+    assert D.dspark_verify_noalloc_status() == 0
 
 
 def test_noalloc_refuses_oversized_problems():
