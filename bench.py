@@ -165,7 +165,7 @@ def kernel_name(path: str, call: str, w) -> str:
     if path == "tcgen05-persistent":
         return "draft_persist_kernel"
     if path == "tcgen05":
-        return "proj_tc_kernel<false> + draft_sample_kernel"
+        return "proj_tc_kernel<false> + draft_sample2_kernel"
     return "draft_proj_simt_kernel + draft_sample_kernel"
 
 

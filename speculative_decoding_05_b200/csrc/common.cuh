@@ -47,15 +47,6 @@ inline void set_smem_once(DeviceOnce& once, Kern* kern, int bytes) {
   });
 }
 
-// Programmatic dependent launch.  wait: block until the kernel this one was
-// launched behind has finished and its writes are visible (returns at once
-// when the launch carried no programmatic dependency).  launch_dependents:
-// let the kernel launched behind this one start its own prologue.
-__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void grid_dep_launch() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-
 // ---------------------------------------------------------------------------
 // sizes and workspace layout
 // ---------------------------------------------------------------------------
@@ -125,6 +116,15 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// An empty asm that takes v as an input: v is computed here, in program
+// order, so every shared-memory load it was computed from has returned.  A
+// warp that releases a buffer for an async-proxy refill (TMA, bulk copy)
+// passes what it computed from its loads through here first, then syncs
+// and arrives.  An arrive issued while the warp's loads were still in
+// flight let the refill overwrite rows before they were read (measured: the
+// first rows of a 128-row stage, read by the warps of lane quarters 0-1).
+__device__ __forceinline__ void consumed(float v) { asm volatile("" ::"f"(v) : "memory"); }
 
 // Softmax partial of a 32-row chunk of one request: A = max_j (bv_j + d_j),
 // s = sum_j 2^(((bv_j - A) + d_j) * it2) (0 when every row is -inf), in four

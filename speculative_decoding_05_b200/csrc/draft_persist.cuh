@@ -881,6 +881,9 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   int* s_units = reinterpret_cast<int*>(s_ud + kGMaxB * 64);  // [9][kGMaxUnits] (type, index, chunk)
   int* s_nunits = s_units + 9 * kGMaxUnits;                    // [9]
   float* s_acta = reinterpret_cast<float*>(s_nunits + 12);     // [kGMaxB] CTA max per request
+  // fill number of each ring stage (consecutive fills of a stage go to
+  // different warps; see tag_wait)
+  volatile int* s_tag = reinterpret_cast<volatile int*>(s_acta + kGMaxB);  // [kPMaxStages]
   // chunk weights relative to the CTA max and their inclusive prefix sums
   double* s_cw = reinterpret_cast<double*>(sPart + (size_t)B * part_cap);  // [B][kGMaxChunks]
   double* s_cp = s_cw + (size_t)B * kGMaxChunks;                                     // [B][kGMaxChunks]
@@ -890,8 +893,9 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(&ringFull[i], 1);
-      mbar_init(&ringEmpty[i], 1);  // one consumer warp per stage
+      mbar_init(&ringEmpty[i], 1);  // one consumer warp per fill
     }
+    for (int i = 0; i < kPMaxStages; ++i) s_tag[i] = -1;
     for (int i = 0; i < 2; ++i) {
       mbar_init(&baseFull[i], 1);
       mbar_init(&baseEmpty[i], 1);
@@ -922,6 +926,7 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             raise_flag(p.flags, DSPARK_FLAG_TIMEOUT);
             break;
           }
+          s_tag[s] = it;
           const int row0 = v0 + (n_tm + n_res + sc) * kChunk;
           const int nr = max(0, min(kChunk, V - row0));
           if (nr > 0) {
@@ -1102,7 +1107,8 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
           const uint8_t* buf;
           if (type == 2) {
             it = k * n_str + idx;
-            ok = ok && mbar_wait_spin(&ringFull[it % S], (uint32_t)(it / S) & 1u);
+            ok = ok && tag_wait(s_tag + it % S, it) &&
+                 mbar_wait_spin(&ringFull[it % S], (uint32_t)(it / S) & 1u);
             buf = sRing + (it % S) * kStageBytes;
           } else {
             buf = (type == 1) ? sRes + idx * kStageBytes : sTail;
@@ -1116,6 +1122,11 @@ draft_gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const PersistArgs p,
             gemv8<NB>(q, u, pr, rr);
           }
           if (type == 2) {
+            // release the stage once every lane's reads of it have returned
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+#pragma unroll
+              for (int j = 0; j < 32; ++j) consumed(pr[b][j]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&ringEmpty[it % S]);
           }

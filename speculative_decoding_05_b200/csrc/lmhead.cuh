@@ -108,7 +108,6 @@ lmhead_tc_kernel(const __grid_constant__ CUtensorMap tm_h, const __grid_constant
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  grid_dep_wait();
 
   if (warp == 0) {
     // ---------------- producer: H block and E block of every k step

@@ -60,6 +60,25 @@ __device__ __forceinline__ double cost_of(const float* __restrict__ xs, const fl
   return staircase ? cost_stair_at(xs, ys, n, tokens) : cost_at(xs, ys, n, tokens);
 }
 
+// cost_of for a non-decreasing sequence of token counts: the table position
+// only moves forward, so each lookup is amortised O(1).  Same arithmetic and
+// results as cost_of.
+struct CostWalker {
+  const float* xs;
+  const float* ys;
+  int n, staircase, i;
+  __device__ double at(double tokens) {
+    if (staircase) {
+      if (tokens > (double)xs[n - 1]) return cost_stair_at(xs, ys, n, tokens);
+      while ((double)xs[i] < tokens) ++i;
+      return ys[i];
+    }
+    while (i < n - 2 && tokens > (double)xs[i + 1]) ++i;
+    const double x0 = xs[i], x1 = xs[i + 1], y0 = ys[i], y1 = ys[i + 1];
+    return y0 + (y1 - y0) * (tokens - x0) / (x1 - x0);
+  }
+};
+
 // key order: larger survival first; equal survival: smaller index first
 __device__ __forceinline__ bool cand_before(double sa, int ia, double sb, int ib) {
   return sa > sb || (sa == sb && ia < ib);
@@ -187,9 +206,10 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   const double excl = block_excl_scan_d<kT>(run, shd, &total);
   // candidate i (0-based) raises the objective iff E_{i+1}/t(B+i+1) > E_i/t(B+i)
   double E = (double)B + excl;
+  CostWalker cw{s_xs, s_ys, n_pts, staircase, 0};
+  double t0 = (i0 < n) ? cw.at((double)B + (double)i0) : 1.0;
   for (int i = i0; i < i0 + per && i < n; ++i) {
-    const double t0 = cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)i);
-    const double t1 = cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)i + 1.0);
+    const double t1 = cw.at((double)B + (double)i + 1.0);
     const double E1 = E + key(i);
     if (!(t0 > 0.0) || !(t1 > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
     if (!(E1 / t1 > E / t0)) {
@@ -197,6 +217,7 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
       break;
     }
     E = E1;
+    t0 = t1;
   }
   __syncthreads();
   // the greedy cut, or the budget's (clamped to [0, n])

@@ -17,20 +17,19 @@
 // partial locally -- no cross-thread reduction, because the request is the
 // TMEM lane.
 //
-// In the draft the projection of position k >= 1 is launched while the
-// sampler of position k - 1 runs (programmatic dependent launch), and its two
-// producer warps start filling the W and base rings at once: neither depends
-// on the sampled tokens, and both inputs were complete before the call's
-// first projection got past its own wait (which its producers take too).
-// The other warps wait for the sampler to finish before reading tokens;
-// every write of the kernel comes after that wait.
+// Launches are plain (stream-ordered).  A launch with programmatic stream
+// serialisation, which let the next position's producers fill the rings
+// while the sampler ran, gained about 3 % on the draft; it was taken out
+// while launch failures were traced, before the ring faults described at
+// tc_b_stages and at the epilogue's stage release were found.
 //
 //   warp 0       W producer (TMA, evict-last: W is re-read every position)
 //   warp 1       TMEM allocator + MMA issuer (one thread)
 //   warp 2       base-logit producer (TMA 3-D boxes, evict-first)   [draft]
 //                target / base row-segment producer (TMA gather4)   [residual]
-//   warps 3..10  epilogue: two warpgroups of 128 threads (= 128 requests),
-//                each taking half of every tile's 32-column chunks
+//   warps 3..10  epilogue: two warpgroups of 128 threads (= 128 requests);
+//                warpgroup g takes the 32-column chunks g, g + 2 of every
+//                tile
 //
 // Draft mode streams base[b, k, v0:v0+32] boxes through a second TMA ring.
 // Residual mode needs the per-request rows target[row_b, :] and
@@ -103,23 +102,29 @@ inline size_t tc_fixed_bytes(int ra, int B, bool residual) {
 // Ring depths.  Each copy in flight waits about the same time for its
 // bytes, so the two rings share what is left in proportion to what they
 // move per tile: W r / 64 stages of 16 KB, the second ring kTileN / 32
-// stages.  W keeps at least two stages (a ring shorter than a tile still
-// flows: the MMAs free its stages in order).
+// stages.  The second ring's depth is even: chunk parity picks the epilogue
+// warpgroup, so every stage is then read by one warpgroup only, which waits
+// on each fill of it in turn.  (With an odd depth a stage alternates between
+// the warpgroups, and a parity wait on fill f can pass while fill f - 1,
+// meant for the other warpgroup, is still landing: the waiter would read the
+// wrong chunk and release the stage early.)  W takes what is left, at least
+// two stages (a ring shorter than a tile still flows: the MMAs free its
+// stages in order).
+inline int tc_b_stages(int r, int B, bool residual, int a_split = 0) {
+  const size_t ring = kTcSmemLimit - tc_fixed_bytes(r << a_split, B, residual);
+  const size_t w_tile = (size_t)(r / 64) * kStageBytes;
+  const size_t rstage = tc_r_stage_bytes(B, residual);
+  const size_t b_tile = (size_t)(kTileN / 32) * rstage;
+  int s = (int)(ring * b_tile / (w_tile + b_tile) / rstage);
+  while (s > 2 && ring < (size_t)s * rstage + 2 * kStageBytes) --s;
+  if (s > kBStagesMax) s = kBStagesMax;
+  return s & ~1;
+}
 inline int tc_w_stages(int r, int B, bool residual, int a_split = 0) {
   const size_t ring = kTcSmemLimit - tc_fixed_bytes(r << a_split, B, residual);
-  const int nkb = r / 64;
-  const size_t w_tile = (size_t)nkb * kStageBytes;
-  const size_t b_tile = (size_t)(kTileN / 32) * tc_r_stage_bytes(B, residual);
-  int s = (int)(ring * w_tile / (w_tile + b_tile) / kStageBytes);
-  if (s < 2) s = 2;
+  const size_t left = ring - (size_t)tc_b_stages(r, B, residual, a_split) * tc_r_stage_bytes(B, residual);
+  int s = (int)(left / kStageBytes);
   if (s > kWStagesMax) s = kWStagesMax;
-  return s;
-}
-inline int tc_b_stages(int r, int B, bool residual, int a_split = 0) {
-  const size_t left = kTcSmemLimit - tc_fixed_bytes(r << a_split, B, residual) -
-                      (size_t)tc_w_stages(r, B, residual, a_split) * kStageBytes;
-  int s = (int)(left / tc_r_stage_bytes(B, residual));
-  if (s > kBStagesMax) s = kBStagesMax;
   return s;
 }
 inline size_t tc_smem_bytes(int r, int B, bool residual, int a_split = 0) {
@@ -201,10 +206,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Producers (warps 0 and 2) read only W and base; at k = 0 they too wait
-  // for the kernel before the call, which may have written either.
   const bool producer = warp == 0 || warp == 2;
-  if (!producer || k == 0) grid_dep_wait();
 
   // operand A: the previous-token rows of U for this block of requests,
   // gathered by the non-producer warps.  The 128 token ids go to shared
@@ -262,7 +264,6 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
     fence_proxy_async_smem();
     named_sync(1, kGather);
-    grid_dep_launch();
   }
 
   if (warp == 0) {
@@ -406,7 +407,10 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
   } else {
     // ---------------- epilogue: thread = request (TMEM lane)
-    const int eg = (warp - 3) >> 2;  // warpgroup: chunks eg * kCpg .. of every tile
+    // warpgroup eg takes chunks eg, eg + kEpi, ... of every tile: chunk
+    // parity picks the warpgroup, so with an even depth every stage of the
+    // second ring is always read by the same warpgroup (see tc_b_stages)
+    const int eg = (warp - 3) >> 2;
     const int quarter = warp & 3;
     const int m = quarter * 32 + lane;
     const int b = bb * kBlockM + m;
@@ -435,7 +439,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         // ---- draft: softmax partial of every 32-row chunk of the tile
 #pragma unroll 1
         for (int ci = 0; ci < kCpg; ++ci) {
-          const int cb = eg * kCpg + ci;
+          const int cb = eg + kEpi * ci;
           float d[32];
           if (wval) tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
           float bv[32];
@@ -458,19 +462,26 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
               bv[4 * j] = q4.x; bv[4 * j + 1] = q4.y; bv[4 * j + 2] = q4.z; bv[4 * j + 3] = q4.w;
             }
           }
+          float2 cpv = make_float2(-CUDART_INF_F, 0.0f);
+          if (wval) {
+            if (v0 + 32 > V) {
+              // the ragged end of the vocabulary: rows past V carry no mass
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (v0 + j >= V) {
+                  bv[j] = -CUDART_INF_F;
+                  d[j] = 0.0f;
+                }
+            }
+            cpv = chunk_partial32(bv, d, it2);
+          }
+          // the stage is released only once every lane's reads have returned
+          consumed(cpv.x);
+          consumed(cpv.y);
           __syncwarp();
           if (lane == 0) mbar_arrive(&emptyB[s]);
           if (!wval) continue;
-          if (v0 + 32 > V) {
-            // the ragged end of the vocabulary: rows past V carry no mass
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (v0 + j >= V) {
-                bv[j] = -CUDART_INF_F;
-                d[j] = 0.0f;
-              }
-          }
-          pp[ci] = chunk_partial32(bv, d, it2);
+          pp[ci] = cpv;
           merge_partial(Mr, Sr, pp[ci].x, pp[ci].y, it2);
           if (draft_bias != nullptr && bval) {
             float* dst = draft_bias + ((size_t)b * K + k) * (size_t)V + v0;
@@ -493,7 +504,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         // ---- residual: sums of max(0, p_t - p_d) and of p_t per chunk
 #pragma unroll 1
         for (int ci = 0; ci < kCpg; ++ci) {
-          const int cb = eg * kCpg + ci;
+          const int cb = eg + kEpi * ci;
           float d[32], bv[32];
           if (wval) tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
           const int v0 = t * kTileN + cb * 32;
@@ -530,8 +541,6 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
               bv[4 * j] = b4.x; bv[4 * j + 1] = b4.y; bv[4 * j + 2] = b4.z; bv[4 * j + 3] = b4.w;
             }
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&emptyB[s]);
           float qs4[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ps4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
           if (bval) {
 #pragma unroll
@@ -544,16 +553,20 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             }
           }
           pp[ci] = make_float2((qs4[0] + qs4[1]) + (qs4[2] + qs4[3]), (ps4[0] + ps4[1]) + (ps4[2] + ps4[3]));
+          consumed(pp[ci].x);
+          consumed(pp[ci].y);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&emptyB[s]);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&accEmpty[a]);
-      if (bval) {
+      if (bval && part != nullptr) {
         float2* dst = part + (size_t)b * n_chunks;
 #pragma unroll
         for (int ci = 0; ci < kCpg; ++ci) {
-          const int c = t * (kTileN / 32) + eg * kCpg + ci;
+          const int c = t * (kTileN / 32) + eg + kEpi * ci;
           if (c < n_chunks) dst[c] = pp[ci];
         }
       }
@@ -704,35 +717,16 @@ inline void tc_set_attr() {
   set_smem_once(once, proj_tc_kernel<kRes>, (int)kTcSmemLimit);
 }
 
-// Launch configuration with programmatic stream serialisation: the kernel
-// may start while the one before it in the stream is still running, and
-// orders itself behind it with griddepcontrol.wait.
-struct PdlLaunch {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  PdlLaunch(unsigned grid, unsigned block, size_t smem, cudaStream_t s) {
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  }
-};
-
 inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const int32_t* tokens,
                             const float* it, float* dl, float* dbias, float2* part,
                             float2* cta_part, unsigned* flags, cudaStream_t s) {
   tc_set_attr<false>();
-  PdlLaunch L(p.n_bb * p.ctas_per_bb, tc_threads<false>(),
-              tc_smem_bytes(p.r, p.B, false, p.a_split), s);
-  cudaLaunchKernelEx(&L.cfg, proj_tc_kernel<false>, p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r,
-                     p.B, p.K, k, prev, tokens, it, (const float*)nullptr, p.base,
-                     (const ResInfo*)nullptr, dl, dbias, part, cta_part, n_chunks_of(p.V),
-                     p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, p.a_rows,
-                     p.a_split, flags);
+  proj_tc_kernel<false><<<p.n_bb * p.ctas_per_bb, tc_threads<false>(),
+                          tc_smem_bytes(p.r, p.B, false, p.a_split), s>>>(
+      p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r, p.B, p.K, k, prev, tokens, it,
+      (const float*)nullptr, p.base, (const ResInfo*)nullptr, dl, dbias, part, cta_part,
+      n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, p.a_rows,
+      p.a_split, flags);
 }
 
 inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,

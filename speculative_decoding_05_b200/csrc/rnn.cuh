@@ -34,10 +34,6 @@ rnn_state_kernel(const TW* __restrict__ U, const TW* __restrict__ R, int V, int 
                  __nv_bfloat16* __restrict__ a_rows, float* __restrict__ states_out,
                  unsigned* flags) {
   extern __shared__ float s_prev[];  // [r]
-  // a plain launch behind the previous position's sampler; the projection
-  // launched behind this kernel may start its W and base producers now
-  grid_dep_wait();
-  grid_dep_launch();
   const int b = blockIdx.x;
   int x = (k == 0) ? prev_token[b] : tokens[(size_t)b * K + (k - 1)];
   x = checked_token(x, V, k == 0, flags);

@@ -124,11 +124,6 @@ draft_sample_kernel(const float* __restrict__ base, const TW* __restrict__ U,
                     float* __restrict__ ref_sum, unsigned* flags) {
   __shared__ __align__(16) float u_s[kMaxRank];
   __shared__ float shf[32];
-  // The next position's projection is launched behind this kernel with a
-  // programmatic dependency; let it start its prologue once this kernel is
-  // running (the wait is a no-op for a plain launch).
-  grid_dep_wait();
-  grid_dep_launch();
   const int b = blockIdx.x;
   const float it = checked_inv_temp(inv_temp, b, flags);
   const float it2 = it * kLog2e;
@@ -299,10 +294,6 @@ draft_sample2_kernel(const float* __restrict__ base, const TW* __restrict__ U,
   // state [B, r] fp32 (RNN head): the re-computed bias is state[b] . W[v]
   // instead of U[x_prev] . W[v]
   __shared__ __align__(16) float u_s[kS2Warps][kMaxRank];
-  // the next position's projection is launched behind this kernel with a
-  // programmatic dependency: let its producers start now
-  grid_dep_wait();
-  grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x * kS2Warps + warp;
   if (b >= B) return;  // whole warps only; no block-wide synchronisation follows

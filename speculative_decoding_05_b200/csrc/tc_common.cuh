@@ -104,6 +104,21 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Bounded wait until the shared word *tag holds `want`: the fill number a
+// ring's producer writes into a stage's tag before it issues that fill.
+// Where consecutive fills of one stage go to different consumers, a parity
+// wait alone cannot tell fill f from fill f - 2 (the parities match); a
+// consumer that first sees its own fill number knows fill f - 1 has landed
+// and been released, so the parity wait that follows can only mean fill f.
+__device__ __forceinline__ bool tag_wait(const volatile int* tag, int want) {
+  if (*tag == want) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (*tag == want) return true;
+    if ((i & 1023u) == 0 && wait_expired(t0, i)) return false;
+  }
+}
+
 // Producer tail of a ring of `n` stages whose stage it % n was filled for
 // uses it = 0 .. issued - 1 and is released by a tcgen05.commit arrive on
 // empty[it % n]: waits until the last min(n, issued) uses are released.

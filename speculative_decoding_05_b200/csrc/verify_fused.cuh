@@ -258,6 +258,8 @@ __global__ void __launch_bounds__(kFThreads, 1) verify_fused_kernel(const FusedA
         if (inB) sb += e4;
         else sa += e4;
       }
+      consumed(sa);  // every read of this piece has returned
+      consumed(sb);
       merge_partial(mA, sA, ma, sa, it2A);
       merge_partial(mB, sB, mb, sb, it2B);
       __syncthreads();  // s_buf is refilled by the next piece
