@@ -44,3 +44,60 @@ def test_persistent_draft_repeats_bit_identically(oracle_mod, B):
         if f != 0 or not same:
             bad.append((i, f, same))
     assert not bad, bad[:10]
+
+
+def test_large_batch_step_repeats_bit_identically():
+    """The tensor-core draft and verify at the stress shape, repeated.
+
+    B = 512, V = 151936, K = 16: the projection streams base-logit boxes
+    through a shared-memory ring that its epilogue warps release for TMA
+    refills.  A stage released before every reader's loads have returned,
+    or a parity wait that takes another fill for its own, corrupts one
+    chunk for a warp's 32 requests -- an error of 1e-5 to 1e-3 in their
+    partition sums that the sampled tokens mostly hide.  Six draft calls
+    (eager, then graph replays, on a stream of their own) and two full
+    steps with the same inputs must give bit-identical tokens, p_tok, lse
+    and verify outputs.
+    """
+    w = WL.get("stress")
+    inp = WL.make_inputs(w, device="cuda")
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype)
+    assert step.path == "tcgen05"
+    s = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        step.run(inp, enable_prefix=True)
+    torch.cuda.synchronize()
+    assert all(f == 0 for f in step.flags().values())
+    draft_out = lambda: (step.tokens, step.p_tok, step.lse, step.ref_max, step.ref_sum)
+    verify_out = lambda: (step.n_accepted, step.out_tokens, step.last_token)
+    first_d = [t.clone() for t in draft_out()]
+    first_v = [t.clone() for t in verify_out()]
+    bad = []
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step.draft(inp)
+    for i in range(6):
+        with torch.cuda.stream(s):
+            if i < 2:
+                step.draft(inp)
+            else:
+                g.replay()
+        torch.cuda.synchronize()
+        f = D.dspark_get_device_flags(step.ws_draft)
+        diff = [j for j, (a, b) in enumerate(zip(first_d, draft_out())) if not torch.equal(a, b)]
+        if f != 0 or diff:
+            bad.append(("draft", i, f, diff))
+    del g
+    for i in range(2):
+        with torch.cuda.stream(s):
+            step.run(inp, enable_prefix=True)
+        torch.cuda.synchronize()
+        fl = step.flags()
+        diff = [j for j, (a, b) in enumerate(zip(first_d + first_v, draft_out() + verify_out()))
+                if not torch.equal(a, b)]
+        if any(fl.values()) or diff:
+            bad.append(("step", i, fl, diff))
+    assert not bad, bad
+    del inp, step
+    torch.cuda.empty_cache()
