@@ -34,9 +34,10 @@
 // Draft mode streams base[b, k, v0:v0+32] boxes through a second TMA ring.
 // Residual mode needs the per-request rows target[row_b, :] and
 // base[b, j_b, :] (j_b differs between requests): warp 2 fetches each
-// request's 128-byte segment of every 32-column chunk with TMA tile::gather4
-// loads (four rows of a one-row-high box per instruction) into a second
-// ring, unswizzled (rows at a 128-byte stride).  A gather through the
+// request's 256-byte segment of every kResCols = 64 columns (two chunks)
+// with TMA tile::gather4 loads (four rows of a one-row-high box per
+// instruction) into a second ring, unswizzled (rows at a 256-byte stride);
+// both warpgroups read every stage.  A gather through the
 // load/store units instead (per-thread loads, or 16-byte cp.async copies)
 // was capped near 5 GB/s per SM by the SM's outstanding misses.  The
 // epilogue thread of request m reads its row's 16-byte chunks starting at
@@ -61,6 +62,9 @@ __host__ __device__ constexpr int tc_epi_groups() { return 2; }
 template <bool kRes>
 __host__ __device__ constexpr int tc_threads() { return 96 + 128 * tc_epi_groups<kRes>(); }
 constexpr int kTileN = 128;
+// Columns of one residual stage: two 32-column chunks, so each gather4 load
+// moves four 256-byte row segments (the loads' issue rate bounds the mode).
+constexpr int kResCols = 64;
 constexpr int kWStagesMax = 12;     // W ring depth: as deep as shared memory allows
 constexpr int kBStagesMax = 16;     // base ring depth (draft): likewise
 constexpr int kStageBytes = 16384;  // 128 rows x 128 bytes
@@ -88,11 +92,14 @@ inline int tc_base_rows(int B) { return B < kBlockM ? (B + 7) / 8 * 8 : kBlockM;
 // Bytes of one k-block of operand A (and of one base box): the block's
 // request rows, 128 bytes each.  A multiple of 1024, the swizzle atom.
 inline size_t tc_a_stage_bytes(int B) { return (size_t)tc_base_rows(B) * 128; }
-// One stage of the second ring, per 32-column chunk: the base box (draft),
-// or the target and base segments of every request (residual).
+// One stage of the second ring: the base box of a 32-column chunk (draft),
+// or the target and base segments of kResCols columns of every request
+// (residual).
 inline size_t tc_r_stage_bytes(int B, bool residual) {
-  return (residual ? 2 : 1) * tc_a_stage_bytes(B);
+  return residual ? (size_t)2 * tc_base_rows(B) * kResCols * 4 : tc_a_stage_bytes(B);
 }
+// Stages of the second ring per tile.
+inline int tc_r_stages_per_tile(bool residual) { return residual ? kTileN / kResCols : kTileN / 32; }
 // Alignment slack, operand A (ra / 64 k-blocks, ra = r or a split state's
 // 2r columns) and the barriers.
 inline size_t tc_fixed_bytes(int ra, int B, bool residual) {
@@ -114,8 +121,9 @@ inline int tc_b_stages(int r, int B, bool residual, int a_split = 0) {
   const size_t ring = kTcSmemLimit - tc_fixed_bytes(r << a_split, B, residual);
   const size_t w_tile = (size_t)(r / 64) * kStageBytes;
   const size_t rstage = tc_r_stage_bytes(B, residual);
-  const size_t b_tile = (size_t)(kTileN / 32) * rstage;
+  const size_t b_tile = (size_t)tc_r_stages_per_tile(residual) * rstage;
   int s = (int)(ring * b_tile / (w_tile + b_tile) / rstage);
+  if (s < 2) s = 2;
   while (s > 2 && ring < (size_t)s * rstage + 2 * kStageBytes) --s;
   if (s > kBStagesMax) s = kBStagesMax;
   return s & ~1;
@@ -161,7 +169,10 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   const int bstage = base_rows * 128;  // bytes of one base box and of one k-block of A
   uint8_t* sW = sA + (ra >> 6) * bstage;
   uint8_t* sBase = sW + n_ws * kStageBytes;
-  const int rstage = (kRes ? 2 : 1) * bstage;  // one stage of the second ring
+  // one stage of the second ring; residual: target segments, then (at
+  // bhalf) base segments, kResCols columns of each request at a 256-byte stride
+  const int bhalf = base_rows * kResCols * 4;
+  const int rstage = kRes ? 2 * bhalf : bstage;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sBase + n_bs * rstage);
   uint64_t* fullW = bars;
   uint64_t* emptyW = fullW + kWStagesMax;
@@ -190,7 +201,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     }
     for (int i = 0; i < n_bs; ++i) {
       mbar_init(&fullB[i], 1);
-      mbar_init(&emptyB[i], 4);
+      // draft: the four warps of the chunk's warpgroup; residual: a stage
+      // holds one chunk of each warpgroup
+      mbar_init(&emptyB[i], kRes ? 4 * kEpi : 4);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&accFull[i], 1);
@@ -359,20 +372,20 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     for (int i = 0; i < nt && !*s_abort; ++i) {
       const int t = tile_at(i);
       bool ok = true;
-      for (int cb = 0; cb < kTileN / 32; ++cb, ++it) {
+      for (int cs = 0; cs < kTileN / kResCols; ++cs, ++it) {
         const int s = it % n_bs;
         const uint32_t ph = (uint32_t)(it / n_bs) & 1u;
         if (!__all_sync(0xffffffffu, mbar_wait(&emptyB[s], ph ^ 1u))) {
           ok = false;
           break;
         }
-        if (lane == 0) mbar_arrive_expect_tx(&fullB[s], (uint32_t)(2 * groups * 512));
+        if (lane == 0) mbar_arrive_expect_tx(&fullB[s], (uint32_t)(2 * groups * 4 * kResCols * 4));
         __syncwarp();
         if (lane < groups) {
-          const int v0 = t * kTileN + cb * 32;
-          uint8_t* st = sBase + s * rstage + lane * 512;
+          const int v0 = t * kTileN + cs * kResCols;
+          uint8_t* st = sBase + s * rstage + lane * (4 * kResCols * 4);
           tma_gather4_hint(st, &tm_tgt, &fullB[s], v0, trow[0], trow[1], trow[2], trow[3], pol);
-          tma_gather4_hint(st + bstage, &tm_base, &fullB[s], v0, brow[0], brow[1], brow[2], brow[3],
+          tma_gather4_hint(st + bhalf, &tm_base, &fullB[s], v0, brow[0], brow[1], brow[2], brow[3],
                            pol);
         }
       }
@@ -508,7 +521,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           float d[32], bv[32];
           if (wval) tmem_ld32(tmem + ((uint32_t)(quarter * 32) << 16) + a * kTileN + cb * 32, d);
           const int v0 = t * kTileN + cb * 32;
-          const int itB = i * (kTileN / 32) + cb;
+          const int itB = i * (kTileN / kResCols) + cb / (kResCols / 32);
           const int s = itB % n_bs;
           const uint32_t ph = (uint32_t)(itB / n_bs) & 1u;
           if (!mbar_wait(&fullB[s], ph)) {
@@ -517,7 +530,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           }
           // this request's segments, staged by warp 2 (m < base_rows when
           // bval): slot j holds chunk (j + rot) & 7, and the TMEM values are
-          // rotated to match (three select stages, static register indices)
+          // rotated to match (three select stages, static register indices).
+          // Rows sit at a 256-byte stride, so the rotation still sends the
+          // eight lanes of a shared-memory phase to eight bank groups.
           const int rot = lane & 7;
           float tq[32], dr[32];
           if (bval) {
@@ -527,8 +542,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
             for (int x = 0; x < 32; ++x) d[x] = (rot & 2) ? dr[(x + 8) & 31] : dr[x];
 #pragma unroll
             for (int x = 0; x < 32; ++x) dr[x] = (rot & 4) ? d[(x + 16) & 31] : d[x];
-            const uint8_t* trow = sBase + s * rstage + m * 128;
-            const uint8_t* brow = trow + bstage;
+            const uint8_t* trow = sBase + s * rstage + m * (kResCols * 4) + (cb % (kResCols / 32)) * 128;
+            const uint8_t* brow = trow + bhalf;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const int c = (j + rot) & 7;
@@ -632,14 +647,14 @@ inline bool encode_w_map(CUtensorMap* m, const void* W, int V, int r) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// rows [n, V] fp32 as 32 x 1 boxes (one row's 128-byte segment), no swizzle:
-// the box of a tile::gather4 load, which takes four rows at once.
+// rows [n, V] fp32 as kResCols x 1 boxes (one row's 256-byte segment), no
+// swizzle: the box of a tile::gather4 load, which takes four rows at once.
 inline bool encode_rows_map(CUtensorMap* m, const float* p, int V, long long rows) {
   auto enc = tensor_map_encoder();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)V, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)V * 4};
-  cuuint32_t box[2] = {32, 1};
+  cuuint32_t box[2] = {(cuuint32_t)kResCols, 1};
   cuuint32_t es[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(p), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
