@@ -69,7 +69,8 @@ constexpr int kWStagesMax = 12;     // W ring depth: as deep as shared memory al
 constexpr int kBStagesMax = 16;     // base ring depth (draft): likewise
 constexpr int kStageBytes = 16384;  // 128 rows x 128 bytes
 constexpr size_t kTcSmemLimit = 232448 - 1024;  // dynamic: 227 KB less the static arrays
-constexpr int kTmemCols = 256;
+constexpr int kTmemCols = 512;     // two 128-column accumulators, then operand A
+constexpr uint32_t kACol = 256;    // operand A's first column (ra / 2 columns)
 
 struct TcPlan {
   CUtensorMap tm_w;
@@ -100,11 +101,12 @@ inline size_t tc_r_stage_bytes(int B, bool residual) {
 }
 // Stages of the second ring per tile.
 inline int tc_r_stages_per_tile(bool residual) { return residual ? kTileN / kResCols : kTileN / 32; }
-// Alignment slack, operand A (ra / 64 k-blocks, ra = r or a split state's
-// 2r columns) and the barriers.
+// Alignment slack and the barriers (operand A lives in tensor memory).
 inline size_t tc_fixed_bytes(int ra, int B, bool residual) {
+  (void)ra;
+  (void)B;
   (void)residual;
-  return 1024 + (size_t)(ra / 64) * tc_a_stage_bytes(B) + 512;
+  return 1024 + 512;
 }
 // Ring depths.  Each copy in flight waits about the same time for its
 // bytes, so the two rings share what is left in proportion to what they
@@ -165,9 +167,8 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   // row of a_rows, r << a_split columns: a state split into bf16 high and
   // low parts, both multiplied by the same W block and accumulated
   const int ra = r << a_split;
-  uint8_t* sA = sm;
-  const int bstage = base_rows * 128;  // bytes of one base box and of one k-block of A
-  uint8_t* sW = sA + (ra >> 6) * bstage;
+  const int bstage = base_rows * 128;  // bytes of one base box
+  uint8_t* sW = sm;
   uint8_t* sBase = sW + n_ws * kStageBytes;
   // one stage of the second ring; residual: target segments, then (at
   // bhalf) base segments, kResCols columns of each request at a 256-byte stride
@@ -219,18 +220,17 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const bool producer = warp == 0 || warp == 2;
-
-  // operand A: the previous-token rows of U for this block of requests,
-  // gathered by the non-producer warps.  The 128 token ids go to shared
-  // memory first (one round of loads), then every thread issues all of its U
-  // loads before storing any, so the gather costs two memory round trips
-  // rather than one per loop iteration.
-  constexpr int kGather = tc_threads<kRes>() - 64;
-  const int gtid = warp == 1 ? lane : threadIdx.x - 64;  // 0..kGather-1 off the producers
-  __shared__ int s_x[kBlockM];
-  if (!producer && gtid < kBlockM) {
-    const int m = gtid;
+  // operand A -> tensor memory, written by the epilogue warps: lane = the
+  // request's row m, 32-bit column kACol + c holds the bf16 pair (2c, 2c + 1)
+  // of U[x_m] (or of its a_rows row); rows past the batch are zero.  A warp
+  // reaches only its lane quarter, so each warpgroup covers all 128 rows and
+  // takes every other 64-element unit of them; a lane loads and stores its
+  // units, 8 16-byte pieces per unit.  The MMA warp joins the barrier that
+  // ends the writes.
+  constexpr int kGather = tc_threads<kRes>() - 64;  // warp 1 + the epilogue warps
+  if (warp >= 3) {
+    const int eg = (warp - 3) >> 2;
+    const int m = (warp & 3) * 32 + lane;
     const int b = bb * kBlockM + m;
     int x = -1;
     if (b < B) {
@@ -247,35 +247,27 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         }
       }
     }
-    s_x[m] = x;
-  }
-  if (!producer) {
-    named_sync(1, kGather);
-    const int cpr = ra >> 3;  // 16-byte chunks per row
     const __nv_bfloat16* src = a_rows != nullptr ? a_rows : U;
-    constexpr int kPer = (kBlockM * 32 + kGather - 1) / kGather;  // 256 columns per pass
-    for (int q0 = 0; q0 < base_rows * cpr; q0 += kPer * kGather) {
-      uint4 val[kPer];
+    const uint4* row = reinterpret_cast<const uint4*>(src + (size_t)(x < 0 ? 0 : x) * ra);
+    const uint32_t lanes = tmem + ((uint32_t)((warp & 3) * 32) << 16) + kACol;
+    const int units = ra >> 6;  // 64 elements = 32 columns each
+    for (int u = eg; u < units; u += kEpi) {
+      uint32_t regs[32];
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int q = q0 + gtid + i * kGather;
-        val[i] = make_uint4(0, 0, 0, 0);
-        if (q < base_rows * cpr) {
-          const int x = s_x[q / cpr];
-          if (x >= 0) val[i] = __ldg(reinterpret_cast<const uint4*>(src + (size_t)x * ra) + (q % cpr));
-        }
+      for (int q = 0; q < 8; ++q) {
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (x >= 0) val = __ldg(row + u * 8 + q);
+        regs[4 * q] = val.x;
+        regs[4 * q + 1] = val.y;
+        regs[4 * q + 2] = val.z;
+        regs[4 * q + 3] = val.w;
       }
-#pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int q = q0 + gtid + i * kGather;
-        if (q < base_rows * cpr) {
-          const int m = q / cpr, c = q % cpr;
-          const int kb = c >> 3, j = c & 7;
-          *reinterpret_cast<uint4*>(sA + kb * bstage + m * 128 + ((j ^ (m & 7)) << 4)) = val[i];
-        }
-      }
+      tmem_st32(lanes + (uint32_t)(u * 32), regs);
     }
-    fence_proxy_async_smem();
+    tmem_st_wait();
+  }
+  if (warp == 1 || warp >= 3) {
+    tc_fence_before();
     named_sync(1, kGather);
   }
 
@@ -310,7 +302,7 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(kBlockM, kTileN);
-      const uint32_t a0 = smem_u32(sA), w0 = smem_u32(sW);
+      const uint32_t aT = tmem + kACol, w0 = smem_u32(sW);
       int it = 0;
       for (int i = 0; i < nt && !*s_abort; ++i) {
         const int a = i & 1;
@@ -333,9 +325,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
           for (int h = 0; h <= a_split; ++h) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(a0 + (h * nkb + kb) * bstage + kk * 32);
               const uint64_t bd = sdesc_sw128(w0 + s * kStageBytes + kk * 32);
-              mma_bf16_ss(tmem + a * kTileN, ad, bd, idesc, (kb | kk | h) != 0);
+              mma_bf16_ts(tmem + a * kTileN, aT + (uint32_t)(((h * nkb + kb) * 4 + kk) * 8), bd,
+                          idesc, (kb | kk | h) != 0);
             }
           }
           mma_commit(&emptyW[s]);
