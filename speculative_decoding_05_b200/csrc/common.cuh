@@ -47,6 +47,16 @@ inline void set_smem_once(DeviceOnce& once, Kern* kern, int bytes) {
   });
 }
 
+// Programmatic dependent launch.  grid_dep_wait blocks until the kernel
+// before this one in the stream has completed and its writes are visible
+// (it returns at once when this launch carries no programmatic dependency);
+// grid_dep_launch lets a kernel launched behind this one with that
+// dependency begin before this one ends.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // sizes and workspace layout
 // ---------------------------------------------------------------------------

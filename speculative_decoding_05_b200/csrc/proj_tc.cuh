@@ -17,11 +17,9 @@
 // partial locally -- no cross-thread reduction, because the request is the
 // TMEM lane.
 //
-// Launches are plain (stream-ordered).  A launch with programmatic stream
-// serialisation, which let the next position's producers fill the rings
-// while the sampler ran, gained about 3 % on the draft; it was taken out
-// while launch failures were traced, before the ring faults described at
-// tc_b_stages and at the epilogue's stage release were found.
+// The draft launch carries programmatic stream serialisation: the next
+// position's producers fill the rings while the sampler runs (see the
+// grid_dep_wait below); the residual launch is plain.
 //
 //   warp 0       W producer (TMA, evict-last: W is re-read every position)
 //   warp 1       TMEM allocator + MMA issuer (one thread)
@@ -219,6 +217,14 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
+  // The draft projection is launched with a programmatic dependency on the
+  // kernel before it (the previous position's sampler).  Every warp that
+  // reads what that kernel wrote (tokens, operand rows) or writes what it
+  // reads (the partials) waits for it here; the producers read only W and
+  // the base logits, which no kernel of the call writes, so from position 1
+  // on they start filling the rings at once.
+  if (warp == 1 || warp >= 3 || k == 0) grid_dep_wait();
 
   // operand A -> tensor memory, written by the epilogue warps: lane = the
   // request's row m, 32-bit column kACol + c holds the bf16 pair (2c, 2c + 1)
@@ -724,16 +730,28 @@ inline void tc_set_attr() {
   set_smem_once(once, proj_tc_kernel<kRes>, (int)kTcSmemLimit);
 }
 
+// The draft projection, launched with programmatic stream serialisation: it
+// may start while the kernel before it (the sampler) runs, and orders
+// itself behind it with griddepcontrol.wait.
 inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const int32_t* tokens,
                             const float* it, float* dl, float* dbias, float2* part,
                             float2* cta_part, unsigned* flags, cudaStream_t s) {
   tc_set_attr<false>();
-  proj_tc_kernel<false><<<p.n_bb * p.ctas_per_bb, tc_threads<false>(),
-                          tc_smem_bytes(p.r, p.B, false, p.a_split), s>>>(
-      p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r, p.B, p.K, k, prev, tokens, it,
-      (const float*)nullptr, p.base, (const ResInfo*)nullptr, dl, dbias, part, cta_part,
-      n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, p.a_rows,
-      p.a_split, flags);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = dim3(p.n_bb * p.ctas_per_bb);
+  cfg.blockDim = dim3(tc_threads<false>());
+  cfg.dynamicSmemBytes = tc_smem_bytes(p.r, p.B, false, p.a_split);
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, proj_tc_kernel<false>, p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r,
+                     p.B, p.K, k, prev, tokens, it, (const float*)nullptr, p.base,
+                     (const ResInfo*)nullptr, dl, dbias, part, cta_part, n_chunks_of(p.V),
+                     p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, p.a_rows,
+                     p.a_split, flags);
 }
 
 inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,

@@ -33,6 +33,9 @@ rnn_state_kernel(const TW* __restrict__ U, const TW* __restrict__ R, int V, int 
                  const float* __restrict__ h0, float* __restrict__ state,
                  __nv_bfloat16* __restrict__ a_rows, float* __restrict__ states_out,
                  unsigned* flags) {
+  // the projection of this position may begin launching (its producers
+  // read only W and the base logits; the rest of it waits for this kernel)
+  grid_dep_launch();
   extern __shared__ float s_prev[];  // [r]
   const int b = blockIdx.x;
   int x = (k == 0) ? prev_token[b] : tokens[(size_t)b * K + (k - 1)];

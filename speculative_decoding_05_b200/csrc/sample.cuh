@@ -294,6 +294,9 @@ draft_sample2_kernel(const float* __restrict__ base, const TW* __restrict__ U,
   // state [B, r] fp32 (RNN head): the re-computed bias is state[b] . W[v]
   // instead of U[x_prev] . W[v]
   __shared__ __align__(16) float u_s[kS2Warps][kMaxRank];
+  // the next position's projection may begin launching now (it waits for
+  // this kernel before it touches anything this kernel reads or writes)
+  grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x * kS2Warps + warp;
   if (b >= B) return;  // whole warps only; no block-wide synchronisation follows
