@@ -114,16 +114,18 @@ def whole_job_rate(units_per_rank: int, world: int, ms_max: float) -> float:
 
 # ---------------------------------------------------------------- traffic --
 
-def source_closure(root: str | None = None) -> list:
-    """The CUDA sources a kernel is built from: its header and every file it
-    includes, transitively (each kernel's header also holds its launcher);
-    every source when no header is named."""
+def source_closure(root=None) -> list:
+    """The CUDA sources a kernel is built from: its header (or each of a
+    list of headers) and every file they include, transitively (each
+    kernel's header also holds its launcher); every source when no header is
+    named."""
     import glob
     import re
     csrc = os.path.join(ROOT, "speculative_decoding_05_b200", "csrc")
     if root is None:
         return sorted(glob.glob(os.path.join(csrc, "*")))
-    seen, todo = set(), [os.path.join(csrc, root)]
+    roots = [root] if isinstance(root, str) else list(root)
+    seen, todo = set(), [os.path.join(csrc, r) for r in roots]
     while todo:
         f = os.path.normpath(todo.pop())
         if f in seen or not os.path.exists(f):
@@ -136,7 +138,7 @@ def source_closure(root: str | None = None) -> list:
     return sorted(seen)
 
 
-def source_digest(root: str | None = None) -> str:
+def source_digest(root=None) -> str:
     """Hash of the sources a stored DRAM-traffic figure depends on (see
     source_closure).  A figure is only valid for the kernel code it was
     measured on."""
