@@ -604,10 +604,11 @@ dspark_status dspark_confidence_prefix_async(const float* z, const float* temps,
   if (!cost_tokens || !cost_ms || !verify_len || !objective) return DSPARK_ERR_INVALID_ARG;
   if (B * K > 0 && (!z || !temps || !c || !survival)) return DSPARK_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  // survivals (fp64), two order buffers of the merge and the per-request counts
+  // the merge's two buffers of (survival fp64, candidate id) and the
+  // per-request counts
   const int n = B * K;
-  const size_t smem = (size_t)n * (sizeof(double) + 2 * sizeof(int)) + (size_t)B * sizeof(int);
-  constexpr int kPrefixSmemMax = kMaxCand * 16 + kMaxCand * 4;
+  const size_t smem = (size_t)n * 2 * (sizeof(double) + sizeof(int)) + (size_t)B * sizeof(int);
+  constexpr int kPrefixSmemMax = kMaxCand * 24 + kMaxCand * 4;
   static DeviceOnce once;
   set_smem_once(once, prefix_kernel<kPrefixThreads>, kPrefixSmemMax);
   if (smem > (size_t)kPrefixSmemMax) return DSPARK_ERR_UNSUPPORTED;

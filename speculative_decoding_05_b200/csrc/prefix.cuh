@@ -8,6 +8,9 @@
 // already a sorted run: the order is a merge of B runs, done as a merge tree
 // in shared memory (log2 B levels; each thread finds its output chunk's
 // split by a merge-path binary search, then merges it sequentially).  The
+// buffers carry the survival keys with the candidate ids: an earlier form
+// that merged ids and looked every key up by id spent 65 of its 86 us at
+// the stress shape in the merge.  The
 // expected-emitted-token prefix sums are a block scan in fp64, and the early
 // stop is the first index where E/t(N) does not increase.
 //
@@ -94,10 +97,13 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
               int32_t* budget_out, unsigned* flags) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int n = B * K;
-  double* surv = reinterpret_cast<double*>(smem_raw);          // [n], candidate k*B + b
-  int* ordA = reinterpret_cast<int*>(surv + n);                 // [n] candidate order
-  int* ordB = ordA + n;                                         // [n] merge buffer
-  int* lcount = ordB + n;                                       // [B]
+  // The merge buffers hold the keys themselves (survival, fp64) beside the
+  // candidate ids k*B + b, so a comparison reads no index first.
+  double* keyA = reinterpret_cast<double*>(smem_raw);  // [n]
+  double* keyB = keyA + n;                              // [n]
+  int* idxA = reinterpret_cast<int*>(keyB + n);         // [n]
+  int* idxB = idxA + n;                                 // [n]
+  int* lcount = idxB + n;                               // [B]
   __shared__ float s_xs[64], s_ys[64];
   __shared__ double shd[32];
   __shared__ int s_stop, s_budget;
@@ -122,21 +128,21 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
 
   // c = sigmoid(z / T_k), one candidate per thread, in fp64
   for (int o = tid; o < n; o += kT) {
-    const int b = o / K, k = o - b * K;
+    const int k = o % K;
     const double ck = 1.0 / (1.0 + exp(-(double)z[o] / (double)temps[k]));
     c_out[o] = (float)ck;
-    surv[k * B + b] = ck;
+    keyA[o] = ck;
   }
   __syncthreads();
   // survival = running product over k (one thread per request); request b's
-  // run of the merge starts at b * K
+  // run of the merge is b * K .. b * K + K - 1, already in order
   for (int b = tid; b < B; b += kT) {
     double run = 1.0;
     for (int k = 0; k < K; ++k) {
-      run *= surv[k * B + b];
+      run *= keyA[b * K + k];
       s_out[(size_t)b * K + k] = (float)run;
-      surv[k * B + b] = run;
-      ordA[b * K + k] = k * B + b;
+      keyA[b * K + k] = run;
+      idxA[b * K + k] = k * B + b;
     }
     lcount[b] = 0;
   }
@@ -144,7 +150,7 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
 
   if (!enable) {
     double e = 0.0;
-    for (int i = tid; i < n; i += kT) e += surv[i];
+    for (int i = tid; i < n; i += kT) e += keyA[i];
     const double E = (double)B + block_sum_d<kT>(e, shd);
     for (int b = tid; b < B; b += kT) verify_len[b] = K;
     if (tid == 0) {
@@ -157,14 +163,20 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   }
 
   // merge tree: runs of width w = K, 2K, 4K, ...; each level merges pairs
-  // of neighbouring runs from src into dst (an unpaired last run is copied)
-  auto before = [&](int ia, int ib) { return cand_before(surv[ia], ia, surv[ib], ib); };
-  int* src = ordA;
-  int* dst = ordB;
-  const int chunk = (n + kT - 1) / kT;  // outputs per thread and level
+  // of neighbouring runs from (skey, sidx) into (dkey, didx) (an unpaired
+  // last run is copied); the heads of the two runs stay in registers
+  double* skey = keyA;
+  int* sidx = idxA;
+  double* dkey = keyB;
+  int* didx = idxB;
+  // outputs per thread and level; odd, so the lanes of a warp writing their
+  // runs' k-th outputs (a stride of chunk elements) fall in different banks
+  const int chunk = ((n + kT - 1) / kT) | 1;
   for (long long w = K; w < n; w <<= 1) {
     const int o0 = min(tid * chunk, n), o1 = min(o0 + chunk, n);
     int i = 0, j = 0, a1 = 0, b1 = 0;  // cursors into the current pair's two runs
+    double ka = 0.0, kb = 0.0;
+    int ia = 0, ib = 0;
     int pair_end = -1;
     for (int o = o0; o < o1; ++o) {
       if (o >= pair_end) {
@@ -180,22 +192,36 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
         while (lo < hi) {
           const int mid = (lo + hi) >> 1;
           // does A[mid] come before B[q - mid - 1]?  then more of A is in
-          if (before(src[a0 + mid], src[b0 + q - mid - 1])) lo = mid + 1;
+          const int x = a0 + mid, y = b0 + q - mid - 1;
+          if (cand_before(skey[x], sidx[x], skey[y], sidx[y])) lo = mid + 1;
           else hi = mid;
         }
         i = a0 + lo;
         j = b0 + (q - lo);
+        if (i < a1) { ka = skey[i]; ia = sidx[i]; }
+        if (j < b1) { kb = skey[j]; ib = sidx[j]; }
       }
-      if (j >= b1 || (i < a1 && before(src[i], src[j]))) dst[o] = src[i++];
-      else dst[o] = src[j++];
+      if (j >= b1 || (i < a1 && cand_before(ka, ia, kb, ib))) {
+        dkey[o] = ka;
+        didx[o] = ia;
+        if (++i < a1) { ka = skey[i]; ia = sidx[i]; }
+      } else {
+        dkey[o] = kb;
+        didx[o] = ib;
+        if (++j < b1) { kb = skey[j]; ib = sidx[j]; }
+      }
     }
     __syncthreads();
-    int* t = src;
-    src = dst;
-    dst = t;
+    double* tk = skey;
+    skey = dkey;
+    dkey = tk;
+    int* ti = sidx;
+    sidx = didx;
+    didx = ti;
   }
-  const int* idx = src;  // candidates in order
-  auto key = [&](int i) { return surv[idx[i]]; };
+  const double* skeys = skey;  // survivals in order
+  const int* idx = sidx;       // their candidate ids
+  auto key = [&](int i) { return skeys[i]; };
 
   // E_i = B + sum of the first i survivals; each thread owns a contiguous run
   const int per = chunk;
