@@ -57,6 +57,27 @@ __device__ __forceinline__ void grid_dep_launch() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Launches kern<<<grid, block, smem, s>>>(args...) with programmatic stream
+// serialisation: the kernel may start while the one before it in the stream
+// runs (once every CTA of that one has called grid_dep_launch or exited),
+// and orders itself behind it with grid_dep_wait.  Every kernel argument is
+// passed explicitly (defaults do not apply through the pointer).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                    cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---------------------------------------------------------------------------
 // sizes and workspace layout
 // ---------------------------------------------------------------------------
@@ -232,6 +253,30 @@ __device__ __forceinline__ float4 ld_stream4(const float* p, uint64_t pol) {
 // projection's bias bit for bit on the CUDA-core path.
 template <typename TW>
 __device__ __forceinline__ float dot_row(const TW* __restrict__ wrow, const float* __restrict__ u, int r) {
+  if constexpr (sizeof(TW) == 2) {
+    if (r == 256) {
+      // the whole 512-byte row in one round of loads, then the same
+      // ascending-index FMA chain as the general loop below
+      uint4 q[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) q[i] = __ldg(reinterpret_cast<const uint4*>(wrow) + i);
+      float acc = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float4 ua = *reinterpret_cast<const float4*>(u + 8 * i);
+        const float4 ub = *reinterpret_cast<const float4*>(u + 8 * i + 4);
+        acc = fmaf(__uint_as_float(q[i].x << 16), ua.x, acc);
+        acc = fmaf(__uint_as_float(q[i].x & 0xffff0000u), ua.y, acc);
+        acc = fmaf(__uint_as_float(q[i].y << 16), ua.z, acc);
+        acc = fmaf(__uint_as_float(q[i].y & 0xffff0000u), ua.w, acc);
+        acc = fmaf(__uint_as_float(q[i].z << 16), ub.x, acc);
+        acc = fmaf(__uint_as_float(q[i].z & 0xffff0000u), ub.y, acc);
+        acc = fmaf(__uint_as_float(q[i].w << 16), ub.z, acc);
+        acc = fmaf(__uint_as_float(q[i].w & 0xffff0000u), ub.w, acc);
+      }
+      return acc;
+    }
+  }
   float acc = 0.0f;
   for (int i0 = 0; i0 < r; i0 += 64) {
     // issue up to eight independent 16-byte loads before using any of them

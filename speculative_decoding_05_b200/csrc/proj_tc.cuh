@@ -737,21 +737,12 @@ inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const i
                             const float* it, float* dl, float* dbias, float2* part,
                             float2* cta_part, unsigned* flags, cudaStream_t s) {
   tc_set_attr<false>();
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.gridDim = dim3(p.n_bb * p.ctas_per_bb);
-  cfg.blockDim = dim3(tc_threads<false>());
-  cfg.dynamicSmemBytes = tc_smem_bytes(p.r, p.B, false, p.a_split);
-  cfg.stream = s;
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, proj_tc_kernel<false>, p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r,
-                     p.B, p.K, k, prev, tokens, it, (const float*)nullptr, p.base,
-                     (const ResInfo*)nullptr, dl, dbias, part, cta_part, n_chunks_of(p.V),
-                     p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, p.a_rows,
-                     p.a_split, flags);
+  launch_dependent(proj_tc_kernel<false>, dim3(p.n_bb * p.ctas_per_bb), dim3(tc_threads<false>()),
+                   tc_smem_bytes(p.r, p.B, false, p.a_split), s, p.tm_w, p.tm_base, p.tm_tgt, p.U,
+                   p.V, p.r, p.B, p.K, k, prev, tokens, it, (const float*)nullptr, p.base,
+                   (const ResInfo*)nullptr, dl, dbias, part, cta_part, n_chunks_of(p.V),
+                   p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, p.a_rows,
+                   p.a_split, flags);
 }
 
 inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,

@@ -295,7 +295,9 @@ draft_sample2_kernel(const float* __restrict__ base, const TW* __restrict__ U,
   // instead of U[x_prev] . W[v]
   __shared__ __align__(16) float u_s[kS2Warps][kMaxRank];
   // the next position's projection may begin launching now (it waits for
-  // this kernel before it touches anything this kernel reads or writes)
+  // this kernel before it touches anything this kernel reads or writes).
+  // This kernel itself is a plain launch: launching it behind the
+  // projection with a dependency as well measured 10 % slower on the draft.
   grid_dep_launch();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.x * kS2Warps + warp;
