@@ -80,6 +80,7 @@ struct TcPlan {
   int V, r, B, K;
   int n_tiles, n_bb, ctas_per_bb;
   int w_stages, b_stages, base_rows;  // ring depths, request rows per base box
+  int w_group;                        // W k-blocks per ring stage
   const __nv_bfloat16* a_rows;        // draft: per-request A rows (split state) or NULL
   int a_split;                         // 1: a_rows hold 2r columns (high, low halves)
 };
@@ -155,7 +156,10 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
                float* __restrict__ draft_logits, float* __restrict__ draft_bias,
                float2* __restrict__ part, float2* __restrict__ cta_part, int n_chunks,
                int n_tiles, int ctas_per_bb, int n_ws, int n_bs, int base_rows,
-               const __nv_bfloat16* __restrict__ a_rows, int a_split, unsigned* flags) {
+               const __nv_bfloat16* __restrict__ a_rows, int a_split, int w_group,
+               unsigned* flags) {
+  // n_ws: W ring space in 16 KB k-block units; w_group: k-blocks per ring
+  // stage (one barrier pair, one commit), so the ring has n_ws / w_group stages
   constexpr int kEpi = tc_epi_groups<kRes>();
   constexpr int kCpg = (kTileN / 32) / kEpi;  // chunks of a tile per epilogue warpgroup
   extern __shared__ uint8_t smem_raw[];
@@ -282,18 +286,22 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();
       int it = 0;
+      const int ngrp = (nkb + w_group - 1) / w_group, nslot = n_ws / w_group;
       for (int i = 0; i < nt && !*s_abort; ++i) {
         const int t = tile_at(i);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % n_ws;
-          const uint32_t ph = (uint32_t)(it / n_ws) & 1u;
+        for (int g = 0; g < ngrp; ++g, ++it) {
+          const int s = it % nslot;
+          const uint32_t ph = (uint32_t)(it / nslot) & 1u;
           if (!mbar_wait(&emptyW[s], ph ^ 1u)) {
             *s_abort = 1;
             raise_flag(flags, DSPARK_FLAG_TIMEOUT);
             break;
           }
-          mbar_arrive_expect_tx(&fullW[s], kStageBytes);
-          tma_load_2d_hint(sW + s * kStageBytes, &tm_w, &fullW[s], kb * 64, t * kTileN, pol);
+          const int nk = min(w_group, nkb - g * w_group);
+          mbar_arrive_expect_tx(&fullW[s], (uint32_t)(nk * kStageBytes));
+          for (int h = 0; h < nk; ++h)
+            tma_load_2d_hint(sW + (s * w_group + h) * kStageBytes, &tm_w, &fullW[s],
+                             (g * w_group + h) * 64, t * kTileN, pol);
         }
       }
       // Tail: a stage is released by a commit of the MMAs that read it, an
@@ -301,14 +309,15 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       // complete.  Wait for the releases of the last stages filled, so the
       // CTA never exits with such an arrive still in flight; after an abort,
       // wait for the copies still in flight instead.
-      if (!*s_abort) wait_ring_released(emptyW, n_ws, it, flags);
-      else drain_ring_loads(fullW, n_ws, it);
+      if (!*s_abort) wait_ring_released(emptyW, nslot, it, flags);
+      else drain_ring_loads(fullW, nslot, it);
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(kBlockM, kTileN);
       const uint32_t aT = tmem + kACol, w0 = smem_u32(sW);
+      const int ngrp = (nkb + w_group - 1) / w_group, nslot = n_ws / w_group;
       int it = 0;
       for (int i = 0; i < nt && !*s_abort; ++i) {
         const int a = i & 1;
@@ -320,20 +329,24 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
         }
         tc_fence_after();
         bool ok = true;
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = it % n_ws;
-          const uint32_t ph = (uint32_t)(it / n_ws) & 1u;
+        for (int g = 0; g < ngrp; ++g, ++it) {
+          const int s = it % nslot;
+          const uint32_t ph = (uint32_t)(it / nslot) & 1u;
           if (!mbar_wait(&fullW[s], ph)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          for (int h = 0; h <= a_split; ++h) {
+          const int nk = min(w_group, nkb - g * w_group);
+          for (int hk = 0; hk < nk; ++hk) {
+            const int kb = g * w_group + hk;
+            for (int h = 0; h <= a_split; ++h) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bd = sdesc_sw128(w0 + s * kStageBytes + kk * 32);
-              mma_bf16_ts(tmem + a * kTileN, aT + (uint32_t)(((h * nkb + kb) * 4 + kk) * 8), bd,
-                          idesc, (kb | kk | h) != 0);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t bd = sdesc_sw128(w0 + (s * w_group + hk) * kStageBytes + kk * 32);
+                mma_bf16_ts(tmem + a * kTileN, aT + (uint32_t)(((h * nkb + kb) * 4 + kk) * 8), bd,
+                            idesc, (kb | kk | h) != 0);
+              }
             }
           }
           mma_commit(&emptyW[s]);
@@ -672,6 +685,16 @@ inline bool encode_base_map(CUtensorMap* m, const float* base, int V, int K, int
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// k-blocks per W ring stage: a whole tile's (one wait and one commit per
+// tile in the MMA thread, which issues every MMA and commit of the CTA:
+// 1, 2 and 4 k-blocks per stage measured 1.61, 1.57 and 1.56 ms for the
+// stress draft), halved until the ring still holds two stages.
+inline int tc_w_group(int r, int w_units) {
+  int g = r / 64;
+  while (g > 1 && w_units / g < 2) g = (g + 1) / 2;
+  return g;
+}
+
 // CTAs per request block, at most this many (the workspace holds this many
 // partials per request and epilogue warpgroup).
 constexpr int kTcMaxCtasPerBlock = 256;
@@ -701,6 +724,7 @@ inline dspark_status tc_plan_draft(TcPlan& p, const float* base, const void* U, 
   tc_grid(p);
   p.w_stages = tc_w_stages(r, B, false, p.a_split);
   p.b_stages = tc_b_stages(r, B, false, p.a_split);
+  p.w_group = tc_w_group(r, p.w_stages);
   p.base_rows = tc_base_rows(B);
   return DSPARK_OK;
 }
@@ -720,6 +744,7 @@ inline dspark_status tc_plan_residual(TcPlan& p, const float* target, long long 
   tc_grid(p);
   p.w_stages = tc_w_stages(r, B, true);
   p.b_stages = tc_b_stages(r, B, true);
+  p.w_group = tc_w_group(r, p.w_stages);
   p.base_rows = tc_base_rows(B);
   return DSPARK_OK;
 }
@@ -742,7 +767,7 @@ inline void tc_launch_draft(const TcPlan& p, int k, const int32_t* prev, const i
                    p.V, p.r, p.B, p.K, k, prev, tokens, it, (const float*)nullptr, p.base,
                    (const ResInfo*)nullptr, dl, dbias, part, cta_part, n_chunks_of(p.V),
                    p.n_tiles, p.ctas_per_bb, p.w_stages, p.b_stages, p.base_rows, p.a_rows,
-                   p.a_split, flags);
+                   p.a_split, p.w_group, flags);
 }
 
 inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float* it,
@@ -752,7 +777,8 @@ inline void tc_launch_residual(const TcPlan& p, const ResInfo* info, const float
                          s>>>(p.tm_w, p.tm_base, p.tm_tgt, p.U, p.V, p.r, p.B, p.K, 0, nullptr,
                               nullptr, it, p.target, p.base, info, nullptr, nullptr, rpart,
                               nullptr, n_chunks_of(p.V), p.n_tiles, p.ctas_per_bb, p.w_stages,
-                              p.b_stages, p.base_rows, (const __nv_bfloat16*)nullptr, 0, flags);
+                              p.b_stages, p.base_rows, (const __nv_bfloat16*)nullptr, 0,
+                              p.w_group, flags);
 }
 
 }  // namespace dspark
