@@ -40,8 +40,9 @@
  *     between calls.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Every call only enqueues work on it: no host
- *     synchronisation, fixed launch shapes for fixed sizes, so a whole
- *     step can be captured in a CUDA graph.
+ *     synchronisation, fixed launch shapes for fixed sizes.  The calls that
+ *     take a workspace can be captured in a CUDA graph (the benchmark
+ *     replays whole steps that way).
  *   - Argument errors (NULL required pointers, bad sizes, misaligned
  *     pointers, too small workspace) are reported synchronously by the
  *     return value, before anything is enqueued.
@@ -401,9 +402,9 @@ dspark_status dspark_verify_lmhead(
  * is about B <= 50 requests; B <= 16, K <= 16 always fits).
  *
  * Set-up: the first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) with that device current and caches it; make that
- * first call before any stream capture.  The function allocates nothing
- * (no cudaMalloc, no cudaFree, no allocating library call).
+ * (cudaGetSymbolAddress) with that device current and caches it.  The
+ * function allocates nothing (no cudaMalloc, no cudaFree, no allocating
+ * library call).
  *
  * Sharing: every call on a device uses the same array and leaves its
  * contents behind; each call clears the part that must start at zero (the
