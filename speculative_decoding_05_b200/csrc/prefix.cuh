@@ -5,10 +5,10 @@
 // survival descending, ties by candidate index k*B + b ascending (position
 // then request).  Survival never rises along a request's positions (each
 // step multiplies by c in (0, 1]), so each request's K candidates are
-// already a sorted run: the order is a merge of B runs, done as a merge tree
-// in shared memory (log2 B levels; each thread finds its output chunk's
-// split by a merge-path binary search, then merges it sequentially).  The
-// buffers carry the survival keys with the candidate ids: an earlier form
+// already a sorted run.  Blocks of 256 or 512 candidates are sorted by one
+// warp each (a bitonic network in registers and shuffles), then merged as a
+// tree in shared memory (each thread finds its output chunk's split by a
+// merge-path binary search, then merges it sequentially).  The buffers carry the survival keys with the candidate ids: an earlier form
 // that merged ids and looked every key up by id spent 65 of its 86 us at
 // the stress shape in the merge.  The
 // expected-emitted-token prefix sums are a block scan in fp64, and the early
@@ -87,6 +87,71 @@ __device__ __forceinline__ bool cand_before(double sa, int ia, double sb, int ib
   return sa > sb || (sa == sb && ia < ib);
 }
 
+// Sorts the elements [e0, e0 + 32 kE) of (key, idx) in place by cand_before
+// with a bitonic network run by one warp: lane l holds elements e0 + kE l ..
+// e0 + kE l + kE - 1 in registers; exchanges at distances below kE stay
+// inside a lane, longer ones cross lanes by shuffles.  Elements at or past
+// n are padding that sorts last and is not written back.  cand_before is a
+// strict total order on distinct ids, so the result is the unique sorted
+// order.
+template <int kE>
+__device__ __forceinline__ void warp_sort(double* key, int* idx, int e0, int n) {
+  constexpr int kN = 32 * kE;
+  const int lane = threadIdx.x & 31;
+  double kv[kE];
+  int iv[kE];
+#pragma unroll
+  for (int i = 0; i < kE; ++i) {
+    const int e = e0 + kE * lane + i;
+    kv[i] = e < n ? key[e] : -1.0;  // survivals are >= 0
+    iv[i] = e < n ? idx[e] : 0x7fffffff;
+  }
+#pragma unroll
+  for (int sz = 2; sz <= kN; sz <<= 1) {
+#pragma unroll
+    for (int d = sz >> 1; d > 0; d >>= 1) {
+      if (d >= kE) {
+        const int ld = d / kE;
+        const bool lower = (lane & ld) == 0;
+#pragma unroll
+        for (int i = 0; i < kE; ++i) {
+          const bool up = ((kE * lane + i) & sz) == 0;
+          const double pk = __shfl_xor_sync(0xffffffffu, kv[i], ld);
+          const int pi = __shfl_xor_sync(0xffffffffu, iv[i], ld);
+          const bool mine_first = cand_before(kv[i], iv[i], pk, pi);
+          if (!((lower == up) ? mine_first : !mine_first)) {
+            kv[i] = pk;
+            iv[i] = pi;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < kE; ++i) {
+          if (i & d) continue;
+          const int j = i | d;
+          const bool up = ((kE * lane + i) & sz) == 0;
+          if (cand_before(kv[i], iv[i], kv[j], iv[j]) != up) {
+            const double tk = kv[i];
+            kv[i] = kv[j];
+            kv[j] = tk;
+            const int ti = iv[i];
+            iv[i] = iv[j];
+            iv[j] = ti;
+          }
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kE; ++i) {
+    const int e = e0 + kE * lane + i;
+    if (e < n) {
+      key[e] = kv[i];
+      idx[e] = iv[i];
+    }
+  }
+}
+
 template <int kT>
 __global__ void __launch_bounds__(kT)
 prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
@@ -131,20 +196,22 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     const int k = o % K;
     const double ck = 1.0 / (1.0 + exp(-(double)z[o] / (double)temps[k]));
     c_out[o] = (float)ck;
-    keyA[o] = ck;
+    keyB[o] = ck;
   }
+  for (int b = tid; b < B; b += kT) lcount[b] = 0;
   __syncthreads();
-  // survival = running product over k (one thread per request); request b's
-  // run of the merge is b * K .. b * K + K - 1, already in order
-  for (int b = tid; b < B; b += kT) {
+  // survival = running product over k: candidate (b, k) multiplies its
+  // request's c values 0..k in order, the product a sequential loop forms,
+  // so neighbouring threads write neighbouring words (one thread per
+  // request, striding K words, met many-way bank conflicts).  Request b's
+  // run of the merge is b * K .. b * K + K - 1, already in order.
+  for (int o = tid; o < n; o += kT) {
+    const int b = o / K, k = o - b * K;
     double run = 1.0;
-    for (int k = 0; k < K; ++k) {
-      run *= keyA[b * K + k];
-      s_out[(size_t)b * K + k] = (float)run;
-      keyA[b * K + k] = run;
-      idxA[b * K + k] = k * B + b;
-    }
-    lcount[b] = 0;
+    for (int j = 0; j <= k; ++j) run *= keyB[b * K + j];
+    s_out[o] = (float)run;
+    keyA[o] = run;
+    idxA[o] = k * B + b;
   }
   __syncthreads();
 
@@ -162,9 +229,19 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     return;
   }
 
-  // merge tree: runs of width w = K, 2K, 4K, ...; each level merges pairs
-  // of neighbouring runs from (skey, sidx) into (dkey, didx) (an unpaired
-  // last run is copied); the heads of the two runs stay in registers
+  // blocks of kWarpSort candidates sorted by one warp each in registers
+  // (the merge levels they replace, runs of K up to kWarpSort, cost about
+  // 5 us each in shared memory), then a merge tree from runs of width
+  // w = kWarpSort: each level merges pairs of neighbouring runs from
+  // (skey, sidx) into (dkey, didx) (an unpaired last run is copied); the
+  // heads of the two runs stay in registers
+  // elements per lane: 8 where the register budget is 64 per thread (1024
+  // threads), else 16
+  constexpr int kE = kT >= 1024 ? 8 : 16;
+  constexpr int kWarpSort = 32 * kE;
+  for (int e0 = (tid >> 5) * kWarpSort; e0 < n; e0 += (kT >> 5) * kWarpSort)
+    warp_sort<kE>(keyA, idxA, e0, n);
+  __syncthreads();
   double* skey = keyA;
   int* sidx = idxA;
   double* dkey = keyB;
@@ -172,7 +249,7 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   // outputs per thread and level; odd, so the lanes of a warp writing their
   // runs' k-th outputs (a stride of chunk elements) fall in different banks
   const int chunk = ((n + kT - 1) / kT) | 1;
-  for (long long w = K; w < n; w <<= 1) {
+  for (long long w = kWarpSort; w < n; w <<= 1) {
     const int o0 = min(tid * chunk, n), o1 = min(o0 + chunk, n);
     int i = 0, j = 0, a1 = 0, b1 = 0;  // cursors into the current pair's two runs
     double ka = 0.0, kb = 0.0;
