@@ -515,10 +515,9 @@ size_t dspark_verify_workspace_size(int V, int r, int B, int K) {
 }
 
 size_t dspark_prefix_workspace_size(int B, int K, int n_pts) {
-  (void)B;
-  (void)K;
   (void)n_pts;
-  return kHeaderBytes;
+  if (B < 0 || K < 0 || (long long)B * K > kMaxCand) return kHeaderBytes;
+  return prefix_ws_bytes(B * K);
 }
 
 dspark_status dspark_draft_markov(const float* base_logits, const void* U, const void* W,
@@ -604,9 +603,40 @@ dspark_status dspark_confidence_prefix_async(const float* z, const float* temps,
   if (!cost_tokens || !cost_ms || !verify_len || !objective) return DSPARK_ERR_INVALID_ARG;
   if (B * K > 0 && (!z || !temps || !c || !survival)) return DSPARK_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int n = B * K;
+  const PrefixArgs a{z, temps, cost_tokens, cost_ms, n_pts, staircase, B, K, enable,
+                     budget_in, c, survival, verify_len, objective, budget_out,
+                     static_cast<unsigned*>(workspace)};
+  if (prefix_multi(n, enable)) {
+    // survival pass, then the rank pass behind it (dependent launch); the
+    // survival pass clears the status word and the rank counter
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    double* surv = reinterpret_cast<double*>(ws + kHeaderBytes);
+    double* okey = reinterpret_cast<double*>(ws + kHeaderBytes + align256((size_t)n * 8));
+    int* oidx = reinterpret_cast<int*>(ws + kHeaderBytes + 2 * align256((size_t)n * 8));
+    unsigned* counter = reinterpret_cast<unsigned*>(ws + kPrefixCounterOff);
+    static DeviceOnce once_multi;
+    once_per_device(once_multi, [] {
+      cudaFuncSetAttribute(prefix_surv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kMaxCand * (int)sizeof(double));
+      cudaFuncSetAttribute(prefix_rank_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           kMaxCand * 16);
+    });
+    const int rb = K >= kSurvThreads ? 1 : kSurvThreads / K;
+    prefix_surv_kernel<<<(B + rb - 1) / rb, kSurvThreads, (size_t)rb * K * sizeof(double), s>>>(
+        a, surv, counter);
+    dspark_status st = check_launch();
+    if (st != DSPARK_OK) return st;
+    // the last CTA's copy of the order and the per-request counts
+    const size_t smem = (size_t)n * (sizeof(double) + sizeof(int)) + (size_t)B * sizeof(int);
+    if (launch_dependent(prefix_rank_kernel, dim3((n + kRankSlice - 1) / kRankSlice),
+                         dim3(kRankThreads), smem, s, a, static_cast<const double*>(surv), okey,
+                         oidx, counter) != cudaSuccess)
+      return DSPARK_ERR_CUDA;
+    return check_launch();
+  }
   // the merge's two buffers of (survival fp64, candidate id) and the
   // per-request counts
-  const int n = B * K;
   const size_t smem = (size_t)n * 2 * (sizeof(double) + sizeof(int)) + (size_t)B * sizeof(int);
   constexpr int kPrefixSmemMax = kMaxCand * 24 + kMaxCand * 4;
   static DeviceOnce once;
@@ -614,13 +644,9 @@ dspark_status dspark_confidence_prefix_async(const float* z, const float* temps,
   if (smem > (size_t)kPrefixSmemMax) return DSPARK_ERR_UNSUPPORTED;
   // the kernel clears the status word itself (one CTA: before any flag is raised)
   if (n <= kPrefixSmallCand)
-    prefix_kernel<kPrefixThreadsSmall><<<1, kPrefixThreadsSmall, smem, s>>>(
-        z, temps, cost_tokens, cost_ms, n_pts, staircase, B, K, enable, budget_in, c, survival,
-        verify_len, objective, budget_out, static_cast<unsigned*>(workspace));
+    prefix_kernel<kPrefixThreadsSmall><<<1, kPrefixThreadsSmall, smem, s>>>(a);
   else
-    prefix_kernel<kPrefixThreads><<<1, kPrefixThreads, smem, s>>>(
-        z, temps, cost_tokens, cost_ms, n_pts, staircase, B, K, enable, budget_in, c, survival,
-        verify_len, objective, budget_out, static_cast<unsigned*>(workspace));
+    prefix_kernel<kPrefixThreads><<<1, kPrefixThreads, smem, s>>>(a);
   return check_launch();
 }
 

@@ -1,18 +1,25 @@
 // prefix.cuh -- sequential temperature scaling, survival and the greedy
-// hardware-aware prefix cut, in one CTA.
+// hardware-aware prefix cut.
 //
 // The whole batch has at most kMaxCand = 8192 candidates (B*K), ordered by
 // survival descending, ties by candidate index k*B + b ascending (position
 // then request).  Survival never rises along a request's positions (each
 // step multiplies by c in (0, 1]), so each request's K candidates are
-// already a sorted run.  Blocks of 256 or 512 candidates are sorted by one
-// warp each (a bitonic network in registers and shuffles), then merged as a
-// tree in shared memory (each thread finds its output chunk's split by a
-// merge-path binary search, then merges it sequentially).  The buffers carry the survival keys with the candidate ids: an earlier form
-// that merged ids and looked every key up by id spent 65 of its 86 us at
-// the stress shape in the merge.  The
-// expected-emitted-token prefix sums are a block scan in fp64, and the early
-// stop is the first index where E/t(N) does not increase.
+// already a sorted run.  Two forms give the same order and outputs:
+//  - one CTA (up to kPrefixSmallCand candidates, or the scheduler off):
+//    blocks of 256 or 512 candidates are sorted by one warp each (a bitonic
+//    network in registers and shuffles), then merged as a tree in shared
+//    memory (each thread finds its output chunk's split by a merge-path
+//    binary search, then merges it sequentially).  The buffers carry the
+//    survival keys with the candidate ids: an earlier form that merged ids
+//    and looked every key up by id spent 65 of its 86 us at the stress
+//    shape in the merge.
+//  - many CTAs (more candidates): each places a slice of at most 63
+//    candidates in the order by counting, for every candidate, how many
+//    slice members precede it (see prefix_rank_kernel); the last CTA runs
+//    the scan.
+// The expected-emitted-token prefix sums are a block scan in fp64, and the
+// early stop is the first index where E/t(N) does not increase.
 //
 // Asynchronous budget (yage.ai, engineering paragraph: how many tokens a
 // step verifies is decided from the confidences of two steps back, which
@@ -152,16 +159,112 @@ __device__ __forceinline__ void warp_sort(double* key, int* idx, int e0, int n) 
   }
 }
 
+// Arguments of the prefix-cut kernels (device pointers; see the C entry
+// dspark_confidence_prefix_async).
+struct PrefixArgs {
+  const float* z;
+  const float* temps;
+  const float* cost_tokens;
+  const float* cost_ms;
+  int n_pts, staircase, B, K, enable;
+  const int32_t* budget_in;
+  float* c_out;
+  float* s_out;
+  int32_t* verify_len;
+  float* objective;
+  int32_t* budget_out;
+  unsigned* flags;
+};
+
+// The cost table into shared memory (thread 0 checks that it ascends), the
+// budget of this call (read before any budget_out write) and the stop index
+// preset to n.  Contains one barrier.
 template <int kT>
-__global__ void __launch_bounds__(kT)
-prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
-              const float* __restrict__ cost_tokens, const float* __restrict__ cost_ms, int n_pts,
-              int staircase, int B, int K, int enable, const int32_t* budget_in,
-              float* __restrict__ c_out, float* __restrict__ s_out,
-              int32_t* __restrict__ verify_len, float* __restrict__ objective,
-              int32_t* budget_out, unsigned* flags) {
+__device__ __forceinline__ void prefix_setup(const PrefixArgs& a, float* s_xs, float* s_ys,
+                                             int* s_budget, int* s_stop, int n) {
+  for (int i = threadIdx.x; i < a.n_pts; i += kT) {
+    s_xs[i] = a.cost_tokens[i];
+    s_ys[i] = a.cost_ms[i];
+  }
+  if (threadIdx.x == 0) *s_budget = a.budget_in != nullptr ? *a.budget_in : -1;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    bool ok = true;
+    for (int i = 0; i + 1 < a.n_pts; ++i) ok = ok && (s_xs[i + 1] > s_xs[i]);
+    if (!ok) raise_flag(a.flags, DSPARK_FLAG_BAD_TABLE);
+    *s_stop = n;
+  }
+}
+
+// The greedy scan and the commit over the candidates in order (survivals
+// skeys, candidate ids idx = k*B + b), in one CTA of kT threads.  lcount
+// [B] must be zero and every input visible to the block on entry.
+template <int kT>
+__device__ __forceinline__ void prefix_cut(const PrefixArgs& a, const double* skeys,
+                                           const int* idx, int* lcount, const float* s_xs,
+                                           const float* s_ys, int budget, int* s_stop,
+                                           double* shd) {
+  const int B = a.B, n = a.B * a.K, tid = threadIdx.x;
+  // E_i = B + sum of the first i survivals; each thread owns a contiguous run
+  const int per = ((n + kT - 1) / kT) | 1;
+  const int i0 = tid * per;
+  double run = 0.0;
+  for (int i = i0; i < i0 + per && i < n; ++i) run += skeys[i];
+  double total;
+  const double excl = block_excl_scan_d<kT>(run, shd, &total);
+  // candidate i (0-based) raises the objective iff E_{i+1}/t(B+i+1) >
+  // E_i/t(B+i); the right side is the left side of the step before
+  double E = (double)B + excl;
+  CostWalker cw{s_xs, s_ys, a.n_pts, a.staircase, 0};
+  double t0 = (i0 < n) ? cw.at((double)B + (double)i0) : 1.0;
+  double obj0 = E / t0;
+  for (int i = i0; i < i0 + per && i < n; ++i) {
+    const double t1 = cw.at((double)B + (double)i + 1.0);
+    const double E1 = E + skeys[i];
+    if (!(t0 > 0.0) || !(t1 > 0.0)) raise_flag(a.flags, DSPARK_FLAG_BAD_TABLE);
+    const double obj1 = E1 / t1;
+    if (!(obj1 > obj0)) {
+      atomicMin(s_stop, i);
+      break;
+    }
+    E = E1;
+    t0 = t1;
+    obj0 = obj1;
+  }
+  __syncthreads();
+  // the greedy cut, or the budget's (clamped to [0, n])
+  const int stop = *s_stop;
+  int n_commit = stop;
+  if (budget >= 0) {
+    const long long want = (long long)budget - B;
+    n_commit = want < 0 ? 0 : (want > n ? n : (int)want);
+  }
+  if (tid == 0 && a.budget_out != nullptr) *a.budget_out = B + stop;
+  for (int i = tid; i < n_commit; i += kT) {
+    const int id = idx[i];
+    if ((unsigned)id < (unsigned)n) atomicAdd(&lcount[id % B], 1);
+  }
+  __syncthreads();
+  for (int b = tid; b < B; b += kT) a.verify_len[b] = lcount[b];
+  // objective of the committed set: E at n_commit from the owning thread's run
+  const bool owner = (n_commit == n) ? (tid == 0) : (n_commit >= i0 && n_commit < i0 + per);
+  if (owner) {
+    double Ec = (double)B + total;
+    if (n_commit < n) {
+      Ec = (double)B + excl;
+      for (int i = i0; i < n_commit; ++i) Ec += skeys[i];
+    }
+    a.objective[0] =
+        (float)(Ec / cost_of(s_xs, s_ys, a.n_pts, a.staircase, (double)B + (double)n_commit));
+  }
+}
+
+// Single-CTA form: every step in one block (the form for up to
+// kPrefixSmallCand candidates, and for enable == 0).
+template <int kT>
+__global__ void __launch_bounds__(kT) prefix_kernel(const PrefixArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int n = B * K;
+  const int B = a.B, K = a.K, n = B * K;
   // The merge buffers hold the keys themselves (survival, fp64) beside the
   // candidate ids k*B + b, so a comparison reads no index first.
   double* keyA = reinterpret_cast<double*>(smem_raw);  // [n]
@@ -174,28 +277,14 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
   __shared__ int s_stop, s_budget;
   const int tid = threadIdx.x;
 
-  if (tid == 0) {
-    *flags = 0u;  // status of this call
-    s_budget = budget_in != nullptr ? *budget_in : -1;  // read before budget_out is written
-  }
-  // cost table into shared memory; it must be ascending in tokens
-  for (int i = tid; i < n_pts; i += kT) {
-    s_xs[i] = cost_tokens[i];
-    s_ys[i] = cost_ms[i];
-  }
-  __syncthreads();
-  if (tid == 0) {
-    bool ok = true;
-    for (int i = 0; i + 1 < n_pts; ++i) ok = ok && (s_xs[i + 1] > s_xs[i]);
-    if (!ok) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
-    s_stop = n;
-  }
+  if (tid == 0) *a.flags = 0u;  // status of this call
+  prefix_setup<kT>(a, s_xs, s_ys, &s_budget, &s_stop, n);
 
   // c = sigmoid(z / T_k), one candidate per thread, in fp64
   for (int o = tid; o < n; o += kT) {
     const int k = o % K;
-    const double ck = 1.0 / (1.0 + exp(-(double)z[o] / (double)temps[k]));
-    c_out[o] = (float)ck;
+    const double ck = 1.0 / (1.0 + exp(-(double)a.z[o] / (double)a.temps[k]));
+    a.c_out[o] = (float)ck;
     keyB[o] = ck;
   }
   for (int b = tid; b < B; b += kT) lcount[b] = 0;
@@ -209,22 +298,22 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     const int b = o / K, k = o - b * K;
     double run = 1.0;
     for (int j = 0; j <= k; ++j) run *= keyB[b * K + j];
-    s_out[o] = (float)run;
+    a.s_out[o] = (float)run;
     keyA[o] = run;
     idxA[o] = k * B + b;
   }
   __syncthreads();
 
-  if (!enable) {
+  if (!a.enable) {
     double e = 0.0;
     for (int i = tid; i < n; i += kT) e += keyA[i];
     const double E = (double)B + block_sum_d<kT>(e, shd);
-    for (int b = tid; b < B; b += kT) verify_len[b] = K;
+    for (int b = tid; b < B; b += kT) a.verify_len[b] = K;
     if (tid == 0) {
-      const double t = cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)n);
-      if (!(t > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
-      objective[0] = (float)(E / t);
-      if (budget_out != nullptr) *budget_out = B + n;
+      const double t = cost_of(s_xs, s_ys, a.n_pts, a.staircase, (double)B + (double)n);
+      if (!(t > 0.0)) raise_flag(a.flags, DSPARK_FLAG_BAD_TABLE);
+      a.objective[0] = (float)(E / t);
+      if (a.budget_out != nullptr) *a.budget_out = B + n;
     }
     return;
   }
@@ -296,53 +385,174 @@ prefix_kernel(const float* __restrict__ z, const float* __restrict__ temps,
     sidx = didx;
     didx = ti;
   }
-  const double* skeys = skey;  // survivals in order
-  const int* idx = sidx;       // their candidate ids
-  auto key = [&](int i) { return skeys[i]; };
+  prefix_cut<kT>(a, skey, sidx, lcount, s_xs, s_ys, s_budget, &s_stop, shd);
+}
 
-  // E_i = B + sum of the first i survivals; each thread owns a contiguous run
-  const int per = chunk;
-  const int i0 = tid * per;
-  double run = 0.0;
-  for (int i = i0; i < i0 + per && i < n; ++i) run += key(i);
-  double total;
-  const double excl = block_excl_scan_d<kT>(run, shd, &total);
-  // candidate i (0-based) raises the objective iff E_{i+1}/t(B+i+1) > E_i/t(B+i)
-  double E = (double)B + excl;
-  CostWalker cw{s_xs, s_ys, n_pts, staircase, 0};
-  double t0 = (i0 < n) ? cw.at((double)B + (double)i0) : 1.0;
-  for (int i = i0; i < i0 + per && i < n; ++i) {
-    const double t1 = cw.at((double)B + (double)i + 1.0);
-    const double E1 = E + key(i);
-    if (!(t0 > 0.0) || !(t1 > 0.0)) raise_flag(flags, DSPARK_FLAG_BAD_TABLE);
-    if (!(E1 / t1 > E / t0)) {
-      atomicMin(&s_stop, i);
-      break;
-    }
-    E = E1;
-    t0 = t1;
+// ---------------------------------------------------------------------------
+// Multi-CTA form (more than kPrefixSmallCand candidates, scheduler on)
+// ---------------------------------------------------------------------------
+//
+// The single CTA above is bound by one SM's issue rate (about 70 us for
+// 8192 candidates, most of it in the sort).  This form spreads the order
+// over the GPU:
+//   1. prefix_surv_kernel: c and survival exactly as prefix_kernel forms
+//      them, each CTA over whole requests; the fp64 survivals go to the
+//      workspace indexed by candidate id k*B + b.
+//   2. prefix_rank_kernel: CTA j takes the candidates with ids in
+//      [j n / G, (j+1) n / G) (at most kRankSlice) as its slice and sorts
+//      them in one warp.  For every candidate e of the batch, q(e) = the
+//      number of slice members that come before e (a binary search in
+//      shared memory).  e comes before slice member p exactly when
+//      q(e) <= p (e not p itself), so with h[q] = #{e : q(e) = q}, member p
+//      has h[0] + ... + h[p] - 1 candidates before it: its place in the
+//      order.  Each CTA writes its members' (survival, id) there; the last
+//      CTA to finish (a counter) reads the whole order back and runs
+//      prefix_cut, the same greedy scan as the single-CTA form.
+// The order is the same strict total order (a NaN survival ranks as -1,
+// after every real one, so the places stay a permutation), hence the same
+// outputs.
+
+constexpr int kSurvThreads = 256;
+constexpr int kRankThreads = kPrefixThreads;
+constexpr int kRankSlice = 63;  // slice members per CTA; slot 63 stays a sentinel
+constexpr int kRankPer = kMaxCand / kRankThreads;  // candidates per thread in the count
+// the rank pass's counter sits in the workspace header, after the status word
+constexpr size_t kPrefixCounterOff = 128;
+
+__device__ __forceinline__ double rank_key(double s) { return s == s ? s : -1.0; }
+
+__global__ void __launch_bounds__(kSurvThreads)
+prefix_surv_kernel(const PrefixArgs a, double* __restrict__ surv_id, unsigned* counter) {
+  extern __shared__ double s_c[];  // c of this CTA's requests
+  // the rank pass may be scheduled now; it waits for this grid to complete
+  grid_dep_launch();
+  const int B = a.B, K = a.K;
+  const int rb = max(1, kSurvThreads / K);  // requests per CTA
+  const int b0 = blockIdx.x * rb, nb = min(rb, B - b0);
+  const int m = nb * K;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *a.flags = 0u;  // status of this call
+    *counter = 0u;
+  }
+  for (int l = threadIdx.x; l < m; l += kSurvThreads) {
+    const int o = b0 * K + l, k = l % K;
+    const double ck = 1.0 / (1.0 + exp(-(double)a.z[o] / (double)a.temps[k]));
+    a.c_out[o] = (float)ck;
+    s_c[l] = ck;
   }
   __syncthreads();
-  // the greedy cut, or the budget's (clamped to [0, n])
-  int n_commit = s_stop;
-  if (s_budget >= 0) {
-    const long long want = (long long)s_budget - B;
-    n_commit = want < 0 ? 0 : (want > n ? n : (int)want);
+  for (int l = threadIdx.x; l < m; l += kSurvThreads) {
+    const int bl = l / K, k = l - bl * K;
+    double run = 1.0;
+    for (int j = 0; j <= k; ++j) run *= s_c[bl * K + j];
+    a.s_out[b0 * K + l] = (float)run;
+    surv_id[(size_t)k * B + b0 + bl] = run;
   }
-  if (tid == 0 && budget_out != nullptr) *budget_out = B + s_stop;
-  for (int i = tid; i < n_commit; i += kT) atomicAdd(&lcount[idx[i] % B], 1);
-  __syncthreads();
-  for (int b = tid; b < B; b += kT) verify_len[b] = lcount[b];
-  // objective of the committed set: E at n_commit from the owning thread's run
-  const bool owner = (n_commit == n) ? (tid == 0) : (n_commit >= i0 && n_commit < i0 + per);
-  if (owner) {
-    double Ec = (double)B + total;
-    if (n_commit < n) {
-      Ec = (double)B + excl;
-      for (int i = i0; i < n_commit; ++i) Ec += key(i);
+}
+
+__global__ void __launch_bounds__(kRankThreads, 1)
+prefix_rank_kernel(const PrefixArgs a, const double* surv_id, double* okey, int* oidx,
+                   unsigned* counter) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  __shared__ double sl_key[64];
+  __shared__ int sl_id[64];
+  __shared__ int hist[64];
+  __shared__ int s_last;
+  __shared__ float s_xs[64], s_ys[64];
+  __shared__ double shd[32];
+  __shared__ int s_stop, s_budget;
+  const int B = a.B, n = a.B * a.K, tid = threadIdx.x, lane = tid & 31;
+  const int G = gridDim.x;
+  const int p0 = (int)((long long)blockIdx.x * n / G);
+  const int P = (int)((long long)(blockIdx.x + 1) * n / G) - p0;  // 1..kRankSlice
+  if (tid < 64) hist[tid] = 0;
+  // Every read of the survival pass's output comes after this wait, as a
+  // volatile load (__ldcg) that the compiler keeps behind it: an ordinary
+  // load of read-only data may be issued before the wait and return what
+  // the workspace held before the survival pass wrote it.
+  grid_dep_wait();
+  // this thread's candidates: ids tid, tid + kRankThreads, ...
+  double ek[kRankPer];
+#pragma unroll
+  for (int j = 0; j < kRankPer; ++j) {
+    const int e = tid + j * kRankThreads;
+    ek[j] = e < n ? rank_key(__ldcg(surv_id + e)) : 0.0;
+  }
+  if (tid < 32) {
+    // the slice, sorted by one warp; slots past P are sentinels that come
+    // before no candidate
+    for (int p = lane; p < 64; p += 32) {
+      sl_key[p] = p < P ? rank_key(__ldcg(surv_id + p0 + p)) : -CUDART_INF;
+      sl_id[p] = p < P ? p0 + p : 0x7fffffff;
     }
-    objective[0] = (float)(Ec / cost_of(s_xs, s_ys, n_pts, staircase, (double)B + (double)n_commit));
+    __syncwarp();
+    warp_sort<2>(sl_key, sl_id, 0, P);
   }
+  __syncthreads();
+  // q(e) by binary lifting over the 64 slots (q <= P <= 63)
+#pragma unroll
+  for (int j = 0; j < kRankPer; ++j) {
+    const int e = tid + j * kRankThreads;
+    const bool valid = e < n;
+    int q = 0;
+#pragma unroll
+    for (int step = 32; step > 0; step >>= 1) {
+      const int t = q + step - 1;
+      if (cand_before(sl_key[t], sl_id[t], ek[j], e)) q += step;
+    }
+    // most candidates fall before or after the whole slice: those before
+    // are counted per warp, those after are not needed
+    const unsigned m0 = __ballot_sync(0xffffffffu, valid && q == 0);
+    if (lane == 0 && m0 != 0u) atomicAdd(&hist[0], __popc(m0));
+    if (valid && q > 0 && q < P) atomicAdd(&hist[q], 1);
+  }
+  __syncthreads();
+  if (tid < 32) {
+    // place of member p = h[0] + ... + h[p] - 1 (lane l holds p = 2l, 2l+1)
+    const int pa = 2 * lane, pb = pa + 1;
+    const int ha = pa < P ? hist[pa] : 0, hb = pb < P ? hist[pb] : 0;
+    int incl = ha + hb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - ha - hb;
+    if (pa < P) {
+      const int r = min(max(excl + ha - 1, 0), n - 1);
+      okey[r] = __ldcg(surv_id + sl_id[pa]);
+      oidx[r] = sl_id[pa];
+    }
+    if (pb < P) {
+      const int r = min(max(excl + ha + hb - 1, 0), n - 1);
+      okey[r] = __ldcg(surv_id + sl_id[pb]);
+      oidx[r] = sl_id[pb];
+    }
+  }
+  // the last CTA to get here runs the scan over the whole order
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(counter, 1u) == (unsigned)(G - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  double* skeys = reinterpret_cast<double*>(smem_raw);  // [n]
+  int* sidx = reinterpret_cast<int*>(skeys + n);        // [n]
+  int* lcount = sidx + n;                               // [B]
+  for (int i = tid; i < n; i += kRankThreads) {
+    skeys[i] = __ldcg(okey + i);
+    sidx[i] = __ldcg(oidx + i);
+  }
+  for (int b = tid; b < B; b += kRankThreads) lcount[b] = 0;
+  prefix_setup<kRankThreads>(a, s_xs, s_ys, &s_budget, &s_stop, n);
+  prefix_cut<kRankThreads>(a, skeys, sidx, lcount, s_xs, s_ys, s_budget, &s_stop, shd);
+}
+
+// Workspace of the prefix cut: the header, then (multi-CTA form) the
+// survivals by candidate id and the order's keys and ids.
+inline bool prefix_multi(int n, int enable) { return enable && n > kPrefixSmallCand; }
+inline size_t prefix_ws_bytes(int n) {
+  return kHeaderBytes + align256((size_t)n * 8) * 2 + align256((size_t)n * 4);
 }
 
 }  // namespace dspark

@@ -250,7 +250,9 @@ proj_tc_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__
       } else if (a_rows != nullptr) {
         x = b;
       } else {
-        x = (k == 0) ? prev_token[b] : tokens[(size_t)b * K + (k - 1)];
+        // volatile loads (__ldcg), kept behind grid_dep_wait: the token of
+        // position k - 1 comes from the sampler this launch overlaps
+        x = (k == 0) ? __ldcg(prev_token + b) : __ldcg(tokens + (size_t)b * K + (k - 1));
         if (x >= V || (k > 0 && x < 0)) {
           raise_flag(flags, DSPARK_FLAG_BAD_TOKEN);
           x = (k > 0) ? (x < 0 ? 0 : V - 1) : -1;

@@ -153,6 +153,56 @@ def compare_requests(oracle, h, g, L_or, rep=None):
     return rep
 
 
+def cut_problems(oracle, S, cost_tokens, cost_ms, L_g, staircase=False, budget=None,
+                 tol=MARGIN):
+    """Why the verify lengths L_g are not a cut the method could have made:
+    the empty list when they are one.  For where the oracle's own stopping
+    decision lies inside the margin, so the GPU may stop elsewhere.
+
+    The candidates in the oracle's order (survival S descending, then k,
+    then b; S from the oracle, fp64) must give L_g as the per-request counts
+    of the first N = sum(L_g) of them (a swap across the cut of two
+    survivals equal to 1e-9 relative is allowed: the two sides' exp may
+    differ by an ulp).  Greedy cut (budget None): the objective E/t(N) of
+    the oracle's order may fall by at most tol (relative) at every step
+    before N, and may rise by at most tol at the step after it.  Budget cut:
+    N = the budget minus B, clamped to [0, B*K]."""
+    B, K = S.shape
+    n = B * K
+    L_g = np.asarray(L_g)
+    kk, bb = np.meshgrid(np.arange(K), np.arange(B))
+    order = np.lexsort((bb.ravel(), kk.ravel(), -S.ravel()))
+    s_sorted = S.ravel()[order]
+    b_sorted = bb.ravel()[order]
+    N = int(L_g.sum())
+    if L_g.min(initial=0) < 0 or L_g.max(initial=0) > K or not 0 <= N <= n:
+        return [f"lengths out of range (sum {N})"]
+    problems = []
+    counts = np.bincount(b_sorted[:N], minlength=B)
+    if not np.array_equal(counts, L_g):
+        d = L_g - counts
+        swap = (0 < N < n and np.abs(d).sum() == 2 and d[b_sorted[N]] == 1
+                and d[b_sorted[N - 1]] == -1
+                and abs(s_sorted[N - 1] - s_sorted[N]) <= 1e-9 * s_sorted[N - 1])
+        if not swap:
+            problems.append(f"lengths are not the first {N} candidates of the order")
+    if budget is not None:
+        want = min(max(int(budget) - B, 0), n)
+        if N != want:
+            problems.append(f"budget cut of {want} candidates, got {N}")
+        return problems
+    cost = oracle.cost_stair_ms if staircase else oracle.cost_ms
+    E = B + np.concatenate([[0.0], np.cumsum(s_sorted)])
+    t = np.array([cost(cost_tokens, cost_ms, B + m) for m in range(n + 1)])
+    obj = E / t
+    falls = np.nonzero(obj[1:N + 1] < obj[:N] * (1.0 - tol))[0]
+    if falls.size:
+        problems.append(f"went on past a clear fall of the objective at {int(falls[0])} (cut {N})")
+    if N < n and obj[N + 1] > obj[N] * (1.0 + tol):
+        problems.append(f"stopped at {N} while the objective still rose")
+    return problems
+
+
 def compare_prefix(oracle, inp, step, enable_prefix, rep):
     """The prefix cut over the whole batch (it is global over requests);
     returns the oracle's verify lengths."""
@@ -165,7 +215,14 @@ def compare_prefix(oracle, inp, step, enable_prefix, rep):
     rep.checked["prefix"] += 1
     if not np.array_equal(L_g, pr["L"]):
         if pr["margin"] < MARGIN:
-            rep.near["prefix"] += 1
+            # the two sides may stop at different places, but each must
+            # still be a greedy cut of the same order
+            why = cut_problems(oracle, pr["S"], host(inp["cost_tokens"]), host(inp["cost_ms"]),
+                               L_g) if enable_prefix else ["lengths differ with the cut off"]
+            if why:
+                rep.fail("prefix: " + "; ".join(why))
+            else:
+                rep.near["prefix"] += 1
         else:
             rep.fail(f"prefix: verify_len differs (margin {pr['margin']:.3g})")
     elif abs(float(host(step.objective)[0]) - pr["objective"]) > 1e-5 * abs(pr["objective"]):

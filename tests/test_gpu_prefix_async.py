@@ -14,19 +14,21 @@ import torch
 
 from speculative_decoding_05_b200 import dspark as D
 from speculative_decoding_05_b200 import workloads as WL
+from tests.parity import cut_problems
 
 pytestmark = pytest.mark.gpu
 MARGIN = 1e-6
 
 
-def run_gpu(z, temps, xs, ys, staircase, budget=None, enable=True, alias=False):
+def run_gpu(z, temps, xs, ys, staircase, budget=None, enable=True, alias=False, ws=None):
     B, K = z.shape
     c = torch.empty(B, K, device="cuda")
     S = torch.empty(B, K, device="cuda")
     L = torch.empty(B, dtype=torch.int32, device="cuda")
     obj = torch.empty(1, device="cuda")
-    ws = torch.zeros(D.dspark_prefix_workspace_size(B, K, xs.numel()), dtype=torch.uint8,
-                     device="cuda")
+    if ws is None:
+        ws = torch.zeros(D.dspark_prefix_workspace_size(B, K, xs.numel()), dtype=torch.uint8,
+                         device="cuda")
     bin_ = None if budget is None else torch.tensor([budget], dtype=torch.int32, device="cuda")
     bout = bin_ if alias else torch.full((1,), -7, dtype=torch.int32, device="cuda")
     D.dspark_confidence_prefix_async(z, temps, xs, ys, enable, c, S, L, obj, ws,
@@ -48,8 +50,15 @@ def compare(oracle_mod, g, z, temps, xs, ys, staircase, budget=None, enable=True
     if r["margin"] >= MARGIN:
         assert np.array_equal(g["L"], r["L"])
         assert g["objective"] == pytest.approx(r["objective"], rel=1e-5)
-    else:  # a near-tie at the cut: the lengths still form a cut of the same size
-        assert g["L"].sum() == r["L"].sum() or budget is None
+    elif enable:
+        # a near-tie at the cut: the lengths must still be a cut of the same
+        # order (for a budget, of the same size)
+        why = cut_problems(oracle_mod, r["S"], args[2], args[3], g["L"], staircase=staircase,
+                           budget=budget)
+        assert not why, why
+    if enable and budget is None:
+        # the greedy N it returns is its own cut's
+        assert g["n_greedy"] == z.shape[0] + int(g["L"].sum())
     return r
 
 
@@ -80,6 +89,26 @@ def test_small_and_ragged(oracle_mod, B, K):
                     ys, staircase, budget=budget)
         compare(oracle_mod, run_gpu(z, temps, xs, ys, staircase, enable=False), z, temps, xs, ys,
                 staircase, enable=False)
+
+
+@pytest.mark.parametrize("B,K", [(512, 16), (256, 6), (129, 8), (100, 81), (1, 4096),
+                                 (8192, 1)])
+def test_one_workspace_many_calls(oracle_mod, B, K):
+    """Calls in a row on one workspace that starts as garbage, each with new
+    confidences.  Above 1024 candidates the cut runs as several CTAs that
+    pass the survivals and the order through the workspace: a read of what
+    an earlier call left there shows up as a wrong cut here."""
+    temps = WL.seq_temps(K).cuda()
+    xs, ys = (t.cuda() for t in WL.cost_table())
+    ws = torch.full((D.dspark_prefix_workspace_size(B, K, xs.numel()),), 0xA5, dtype=torch.uint8,
+                    device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(B + 7 * K)
+    for t in range(4):
+        z = torch.randn(B, K, generator=g, device="cuda").mul_(1.0 + 0.3 * t).add_(2.0 - 0.4 * t)
+        staircase = t % 2 == 1
+        budget = None if t < 3 else B + (B * K) // 3
+        compare(oracle_mod, run_gpu(z, temps, xs, ys, staircase, budget=budget, ws=ws), z, temps,
+                xs, ys, staircase, budget=budget)
 
 
 def test_budget_word_may_be_shared(oracle_mod):
