@@ -231,6 +231,9 @@ dspark_status dspark_draft_rnn(
 /* 2. Confidence-scheduled prefix cut                                      */
 /* ---------------------------------------------------------------------- */
 
+/* Bytes of the workspace of the two prefix calls: the status word, and for
+ * more than 1024 candidates (B*K) the survivals and the candidate order that
+ * the call's two kernels pass between them (20 bytes per candidate). */
 size_t dspark_prefix_workspace_size(int B, int K, int n_pts);
 
 /*
