@@ -111,6 +111,46 @@ def test_one_workspace_many_calls(oracle_mod, B, K):
                 xs, ys, staircase, budget=budget)
 
 
+def test_large_batch_bad_table_and_nan(oracle_mod):
+    """The multi-CTA form (above 1024 candidates) raises the bad-table flag
+    as the single CTA does, and the next call clears it.  A NaN confidence
+    makes its request's survival NaN from that position on; such candidates
+    are placed after every real one, so the cut equals the oracle's with
+    those confidences at -inf (survival 0, which never raises the
+    objective)."""
+    B, K = 256, 6
+    temps = WL.seq_temps(K).cuda()
+    xs, ys = (t.cuda() for t in WL.cost_table())
+    g = torch.Generator(device="cuda").manual_seed(77)
+    z = torch.randn(B, K, generator=g, device="cuda").add_(1.5)
+    ws = torch.full((D.dspark_prefix_workspace_size(B, K, xs.numel()),), 0x5A, dtype=torch.uint8,
+                    device="cuda")
+    c = torch.empty(B, K, device="cuda")
+    S = torch.empty(B, K, device="cuda")
+    L = torch.empty(B, dtype=torch.int32, device="cuda")
+    obj = torch.empty(1, device="cuda")
+    D.dspark_confidence_prefix(z, temps, xs.flip(0).contiguous(), ys, True, c, S, L, obj, ws)
+    torch.cuda.synchronize()
+    assert D.dspark_get_device_flags(ws, None) & D.FLAG_BAD_TABLE
+    D.dspark_confidence_prefix(z, temps, xs, ys, True, c, S, L, obj, ws)
+    torch.cuda.synchronize()
+    assert D.dspark_get_device_flags(ws, None) == 0
+    zn = z.clone()
+    zn[3, 2] = float("nan")
+    zn[7, 0] = float("nan")
+    D.dspark_confidence_prefix(zn, temps, xs, ys, True, c, S, L, obj, ws)
+    torch.cuda.synchronize()
+    Lg = L.cpu().numpy()
+    assert Lg[3] <= 2 and Lg[7] == 0 and np.isfinite(obj.item())
+    zi = zn.cpu().numpy().copy()
+    zi[np.isnan(zi)] = -np.inf
+    r = oracle_mod.prefix_async(zi, temps.cpu().numpy(), xs.cpu().numpy(), ys.cpu().numpy())
+    if r["margin"] >= MARGIN:
+        assert np.array_equal(Lg, r["L"])
+    else:
+        assert not cut_problems(oracle_mod, r["S"], xs.cpu().numpy(), ys.cpu().numpy(), Lg)
+
+
 def test_budget_word_may_be_shared(oracle_mod):
     w = WL.get("serving")
     z = torch.randn(w.B, w.K, device="cuda").add_(1.5)
