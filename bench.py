@@ -576,6 +576,7 @@ def main():
             print(json.dumps(out), flush=True)
         return
 
+    import numpy as np
     import torch
     import torch.distributed as dist
     from speculative_decoding_05_b200 import build as BLD
@@ -717,22 +718,32 @@ def main():
     # (the logits, temperatures, confidences and row offsets, and that step's
     # uniforms) and its results out; the previous token of a multi-step run
     # stays on the device (the graph carries it), that of a one-step run is
-    # copied in too
+    # copied in too.  With the scheduler on, the target rows come in after
+    # the cut, and only the verified ones (each request's first L_b + 1
+    # rows, packed, with their row offsets): the rows a target model would
+    # compute for that verify.  The host waits for the cut inside the timed
+    # region.
     e2e = None
     if rank == 0 or world > 1:
-        names_in = ["base", "target", "inv_temp", "z", "row_start"]
+        K1 = w.K + 1
+        names_in = ["base", "inv_temp", "z"] + ([] if w.scheduler else ["target", "row_start"])
         if w.steps <= 1:
             names_in.append("prev_token")
         host_in = {k: inp[k].cpu().pin_memory() for k in names_in}
+        host_tgt = inp["target"].cpu().pin_memory() if w.scheduler else None
+        host_rs = torch.empty(w.B, dtype=torch.int64, pin_memory=True)
+        host_vl = torch.empty(w.B, dtype=torch.int32, pin_memory=True)
         host_uni = {k: v.cpu().pin_memory() for k, v in uni.items()}
         outs = [step.n_accepted, step.out_tokens, step.last_token]
         host_out = [torch.empty(o.shape, dtype=o.dtype, pin_memory=True) for o in outs]
-        h2d = sum(t.numel() * t.element_size() for t in host_in.values()) + \
+        h2d_fixed = sum(t.numel() * t.element_size() for t in host_in.values()) + \
             sum(t[0].numel() * t.element_size() for t in host_uni.values())
         d2h = sum(t.numel() * t.element_size() for t in host_out)
+        row_bytes = w.V * inp["target"].element_size()
         n_e2e = max(1, min(args.e2e_steps, args.steps))
         e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                   for _ in range(n_e2e)]
+        h2d_steps = []
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):
             for i in range(n_e2e):
@@ -743,15 +754,47 @@ def main():
                     inp[k].copy_(host_in[k], non_blocking=True)
                 for k, v in host_uni.items():
                     inp[k].copy_(v[j], non_blocking=True)
-                replay()
+                h2d = h2d_fixed
+                if w.scheduler:
+                    graphs[0].replay()
+                    graphs[1].replay()
+                    host_vl.copy_(step.verify_len, non_blocking=True)
+                    stream.synchronize()
+                    rows = host_vl.numpy().clip(0, w.K).astype(np.int64) + 1
+                    rs = host_rs.numpy()
+                    rs[0] = 0
+                    np.cumsum(rows[:-1], out=rs[1:])
+                    for bb in range(w.B):
+                        o, n = int(rs[bb]), int(rows[bb])
+                        inp["target"][o:o + n].copy_(host_tgt[bb * K1:bb * K1 + n],
+                                                     non_blocking=True)
+                    off = int(rs[-1] + rows[-1])
+                    inp["row_start"].copy_(host_rs, non_blocking=True)
+                    h2d += off * row_bytes + host_rs.numel() * 8
+                    d2h_cut = host_vl.numel() * 4
+                    graphs[2].replay()
+                    if w.steps > 1:
+                        inp["prev_token"].copy_(step.last_token)
+                else:
+                    d2h_cut = 0
+                    replay()
                 for o, ho in zip(outs, host_out):
                     ho.copy_(o, non_blocking=True)
                 e2e_ev[i][1].record(stream)
+                h2d_steps.append(h2d)
         torch.cuda.synchronize()
+        if w.scheduler:
+            # the packed layout is what the device buffers now hold; put the
+            # full-batch layout back for anything that runs after this
+            inp["target"].copy_(host_tgt)
+            inp["row_start"].copy_(torch.arange(w.B, dtype=torch.int64) * K1)
+            torch.cuda.synchronize()
         e2e_ms = reduce_max(statistics.mean(a.elapsed_time(b) for a, b in e2e_ev), dev)
         e2e = {"value": whole_job_rate(units_per_rank, world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
-        del host_in, host_uni
+               "h2d_bytes_per_step": statistics.mean(h2d_steps),
+               "d2h_bytes_per_step": d2h + d2h_cut, "ms_per_step": e2e_ms,
+               "target_rows": "verified rows only, after the cut" if w.scheduler else "all"}
+        del host_in, host_uni, host_tgt
 
     vpath = D.dspark_verify_path(w.V, w.r, w.B, w.K, inp["U"].dtype, step.draft_bias is not None)
     n_launch = launches_per_step(step.path, vpath, w.K)

@@ -72,3 +72,38 @@ def test_single_launch_verify_twice_in_a_row(oracle_mod):
         assert not rep.failures, rep.failures[:10]
         outs.append(step.out_tokens.clone())
     assert step.flags()["verify"] == 0
+
+
+PACKED = [
+    (9000, 256, 2, 9, [0, 9], True),             # single-launch verify
+    (4096, 64, 4, 17, [17, 0, 8, 16], False),    # staged, CUDA-core residual
+    (8192, 256, 40, 5, None, False),             # staged, tcgen05 residual
+]
+
+
+@pytest.mark.parametrize("V,r,B,K,lens,keep_bias", PACKED)
+def test_packed_target_rows_match_dense(V, r, B, K, lens, keep_bias):
+    """The target rows may come packed: request b's L_b + 1 verified rows
+    back to back, row_start holding their offsets (what a caller that only
+    computes the verified rows passes).  The outputs equal those of the
+    full (K + 1)-rows-per-request layout bit for bit."""
+    w = WL.get("single", V=V, r=r, B=B, K=K, seed=90 + B + K)
+    inp = WL.make_inputs(w, device="cuda")
+    if lens is None:
+        lens = torch.randint(0, K + 1, (B,), generator=torch.Generator().manual_seed(B)).tolist()
+    step = DSparkStep(w.V, w.r, w.B, w.K, inp["target"].shape[0], inp["U"].dtype,
+                      keep_bias=keep_bias)
+    step.draft(inp)
+    step.verify_len.copy_(torch.tensor(lens, dtype=torch.int32))
+    step.verify(inp)
+    torch.cuda.synchronize()
+    dense = [t.clone() for t in (step.n_accepted, step.out_tokens, step.last_token)]
+    rows = [L + 1 for L in lens]
+    offs = [sum(rows[:b]) for b in range(B)]
+    tgt = torch.cat([inp["target"][b * (K + 1):b * (K + 1) + rows[b]] for b in range(B)])
+    rs = torch.tensor(offs, dtype=torch.int64, device="cuda")
+    step.verify(dict(inp, target=tgt.contiguous(), row_start=rs))
+    torch.cuda.synchronize()
+    assert step.flags()["verify"] == 0
+    for a, b in zip(dense, (step.n_accepted, step.out_tokens, step.last_token)):
+        assert torch.equal(a, b)
