@@ -149,14 +149,16 @@ def source_digest(root=None) -> str:
     return h.hexdigest()[:16]
 
 
-def launches_per_step(draft_path: str, verify_path: str, K: int) -> int:
+def launches_per_step(draft_path: str, verify_path: str, K: int,
+                      prefix_path: str = "single-cta") -> int:
     """Kernels one step launches: the draft (one persistent launch, else a
-    projection and a sampler per position), the prefix cut (one), the verify
-    (one single-launch kernel, else statistics, accept, residual and
-    sample)."""
+    projection and a sampler per position), the prefix cut (one, or a
+    survival and a rank kernel), the verify (one single-launch kernel, else
+    statistics, accept, residual and sample)."""
     draft = 1 if draft_path.startswith(("persistent", "tcgen05-persistent")) else 2 * K
+    prefix = 2 if prefix_path == "multi-cta" else 1
     verify = 1 if verify_path == "single-launch" else 4
-    return draft + 1 + verify
+    return draft + prefix + verify
 
 
 def kernel_name(path: str, call: str, w) -> str:
@@ -797,7 +799,7 @@ def main():
         del host_in, host_uni, host_tgt
 
     vpath = D.dspark_verify_path(w.V, w.r, w.B, w.K, inp["U"].dtype, step.draft_bias is not None)
-    n_launch = launches_per_step(step.path, vpath, w.K)
+    n_launch = launches_per_step(step.path, vpath, w.K, D.dspark_prefix_path(w.B, w.K, w.scheduler))
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inp, args.cpu_seconds)

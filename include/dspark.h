@@ -480,6 +480,13 @@ const char *dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype)
  * either way, up to floating-point summation order. */
 const char *dspark_verify_path(int V, int r, int B, int K, dspark_dtype uw_dtype, int have_bias);
 
+/* Name of the path the prefix calls take for B*K candidates with the
+ * scheduler on (enable != 0) or off: "multi-cta" (more than 1024 candidates,
+ * scheduler on: a survival kernel, then a rank kernel over about B*K / 63
+ * CTAs whose last CTA runs the scan) or "single-cta" (one kernel, one CTA).
+ * Same results either way. */
+const char *dspark_prefix_path(int B, int K, int enable);
+
 /* Library ABI version (major*100 + minor). */
 int dspark_version(void);
 

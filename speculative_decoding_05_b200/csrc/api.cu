@@ -472,7 +472,7 @@ dspark_status noalloc_scratch(void** out) {
 
 extern "C" {
 
-int dspark_version(void) { return 100; }
+int dspark_version(void) { return 101; }
 
 const char* dspark_status_string(dspark_status s) {
   switch (s) {
@@ -492,6 +492,11 @@ const char* dspark_draft_path(int V, int r, int B, int K, dspark_dtype uw_dtype)
   if (use_persist(V, r, B, uw_dtype))
     return gemv_path(r, B) ? "persistent-cuda-core" : "tcgen05-persistent";
   return use_tc(V, r, B, uw_dtype) ? "tcgen05" : "cuda-core";
+}
+
+const char* dspark_prefix_path(int B, int K, int enable) {
+  if (B < 0 || K < 0) return "single-cta";
+  return prefix_multi(B * K, enable) ? "multi-cta" : "single-cta";
 }
 
 const char* dspark_verify_path(int V, int r, int B, int K, dspark_dtype uw_dtype, int have_bias) {

@@ -35,7 +35,8 @@ SYMBOLS = [
     "dspark_prefix_workspace_size", "dspark_confidence_prefix",
     "dspark_verify_workspace_size", "dspark_verify",
     "dspark_get_device_status", "dspark_get_device_flags",
-    "dspark_status_string", "dspark_draft_path", "dspark_verify_path", "dspark_version",
+    "dspark_status_string", "dspark_draft_path", "dspark_verify_path", "dspark_prefix_path",
+    "dspark_version",
     "dspark_verify_noalloc",
     "dspark_verify_noalloc_status",
     "dspark_verify_lmhead_workspace_size",
@@ -116,6 +117,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
     lib.dspark_draft_path.restype = ctypes.c_char_p
     lib.dspark_verify_path.argtypes = [I, I, I, I, I, I]
     lib.dspark_verify_path.restype = ctypes.c_char_p
+    lib.dspark_prefix_path.argtypes = [I, I, I]
+    lib.dspark_prefix_path.restype = ctypes.c_char_p
     lib.dspark_version.argtypes = []
     lib.dspark_version.restype = I
     if path is None:
@@ -168,6 +171,10 @@ def dspark_verify_path(V, r, B, K, uw_dtype, have_bias) -> str:
     code = uw_dtype if isinstance(uw_dtype, int) else (
         DSPARK_BF16 if uw_dtype == torch.bfloat16 else DSPARK_F32)
     return load().dspark_verify_path(V, r, B, K, code, int(bool(have_bias))).decode()
+
+
+def dspark_prefix_path(B, K, enable) -> str:
+    return load().dspark_prefix_path(B, K, int(bool(enable))).decode()
 
 
 def dspark_draft_workspace_size(V, r, B, K) -> int:

@@ -174,6 +174,14 @@ def test_bench_launch_count_follows_the_paths():
     v = D.dspark_verify_path(129280, 256, 256, 6, torch.bfloat16, False)
     assert (d, v) == ("tcgen05", "staged-tcgen05")
     assert bench.launches_per_step(d, v, 6) == 2 * 6 + 1 + 4
+    # the prefix cut of more than 1024 candidates with the scheduler on is
+    # two kernels
+    p = D.dspark_prefix_path(256, 6, True)
+    assert p == "multi-cta"
+    assert bench.launches_per_step(d, v, 6, p) == 2 * 6 + 2 + 4
+    assert D.dspark_prefix_path(256, 6, False) == "single-cta"
+    assert D.dspark_prefix_path(64, 16, True) == "single-cta"   # exactly 1024
+    assert D.dspark_prefix_path(1, 1025, True) == "multi-cta"
 
 
 def test_temperature_fit_workspace_is_bounded(lib):
