@@ -74,6 +74,14 @@ def test_workspace_sizes(lib):
     assert lib.dspark_verify_workspace_size(V, r, B, K) >= 256 + B * nch * 8
     assert lib.dspark_prefix_workspace_size(B, K, 16) >= 4
     assert lib.dspark_draft_workspace_size(0, r, B, K) == 0
+    # the prefix workspace: the 2 KB header, plus (for a valid batch) the
+    # survivals and the order the multi-CTA form passes between its kernels,
+    # 20 bytes per candidate; invalid or oversized batches get the header
+    n = B * K
+    assert lib.dspark_prefix_workspace_size(B, K, 16) >= 2048 + 20 * n
+    assert lib.dspark_prefix_workspace_size(B, K, 16) < 2048 + 20 * n + 3 * 256
+    assert lib.dspark_prefix_workspace_size(1024, 9, 16) == 2048
+    assert lib.dspark_prefix_workspace_size(-1, 4, 16) == 2048
 
 
 def _draft(lib, V=1024, r=16, B=2, K=3, base=1 << 20, U=1 << 21, W=1 << 22, ws=1 << 24,
