@@ -66,6 +66,7 @@ def compare(oracle_mod, g, z, temps, xs, ys, staircase, budget=None, enable=True
 @pytest.mark.parametrize("name", ["serving", "stress"])
 def test_greedy_and_budgets(oracle_mod, name, staircase):
     w = WL.get(name)
+    assert D.dspark_prefix_path(w.B, w.K, True) == "multi-cta"  # 1536 and 8192 candidates
     g = torch.Generator(device="cuda").manual_seed(5)
     z = torch.randn(w.B, w.K, generator=g, device="cuda").add_(1.5)
     temps = WL.seq_temps(w.K).cuda()
@@ -79,6 +80,7 @@ def test_greedy_and_budgets(oracle_mod, name, staircase):
 
 @pytest.mark.parametrize("B,K", [(1, 1), (3, 4), (37, 5), (130, 7)])
 def test_small_and_ragged(oracle_mod, B, K):
+    assert D.dspark_prefix_path(B, K, True) == "single-cta"
     g = torch.Generator(device="cuda").manual_seed(B * 31 + K)
     z = torch.randn(B, K, generator=g, device="cuda").add_(1.0)
     temps = WL.seq_temps(K).cuda()
@@ -98,6 +100,7 @@ def test_one_workspace_many_calls(oracle_mod, B, K):
     confidences.  Above 1024 candidates the cut runs as several CTAs that
     pass the survivals and the order through the workspace: a read of what
     an earlier call left there shows up as a wrong cut here."""
+    assert D.dspark_prefix_path(B, K, True) == "multi-cta"
     temps = WL.seq_temps(K).cuda()
     xs, ys = (t.cuda() for t in WL.cost_table())
     ws = torch.full((D.dspark_prefix_workspace_size(B, K, xs.numel()),), 0xA5, dtype=torch.uint8,
