@@ -112,6 +112,10 @@ def test_one_workspace_many_calls(oracle_mod, B, K):
         budget = None if t < 3 else B + (B * K) // 3
         compare(oracle_mod, run_gpu(z, temps, xs, ys, staircase, budget=budget, ws=ws), z, temps,
                 xs, ys, staircase, budget=budget)
+    # the scheduler off: one CTA (of 1024 threads above 1024 candidates)
+    assert D.dspark_prefix_path(B, K, False) == "single-cta"
+    compare(oracle_mod, run_gpu(z, temps, xs, ys, False, enable=False, ws=ws), z, temps, xs, ys,
+            False, enable=False)
 
 
 def test_large_batch_bad_table_and_nan(oracle_mod):
